@@ -1,0 +1,161 @@
+"""Block manager model in plain Python (oracle; test infrastructure only).
+
+Sources (page title, section):
+  [BLOG] "How PagedAttention Powers vLLM's KV Cache":
+    "PagedAttention: paging, borrowed from the operating system" - when a sequence
+      needs room it takes a free physical block from a shared pool and appends it to
+      its block table; a finished sequence's blocks go back to the pool; nothing is
+      reserved up front.
+    "The bonus contiguous storage can't give you: sharing" - block tables of several
+      sequences may point at one physical block, which carries a reference count;
+      before a sequence writes past the shared region it copies that block
+      (copy-on-write); parallel sampling branches share the prompt's blocks.
+  [LAB] "PagedAttention" explainer:
+    "Add pages as the request grows" / "Block allocation" - a new block only when
+      the current one is full, so only the last block has unused slots.
+    "Share matching prefixes" / "Shared blocks and copy-on-write" - writing into a
+      shared block needs a private copy; appending after a full shared block only
+      needs a new block.
+
+Readings where the pages are silent (the C-ABI allocator follows the same ones):
+  * free pool order: a LIFO stack whose successive pops return free_order[0],
+    free_order[1], ...; a block whose count drops to zero is pushed on top;
+  * a finished sequence releases its blocks in logical order;
+  * copy-on-write fires when the block the next token goes into has count > 1;
+    the writer gets a fresh block, the shared block's count drops by one;
+  * a failing call leaves the state unchanged; a batch of appends is all or nothing;
+  * block-table rows are padded with -1.
+"""
+from __future__ import annotations
+
+import copy
+
+
+class AllocError(Exception):
+    def __init__(self, code: str, msg: str = ""):
+        super().__init__(f"{code}: {msg}")
+        self.code = code
+
+
+NO_FREE_BLOCKS = "NO_FREE_BLOCKS"
+UNKNOWN_SEQ = "UNKNOWN_SEQ"
+SEQ_EXISTS = "SEQ_EXISTS"
+INVALID_ARG = "INVALID_ARG"
+
+
+class BlockManager:
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        if num_blocks <= 0 or block_size <= 0:
+            raise AllocError(INVALID_ARG, "pool and block size must be positive")
+        order = list(range(num_blocks)) if free_order is None else [int(b) for b in free_order]
+        if sorted(order) != list(range(num_blocks)):
+            raise AllocError(INVALID_ARG, "free_order must be a permutation of the pool")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        self.free = order[::-1]          # top of the stack is the end of the list
+        self.ref = [0] * num_blocks
+        self.tables: dict[int, list[int]] = {}
+        self.lens: dict[int, int] = {}
+        self.cow_copies = 0
+        self.blocks_allocated = 0
+
+    # -- helpers -------------------------------------------------------------
+    def _pop(self) -> int:
+        b = self.free.pop()
+        self.ref[b] = 1
+        self.blocks_allocated += 1
+        return b
+
+    def _blocks_for(self, n_tokens: int) -> int:
+        return (n_tokens + self.block_size - 1) // self.block_size
+
+    # -- operations ----------------------------------------------------------
+    def add(self, seq_id: int, n_tokens: int) -> None:
+        """A new sequence with n_tokens cached tokens: ceil(n/bs) fresh blocks."""
+        if seq_id in self.tables:
+            raise AllocError(SEQ_EXISTS, str(seq_id))
+        if n_tokens < 0:
+            raise AllocError(INVALID_ARG, "negative length")
+        need = self._blocks_for(n_tokens)
+        if need > len(self.free):
+            raise AllocError(NO_FREE_BLOCKS, f"need {need}, have {len(self.free)}")
+        self.tables[seq_id] = [self._pop() for _ in range(need)]
+        self.lens[seq_id] = n_tokens
+
+    def fork(self, parent: int, child: int) -> None:
+        """child shares every block of parent (each count + 1)."""
+        if parent not in self.tables:
+            raise AllocError(UNKNOWN_SEQ, str(parent))
+        if child in self.tables:
+            raise AllocError(SEQ_EXISTS, str(child))
+        self.tables[child] = list(self.tables[parent])
+        self.lens[child] = self.lens[parent]
+        for b in self.tables[child]:
+            self.ref[b] += 1
+
+    def append_slot(self, seq_id: int):
+        """Room for one more token: returns (slot, cow_src, cow_dst), -1 = no copy."""
+        if seq_id not in self.tables:
+            raise AllocError(UNKNOWN_SEQ, str(seq_id))
+        table, n = self.tables[seq_id], self.lens[seq_id]
+        off = n % self.block_size
+        src = dst = -1
+        if off == 0:
+            if not self.free:
+                raise AllocError(NO_FREE_BLOCKS, "append")
+            table.append(self._pop())
+        elif self.ref[table[-1]] > 1:
+            if not self.free:
+                raise AllocError(NO_FREE_BLOCKS, "copy-on-write")
+            src = table[-1]
+            dst = self._pop()
+            self.ref[src] -= 1
+            table[-1] = dst
+            self.cow_copies += 1
+        self.lens[seq_id] = n + 1
+        return table[-1] * self.block_size + off, src, dst
+
+    def append_slots(self, seq_ids):
+        """One append per listed sequence, in order; all or nothing."""
+        saved = copy.deepcopy(self.__dict__)
+        try:
+            return [self.append_slot(s) for s in seq_ids]
+        except AllocError:
+            self.__dict__.clear()
+            self.__dict__.update(saved)
+            raise
+
+    def free_seq(self, seq_id: int) -> None:
+        if seq_id not in self.tables:
+            raise AllocError(UNKNOWN_SEQ, str(seq_id))
+        for b in self.tables.pop(seq_id):
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                self.free.append(b)
+        del self.lens[seq_id]
+
+    # -- views ---------------------------------------------------------------
+    def block_tables(self, seq_ids, max_blocks: int):
+        rows, lens = [], []
+        for s in seq_ids:
+            t = self.tables[s]
+            if len(t) > max_blocks:
+                raise AllocError(INVALID_ARG, "table wider than max_blocks")
+            rows.append(t + [-1] * (max_blocks - len(t)))
+            lens.append(self.lens[s])
+        return rows, lens
+
+    def free_list(self):
+        """Free blocks in the order the next pops return them."""
+        return self.free[::-1]
+
+    def stats(self) -> dict:
+        bs = self.block_size
+        used = self.num_blocks - len(self.free)
+        return dict(
+            num_blocks=self.num_blocks, block_size=bs, free_blocks=len(self.free),
+            used_blocks=used, shared_blocks=sum(1 for r in self.ref if r > 1),
+            total_refs=sum(self.ref), num_seqs=len(self.tables),
+            logical_tokens=sum(self.lens.values()), allocated_slots=used * bs,
+            tail_waste_slots=sum(len(t) * bs - self.lens[s] for s, t in self.tables.items()),
+            cow_copies=self.cow_copies, blocks_allocated=self.blocks_allocated)
