@@ -1,0 +1,455 @@
+"""Benchmark of the paged KV-cache decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one decode step of one layer over the whole batch: the block manager
+appends one slot per sequence (copy-on-write pairs where a block is shared), the
+metadata goes to the device, pa_copy_blocks, pa_reshape_and_cache and
+pa_decode_attention run.  Inputs are synthetic (seeded, see ``workloads``) and
+resident in HBM before the timed region; the K/V pool is far larger than L2, so no
+flush is needed between steps.
+
+Under torchrun each rank runs its own replica (its own pool, sequences and seed):
+the path has no exchange step, so there is no collective on the data path; the
+ranks meet only at the barriers around the timed region and in the max-reduction
+of the elapsed time.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (rank 0 only) on bounded samples of the
+same workload and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "paged decode attention: achieved HBM GB/s vs peak; sequences/sec per layer"
+PEAKS_FILE = os.path.join(HERE, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what one step must move at least once)
+# ---------------------------------------------------------------------------
+
+def decode_bytes(cfg, lens, unique_tokens=None) -> int:
+    """K/V of every cached token once + q + out + block-table entries + lengths.
+    ``unique_tokens`` (shared-prefix workloads) counts each physical slot once."""
+    E = cfg.elem_bytes
+    tokens = int(np.sum(lens)) if unique_tokens is None else int(unique_tokens)
+    kv = tokens * cfg.num_kv_heads * cfg.head_dim * 2 * E
+    qo = 2 * cfg.num_seqs * cfg.num_heads * cfg.head_dim * E
+    tab = int(np.sum((np.asarray(lens) + cfg.block_size - 1) // cfg.block_size)) * 4
+    return kv + qo + tab + 4 * cfg.num_seqs
+
+
+def cache_op_bytes(cfg, num_tokens, num_pairs) -> int:
+    E = cfg.elem_bytes
+    row = cfg.num_kv_heads * cfg.head_dim * E
+    reshape = 2 * (2 * num_tokens * row) + 8 * num_tokens       # K and V: read + write
+    copy = 2 * 2 * num_pairs * cfg.block_size * row              # K and V blocks: read + write
+    return reshape + copy
+
+
+def unique_context_tokens(dec, cfg, seq_ids) -> int:
+    """Distinct physical slots the decode reads: a shared block counts once, at the
+    longest fill among the sequences that map it."""
+    fill = {}
+    for s in seq_ids:
+        blocks = dec.alloc.seq_blocks(int(s))
+        L = dec.alloc.seq_len(int(s))
+        for j, b in enumerate(blocks):
+            n = min(cfg.block_size, L - j * cfg.block_size)
+            fill[b] = max(fill.get(b, 0), n)
+    return sum(fill.values())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleTimer:
+    """The CPU oracle's decode attention on whole sequences (all heads)."""
+
+    def __init__(self, cfg, inp):
+        from oracle.step import build_context
+        self.cfg, self.inp = cfg, inp
+        bm, self.k, self.v, _ = build_context(inp, copy_pool=False)
+        ids = list(range(cfg.num_seqs))
+        width = max(len(bm.tables[s]) for s in ids) + 1
+        rows, lens = bm.block_tables(ids, width)
+        self.tables, self.lens = np.array(rows, np.int32), np.array(lens, np.int64)
+        try:
+            from threadpoolctl import threadpool_info
+            self.threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        except Exception:
+            self.threads = 1
+
+    def run(self, seqs):
+        """Seconds spent and algorithmic bytes covered for the listed sequences."""
+        from oracle.attention import paged_decode_attention
+        cfg = self.cfg
+        t0 = time.perf_counter()
+        paged_decode_attention(self.inp.q, self.k, self.v, self.tables, self.lens, cfg.scale,
+                               cfg.block_size, cfg.num_kv_heads, cfg.dtype, seqs=seqs)
+        dt = time.perf_counter() - t0
+        return dt, decode_bytes(cfg.with_(num_seqs=len(seqs)), self.lens[list(seqs)])
+
+    def budgeted(self, budget_s: float):
+        """Sequences in index order until the budget is spent: (GB/s, seq/s, text)."""
+        t_all, b_all, n = 0.0, 0, 0
+        for s in range(self.cfg.num_seqs):
+            dt, b = self.run([s])
+            t_all, b_all, n = t_all + dt, b_all + b, n + 1
+            if t_all > budget_s:
+                break
+        desc = (f"oracle decode attention (float64, all {self.cfg.num_heads} heads) on the "
+                f"first {n} of {self.cfg.num_seqs} sequences "
+                f"({int(self.lens[:n].sum())} tokens), {t_all:.1f} s")
+        return b_all / t_all / 1e9, n / t_all, desc
+
+
+def run_reference(args, cfg):
+    """The oracle as the reference arm: rank 0 only; each step is the oracle on a
+    bounded sample of the workload (two sequences, all heads)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    from workloads import make_inputs
+    timer = OracleTimer(cfg, make_inputs(cfg, args.seed))
+    per_step = 2
+    t_all, b_all = 0.0, 0
+    for i in range(args.warmup + args.steps):
+        seqs = [(i * per_step + j) % cfg.num_seqs for j in range(per_step)]
+        dt, b = timer.run(seqs)
+        if i >= args.warmup:
+            t_all, b_all = t_all + dt, b_all + b
+    value = b_all / t_all / 1e9
+    sample = (f"per step: oracle decode attention (float64, all {cfg.num_heads} heads) of "
+              f"{per_step} of the {cfg.num_seqs} sequences, cycling through the batch")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t_all / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "seqs_per_s": round(per_step * args.steps / t_all, 4),
+        "config": {"workload": cfg.name, "description": cfg.description},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": timer.threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    import paged_kv_cache_342_b200 as pa
+    from paged_kv_cache_342_b200.runtime import PagedDecoder
+    from workloads import TORCH_DTYPES, make_inputs, step_tokens, storage_to_torch
+
+    # CPU baseline first (before any GPU work), rank 0 at N=1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        timer = OracleTimer(cfg, make_inputs(cfg, args.seed))
+        gbs, sps, desc = timer.budgeted(12.0)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": timer.threads, "kind": "oracle",
+               "sample": desc, "seqs_per_s": round(sps, 3)}
+        del timer
+
+    seed = args.seed + rank
+    inp = make_inputs(cfg, seed)
+    S, Hq, Hkv, D, bs = cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
+    nsteps = args.warmup + args.steps
+    max_len = int((inp.context_lens + 1).max()) + nsteps + 1
+    max_blocks = (max_len + bs - 1) // bs
+    kd = storage_to_torch(inp.k_pool, cfg.dtype).to(dev)
+    vd = storage_to_torch(inp.v_pool, cfg.dtype).to(dev)
+    del inp.k_pool, inp.v_pool
+    dec = PagedDecoder(kd, vd, Hq, cfg.scale, max_blocks, inp.free_order, cfg.partition_size)
+    if inp.prefix is None:
+        for s in range(S):
+            dec.admit(s, int(inp.context_lens[s]))
+    else:
+        p = inp.prefix
+        dec.apply_copies(dec.admit_shared_prefix(p.groups, p.samples, p.prefix_len,
+                                                 p.private_lens))
+    dec.bind(range(S))
+
+    # per-step new tokens: host (pinned) and device-resident copies
+    toks_h, toks_d = [], []
+    for i in range(nsteps + (0 if args.no_e2e else args.steps)):
+        q, nk, nv = (inp.q, inp.new_k, inp.new_v) if i == 0 else step_tokens(cfg, seed, i)
+        h = [storage_to_torch(a, cfg.dtype).pin_memory() for a in (q, nk, nv)]
+        toks_h.append(h)
+        if i < nsteps:
+            toks_d.append([t.to(dev) for t in h])
+    out = torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one_step(i, ev=None, tokens=None):
+        q, nk, nv = tokens if tokens is not None else toks_d[i]
+        meta = dec.prepare()
+        n = meta["num_cow"]
+        if n:
+            pa.pa_copy_blocks(kd, vd, dec.d_pairs[:n], meta["pairs"])
+        pa.pa_reshape_and_cache(nk, nv, kd, vd, dec.d_slots)
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_decode_attention(out, q, kd, vd, dec.d_tables, dec.d_lens, cfg.scale, bs, Hkv,
+                               meta["max_len"], cfg.partition_size,
+                               dec._ws if dec._ws.numel() else None)
+        if ev is not None:
+            ev[1].record(stream)
+        parts = max(1, -(-meta["max_len"] // cfg.partition_size))
+        launches = (1 if n else 0) + 1 + 1 + (1 if parts > 1 else 0)
+        return meta, launches
+
+    for i in range(args.warmup):
+        one_step(i)
+    torch.cuda.synchronize(dev)
+    if pa.pa_device_error_read() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    # bytes of the timed steps (lengths grow by one per step)
+    lens0 = np.array([dec.alloc.seq_len(s) for s in range(S)], np.int64)
+    step_bytes, dec_bytes, seqs_done, launches, cows = [], [], 0, 0, 0
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for k in range(args.steps):
+            meta, nl = one_step(args.warmup + k, evs[k])
+            launches += nl
+            cows += meta["num_cow"]
+            L = lens0 + k + 1
+            uniq = unique_context_tokens(dec, cfg, range(S)) if inp.prefix is not None else None
+            db = decode_bytes(cfg, L, uniq)
+            dec_bytes.append(db)
+            step_bytes.append(db + cache_op_bytes(cfg, S, meta["num_cow"]))
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    err = pa.pa_device_error_read()
+    if err:
+        raise RuntimeError(f"device error word {err} after the timed region")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        tb = torch.tensor([float(sum(step_bytes))], device=dev, dtype=torch.float64)
+        dist.all_reduce(tb)
+        total_bytes = float(tb.item())
+    else:
+        total_bytes = float(sum(step_bytes))
+    value = total_bytes / (elapsed_ms * 1e-3) / 1e9
+    seqs_per_s = S * world * args.steps / (elapsed_ms * 1e-3)
+
+    # ---- end to end through the public API with host buffers ----------------------
+    e2e = None
+    if not args.no_e2e:
+        out_h = torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], pin_memory=True)
+        tok_bufs = [torch.empty_like(t, device=dev) for t in toks_d[0]]
+        base = nsteps
+        e_bytes = []
+        # warm-up of this mode
+        for k in range(3):
+            for dst, src in zip(tok_bufs, toks_h[base + k % args.steps]):
+                dst.copy_(src, non_blocking=True)
+            one_step(0, tokens=tok_bufs)
+            out_h.copy_(out, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        lens1 = np.array([dec.alloc.seq_len(s) for s in range(S)], np.int64)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in range(args.steps):
+            for dst, src in zip(tok_bufs, toks_h[base + k]):
+                dst.copy_(src, non_blocking=True)
+            meta, _ = one_step(0, tokens=tok_bufs)
+            out_h.copy_(out, non_blocking=True)
+            L = lens1 + k + 1
+            uniq = unique_context_tokens(dec, cfg, range(S)) if inp.prefix is not None else None
+            e_bytes.append(decode_bytes(cfg, L, uniq) + cache_op_bytes(cfg, S, meta["num_cow"]))
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        E = sum(e_bytes) * world / (e_ms * 1e-3) / 1e9
+        h2d = sum(t.numel() * t.element_size() for t in toks_h[0])
+        h2d += S * 8 + S * max_blocks * 4 + S * 4          # slots, tables, lengths
+        d2h = S * Hq * D * cfg.elem_bytes
+        e2e = {"value": round(E, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / args.steps, 4)}
+
+    # ---- roofline of the decode call --------------------------------------------
+    peak, peak_kind = hbm_peak()
+    dec_avg_ms = statistics.mean(dec_ms)
+    achieved = statistics.mean(dec_bytes) / (dec_avg_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+            "kernel": "pa_decode_attention (partition kernel + log-sum-exp merge)",
+            "bytes_per_launch": int(statistics.mean(dec_bytes)),
+            "avg_launch_us": round(dec_avg_ms * 1e3, 2),
+            "frac_of_nominal_8000": round(achieved / 8000.0, 4),
+            "traffic": None}
+    prof = os.path.join(HERE, "profiles", f"traffic_{cfg.name}.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                roof["traffic"] = json.load(f).get("traffic_bytes_per_launch")
+        except (OSError, ValueError):
+            pass
+
+    if rank == 0:
+        ws = dec._ws.numel()
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "seqs_per_s": round(seqs_per_s, 1),
+            "config": {"workload": cfg.name, "description": cfg.description,
+                       "num_seqs": S, "num_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
+                       "block_size": bs, "num_blocks": cfg.num_blocks,
+                       "partition_size": cfg.partition_size,
+                       "mean_seq_len": round(float((lens0 + 1).mean()), 1),
+                       "l2": "inputs larger than L2 (K/V pool %.2f GB per rank), no flush"
+                             % (2 * kd.numel() * kd.element_size() / 1e9),
+                       "parallelism": f"replicas x{world}", "workspace_bytes": int(ws),
+                       "cow_pairs_in_timed_steps": cows},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    from workloads import CONFIGS, HEADLINE
+    cfg = CONFIGS[args.workload or HEADLINE]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

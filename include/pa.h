@@ -1,0 +1,253 @@
+/*
+ * pa.h - C ABI of the B200 (sm_100a) paged KV-cache decode library (libpa.so).
+ *
+ * The operation is PagedAttention's data path as three web pages describe it:
+ *   [GLOSS] "PagedAttention", inferensys.com LLM-operations glossary;
+ *   [BLOG]  "How PagedAttention Powers vLLM's KV Cache", hassanahmed.net;
+ *   [LAB]   "PagedAttention", divagr.pages.dev attention-lab explainer.
+ * Keys and values of each sequence live in fixed-size physical blocks of one shared
+ * pool; a per-sequence block table maps logical block j to a physical block ([BLOG]
+ * "PagedAttention: paging, borrowed from the operating system"; [LAB] "Keep pages in
+ * order").  The attention kernel walks that table and gathers K/V block by block
+ * ([BLOG] "The attention kernel has to read scattered blocks"); blocks are shared
+ * between sequences with reference counts and copied before a shared block is
+ * written ([BLOG] "The bonus contiguous storage can't give you: sharing"; [LAB]
+ * "Share matching prefixes").
+ *
+ * Conventions shared by every entry point
+ *   - Return value: a pa_status.  PA_OK is 0; anything else means the call did
+ *     nothing (argument errors are found before any launch) or, for PA_ERR_CUDA,
+ *     that a launch failed.
+ *   - Tensor arguments of the GPU entry points are DEVICE pointers owned by the
+ *     caller, contiguous, 16-byte aligned, in the layouts stated below.  The
+ *     library never allocates, frees or keeps device memory; scratch space is
+ *     passed in by the caller (see pa_decode_workspace_bytes).
+ *   - GPU work is enqueued on the caller's stream (a cudaStream_t passed as
+ *     pa_stream_t; NULL = legacy default stream) and is asynchronous: no entry
+ *     point synchronises, except pa_device_error_read.
+ *   - Element types: PA_F32, PA_BF16, PA_F16.  q, out and both caches share one.
+ *   - Cache layout (K and V alike): [num_blocks, num_kv_heads, block_size, head_dim];
+ *     so each (block, kv head) pair is one contiguous block_size*head_dim run.
+ *     Slot s means block s / block_size, offset s % block_size.
+ *   - Kernels check every block id and slot they dereference against num_blocks.
+ *     An out-of-range index is skipped (never dereferenced) and recorded in a
+ *     device error word; pa_device_error_read returns and clears it.
+ *   - Allocator handles are host objects owned by the library; not thread-safe.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,    /* bad pointer, size, dtype, alignment or workspace   */
+  PA_ERR_NO_FREE_BLOCKS = 2, /* the pool cannot supply the blocks this call needs  */
+  PA_ERR_UNKNOWN_SEQ = 3,    /* sequence id not present in the allocator            */
+  PA_ERR_SEQ_EXISTS = 4,     /* sequence id already present                         */
+  PA_ERR_BAD_INDEX = 5,      /* a kernel met an out-of-range block id / slot / len  */
+  PA_ERR_CUDA = 6,           /* a CUDA runtime call or launch failed                */
+  PA_ERR_UNSUPPORTED = 7     /* valid but not built: head_dim / block_size / dtype  */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
+
+typedef void* pa_stream_t; /* a cudaStream_t */
+
+/* Bits of the device error word (pa_device_error_read). */
+#define PA_DEVERR_SLOT 1u        /* reshape_and_cache: slot >= num_blocks*block_size */
+#define PA_DEVERR_COPY_BLOCK 2u  /* copy_blocks: src or dst outside [0, num_blocks)  */
+#define PA_DEVERR_TABLE 4u       /* decode: block-table entry outside [0, num_blocks)*/
+#define PA_DEVERR_SEQ_LEN 8u     /* decode: seq_len < 0, > max_seq_len or > table    */
+#define PA_DEVERR_TIMEOUT 16u    /* a bounded wait on an async copy gave up          */
+
+/* ------------------------------------------------------------------------- */
+/* GPU entry points                                                           */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * pa_reshape_and_cache - write each new token's K and V into its slot.
+ * ([BLOG] "Quick recap: the KV cache is per token, and it grows": each generated
+ * token adds one key and one value; the slot comes from the block manager.)
+ *
+ *   key, value    [num_tokens, num_kv_heads, head_dim]           (read)
+ *   k_cache, v_cache  cache layout above                          (written)
+ *   slot_mapping  int64 [num_tokens]; slot of token t, or -1 = skip (read)
+ * For every t with slot_mapping[t] >= 0: k_cache[slot/bs, h, slot%bs, :] =
+ * key[t, h, :] for all h, and the same for V.  Bits are copied unchanged.
+ * Slots must be distinct (two tokens with one slot race).  A slot >=
+ * num_blocks*block_size is skipped and sets PA_DEVERR_SLOT.
+ * head_dim*element size must be a multiple of 16 bytes.  num_tokens == 0 is a no-op.
+ */
+int pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int64_t num_blocks, int dtype,
+                         pa_stream_t stream);
+
+/*
+ * pa_copy_blocks - make the private copies of copy-on-write.
+ * ([BLOG] "The bonus contiguous storage can't give you: sharing": a sequence that
+ * writes into a shared block first copies it; [LAB] "Share matching prefixes".)
+ *
+ *   block_mapping_dev   int32 [num_pairs, 2] (src, dst) pairs on the device (read)
+ *   block_mapping_host  the same pairs in host memory, used only to validate;
+ *                       may be NULL to skip validation
+ * Every dst block (all kv heads, all slots) of K and V becomes a copy of its src.
+ * With block_mapping_host given, the call returns PA_ERR_INVALID_ARG unless every
+ * id is in [0, num_blocks), no dst repeats and no dst is also a src (so the result
+ * does not depend on the order the pairs run in).  A src may repeat.  The kernel
+ * re-checks ids and skips (PA_DEVERR_COPY_BLOCK) any outside the pool.
+ * num_pairs == 0 is a no-op.
+ */
+int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_mapping_dev,
+                   const int32_t* block_mapping_host, int num_pairs, int num_kv_heads,
+                   int head_dim, int block_size, int64_t num_blocks, int dtype,
+                   pa_stream_t stream);
+
+/*
+ * pa_decode_workspace_bytes - scratch bytes pa_decode_attention needs.
+ * P = ceil(max_seq_len / partition_size) partitions per sequence; when P > 1 the
+ * workspace holds float32 partial outputs [num_seqs, num_heads, P, head_dim] and
+ * float32 running max / exp-sum [num_seqs, num_heads, P] each.  Returns 0 when
+ * P <= 1 (no merge needed) and 0 for invalid sizes.
+ */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_seq_len,
+                                 int partition_size);
+
+/*
+ * pa_decode_attention - single-query (decode) attention over the paged cache.
+ * ([BLOG] "The attention kernel has to read scattered blocks"; [LAB] "Keep pages in
+ * order" and "Measure memory use across requests": the attention equation is
+ * unchanged, only the K/V addressing goes through the block table; [BLOG] "Where it
+ * bites": grouped-query attention, several query heads sharing one kv head.)
+ *
+ *   out           [num_seqs, num_heads, head_dim]                 (written)
+ *   q             [num_seqs, num_heads, head_dim]                 (read)
+ *   k_cache, v_cache  cache layout above                          (read)
+ *   block_tables  int32 [num_seqs, max_blocks_per_seq]; row s lists the physical
+ *                 blocks of sequence s in logical order; entries past
+ *                 ceil(seq_lens[s]/block_size) are never read   (read)
+ *   seq_lens      int32 [num_seqs]: cached tokens of each sequence, including the
+ *                 token written this step                          (read)
+ *   scale         logit scale (typically 1/sqrt(head_dim))
+ *   block_size, num_kv_heads   as in the cache; num_heads % num_kv_heads == 0
+ *   max_seq_len   host-side upper bound of seq_lens (sizes the grid and workspace
+ *                 without a device-to-host read); a longer seq_len is skipped and
+ *                 sets PA_DEVERR_SEQ_LEN
+ *   partition_size  tokens per partition (multiple of block_size; 0 = 512).  A
+ *                 sequence longer than one partition is split; the partitions are
+ *                 merged by log-sum-exp weights in a second kernel.
+ *   workspace     device scratch of at least pa_decode_workspace_bytes(...) bytes
+ *                 (may be NULL when that is 0); contents need no initialisation.
+ * For each sequence s and query head h (kv head g = h / (num_heads/num_kv_heads)):
+ *   out[s,h,:] = sum_t softmax_t(scale * q[s,h,:] . K_t) V_t over the seq_lens[s]
+ * cached tokens t, K_t/V_t read from block block_tables[s, t / block_size], offset
+ * t % block_size, kv head g.  Accumulation is float32; out is rounded to the cache
+ * dtype (round-to-nearest-even).  seq_lens[s] == 0 gives zeros.
+ * Supported: head_dim in {64, 128, 256}; block_size in {4, 8, 16, 32}; tensor-core
+ * path for num_heads/num_kv_heads a multiple of 8 with bf16/f16, head_dim 64/128/256
+ * and block_size 16/32; other shapes use the CUDA-core path.
+ */
+int pa_decode_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, const int32_t* seq_lens, float scale,
+                        int block_size, int num_kv_heads, int num_seqs, int num_heads,
+                        int head_dim, int max_blocks_per_seq, int64_t num_blocks,
+                        int max_seq_len, int partition_size, int dtype, void* workspace,
+                        size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_decode_uses_tensor_cores - 1 if pa_decode_attention serves this shape with the
+ * tensor-core (mma.sync) partition kernel, 0 if with the CUDA-core kernel.  Host
+ * only; no GPU work.
+ */
+int pa_decode_uses_tensor_cores(int dtype, int num_heads, int num_kv_heads, int head_dim,
+                                int block_size);
+
+/*
+ * pa_device_error_read - synchronise the current device, then return (in *bits) and
+ * clear the device error word that the kernels set on out-of-range indices or on
+ * a bounded wait that gave up (PA_DEVERR_* bits; 0 = none).
+ */
+int pa_device_error_read(uint32_t* bits);
+
+/* ------------------------------------------------------------------------- */
+/* Host block allocator                                                       */
+/* ------------------------------------------------------------------------- */
+/*
+ * The block manager of [BLOG] "PagedAttention: paging, borrowed from the operating
+ * system" and "The bonus contiguous storage can't give you: sharing", and [LAB]
+ * "Add pages as the request grows" / "Share matching prefixes":
+ *   - one pool of num_blocks physical blocks of block_size token slots;
+ *   - a sequence takes a new block only when its last block is full, so only its
+ *     last block can have unused slots;
+ *   - fork shares every block of a parent with a child (reference counts + 1);
+ *   - copy-on-write: when the block the next token goes into is shared (count > 1)
+ *     the writer gets a fresh block and a (src, dst) pair to copy with
+ *     pa_copy_blocks before writing; after a full shared block only a new block is
+ *     taken;
+ *   - a freed sequence drops its counts; blocks that reach zero return to the pool.
+ * Pool order: a LIFO stack whose successive pops return free_order[0],
+ * free_order[1], ... (identity order when free_order is NULL); a block returned to
+ * the pool goes on top; a freed sequence returns its blocks in logical order.
+ * Every failing call leaves the allocator state unchanged.
+ */
+typedef struct pa_alloc pa_alloc_t;
+
+typedef struct {
+  int64_t num_blocks;        /* pool size                                        */
+  int64_t block_size;        /* token slots per block                            */
+  int64_t free_blocks;       /* blocks in the free pool                          */
+  int64_t used_blocks;       /* blocks with reference count > 0                  */
+  int64_t shared_blocks;     /* blocks with reference count > 1                  */
+  int64_t total_refs;        /* sum of reference counts = block-table entries    */
+  int64_t num_seqs;          /* live sequences                                   */
+  int64_t logical_tokens;    /* sum of sequence lengths                          */
+  int64_t allocated_slots;   /* used_blocks * block_size                         */
+  int64_t tail_waste_slots;  /* sum over sequences of blocks*block_size - length */
+  int64_t cow_copies;        /* copy-on-write pairs issued so far                */
+  int64_t blocks_allocated;  /* blocks taken from the pool so far                */
+} pa_stats_t;
+
+/* Create a pool; free_order (host int32 [num_blocks], a permutation) or NULL. */
+int pa_alloc_create(int64_t num_blocks, int block_size, const int32_t* free_order,
+                    pa_alloc_t** out);
+int pa_alloc_destroy(pa_alloc_t* a);
+
+/* Admit seq_id with num_tokens cached tokens: ceil(num_tokens/block_size) blocks. */
+int pa_seq_add(pa_alloc_t* a, int64_t seq_id, int64_t num_tokens);
+/* child shares all of parent's blocks and its length. */
+int pa_seq_fork(pa_alloc_t* a, int64_t parent, int64_t child);
+/* Room for one more token of seq_id: *slot receives its slot; *cow_src/*cow_dst the
+ * copy to make first, or -1/-1.  Length grows by one. */
+int pa_seq_append_slot(pa_alloc_t* a, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                       int32_t* cow_dst);
+/* One append for each of seq_ids[0..n) in order, all or nothing.  slots[i] gets the
+ * slot of seq_ids[i]; the copy pairs go to cow_pairs (int32 [n, 2] capacity) in
+ * order, their count to *num_cow. */
+int pa_seq_append_slots(pa_alloc_t* a, const int64_t* seq_ids, int n, int64_t* slots,
+                        int32_t* cow_pairs, int* num_cow);
+/* Release seq_id. */
+int pa_seq_free(pa_alloc_t* a, int64_t seq_id);
+int pa_seq_len(const pa_alloc_t* a, int64_t seq_id, int64_t* len);
+/* Copy seq_id's block table (logical order) into out[0..cap); *n = its length. */
+int pa_seq_blocks(const pa_alloc_t* a, int64_t seq_id, int32_t* out, int64_t cap,
+                  int64_t* n);
+/* Host int32 tables [num_seqs, max_blocks_per_seq] (rows padded with -1) and int32
+ * seq_lens [num_seqs] for the listed sequences, ready to copy to the device. */
+int pa_build_block_tables(const pa_alloc_t* a, const int64_t* seq_ids, int num_seqs,
+                          int32_t* tables, int max_blocks_per_seq, int32_t* seq_lens);
+int pa_block_refcount(const pa_alloc_t* a, int32_t block, int32_t* refcount);
+/* Free blocks in the order the next pops return them; *n = how many. */
+int pa_alloc_free_list(const pa_alloc_t* a, int32_t* out, int64_t cap, int64_t* n);
+int pa_alloc_stats(const pa_alloc_t* a, pa_stats_t* stats);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

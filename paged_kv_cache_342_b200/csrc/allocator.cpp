@@ -1,0 +1,301 @@
+// Host block manager for the paged KV cache (C ABI in include/pa.h).
+//
+// Behaviour from "How PagedAttention Powers vLLM's KV Cache" (hassanahmed.net),
+// sections "PagedAttention: paging, borrowed from the operating system" (blocks
+// from a shared free pool, appended on demand, returned when a sequence ends) and
+// "The bonus contiguous storage can't give you: sharing" (reference counts,
+// copy-on-write, parallel samples sharing a prompt), and from the "PagedAttention"
+// attention-lab explainer (divagr.pages.dev), sections "Add pages as the request
+// grows" and "Share matching prefixes" (a new block only when the last is full;
+// after a full shared block only a new block, no copy).
+//
+// Pool order (not fixed by the pages): a LIFO stack; pops return free_order[0],
+// free_order[1], ...; a released block goes on top; a freed sequence releases its
+// blocks in logical order.  Every failing call leaves the state unchanged.
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/pa.h"
+
+namespace {
+
+struct Seq {
+  std::vector<int32_t> blocks;  // logical order
+  int64_t len = 0;
+};
+
+}  // namespace
+
+struct pa_alloc {
+  int64_t num_blocks = 0;
+  int block_size = 0;
+  std::vector<int32_t> free_stack;  // back() is the top
+  std::vector<int32_t> ref;
+  std::unordered_map<int64_t, Seq> seqs;
+  int64_t cow_copies = 0;
+  int64_t blocks_allocated = 0;
+  int64_t shared_blocks = 0;  // maintained incrementally: count of ref > 1
+
+  int32_t pop() {
+    int32_t b = free_stack.back();
+    free_stack.pop_back();
+    ref[b] = 1;
+    ++blocks_allocated;
+    return b;
+  }
+  void inc(int32_t b) {
+    if (++ref[b] == 2) ++shared_blocks;
+  }
+  void dec(int32_t b) {
+    if (ref[b]-- == 2) --shared_blocks;
+    if (ref[b] == 0) free_stack.push_back(b);
+  }
+};
+
+namespace {
+
+inline int64_t blocks_for(int64_t n, int bs) { return (n + bs - 1) / bs; }
+
+// Blocks one append to `s` takes from the pool, given the (possibly simulated)
+// reference count of its last block.
+inline bool append_needs_block(const Seq& s, int bs, int32_t last_ref) {
+  if (s.len % bs == 0) return true;
+  return last_ref > 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_alloc_create(int64_t num_blocks, int block_size, const int32_t* free_order,
+                    pa_alloc_t** out) {
+  if (!out || num_blocks <= 0 || block_size <= 0 || num_blocks > INT32_MAX)
+    return PA_ERR_INVALID_ARG;
+  *out = nullptr;
+  pa_alloc* a = new (std::nothrow) pa_alloc();
+  if (!a) return PA_ERR_INVALID_ARG;
+  a->num_blocks = num_blocks;
+  a->block_size = block_size;
+  a->ref.assign(static_cast<size_t>(num_blocks), 0);
+  a->free_stack.resize(static_cast<size_t>(num_blocks));
+  if (free_order) {
+    std::vector<uint8_t> seen(static_cast<size_t>(num_blocks), 0);
+    for (int64_t i = 0; i < num_blocks; ++i) {
+      int32_t b = free_order[i];
+      if (b < 0 || b >= num_blocks || seen[b]) {
+        delete a;
+        return PA_ERR_INVALID_ARG;
+      }
+      seen[b] = 1;
+      a->free_stack[static_cast<size_t>(num_blocks - 1 - i)] = b;
+    }
+  } else {
+    for (int64_t i = 0; i < num_blocks; ++i)
+      a->free_stack[static_cast<size_t>(num_blocks - 1 - i)] = static_cast<int32_t>(i);
+  }
+  *out = a;
+  return PA_OK;
+}
+
+int pa_alloc_destroy(pa_alloc_t* a) {
+  delete a;
+  return PA_OK;
+}
+
+int pa_seq_add(pa_alloc_t* a, int64_t seq_id, int64_t num_tokens) {
+  if (!a || num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (a->seqs.count(seq_id)) return PA_ERR_SEQ_EXISTS;
+  int64_t need = blocks_for(num_tokens, a->block_size);
+  if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_NO_FREE_BLOCKS;
+  Seq s;
+  s.blocks.reserve(static_cast<size_t>(need + 1));
+  for (int64_t i = 0; i < need; ++i) s.blocks.push_back(a->pop());
+  s.len = num_tokens;
+  a->seqs.emplace(seq_id, std::move(s));
+  return PA_OK;
+}
+
+int pa_seq_fork(pa_alloc_t* a, int64_t parent, int64_t child) {
+  if (!a) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(parent);
+  if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
+  if (a->seqs.count(child)) return PA_ERR_SEQ_EXISTS;
+  Seq c = it->second;  // copy of the table and length
+  for (int32_t b : c.blocks) a->inc(b);
+  a->seqs.emplace(child, std::move(c));
+  return PA_OK;
+}
+
+static int64_t append_one(pa_alloc* a, Seq& s, int32_t* src, int32_t* dst) {
+  const int bs = a->block_size;
+  const int64_t off = s.len % bs;
+  *src = -1;
+  *dst = -1;
+  if (off == 0) {
+    s.blocks.push_back(a->pop());
+  } else {
+    int32_t last = s.blocks.back();
+    if (a->ref[last] > 1) {
+      int32_t fresh = a->pop();
+      a->dec(last);  // stays > 0: it was shared
+      s.blocks.back() = fresh;
+      *src = last;
+      *dst = fresh;
+      ++a->cow_copies;
+    }
+  }
+  ++s.len;
+  return static_cast<int64_t>(s.blocks.back()) * bs + off;
+}
+
+int pa_seq_append_slot(pa_alloc_t* a, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                       int32_t* cow_dst) {
+  if (!a || !slot || !cow_src || !cow_dst) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
+  Seq& s = it->second;
+  bool need = append_needs_block(s, a->block_size, s.blocks.empty() ? 0 : a->ref[s.blocks.back()]);
+  if (need && a->free_stack.empty()) return PA_ERR_NO_FREE_BLOCKS;
+  *slot = append_one(a, s, cow_src, cow_dst);
+  return PA_OK;
+}
+
+int pa_seq_append_slots(pa_alloc_t* a, const int64_t* seq_ids, int n, int64_t* slots,
+                        int32_t* cow_pairs, int* num_cow) {
+  if (!a || n < 0 || (n > 0 && (!seq_ids || !slots || !cow_pairs)) || !num_cow)
+    return PA_ERR_INVALID_ARG;
+  // Dry run: count the blocks the batch takes, simulating lengths and the
+  // reference counts that earlier copies in the batch drop.
+  std::unordered_map<int64_t, int64_t> len_delta;
+  std::unordered_map<int32_t, int32_t> ref_drop;
+  std::unordered_map<int64_t, int32_t> last_block;  // seqs whose last block changed
+  int64_t need = 0;
+  const int bs = a->block_size;
+  for (int i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
+    const Seq& s = it->second;
+    int64_t len = s.len + len_delta[seq_ids[i]];
+    if (len % bs == 0) {
+      ++need;
+      last_block[seq_ids[i]] = -1;  // a fresh, private block
+    } else {
+      auto lb = last_block.find(seq_ids[i]);
+      int32_t last = (lb != last_block.end()) ? lb->second : s.blocks.back();
+      if (last >= 0) {
+        int32_t r = a->ref[last] - ref_drop[last];
+        if (r > 1) {
+          ++need;
+          ++ref_drop[last];
+          last_block[seq_ids[i]] = -1;
+        }
+      }
+    }
+    ++len_delta[seq_ids[i]];
+  }
+  if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_NO_FREE_BLOCKS;
+  int nc = 0;
+  for (int i = 0; i < n; ++i) {
+    Seq& s = a->seqs.find(seq_ids[i])->second;
+    int32_t src, dst;
+    slots[i] = append_one(a, s, &src, &dst);
+    if (src >= 0) {
+      cow_pairs[2 * nc] = src;
+      cow_pairs[2 * nc + 1] = dst;
+      ++nc;
+    }
+  }
+  *num_cow = nc;
+  return PA_OK;
+}
+
+int pa_seq_free(pa_alloc_t* a, int64_t seq_id) {
+  if (!a) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
+  for (int32_t b : it->second.blocks) a->dec(b);
+  a->seqs.erase(it);
+  return PA_OK;
+}
+
+int pa_seq_len(const pa_alloc_t* a, int64_t seq_id, int64_t* len) {
+  if (!a || !len) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
+  *len = it->second.len;
+  return PA_OK;
+}
+
+int pa_seq_blocks(const pa_alloc_t* a, int64_t seq_id, int32_t* out, int64_t cap, int64_t* n) {
+  if (!a || !n || cap < 0 || (cap > 0 && !out)) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
+  const auto& b = it->second.blocks;
+  *n = static_cast<int64_t>(b.size());
+  int64_t m = cap < *n ? cap : *n;
+  if (m > 0) std::memcpy(out, b.data(), static_cast<size_t>(m) * sizeof(int32_t));
+  return PA_OK;
+}
+
+int pa_build_block_tables(const pa_alloc_t* a, const int64_t* seq_ids, int num_seqs,
+                          int32_t* tables, int max_blocks_per_seq, int32_t* seq_lens) {
+  if (!a || num_seqs < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs > 0 && (!seq_ids || !tables || !seq_lens)) return PA_ERR_INVALID_ARG;
+  for (int i = 0; i < num_seqs; ++i) {  // validate first: all or nothing
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
+    if (static_cast<int64_t>(it->second.blocks.size()) > max_blocks_per_seq ||
+        it->second.len > INT32_MAX)
+      return PA_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < num_seqs; ++i) {
+    const Seq& s = a->seqs.find(seq_ids[i])->second;
+    int32_t* row = tables + static_cast<int64_t>(i) * max_blocks_per_seq;
+    size_t nb = s.blocks.size();
+    if (nb) std::memcpy(row, s.blocks.data(), nb * sizeof(int32_t));
+    for (int64_t j = static_cast<int64_t>(nb); j < max_blocks_per_seq; ++j) row[j] = -1;
+    seq_lens[i] = static_cast<int32_t>(s.len);
+  }
+  return PA_OK;
+}
+
+int pa_block_refcount(const pa_alloc_t* a, int32_t block, int32_t* refcount) {
+  if (!a || !refcount || block < 0 || block >= a->num_blocks) return PA_ERR_INVALID_ARG;
+  *refcount = a->ref[block];
+  return PA_OK;
+}
+
+int pa_alloc_free_list(const pa_alloc_t* a, int32_t* out, int64_t cap, int64_t* n) {
+  if (!a || !n || cap < 0 || (cap > 0 && !out)) return PA_ERR_INVALID_ARG;
+  const auto& fs = a->free_stack;
+  *n = static_cast<int64_t>(fs.size());
+  int64_t m = cap < *n ? cap : *n;
+  for (int64_t i = 0; i < m; ++i) out[i] = fs[fs.size() - 1 - static_cast<size_t>(i)];
+  return PA_OK;
+}
+
+int pa_alloc_stats(const pa_alloc_t* a, pa_stats_t* st) {
+  if (!a || !st) return PA_ERR_INVALID_ARG;
+  std::memset(st, 0, sizeof(*st));
+  st->num_blocks = a->num_blocks;
+  st->block_size = a->block_size;
+  st->free_blocks = static_cast<int64_t>(a->free_stack.size());
+  st->used_blocks = a->num_blocks - st->free_blocks;
+  st->shared_blocks = a->shared_blocks;
+  st->num_seqs = static_cast<int64_t>(a->seqs.size());
+  for (const auto& kv : a->seqs) {
+    const Seq& s = kv.second;
+    st->total_refs += static_cast<int64_t>(s.blocks.size());
+    st->logical_tokens += s.len;
+    st->tail_waste_slots += static_cast<int64_t>(s.blocks.size()) * a->block_size - s.len;
+  }
+  st->allocated_slots = st->used_blocks * a->block_size;
+  st->cow_copies = a->cow_copies;
+  st->blocks_allocated = a->blocks_allocated;
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,168 @@
+// Cache maintenance kernels: pa_reshape_and_cache (write each new token's K/V into
+// its slot) and pa_copy_blocks (the private copy of copy-on-write).
+//
+// "How PagedAttention Powers vLLM's KV Cache" (hassanahmed.net), "Quick recap: the
+// KV cache is per token, and it grows" and "The bonus contiguous storage can't give
+// you: sharing"; "PagedAttention" attention-lab explainer (divagr.pages.dev),
+// "Share matching prefixes".
+//
+// Both are pure HBM copies: 16-byte vectors, one per thread per step, grid-stride
+// loops sized to the SM count.  Cache layout [num_blocks, num_kv_heads, block_size,
+// head_dim]; one block of one tensor is num_kv_heads*block_size*head_dim elements.
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+
+namespace pa {
+namespace {
+
+// One 16-byte vector of one token row per thread.  nvr = vectors per (token, head) row.
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(
+    const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ k_cache,
+    uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int64_t num_tokens,
+    int num_kv_heads, int nvr, int block_size, int64_t num_slots, uint32_t* err) {
+  const int64_t per_token = static_cast<int64_t>(num_kv_heads) * nvr;
+  const int64_t total = num_tokens * per_token;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_token;
+    const int64_t r = i - t * per_token;
+    const int h = static_cast<int>(r / nvr);
+    const int v = static_cast<int>(r - static_cast<int64_t>(h) * nvr);
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      set_error(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t blk = slot / block_size;
+    const int64_t off = slot - blk * block_size;
+    // cache row (blk, h, off): ((blk * Hkv + h) * bs + off) * nvr vectors
+    const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * nvr + v;
+    k_cache[dst] = __ldg(key + i);
+    v_cache[dst] = __ldg(value + i);
+  }
+}
+
+// grid: x = chunk of the block, y = pair, z = 0 (K) / 1 (V).  Each CTA copies
+// kPerThread*256 vectors of one block of one tensor.
+constexpr int kCopyPerThread = 4;
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_cache,
+                                                          uint4* __restrict__ v_cache,
+                                                          const int32_t* __restrict__ mapping,
+                                                          int64_t vecs_per_block,
+                                                          int64_t num_blocks, uint32_t* err) {
+  const int32_t src = __ldg(mapping + 2 * blockIdx.y);
+  const int32_t dst = __ldg(mapping + 2 * blockIdx.y + 1);
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) set_error(err, PA_DEVERR_COPY_BLOCK);
+    return;
+  }
+  uint4* base = blockIdx.z ? v_cache : k_cache;
+  const uint4* s = base + static_cast<int64_t>(src) * vecs_per_block;
+  uint4* d = base + static_cast<int64_t>(dst) * vecs_per_block;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * (256 * kCopyPerThread) + threadIdx.x;
+  uint4 tmp[kCopyPerThread];
+#pragma unroll
+  for (int u = 0; u < kCopyPerThread; ++u) {
+    const int64_t i = first + u * 256;
+    if (i < vecs_per_block) tmp[u] = __ldg(s + i);
+  }
+#pragma unroll
+  for (int u = 0; u < kCopyPerThread; ++u) {
+    const int64_t i = first + u * 256;
+    if (i < vecs_per_block) d[i] = tmp[u];
+  }
+}
+
+int elem_bytes(int dtype) {
+  switch (dtype) {
+    case PA_F32: return 4;
+    case PA_BF16: return 2;
+    case PA_F16: return 2;
+    default: return 0;
+  }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_cache,
+                                    void* v_cache, const int64_t* slot_mapping,
+                                    int64_t num_tokens, int num_kv_heads, int head_dim,
+                                    int block_size, int64_t num_blocks, int dtype,
+                                    pa_stream_t stream) {
+  const int eb = elem_bytes(dtype);
+  if (eb == 0 || num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if ((static_cast<int64_t>(head_dim) * eb) % 16 != 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  const int nvr = head_dim * eb / 16;
+  const int64_t total = num_tokens * num_kv_heads * nvr;
+  const int64_t want = (total + 255) / 256;
+  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8));
+  uint32_t* err = device_error_word();
+  if (!err) return PA_ERR_CUDA;
+  reshape_and_cache_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, num_tokens,
+      num_kv_heads, nvr, block_size, num_blocks * block_size, err);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_mapping_dev,
+                              const int32_t* block_mapping_host, int num_pairs, int num_kv_heads,
+                              int head_dim, int block_size, int64_t num_blocks, int dtype,
+                              pa_stream_t stream) {
+  const int eb = elem_bytes(dtype);
+  if (eb == 0 || num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0 || num_pairs > 65535)
+    return PA_ERR_INVALID_ARG;
+  const int64_t block_bytes = static_cast<int64_t>(num_kv_heads) * block_size * head_dim * eb;
+  if (block_bytes % 16 != 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !block_mapping_dev) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+  if (block_mapping_host) {
+    // every id in range; destinations distinct and never a source
+    for (int i = 0; i < num_pairs; ++i) {
+      const int32_t s = block_mapping_host[2 * i], d = block_mapping_host[2 * i + 1];
+      if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) return PA_ERR_INVALID_ARG;
+    }
+    std::vector<int32_t> dsts(num_pairs), srcs(num_pairs);
+    for (int i = 0; i < num_pairs; ++i) {
+      srcs[i] = block_mapping_host[2 * i];
+      dsts[i] = block_mapping_host[2 * i + 1];
+    }
+    std::sort(dsts.begin(), dsts.end());
+    std::sort(srcs.begin(), srcs.end());
+    if (std::adjacent_find(dsts.begin(), dsts.end()) != dsts.end()) return PA_ERR_INVALID_ARG;
+    for (int32_t d : dsts)
+      if (std::binary_search(srcs.begin(), srcs.end(), d)) return PA_ERR_INVALID_ARG;
+  }
+  const int64_t vecs = block_bytes / 16;
+  const int64_t chunks = (vecs + 256 * kCopyPerThread - 1) / (256 * kCopyPerThread);
+  if (chunks > 0x7fffffff) return PA_ERR_INVALID_ARG;
+  uint32_t* err = device_error_word();
+  if (!err) return PA_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(num_pairs), 2);
+  copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping_dev, vecs,
+      num_blocks, err);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}

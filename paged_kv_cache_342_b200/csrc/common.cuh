@@ -1,0 +1,176 @@
+// Shared device helpers for the sm_100a kernels: element types, 16-byte vector
+// conversions, mbarrier and bulk-copy (TMA) wrappers, bounded waits, error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pa.h"
+
+namespace pa {
+
+// ---------------------------------------------------------------------------
+// host-side launch parameters (plain data, passed by value to the kernels)
+// ---------------------------------------------------------------------------
+struct DecodeParams {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  float scale_log2;  // scale * log2(e): logits live in the base-2 domain
+  int num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq;
+  int64_t num_blocks;
+  int max_seq_len, partition_size, max_parts;
+  float* ws_o;  // [S, Hq, P, D]  normalised partial outputs
+  float* ws_m;  // [S, Hq, P]     partition max (base-2 logits)
+  float* ws_l;  // [S, Hq, P]     partition exp-sum
+  uint32_t* err;
+};
+
+// Device address of the library's error word on the current device.
+uint32_t* device_error_word();
+
+// ---------------------------------------------------------------------------
+// element types
+// ---------------------------------------------------------------------------
+template <typename T> struct ElemTraits;
+template <> struct ElemTraits<float> { static constexpr int kVec = 4; };
+template <> struct ElemTraits<__nv_bfloat16> { static constexpr int kVec = 8; };
+template <> struct ElemTraits<__half> { static constexpr int kVec = 8; };
+
+// 16 bytes of T -> floats (kVec of them)
+__device__ __forceinline__ void vec_to_float(const uint4& v, float* f, float) {
+  f[0] = __uint_as_float(v.x);
+  f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z);
+  f[3] = __uint_as_float(v.w);
+}
+__device__ __forceinline__ void bf16x2_to_float(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+__device__ __forceinline__ void vec_to_float(const uint4& v, float* f, __nv_bfloat16) {
+  bf16x2_to_float(v.x, f[0], f[1]);
+  bf16x2_to_float(v.y, f[2], f[3]);
+  bf16x2_to_float(v.z, f[4], f[5]);
+  bf16x2_to_float(v.w, f[6], f[7]);
+}
+__device__ __forceinline__ void h2_to_float(uint32_t w, float& lo, float& hi) {
+  __half2 h = *reinterpret_cast<const __half2*>(&w);
+  float2 f = __half22float2(h);
+  lo = f.x;
+  hi = f.y;
+}
+__device__ __forceinline__ void vec_to_float(const uint4& v, float* f, __half) {
+  h2_to_float(v.x, f[0], f[1]);
+  h2_to_float(v.y, f[2], f[3]);
+  h2_to_float(v.z, f[4], f[5]);
+  h2_to_float(v.w, f[6], f[7]);
+}
+
+__device__ __forceinline__ void store_elem(float* p, float x) { *p = x; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void store_elem(__half* p, float x) { *p = __float2half_rn(x); }
+
+// ---------------------------------------------------------------------------
+// shared-memory barriers and bulk asynchronous copies (TMA engine)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for the phase with the given parity to complete; give up after about one
+// second (or 2^26 polls) and return false so the caller can record the timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1; it < (1u << 26); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && global_timer_ns() - t0 > 1000000000ull) return false;
+  }
+  return false;
+}
+// Order this thread's earlier generic-proxy shared-memory accesses before later
+// async-proxy (TMA) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// 1-D bulk copy global -> shared, completion counted on an mbarrier.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void set_error(uint32_t* err, uint32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// exp2 of a base-2 logit difference; -inf - -inf (an empty state) gives 0.
+__device__ __forceinline__ float exp2_safe(float a, float m) {
+  return (m == -INFINITY) ? 0.f : exp2f(a - m);
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute is
+// per device; the flag array is per kernel instantiation).
+template <typename K>
+cudaError_t ensure_smem_limit(K kern, int bytes) {
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
+
+}  // namespace pa

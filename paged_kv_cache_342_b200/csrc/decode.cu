@@ -1,0 +1,222 @@
+// pa_decode_attention: argument checks, workspace layout, choice of partition
+// kernel (tensor-core tile for grouped-query head groups, CUDA cores otherwise) and
+// the log-sum-exp merge kernel that combines partitions.
+//
+// "How PagedAttention Powers vLLM's KV Cache" (hassanahmed.net), "The attention
+// kernel has to read scattered blocks" and "Where it bites" (grouped-query
+// attention); "PagedAttention" attention-lab explainer (divagr.pages.dev), "Keep
+// pages in order" and "Measure memory use across requests" (the attention equation
+// is unchanged by paging).
+#include "common.cuh"
+#include "decode_simt.cuh"
+
+namespace pa {
+
+cudaError_t launch_decode_simt_f32(const DecodeParams& p, int gs, cudaStream_t st);
+cudaError_t launch_decode_simt_bf16(const DecodeParams& p, int gs, cudaStream_t st);
+cudaError_t launch_decode_simt_f16(const DecodeParams& p, int gs, cudaStream_t st);
+cudaError_t launch_decode_mma_bf16(const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st);
+
+namespace {
+
+constexpr int kDefaultPartition = 512;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct WsLayout {
+  int parts = 1;
+  size_t o_off = 0, m_off = 0, l_off = 0, bytes = 0;
+};
+
+WsLayout ws_layout(int64_t num_seqs, int64_t num_heads, int64_t head_dim, int64_t max_seq_len,
+                   int64_t partition_size) {
+  WsLayout w;
+  w.parts = max_seq_len > 0 ? static_cast<int>((max_seq_len + partition_size - 1) / partition_size) : 1;
+  if (w.parts <= 1) return w;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_heads * w.parts;
+  w.o_off = 0;
+  w.m_off = align256(rows * head_dim * sizeof(float));
+  w.l_off = w.m_off + align256(rows * sizeof(float));
+  w.bytes = w.l_off + align256(rows * sizeof(float));
+  return w;
+}
+
+// Merge: one warp per (sequence, head) row with more than one partition.
+//   M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p
+// (m_p in base-2 logits, o_p normalised by its own l_p).  Lanes own head_dim/32
+// consecutive output elements; partitions are walked 4 at a time.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
+  constexpr int DPL = D / 32;
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p.num_seqs * p.num_heads) return;
+  const int s = row / p.num_heads;
+  const int L = checked_len(p, s, false);
+  const int nparts = L > 0 ? (L + p.partition_size - 1) / p.partition_size : 1;
+  if (nparts <= 1) return;
+  const float* mrow = p.ws_m + static_cast<int64_t>(row) * p.max_parts;
+  const float* lrow = p.ws_l + static_cast<int64_t>(row) * p.max_parts;
+  const float* orow = p.ws_o + static_cast<int64_t>(row) * p.max_parts * D + lane * DPL;
+  float M = -INFINITY;
+  for (int i = lane; i < nparts; i += 32) M = fmaxf(M, mrow[i]);
+  M = warp_max(M);
+  float den = 0.f;
+  for (int i = lane; i < nparts; i += 32) den += lrow[i] * exp2_safe(mrow[i], M);
+  den = warp_sum(den);
+  float acc[DPL];
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) acc[j] = 0.f;
+  int i = 0;
+  for (; i + 4 <= nparts; i += 4) {
+    float w[4], o[4][DPL];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      w[u] = lrow[i + u] * exp2_safe(mrow[i + u], M);
+#pragma unroll
+      for (int j = 0; j < DPL; j += 2) {
+        const float2 v = *reinterpret_cast<const float2*>(orow + static_cast<int64_t>(i + u) * D + j);
+        o[u][j] = v.x;
+        o[u][j + 1] = v.y;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w[u], o[u][j], acc[j]);
+  }
+  for (; i < nparts; ++i) {
+    const float w = lrow[i] * exp2_safe(mrow[i], M);
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w, orow[static_cast<int64_t>(i) * D + j], acc[j]);
+  }
+  T* out = static_cast<T*>(p.out) + static_cast<int64_t>(row) * D + lane * DPL;
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) store_elem(out + j, acc[j] * inv);
+}
+
+template <typename T>
+cudaError_t launch_merge(const DecodeParams& p, cudaStream_t st) {
+  const int rows = p.num_seqs * p.num_heads;
+  const int grid = (rows + 3) / 4;
+  switch (p.head_dim) {
+    case 64: merge_kernel<T, 64><<<grid, 128, 0, st>>>(p); break;
+    case 128: merge_kernel<T, 128><<<grid, 128, 0, st>>>(p); break;
+    case 256: merge_kernel<T, 256><<<grid, 128, 0, st>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Heads per CTA on the CUDA-core path: the largest of 4, 2, 1 dividing the group
+// (4 only up to head_dim 128, to bound registers).
+int simt_heads_per_cta(int group, int head_dim) {
+  if (group % 4 == 0 && head_dim <= 128) return 4;
+  if (group % 2 == 0) return 2;
+  return 1;
+}
+
+bool mma_eligible(int dtype, int group, int head_dim, int block_size) {
+  return (dtype == PA_BF16 || dtype == PA_F16) && group % 8 == 0 && group <= 16 &&
+         (head_dim == 64 || head_dim == 128 || head_dim == 256) &&
+         (block_size == 16 || block_size == 32);
+}
+
+}  // namespace
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" int pa_decode_uses_tensor_cores(int dtype, int num_heads, int num_kv_heads,
+                                           int head_dim, int block_size) {
+  if (num_kv_heads <= 0 || num_heads <= 0 || num_heads % num_kv_heads) return 0;
+  return mma_eligible(dtype, num_heads / num_kv_heads, head_dim, block_size) ? 1 : 0;
+}
+
+extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                            int max_seq_len, int partition_size) {
+  if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_seq_len < 0 || partition_size < 0)
+    return 0;
+  if (partition_size == 0) partition_size = kDefaultPartition;
+  return ws_layout(num_seqs, num_heads, head_dim, max_seq_len, partition_size).bytes;
+}
+
+extern "C" int pa_decode_attention(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   const int32_t* seq_lens, float scale, int block_size,
+                                   int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                                   int max_blocks_per_seq, int64_t num_blocks, int max_seq_len,
+                                   int partition_size, int dtype, void* workspace,
+                                   size_t workspace_bytes, pa_stream_t stream) {
+  if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16) return PA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads ||
+      head_dim <= 0 || block_size <= 0 || max_blocks_per_seq < 0 || num_blocks <= 0 ||
+      max_seq_len < 0 || partition_size < 0)
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+  if (block_size != 4 && block_size != 8 && block_size != 16 && block_size != 32)
+    return PA_ERR_UNSUPPORTED;
+  if (partition_size == 0) partition_size = kDefaultPartition;
+  if (partition_size % block_size) return PA_ERR_INVALID_ARG;
+  if (num_seqs > 65535) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  const WsLayout ws = ws_layout(num_seqs, num_heads, head_dim, max_seq_len, partition_size);
+  if (ws.parts > 65535) return PA_ERR_INVALID_ARG;
+  if (ws.bytes > 0 && (!workspace || workspace_bytes < ws.bytes || !aligned16(workspace)))
+    return PA_ERR_INVALID_ARG;
+
+  DecodeParams p{};
+  p.out = out;
+  p.q = q;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_seqs = num_seqs;
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.head_dim = head_dim;
+  p.block_size = block_size;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.max_seq_len = max_seq_len;
+  p.partition_size = partition_size;
+  p.max_parts = ws.parts;
+  if (ws.bytes > 0) {
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    p.ws_o = reinterpret_cast<float*>(base + ws.o_off);
+    p.ws_m = reinterpret_cast<float*>(base + ws.m_off);
+    p.ws_l = reinterpret_cast<float*>(base + ws.l_off);
+  }
+  p.err = device_error_word();
+  if (!p.err) return PA_ERR_CUDA;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int group = num_heads / num_kv_heads;
+  cudaError_t e;
+  if (mma_eligible(dtype, group, head_dim, block_size)) {
+    e = dtype == PA_BF16 ? launch_decode_mma_bf16(p, st) : launch_decode_mma_f16(p, st);
+  } else {
+    const int gs = simt_heads_per_cta(group, head_dim);
+    e = dtype == PA_F32    ? launch_decode_simt_f32(p, gs, st)
+        : dtype == PA_BF16 ? launch_decode_simt_bf16(p, gs, st)
+                           : launch_decode_simt_f16(p, gs, st);
+  }
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (ws.parts > 1) {
+    e = dtype == PA_F32    ? launch_merge<float>(p, st)
+        : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, st)
+                           : launch_merge<__half>(p, st);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}

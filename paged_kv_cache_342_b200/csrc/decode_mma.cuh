@@ -1,0 +1,393 @@
+// Tensor-core paged decode attention for grouped-query head groups (partition
+// kernel).  Same result as the CUDA-core kernel; used when 8 or 16 query heads
+// share one kv head, so that scores and p.V form dense tiles ("How PagedAttention
+// Powers vLLM's KV Cache", hassanahmed.net, "Where it bites": grouped-query
+// attention stacks with paging; "The attention kernel has to read scattered
+// blocks": the kernel walks the block table and gathers K/V block by block).
+//
+// Per block of BS tokens of one kv head (BS = 16 or 32):
+//   S^T [tokens x heads] = K [tokens x D] . Q^T [D x heads]    mma m16n8k16, A = K
+//   online softmax per head (column) in float32, base-2 logits
+//   O^T [D x heads]     += V^T [D x tokens] . P^T [tokens x heads]   A = V^T
+// K/V blocks arrive by tensor-map TMA (cp.async.bulk.tensor.2d, 64-element x BS-row
+// boxes with the 128-byte swizzle, so the 8-row ldmatrix reads hit 8 different bank
+// groups) into NST stages per warp, completing on the stage mbarrier.  A and B
+// operands are bf16 (or f16), accumulators float32.  The score fragment (C layout)
+// becomes the B operand of p.V through one movmatrix.trans per 8x8 quarter.
+// Tokens past the sequence end get -inf scores, and their V rows are zeroed in
+// shared memory first (0 * NaN would otherwise poison the tile).
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "decode_simt.cuh"  // checked_len
+
+namespace pa {
+
+template <typename T> struct MmaOps;
+
+template <> struct MmaOps<__nv_bfloat16> {
+  static __device__ __forceinline__ void mma(float (&c)[4], const uint32_t (&a)[4],
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+
+template <> struct MmaOps<__half> {
+  static __device__ __forceinline__ void mma(float (&c)[4], const uint32_t (&a)[4],
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+// 2-D tiled TMA load of one box into shared memory, completion on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+template <typename T, int D, int BS, int NT, int NW, int NST>
+struct MmaCfg {
+  static constexpr int kHalves = D / 64;         // 128-byte column slabs per row
+  static constexpr int kSlabBytes = BS * 128;    // one slab of one tile
+  static constexpr int kTileBytes = kHalves * kSlabBytes;  // = BS * D * 2
+  static constexpr int kStageBytes = 2 * kTileBytes;       // K tile + V tile
+  static constexpr int kTT = BS / 16;            // 16-token row tiles per block
+  static constexpr int kKS = D / 16;             // k-steps of q.K / m-tiles of V^T
+  static constexpr int kHeads = 8 * NT;
+  static constexpr int kStageArea = NW * NST * kStageBytes;
+  static constexpr int kRedBytes = NW * kHeads * (D + 2) * 4;
+  static constexpr int kSmemBytes =
+      1024 + (kStageArea > kRedBytes ? kStageArea : kRedBytes) + NW * NST * 8;
+  static_assert(sizeof(T) == 2, "tensor-core path takes 16-bit caches");
+  static_assert(BS % 16 == 0 && kSlabBytes % 1024 == 0, "slabs must stay 1024-byte aligned");
+};
+
+// byte offset of (row r, 16-byte chunk c of the full row) inside a tile stored as
+// D/64 slabs of [BS rows][128 bytes] with the 128-byte swizzle (chunk ^= row % 8)
+template <int BS>
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * (BS * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <typename T, int D, int BS, int NT, int NW, int NST>
+__global__ void __launch_bounds__(NW * 32)
+    decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv) {
+  using C = MmaCfg<T, D, BS, NT, NW, NST>;
+  using Ops = MmaOps<T>;
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int TT = C::kTT, KS = C::kKS;
+
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzle atoms
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g8 = lane >> 2, t4 = lane & 3;  // fragment row group / thread in group
+  const int s = blockIdx.y, part = blockIdx.z;
+  const int h0 = blockIdx.x * C::kHeads;
+  const int kvh = h0 / (p.num_heads / p.num_kv_heads);
+
+  const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && part == 0);
+  const int ps = p.partition_size;
+  const int nparts = L > 0 ? (L + ps - 1) / ps : 1;
+  if (part >= nparts) return;
+  const int tok_begin = part * ps;
+  const int tok_end = min(L, tok_begin + ps);
+  const int nblk = tok_end > tok_begin ? (tok_end - tok_begin + BS - 1) / BS : 0;
+  const int32_t* table =
+      p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + tok_begin / BS;
+
+  const uint32_t stage0 = base + warp * NST * C::kStageBytes;
+  const uint32_t bar0 = base + (C::kSmemBytes - 1024 - NW * NST * 8) + warp * NST * 8;
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < NST; ++i) mbar_init(bar0 + 8 * i, 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  // Q^T as B fragments: qb[nt][ks][0] = q[head n0+g8][16ks + 2t4 .. +1], [1] = +8 dims
+  uint32_t qb[NT][KS][2];
+  {
+    const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(s) * p.num_heads + h0) * D;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const T* qp = qrow + (nt * 8 + g8) * D + ks * 16 + 2 * t4;
+        qb[nt][ks][0] = __ldg(reinterpret_cast<const unsigned int*>(qp));
+        qb[nt][ks][1] = __ldg(reinterpret_cast<const unsigned int*>(qp + 8));
+      }
+  }
+
+  // per thread: heads nt*8 + 2t4 + {0,1}
+  float m[NT][2], l[NT][2];
+  float oacc[KS][NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m[nt][0] = m[nt][1] = -INFINITY;
+    l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.f;
+  }
+
+  const int nb_w = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;
+  int tab_base = 0;
+  int32_t tab = (lane < nb_w) ? __ldg(table + warp + lane * NW) : -1;
+  uint32_t bad = 0;
+
+  auto issue = [&](int k) {
+    if (k - tab_base >= 32) {
+      tab_base += 32;
+      const int kk = tab_base + lane;
+      tab = (kk < nb_w) ? __ldg(table + warp + kk * NW) : -1;
+    }
+    const int32_t blk = __shfl_sync(FULL, tab, k - tab_base);
+    const bool ok = blk >= 0 && blk < p.num_blocks;
+    const int st = k % NST;
+    bad = ok ? (bad & ~(1u << st)) : (bad | (1u << st));
+    if (lane == 0) {
+      const uint32_t bar = bar0 + 8 * st;
+      if (ok) {
+        const int row0 = (blk * p.num_kv_heads + kvh) * BS;
+        const uint32_t dst = stage0 + st * C::kStageBytes;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar, C::kStageBytes);
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h) {
+          tma_load_2d(dst + h * C::kSlabBytes, &tmk, 64 * h, row0, bar);
+          tma_load_2d(dst + C::kTileBytes + h * C::kSlabBytes, &tmv, 64 * h, row0, bar);
+        }
+      } else {
+        set_error(p.err, PA_DEVERR_TABLE);
+        mbar_arrive(bar);
+      }
+    }
+  };
+
+  const int npre = nb_w < NST ? nb_w : NST;
+  for (int k = 0; k < npre; ++k) issue(k);
+  int issued = npre;
+  int k = 0;
+  bool aborted = false;
+  for (; k < nb_w; ++k) {
+    const int st = k % NST;
+    const bool ok = mbar_wait_bounded(bar0 + 8 * st, (k / NST) & 1);
+    if (!__all_sync(FULL, ok)) {
+      aborted = true;
+      break;
+    }
+    if (!((bad >> st) & 1u)) {
+      const uint32_t kt = stage0 + st * C::kStageBytes;
+      const uint32_t vt = kt + C::kTileBytes;
+      const int valid = min(BS, tok_end - (tok_begin + (warp + k * NW) * BS));
+      if (valid < BS) {
+        // zero the V rows past the end: 16 bytes per lane per step
+        uint8_t* vg = smem + (vt - base);
+        const int nchunks = (BS - valid) * (D / 8);
+        for (int i = lane; i < nchunks; i += 32) {
+          const int r = valid + i / (D / 8), c = i % (D / 8);
+          *reinterpret_cast<uint4*>(vg + swz<BS>(r, c)) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
+      // ---- S^T = K Q^T --------------------------------------------------
+      float sacc[TT][NT][4];
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sacc[tt][nt][i] = 0.f;
+      {
+        const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+          const int r = tt * 16 + (mi & 1) * 8 + ri;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            uint32_t a[4];
+            ldsm_x4(kt + swz<BS>(r, 2 * ks + (mi >> 1)), a);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) Ops::mma(sacc[tt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+          }
+        }
+      }
+      // ---- online softmax per head column ----------------------------------
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const int tok = tt * 16 + g8 + 8 * r;
+              const float sv = tok < valid ? sacc[tt][nt][2 * r + j] * p.scale_log2 : -INFINITY;
+              sacc[tt][nt][2 * r + j] = sv;
+              mx = fmaxf(mx, sv);
+            }
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+          const float mn = fmaxf(m[nt][j], mx);
+          const float corr = exp2_safe(m[nt][j], mn);
+          m[nt][j] = mn;
+          float ls = 0.f;
+#pragma unroll
+          for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const float pv = exp2_safe(sacc[tt][nt][2 * r + j], mn);
+              sacc[tt][nt][2 * r + j] = pv;
+              ls += pv;
+            }
+          l[nt][j] = l[nt][j] * corr + ls;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            oacc[mt][nt][j] *= corr;
+            oacc[mt][nt][2 + j] *= corr;
+          }
+        }
+      }
+      // ---- P^T as B fragments (movmatrix.trans of each 8x8 quarter) ----------
+      uint32_t pb[TT][NT][2];
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          pb[tt][nt][0] = movmatrix_trans(Ops::pack(sacc[tt][nt][0], sacc[tt][nt][1]));
+          pb[tt][nt][1] = movmatrix_trans(Ops::pack(sacc[tt][nt][2], sacc[tt][nt][3]));
+        }
+      // ---- O^T += V^T P^T -------------------------------------------------
+      {
+        const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+          const int r = tt * 16 + (mi >> 1) * 8 + ri;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            uint32_t a[4];
+            ldsm_x4_trans(vt + swz<BS>(r, 2 * mt + (mi & 1)), a);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) Ops::mma(oacc[mt][nt], a, pb[tt][nt][0], pb[tt][nt][1]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (issued < nb_w) {
+      issue(issued);
+      ++issued;
+    }
+  }
+  if (aborted) {
+    if (lane == 0) set_error(p.err, PA_DEVERR_TIMEOUT);
+    for (; k < issued; ++k) mbar_wait_bounded(bar0 + 8 * (k % NST), (k / NST) & 1);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) m[nt][0] = m[nt][1] = -INFINITY;
+  }
+
+  // exp-sums: add the partial sums of the 8 lanes that share a head column
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float x = l[nt][j];
+      x += __shfl_xor_sync(FULL, x, 4);
+      x += __shfl_xor_sync(FULL, x, 8);
+      x += __shfl_xor_sync(FULL, x, 16);
+      l[nt][j] = aborted ? 0.f : x;
+    }
+
+  // merge warps through shared memory
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(smem);
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float* r = red + (warp * C::kHeads + nt * 8 + 2 * t4 + j) * (D + 2);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        r[mt * 16 + g8] = oacc[mt][nt][j];
+        r[mt * 16 + g8 + 8] = oacc[mt][nt][2 + j];
+      }
+      if (g8 == 0) {
+        r[D] = m[nt][j];
+        r[D + 1] = l[nt][j];
+      }
+    }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < C::kHeads * D; idx += NW * 32) {
+    const int hh = idx / D, d = idx - hh * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red[(w * C::kHeads + hh) * (D + 2) + D]);
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float* r = red + (w * C::kHeads + hh) * (D + 2);
+      const float f = exp2_safe(r[D], M);
+      num = fmaf(r[d], f, num);
+      den = fmaf(r[D + 1], f, den);
+    }
+    const float o = den > 0.f ? num / den : 0.f;
+    const int64_t row = static_cast<int64_t>(s) * p.num_heads + h0 + hh;
+    if (nparts == 1) {
+      store_elem(static_cast<T*>(p.out) + row * D + d, o);
+    } else {
+      const int64_t prow = row * p.max_parts + part;
+      p.ws_o[prow * D + d] = o;
+      if (d == 0) {
+        p.ws_m[prow] = M;
+        p.ws_l[prow] = den;
+      }
+    }
+  }
+}
+
+}  // namespace pa

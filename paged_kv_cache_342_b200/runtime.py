@@ -1,0 +1,141 @@
+"""One decode step of the paged KV-cache path, driven through the C ABI.
+
+Order of a step (the sources are the pages cited in ``include/pa.h``):
+  1. the block manager gives every sequence room for one more token
+     (``pa_seq_append_slots``): a slot, and a (src, dst) copy where the token's
+     block is shared;
+  2. slots, copy pairs, block tables and lengths go to the device in one pinned
+     staging round (the only host-to-device traffic of a step);
+  3. ``pa_copy_blocks`` makes the copy-on-write copies - before the write, since
+     the new token lands in the copy;
+  4. ``pa_reshape_and_cache`` writes the new token's K/V into its slot;
+  5. ``pa_decode_attention`` attends over every cached token, the new one included.
+
+This module only moves arguments: the work of every step is done by the library.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (DEFAULT_PARTITION, BlockAllocator, pa_copy_blocks, pa_decode_attention,
+               pa_decode_workspace_bytes, pa_reshape_and_cache)
+
+
+class PagedDecoder:
+    """Device caches + block manager + staging buffers for a fixed set of sequences.
+
+    ``k_cache``/``v_cache`` are caller-owned CUDA tensors [NB, Hkv, bs, D].
+    ``max_blocks_per_seq`` is the block-table width (capacity per sequence).
+    """
+
+    def __init__(self, k_cache, v_cache, num_heads: int, scale: float, max_blocks_per_seq: int,
+                 free_order=None, partition_size: int = DEFAULT_PARTITION, stream=None):
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim = k_cache.shape
+        self.num_heads, self.scale = num_heads, scale
+        self.max_blocks = max_blocks_per_seq
+        self.partition_size = partition_size
+        self.device = k_cache.device
+        self.stream = stream
+        self.alloc = BlockAllocator(self.num_blocks, self.block_size, free_order)
+        self._seq_ids = None
+        self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
+        self._done = None  # event: the last staging copy has been consumed
+
+    # -- context building ------------------------------------------------------
+    def admit(self, seq_id: int, num_tokens: int) -> None:
+        self.alloc.add(seq_id, num_tokens)
+
+    def admit_shared_prefix(self, groups: int, samples: int, prefix_len: int, private_lens,
+                            first_id: int = 0) -> np.ndarray:
+        """Groups of ``samples`` sequences sharing a prefix: the group's first sample is
+        admitted with the prefix, the others fork from it; then, sample by sample, the
+        private tokens are appended.  Returns the copy-on-write pairs those appends
+        produced (apply them with ``apply_copies`` before reading the cache)."""
+        pairs = []
+        for g in range(groups):
+            parent = first_id + g * samples
+            self.alloc.add(parent, prefix_len)
+            for i in range(1, samples):
+                self.alloc.fork(parent, parent + i)
+        for i, n in enumerate(np.asarray(private_lens, dtype=np.int64)):
+            sid = first_id + i
+            for _ in range(int(n)):
+                _, src, dst = self.alloc.append_slot(sid)
+                if src >= 0:
+                    pairs.append((src, dst))
+        return np.array(pairs, dtype=np.int32).reshape(-1, 2)
+
+    def apply_copies(self, pairs: np.ndarray) -> None:
+        if len(pairs):
+            dev = torch.from_numpy(np.ascontiguousarray(pairs)).to(self.device)
+            pa_copy_blocks(self.k_cache, self.v_cache, dev, pairs, stream=self.stream)
+
+    # -- the step ---------------------------------------------------------------
+    def bind(self, seq_ids) -> None:
+        """Fix the batch of sequences the steps run over and allocate staging."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        self._seq_ids = ids
+        S = ids.size
+        pin = dict(pin_memory=True)
+        self.h_slots = torch.empty(S, dtype=torch.int64, **pin)
+        self.h_pairs = torch.empty((max(S, 1), 2), dtype=torch.int32, **pin)
+        self.h_tables = torch.empty((S, self.max_blocks), dtype=torch.int32, **pin)
+        self.h_lens = torch.empty(S, dtype=torch.int32, **pin)
+        self.d_slots = torch.empty(S, dtype=torch.int64, device=self.device)
+        self.d_pairs = torch.empty((max(S, 1), 2), dtype=torch.int32, device=self.device)
+        self.d_tables = torch.empty((S, self.max_blocks), dtype=torch.int32, device=self.device)
+        self.d_lens = torch.empty(S, dtype=torch.int32, device=self.device)
+        cap = self.max_blocks * self.block_size
+        ws = pa_decode_workspace_bytes(S, self.num_heads, self.head_dim, cap, self.partition_size)
+        if ws > self._ws.numel():
+            self._ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
+
+    def prepare(self) -> dict:
+        """Steps 1-3 of the host side: allocate slots, stage and upload metadata.
+        Returns what the kernels need (counts, max length)."""
+        if self._done is not None:
+            self._done.synchronize()  # staging buffers are free again
+        slots, pairs = self.alloc.append_slots(self._seq_ids, self.h_slots.numpy(),
+                                               self.h_pairs.numpy())
+        n_cow = len(pairs)
+        _, lens = self.alloc.build_block_tables(self._seq_ids, self.max_blocks,
+                                                self.h_tables.numpy(), self.h_lens.numpy())
+        max_len = int(lens.max()) if lens.size else 0
+        s = self._torch_stream()
+        with torch.cuda.stream(s):
+            self.d_slots.copy_(self.h_slots, non_blocking=True)
+            if n_cow:
+                self.d_pairs[:n_cow].copy_(self.h_pairs[:n_cow], non_blocking=True)
+            self.d_tables.copy_(self.h_tables, non_blocking=True)
+            self.d_lens.copy_(self.h_lens, non_blocking=True)
+            self._done = torch.cuda.Event()
+            self._done.record(s)
+        return dict(num_cow=n_cow, max_len=max_len, pairs=self.h_pairs.numpy()[:n_cow])
+
+    def launch(self, meta: dict, q, new_k, new_v, out) -> None:
+        """Steps 3-5 on the device."""
+        n = meta["num_cow"]
+        if n:
+            pa_copy_blocks(self.k_cache, self.v_cache, self.d_pairs[:n], meta["pairs"],
+                           stream=self._stream_arg())
+        pa_reshape_and_cache(new_k, new_v, self.k_cache, self.v_cache, self.d_slots,
+                             stream=self._stream_arg())
+        pa_decode_attention(out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
+                            self.scale, self.block_size, self.num_kv_heads, meta["max_len"],
+                            self.partition_size, self._ws if self._ws.numel() else None,
+                            stream=self._stream_arg())
+
+    def step(self, q, new_k, new_v, out) -> dict:
+        meta = self.prepare()
+        self.launch(meta, q, new_k, new_v, out)
+        return meta
+
+    def _torch_stream(self):
+        if self.stream is None:
+            return torch.cuda.current_stream(self.device)
+        return self.stream
+
+    def _stream_arg(self):
+        return self._torch_stream()

@@ -1,0 +1,127 @@
+"""The C-ABI library loads, exports every function include/pa.h declares, and
+rejects bad arguments before touching a GPU (host-only checks; no kernel runs)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import paged_kv_cache_342_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t)\s+(pa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for must in ("pa_reshape_and_cache", "pa_copy_blocks", "pa_decode_attention",
+                 "pa_decode_workspace_bytes", "pa_alloc_create", "pa_seq_fork",
+                 "pa_seq_append_slot", "pa_alloc_stats"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(pa):
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert missing == []
+
+
+def test_library_is_built_for_sm100a(pa):
+    # the fatbin of an sm_100a build names the architecture; a cheap check without
+    # disassembling anything
+    data = open(pa.LIB_PATH, "rb").read()
+    assert b"sm_100a" in data
+
+
+def test_workspace_bytes(pa):
+    assert pa.pa_decode_workspace_bytes(64, 32, 128, 512, 512) == 0       # one partition
+    assert pa.pa_decode_workspace_bytes(64, 32, 128, 0, 512) == 0
+    b = pa.pa_decode_workspace_bytes(8, 64, 128, 131072, 512)
+    rows = 8 * 64 * 256
+    align = lambda x: (x + 255) // 256 * 256
+    assert b == align(rows * 128 * 4) + 2 * align(rows * 4)
+    assert pa.pa_decode_workspace_bytes(2, 4, 64, 1000, 0) == \
+        pa.pa_decode_workspace_bytes(2, 4, 64, 1000, 512)
+    assert pa.pa_decode_workspace_bytes(-1, 4, 64, 1000, 512) == 0
+
+
+def test_tensor_core_path_selection(pa):
+    assert pa.pa_decode_uses_tensor_cores(pa.PA_BF16, 64, 8, 128, 16)
+    assert pa.pa_decode_uses_tensor_cores(pa.PA_F16, 32, 2, 64, 32)
+    assert not pa.pa_decode_uses_tensor_cores(pa.PA_BF16, 32, 32, 128, 16)   # MHA
+    assert not pa.pa_decode_uses_tensor_cores(pa.PA_F32, 64, 8, 128, 16)     # fp32 cache
+    assert not pa.pa_decode_uses_tensor_cores(pa.PA_BF16, 64, 8, 128, 8)     # block 8
+
+
+FAKE = 1 << 20  # an aligned, never-dereferenced pointer value: every call below fails
+                # its host-side checks before any launch
+
+
+def _decode(pa, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, tables=FAKE, lens=FAKE, scale=0.1, bs=16, hkv=4,
+             S=2, hq=4, D=128, mb=8, nb=64, max_len=100, ps=512, dtype=pa.PA_BF16, ws=None,
+             wsb=0)
+    a.update(kw)
+    return pa.lib.pa_decode_attention(a["out"], a["q"], a["k"], a["v"], a["tables"], a["lens"],
+                                      a["scale"], a["bs"], a["hkv"], a["S"], a["hq"], a["D"],
+                                      a["mb"], a["nb"], a["max_len"], a["ps"], a["dtype"],
+                                      a["ws"], a["wsb"], None)
+
+
+def test_decode_argument_checks(pa):
+    assert _decode(pa, dtype=9) == pa.PA_ERR_INVALID_ARG
+    assert _decode(pa, D=96) == pa.PA_ERR_UNSUPPORTED
+    assert _decode(pa, bs=12) == pa.PA_ERR_UNSUPPORTED
+    assert _decode(pa, hq=6, hkv=4) == pa.PA_ERR_INVALID_ARG
+    assert _decode(pa, ps=520) == pa.PA_ERR_INVALID_ARG          # not a multiple of 16
+    assert _decode(pa, q=FAKE + 4) == pa.PA_ERR_INVALID_ARG     # misaligned
+    assert _decode(pa, tables=None) == pa.PA_ERR_INVALID_ARG
+    assert _decode(pa, max_len=5000) == pa.PA_ERR_INVALID_ARG   # needs a workspace
+    assert _decode(pa, max_len=5000, ws=FAKE, wsb=16) == pa.PA_ERR_INVALID_ARG  # too small
+    assert _decode(pa, S=0) == pa.PA_OK                          # nothing to do
+
+
+def _copy(pa, pairs, nb=16):
+    host = np.ascontiguousarray(pairs, dtype=np.int32)
+    return pa.lib.pa_copy_blocks(FAKE, FAKE, FAKE, host.ctypes.data, len(host), 2, 64, 16, nb,
+                                 pa.PA_BF16, None)
+
+
+def test_copy_blocks_mapping_checks(pa):
+    assert _copy(pa, [(1, 2), (1, 2)]) == pa.PA_ERR_INVALID_ARG    # dst repeats
+    assert _copy(pa, [(1, 2), (2, 3)]) == pa.PA_ERR_INVALID_ARG    # dst is also a src
+    assert _copy(pa, [(1, 16)]) == pa.PA_ERR_INVALID_ARG           # outside the pool
+    assert _copy(pa, [(-1, 3)]) == pa.PA_ERR_INVALID_ARG
+    assert pa.lib.pa_copy_blocks(FAKE, FAKE, FAKE, None, 0, 2, 64, 16, 16, pa.PA_BF16,
+                                 None) == pa.PA_OK                 # no pairs: no-op
+
+
+def test_reshape_argument_checks(pa):
+    f = pa.lib.pa_reshape_and_cache
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 6, 16, 8, pa.PA_BF16, None) == \
+        pa.PA_ERR_INVALID_ARG                                       # 12-byte rows
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 5, None) == pa.PA_ERR_INVALID_ARG
+    assert f(None, None, None, None, None, 0, 2, 64, 16, 8, pa.PA_F16, None) == pa.PA_OK
+
+
+def test_importing_without_library_fails_loudly(tmp_path):
+    """The binding refuses to load rather than fall back to anything else."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "paged_kv_cache_342_b200")
+    dst = tmp_path / "paged_kv_cache_342_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "_build", "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", "import paged_kv_cache_342_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libpa.so is missing" in r.stderr

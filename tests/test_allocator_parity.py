@@ -1,0 +1,166 @@
+"""The C++ block manager in libpa.so against the oracle's model, bit for bit:
+slots, copy-on-write pairs, block tables, reference counts, free-pool order and
+statistics after every operation; errors leave both unchanged.  Host only."""
+import numpy as np
+import pytest
+
+from oracle.allocator import AllocError, BlockManager
+from workloads import CONFIGS, make_inputs
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import paged_kv_cache_342_b200 as m
+    return m
+
+
+def same_state(c, o: BlockManager):
+    assert c.stats() == o.stats()
+    assert c.free_list() == o.free_list()
+    for b in range(o.num_blocks):
+        assert c.refcount(b) == o.ref[b]
+    for s, t in o.tables.items():
+        assert c.seq_blocks(s) == t
+        assert c.seq_len(s) == o.lens[s]
+
+
+def run_both(pa, c, o, op, *args):
+    """Apply one op to both; both must succeed with equal results or fail alike."""
+    err_c = err_o = None
+    res_c = res_o = None
+    try:
+        res_c = getattr(c, op)(*args)
+    except pa.PagedAttentionError as e:
+        err_c = e.code
+    try:
+        res_o = getattr(o, {"free": "free_seq"}.get(op, op))(*args)
+    except AllocError as e:
+        err_o = e.code
+    assert err_c == err_o, (op, args, err_c, err_o)
+    return res_c, res_o
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_op_sequences(pa, seed):
+    g = np.random.default_rng(seed)
+    nb, bs = int(g.integers(8, 40)), int(g.choice([1, 2, 4, 16]))
+    order = g.permutation(nb)
+    c, o = pa.BlockAllocator(nb, bs, order), BlockManager(nb, bs, order)
+    live, next_id = [], 0
+    for step in range(400):
+        op = int(g.integers(0, 12))
+        if op < 2 or not live:
+            n = int(g.integers(0, 3 * bs + 1))
+            run_both(pa, c, o, "add", next_id, n)
+            if next_id in o.tables:
+                live.append(next_id)
+            next_id += 1
+        elif op < 4:
+            p = live[int(g.integers(0, len(live)))]
+            run_both(pa, c, o, "fork", p, next_id)
+            if next_id in o.tables:
+                live.append(next_id)
+            next_id += 1
+        elif op < 8:
+            s = live[int(g.integers(0, len(live)))]
+            rc, ro = run_both(pa, c, o, "append_slot", s)
+            assert rc == ro
+        elif op < 10:
+            k = int(g.integers(1, 6))
+            ids = [live[int(i)] for i in g.integers(0, len(live), k)]
+            rc, ro = run_both(pa, c, o, "append_slots", ids)
+            if ro is not None:
+                slots, pairs = rc
+                assert slots.tolist() == [r[0] for r in ro]
+                assert [tuple(p) for p in pairs.tolist()] == [(r[1], r[2]) for r in ro if r[1] >= 0]
+        elif op < 11:
+            s = live.pop(int(g.integers(0, len(live))))
+            run_both(pa, c, o, "free", s)
+        else:
+            run_both(pa, c, o, "free", 10_000 + step)      # unknown id
+            run_both(pa, c, o, "fork", 10_000 + step, 20_000 + step)
+            if live:
+                run_both(pa, c, o, "add", live[0], 3)        # exists
+        same_state(c, o)
+    ids = sorted(o.tables)
+    if ids:
+        width = max(len(o.tables[s]) for s in ids) + 2
+        t_c, l_c = c.build_block_tables(ids, width)
+        rows, lens = o.block_tables(ids, width)
+        assert t_c.tolist() == rows and l_c.tolist() == lens
+
+
+def test_failed_batch_changes_nothing(pa):
+    c, o = pa.BlockAllocator(5, 4), BlockManager(5, 4)
+    for m in (c, o):
+        m.add(0, 6)          # 2 blocks, last half full
+        m.fork(0, 1)
+        m.add(2, 8)          # 2 full blocks
+    # seq 0: copy (1 block), seq 1: in place, seq 2: new block, seq 2 again: in place
+    # -> needs 2 blocks, pool has 1
+    run_both(pa, c, o, "append_slots", [0, 1, 2, 2, 2, 2, 2])
+    same_state(c, o)
+    rc, ro = run_both(pa, c, o, "append_slots", [0, 1])
+    same_state(c, o)
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "7b_bf16", "13b_fp16", "gqa_long_bf16"])
+def test_workload_context_and_step(pa, name):
+    cfg = CONFIGS[name]
+    inp = make_inputs(cfg, 0, pool=False)
+    c = pa.BlockAllocator(cfg.num_blocks, cfg.block_size, inp.free_order)
+    o = BlockManager(cfg.num_blocks, cfg.block_size, inp.free_order)
+    for s in range(cfg.num_seqs):
+        c.add(s, int(inp.context_lens[s]))
+        o.add(s, int(inp.context_lens[s]))
+    slots, pairs = c.append_slots(range(cfg.num_seqs))
+    ro = o.append_slots(range(cfg.num_seqs))
+    assert slots.tolist() == [r[0] for r in ro] and len(pairs) == 0
+    assert c.stats() == o.stats() and c.free_list() == o.free_list()
+
+
+@pytest.mark.parametrize("fork_step", [False, True])
+def test_prefix_workload(pa, fork_step):
+    from oracle.step import build_context
+    from paged_kv_cache_342_b200.runtime import PagedDecoder  # noqa: F401 (import check)
+    cfg = CONFIGS["prefix_cow_bf16"]
+    inp = make_inputs(cfg, 0, fork_step=fork_step, pool=False)
+    o, _, _, build_pairs = build_context(inp, copy_pool=False)
+    c = pa.BlockAllocator(cfg.num_blocks, cfg.block_size, inp.free_order)
+    p = inp.prefix
+    cp = []
+    for gi in range(p.groups):
+        c.add(gi * p.samples, p.prefix_len)
+        for i in range(1, p.samples):
+            c.fork(gi * p.samples, gi * p.samples + i)
+    for s in range(cfg.num_seqs):
+        for _ in range(int(p.private_lens[s])):
+            _, src, dst = c.append_slot(s)
+            if src >= 0:
+                cp.append((src, dst))
+    assert cp == build_pairs
+    slots, pairs = c.append_slots(range(cfg.num_seqs))
+    ro = o.append_slots(range(cfg.num_seqs))
+    assert slots.tolist() == [r[0] for r in ro]
+    assert [tuple(x) for x in pairs.tolist()] == [(r[1], r[2]) for r in ro if r[1] >= 0]
+    if fork_step:
+        assert len(pairs) == 224
+    assert c.stats() == o.stats()
+    assert c.stats()["cow_copies"] == len(build_pairs) + len(pairs)
+
+
+def test_stats_match_worked_batch_example(pa, golden):
+    ex = golden["batch"]
+    c = pa.BlockAllocator(64, ex["block_size_implied"])
+    for i, n in enumerate(ex["lengths_printed"]):
+        c.add(i, n)
+    st = c.stats()
+    assert st["allocated_slots"] == ex["paged_slots_printed"]
+    assert st["logical_tokens"] == ex["stored_tokens_printed"]
+
+
+def test_bad_create_arguments(pa):
+    with pytest.raises(pa.PagedAttentionError):
+        pa.BlockAllocator(4, 4, [0, 1, 1, 2])        # not a permutation
+    with pytest.raises(pa.PagedAttentionError):
+        pa.BlockAllocator(0, 4)

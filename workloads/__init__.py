@@ -253,3 +253,31 @@ def step_tokens(cfg: DecodeConfig, seed: int, step: int):
     nk = normal_fill((S, Hkv, D), cfg.dtype, cfg.std, seed, base + 1)
     nv = normal_fill((S, Hkv, D), cfg.dtype, cfg.std, seed, base + 2)
     return q, nk, nv
+
+
+# ---------------------------------------------------------------------------
+# torch views of storage arrays (device placement is the caller's business)
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+class _TorchDtypes(dict):
+    def __missing__(self, key):
+        t = _torch()
+        self.update({"f32": t.float32, "bf16": t.bfloat16, "f16": t.float16})
+        return dict.__getitem__(self, key)
+
+
+TORCH_DTYPES = _TorchDtypes()
+
+
+def storage_to_torch(a: np.ndarray, dtype: str):
+    """A CPU torch tensor sharing the bits of a storage array (bf16 from uint16)."""
+    t = _torch()
+    a = np.ascontiguousarray(a)
+    if dtype == "bf16":
+        return t.from_numpy(a.view(np.int16)).view(t.bfloat16)
+    return t.from_numpy(a)
