@@ -175,6 +175,12 @@ int pa_decode_uses_tensor_cores(int dtype, int num_heads, int num_kv_heads, int 
  */
 int pa_device_error_read(uint32_t* bits);
 
+/*
+ * pa_last_cuda_error - text of the last CUDA error an entry point met on this
+ * thread (the reason behind a PA_ERR_CUDA), or "" if none.  Owned by the library.
+ */
+const char* pa_last_cuda_error(void);
+
 /* ------------------------------------------------------------------------- */
 /* Host block allocator                                                       */
 /* ------------------------------------------------------------------------- */

@@ -4,7 +4,7 @@ The binding only marshals arguments: every GPU step runs in the library's CUDA
 kernels and every allocator step in its C++ block manager.  Function names match
 the C ABI in ``include/pa.h``.  Tensor arguments are torch CUDA tensors (torch is
 used for device memory and streams only); importing this package fails loudly if
-the library has not been built (``python -m paged_kv_cache_342_b200.build``).
+the library has not been built (``python paged_kv_cache_342_b200/csrc/build.py``).
 """
 from __future__ import annotations
 
@@ -34,7 +34,7 @@ class PagedAttentionError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m paged_kv_cache_342_b200.build`")
+                      "`python paged_kv_cache_342_b200/csrc/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -62,6 +62,7 @@ _sig("pa_decode_attention", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, 
      _i32, _i64, _i32, _i32, _i32, _p, ctypes.c_size_t, _p)
 _sig("pa_decode_uses_tensor_cores", _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_device_error_read", _i32, ctypes.POINTER(ctypes.c_uint32))
+_sig("pa_last_cuda_error", ctypes.c_char_p)
 _sig("pa_alloc_create", _i32, _i64, _i32, _p, ctypes.POINTER(_p))
 _sig("pa_alloc_destroy", _i32, _p)
 _sig("pa_seq_add", _i32, _p, _i64, _i64)
@@ -79,7 +80,13 @@ _sig("pa_alloc_stats", _i32, _p, ctypes.POINTER(pa_stats_t))
 
 def _check(status: int, where: str) -> None:
     if status != PA_OK:
+        if status == PA_ERR_CUDA:
+            where += " (" + pa_last_cuda_error() + ")"
         raise PagedAttentionError(status, where)
+
+
+def pa_last_cuda_error() -> str:
+    return (lib.pa_last_cuda_error() or b"").decode(errors="replace")
 
 
 # ---------------------------------------------------------------------------

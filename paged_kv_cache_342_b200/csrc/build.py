@@ -1,6 +1,9 @@
 """Build libpa.so (the C-ABI library) in-tree for B200 (sm_100a).
 
-    python -m paged_kv_cache_342_b200.build [--verbose-ptxas] [--jobs N]
+    python paged_kv_cache_342_b200/csrc/build.py [--verbose-ptxas] [--jobs N] [--force]
+
+(A plain script beside the sources: it must run before the package, which refuses
+to import without the library, can be imported.)
 
 Each source compiles to an object under ``_build/`` in parallel; the objects link
 into ``paged_kv_cache_342_b200/libpa.so`` with the CUDA runtime linked statically.
@@ -15,9 +18,9 @@ import subprocess
 import sys
 from concurrent.futures import ThreadPoolExecutor
 
-PKG = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.dirname(os.path.abspath(__file__))
+PKG = os.path.dirname(CSRC)
 ROOT = os.path.dirname(PKG)
-CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libpa.so")
 HEADERS = [os.path.join(ROOT, "include", "pa.h")] + [

@@ -117,12 +117,17 @@ extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_
   const int64_t want = (total + 255) / 256;
   const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8));
   uint32_t* err = device_error_word();
-  if (!err) return PA_ERR_CUDA;
+  if (!err) {
+    note_cuda_error(cudaGetLastError());
+    return PA_ERR_CUDA;
+  }
   reshape_and_cache_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(key), static_cast<const uint4*>(value),
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, num_tokens,
       num_kv_heads, nvr, block_size, num_blocks * block_size, err);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  note_cuda_error(e);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_mapping_dev,
@@ -159,10 +164,15 @@ extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block
   const int64_t chunks = (vecs + 256 * kCopyPerThread - 1) / (256 * kCopyPerThread);
   if (chunks > 0x7fffffff) return PA_ERR_INVALID_ARG;
   uint32_t* err = device_error_word();
-  if (!err) return PA_ERR_CUDA;
+  if (!err) {
+    note_cuda_error(cudaGetLastError());
+    return PA_ERR_CUDA;
+  }
   dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(num_pairs), 2);
   copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping_dev, vecs,
       num_blocks, err);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  note_cuda_error(e);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

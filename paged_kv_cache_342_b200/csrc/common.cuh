@@ -159,16 +159,19 @@ __device__ __forceinline__ float exp2_safe(float a, float m) {
   return (m == -INFINITY) ? 0.f : exp2f(a - m);
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device (the attribute is
-// per device; the flag array is per kernel instantiation).
-template <typename K>
-cudaError_t ensure_smem_limit(K kern, int bytes) {
+// Record a failing CUDA call for pa_last_cuda_error (thread-local text).
+void note_cuda_error(cudaError_t e);
+
+// Raise a kernel's dynamic shared-memory limit once per device.  The kernel is a
+// template argument so every instantiation keeps its own per-device flags.
+template <auto Kern>
+cudaError_t ensure_smem_limit(int bytes) {
   static bool done[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
   return e;
 }

@@ -198,7 +198,10 @@ extern "C" int pa_decode_attention(void* out, const void* q, const void* k_cache
     p.ws_l = reinterpret_cast<float*>(base + ws.l_off);
   }
   p.err = device_error_word();
-  if (!p.err) return PA_ERR_CUDA;
+  if (!p.err) {
+    note_cuda_error(cudaGetLastError());
+    return PA_ERR_CUDA;
+  }
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int group = num_heads / num_kv_heads;
@@ -211,12 +214,18 @@ extern "C" int pa_decode_attention(void* out, const void* q, const void* k_cache
         : dtype == PA_BF16 ? launch_decode_simt_bf16(p, gs, st)
                            : launch_decode_simt_f16(p, gs, st);
   }
-  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (e != cudaSuccess) {
+    note_cuda_error(e);
+    return PA_ERR_CUDA;
+  }
   if (ws.parts > 1) {
     e = dtype == PA_F32    ? launch_merge<float>(p, st)
         : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, st)
                            : launch_merge<__half>(p, st);
-    if (e != cudaSuccess) return PA_ERR_CUDA;
+    if (e != cudaSuccess) {
+      note_cuda_error(e);
+      return PA_ERR_CUDA;
+    }
   }
   return PA_OK;
 }

@@ -20,8 +20,8 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
   if (!make_cache_tensor_map(&tmk, p.k_cache, rows, D, BS, bf16) ||
       !make_cache_tensor_map(&tmv, p.v_cache, rows, D, BS, bf16))
     return cudaErrorInvalidValue;
-  auto kern = decode_mma_kernel<__nv_bfloat16, D, BS, NT, NW, NST>;
-  cudaError_t e = ensure_smem_limit(kern, C::kSmemBytes);
+  constexpr auto kern = decode_mma_kernel<__nv_bfloat16, D, BS, NT, NW, NST>;
+  cudaError_t e = ensure_smem_limit<kern>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_heads / C::kHeads, p.num_seqs, p.max_parts);
   kern<<<grid, NW * 32, C::kSmemBytes, st>>>(p, tmk, tmv);

@@ -315,8 +315,8 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
 template <typename T, int D, int BS, int GS, int NW, int NST>
 cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream) {
   using C = SimtCfg<T, D, BS, GS, NW, NST>;
-  auto kern = decode_simt_kernel<T, D, BS, GS, NW, NST>;
-  cudaError_t attr = ensure_smem_limit(kern, C::kSmemBytes);
+  constexpr auto kern = decode_simt_kernel<T, D, BS, GS, NW, NST>;
+  cudaError_t attr = ensure_smem_limit<kern>(C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
   dim3 grid(p.num_heads / GS, p.num_seqs, p.max_parts);
   kern<<<grid, NW * 32, C::kSmemBytes, stream>>>(p);

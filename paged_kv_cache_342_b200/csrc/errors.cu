@@ -2,6 +2,7 @@
 // skip an out-of-range index or give up a bounded wait; pa_device_error_read
 // returns and clears it.
 #include <atomic>
+#include <cstdio>
 
 #include "common.cuh"
 
@@ -27,16 +28,32 @@ uint32_t* device_error_word() {
   return static_cast<uint32_t*>(addr);
 }
 
+namespace {
+thread_local char g_last_cuda_error[256] = "";
+}  // namespace
+
+void note_cuda_error(cudaError_t e) {
+  if (e == cudaSuccess) return;
+  const char* name = cudaGetErrorName(e);
+  const char* text = cudaGetErrorString(e);
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", name ? name : "?",
+           text ? text : "?");
+}
+
 }  // namespace pa
+
+extern "C" const char* pa_last_cuda_error(void) { return pa::g_last_cuda_error; }
 
 extern "C" int pa_device_error_read(uint32_t* bits) {
   if (!bits) return PA_ERR_INVALID_ARG;
   *bits = 0;
-  if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
-  if (cudaMemcpyFromSymbol(bits, pa::g_error_word, sizeof(uint32_t)) != cudaSuccess)
-    return PA_ERR_CUDA;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(bits, pa::g_error_word, sizeof(uint32_t));
   const uint32_t zero = 0;
-  if (cudaMemcpyToSymbol(pa::g_error_word, &zero, sizeof(uint32_t)) != cudaSuccess)
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(pa::g_error_word, &zero, sizeof(uint32_t));
+  if (e != cudaSuccess) {
+    pa::note_cuda_error(e);
     return PA_ERR_CUDA;
+  }
   return PA_OK;
 }

@@ -19,7 +19,8 @@ def pa():
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "pa.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:int|size_t)\s+(pa_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(pa_\w+)\s*\(", text,
+                                 flags=re.M)))
 
 
 def test_header_declares_the_path():
