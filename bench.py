@@ -41,8 +41,8 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
@@ -101,25 +101,38 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        import threading
+        self.lines, self.first = [], threading.Event()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
+            return self
+
+        def reader():
+            for line in self.proc.stdout:
+                if line.strip():
+                    self.lines.append((time.perf_counter(), line.strip()))
+                    self.first.set()
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        self.first.wait(timeout=10)       # sampling is running before the timed region
+        self.t0 = time.perf_counter()
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        self.t1 = time.perf_counter()
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.thread.join(timeout=5)
+            self.lines = [l for t, l in self.lines if self.t0 <= t <= self.t1]
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -200,22 +213,26 @@ def run_reference(args, cfg):
         return
     from workloads import make_inputs
     timer = OracleTimer(cfg, make_inputs(cfg, args.seed))
-    per_step = 2
+    # bounded: about 2 minutes of oracle work at the default step count
+    per_step = 1 if args.steps * 1 > 500 else 2
+    steps = min(args.steps, 200)
     t_all, b_all = 0.0, 0
-    for i in range(args.warmup + args.steps):
+    warm = min(args.warmup, 3)
+    for i in range(warm + steps):
         seqs = [(i * per_step + j) % cfg.num_seqs for j in range(per_step)]
         dt, b = timer.run(seqs)
-        if i >= args.warmup:
+        if i >= warm:
             t_all, b_all = t_all + dt, b_all + b
     value = b_all / t_all / 1e9
     sample = (f"per step: oracle decode attention (float64, all {cfg.num_heads} heads) of "
-              f"{per_step} of the {cfg.num_seqs} sequences, cycling through the batch")
+              f"{per_step} of the {cfg.num_seqs} sequences, cycling through the batch; "
+              f"{steps} timed steps (at most 200 of the requested {args.steps})")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(1e3 * t_all / args.steps, 3), "higher_is_better": True,
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+        "ms_per_step": round(1e3 * t_all / steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "seqs_per_s": round(per_step * args.steps / t_all, 4),
+        "seqs_per_s": round(per_step * steps / t_all, 4),
         "config": {"workload": cfg.name, "description": cfg.description},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": timer.threads,
                          "kind": "oracle", "sample": sample},
@@ -236,11 +253,6 @@ def run_ours(args, cfg):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     import paged_kv_cache_342_b200 as pa
     from paged_kv_cache_342_b200.runtime import PagedDecoder
@@ -255,14 +267,20 @@ def run_ours(args, cfg):
                "sample": desc, "seqs_per_s": round(sps, 3)}
         del timer
 
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
     seed = args.seed + rank
     inp = make_inputs(cfg, seed)
     S, Hq, Hkv, D, bs = cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
-    nsteps = args.warmup + args.steps
-    max_len = int((inp.context_lens + 1).max()) + nsteps + 1
+    max_len = int((inp.context_lens + 1).max()) + 1
     max_blocks = (max_len + bs - 1) // bs
     kd = storage_to_torch(inp.k_pool, cfg.dtype).to(dev)
     vd = storage_to_torch(inp.v_pool, cfg.dtype).to(dev)
+    pool_bytes = 2 * kd.numel() * kd.element_size()
     del inp.k_pool, inp.v_pool
     dec = PagedDecoder(kd, vd, Hq, cfg.scale, max_blocks, inp.free_order, cfg.partition_size)
     if inp.prefix is None:
@@ -272,21 +290,23 @@ def run_ours(args, cfg):
         p = inp.prefix
         dec.apply_copies(dec.admit_shared_prefix(p.groups, p.samples, p.prefix_len,
                                                  p.private_lens))
-    dec.bind(range(S))
+    # every step decodes the same lengths: sequences roll back one token per step
+    dec.bind(range(S), rolling=True)
 
-    # per-step new tokens: host (pinned) and device-resident copies
+    # a ring of distinct per-step token sets: pinned host copies and device copies
+    ring = 8
     toks_h, toks_d = [], []
-    for i in range(nsteps + (0 if args.no_e2e else args.steps)):
+    for i in range(ring):
         q, nk, nv = (inp.q, inp.new_k, inp.new_v) if i == 0 else step_tokens(cfg, seed, i)
         h = [storage_to_torch(a, cfg.dtype).pin_memory() for a in (q, nk, nv)]
         toks_h.append(h)
-        if i < nsteps:
-            toks_d.append([t.to(dev) for t in h])
+        toks_d.append([t.to(dev) for t in h])
     out = torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], device=dev)
     stream = torch.cuda.current_stream(dev)
+    ws = dec._ws if dec._ws.numel() else None
 
-    def one_step(i, ev=None, tokens=None):
-        q, nk, nv = tokens if tokens is not None else toks_d[i]
+    def one_step(tokens, ev=None):
+        q, nk, nv = tokens
         meta = dec.prepare()
         n = meta["num_cow"]
         if n:
@@ -295,46 +315,52 @@ def run_ours(args, cfg):
         if ev is not None:
             ev[0].record(stream)
         pa.pa_decode_attention(out, q, kd, vd, dec.d_tables, dec.d_lens, cfg.scale, bs, Hkv,
-                               meta["max_len"], cfg.partition_size,
-                               dec._ws if dec._ws.numel() else None)
+                               meta["max_len"], cfg.partition_size, ws)
         if ev is not None:
             ev[1].record(stream)
-        parts = max(1, -(-meta["max_len"] // cfg.partition_size))
-        launches = (1 if n else 0) + 1 + 1 + (1 if parts > 1 else 0)
-        return meta, launches
+        return meta
 
+    warm_cow = 0
     for i in range(args.warmup):
-        one_step(i)
+        warm_cow += one_step(toks_d[i % ring])["num_cow"]
     torch.cuda.synchronize(dev)
     if pa.pa_device_error_read() != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    # bytes of the timed steps (lengths grow by one per step)
-    lens0 = np.array([dec.alloc.seq_len(s) for s in range(S)], np.int64)
-    step_bytes, dec_bytes, seqs_done, launches, cows = [], [], 0, 0, 0
+    # the workload is stationary from here on: bytes per step computed once
+    meta0 = one_step(toks_d[0])
+    torch.cuda.synchronize(dev)
+    lens = np.array([dec.alloc.seq_len(s) for s in range(S)], np.int64)
+    uniq = unique_context_tokens(dec, cfg, range(S)) if inp.prefix is not None else None
+    dec_bytes = decode_bytes(cfg, lens, uniq)
+    step_bytes = dec_bytes + cache_op_bytes(cfg, S, 0)
+    logical_dec_bytes = decode_bytes(cfg, lens)
+    launches_per_step = dec.kernel_launches(meta0)
+
+    # per-call events on a sample of the steps (the decode call's own duration)
+    n_ev = min(args.steps, 200)
+    ev_every = max(1, args.steps // n_ev)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+           for _ in range(n_ev)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cows = 0
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         t_start.record(stream)
+        e = 0
         for k in range(args.steps):
-            meta, nl = one_step(args.warmup + k, evs[k])
-            launches += nl
-            cows += meta["num_cow"]
-            L = lens0 + k + 1
-            uniq = unique_context_tokens(dec, cfg, range(S)) if inp.prefix is not None else None
-            db = decode_bytes(cfg, L, uniq)
-            dec_bytes.append(db)
-            step_bytes.append(db + cache_op_bytes(cfg, S, meta["num_cow"]))
+            ev = None
+            if k % ev_every == 0 and e < n_ev:
+                ev, e = evs[e], e + 1
+            cows += one_step(toks_d[k % ring], ev)["num_cow"]
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
-    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    dec_ms = [a.elapsed_time(b) for a, b in evs[:e]]
     err = pa.pa_device_error_read()
     if err:
         raise RuntimeError(f"device error word {err} after the timed region")
@@ -342,11 +368,7 @@ def run_ours(args, cfg):
         t = torch.tensor([elapsed_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         elapsed_ms = float(t.item())
-        tb = torch.tensor([float(sum(step_bytes))], device=dev, dtype=torch.float64)
-        dist.all_reduce(tb)
-        total_bytes = float(tb.item())
-    else:
-        total_bytes = float(sum(step_bytes))
+    total_bytes = float(step_bytes) * args.steps * world
     value = total_bytes / (elapsed_ms * 1e-3) / 1e9
     seqs_per_s = S * world * args.steps / (elapsed_ms * 1e-3)
 
@@ -354,29 +376,23 @@ def run_ours(args, cfg):
     e2e = None
     if not args.no_e2e:
         out_h = torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], pin_memory=True)
-        tok_bufs = [torch.empty_like(t, device=dev) for t in toks_d[0]]
-        base = nsteps
-        e_bytes = []
-        # warm-up of this mode
-        for k in range(3):
-            for dst, src in zip(tok_bufs, toks_h[base + k % args.steps]):
+        bufs = [torch.empty_like(t, device=dev) for t in toks_d[0]]
+
+        def e2e_step(k):
+            for dst, src in zip(bufs, toks_h[k % ring]):
                 dst.copy_(src, non_blocking=True)
-            one_step(0, tokens=tok_bufs)
+            one_step(bufs)
             out_h.copy_(out, non_blocking=True)
+
+        for k in range(3):
+            e2e_step(k)
         torch.cuda.synchronize(dev)
-        lens1 = np.array([dec.alloc.seq_len(s) for s in range(S)], np.int64)
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for k in range(args.steps):
-            for dst, src in zip(tok_bufs, toks_h[base + k]):
-                dst.copy_(src, non_blocking=True)
-            meta, _ = one_step(0, tokens=tok_bufs)
-            out_h.copy_(out, non_blocking=True)
-            L = lens1 + k + 1
-            uniq = unique_context_tokens(dec, cfg, range(S)) if inp.prefix is not None else None
-            e_bytes.append(decode_bytes(cfg, L, uniq) + cache_op_bytes(cfg, S, meta["num_cow"]))
+            e2e_step(k)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
@@ -384,34 +400,29 @@ def run_ours(args, cfg):
             t = torch.tensor([e_ms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
-        E = sum(e_bytes) * world / (e_ms * 1e-3) / 1e9
-        h2d = sum(t.numel() * t.element_size() for t in toks_h[0])
-        h2d += S * 8 + S * max_blocks * 4 + S * 4          # slots, tables, lengths
+        E = float(step_bytes) * args.steps * world / (e_ms * 1e-3) / 1e9
+        h2d = sum(t.numel() * t.element_size() for t in toks_h[0]) + dec.staging_bytes
         d2h = S * Hq * D * cfg.elem_bytes
         e2e = {"value": round(E, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / args.steps, 4)}
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / args.steps, 4),
+               "seqs_per_s": round(S * world * args.steps / (e_ms * 1e-3), 1)}
 
     # ---- roofline of the decode call --------------------------------------------
     peak, peak_kind = hbm_peak()
     dec_avg_ms = statistics.mean(dec_ms)
-    achieved = statistics.mean(dec_bytes) / (dec_avg_ms * 1e-3) / 1e9
+    achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
             "kernel": "pa_decode_attention (partition kernel + log-sum-exp merge)",
-            "bytes_per_launch": int(statistics.mean(dec_bytes)),
-            "avg_launch_us": round(dec_avg_ms * 1e3, 2),
+            "bytes_per_launch": int(dec_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 2),
+            "launches_timed": len(dec_ms),
             "frac_of_nominal_8000": round(achieved / 8000.0, 4),
-            "traffic": None}
-    prof = os.path.join(HERE, "profiles", f"traffic_{cfg.name}.json")
-    if os.path.exists(prof):
-        try:
-            with open(prof) as f:
-                roof["traffic"] = json.load(f).get("traffic_bytes_per_launch")
-        except (OSError, ValueError):
-            pass
+            "traffic": recorded_traffic(cfg)}
+    if uniq is not None:
+        roof["logical_bytes_per_launch"] = int(logical_dec_bytes)
+        roof["logical_achieved"] = round(logical_dec_bytes / (dec_avg_ms * 1e-3) / 1e9, 1)
 
     if rank == 0:
-        ws = dec._ws.numel()
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -422,21 +433,50 @@ def run_ours(args, cfg):
                        "num_seqs": S, "num_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
                        "block_size": bs, "num_blocks": cfg.num_blocks,
                        "partition_size": cfg.partition_size,
-                       "mean_seq_len": round(float((lens0 + 1).mean()), 1),
+                       "mean_seq_len": round(float(lens.mean()), 1),
+                       "max_seq_len": int(lens.max()),
                        "l2": "inputs larger than L2 (K/V pool %.2f GB per rank), no flush"
-                             % (2 * kd.numel() * kd.element_size() / 1e9),
-                       "parallelism": f"replicas x{world}", "workspace_bytes": int(ws),
-                       "cow_pairs_in_timed_steps": cows},
+                             % (pool_bytes / 1e9),
+                       "steps": "each step appends one token per sequence and rolls the "
+                                "previous one back, so every step decodes these lengths",
+                       "parallelism": f"replicas x{world}",
+                       "workspace_bytes": int(dec._ws.numel()),
+                       "cow_pairs_in_warmup": warm_cow, "cow_pairs_in_timed_steps": cows},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": launches,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def recorded_traffic(cfg):
+    """DRAM bytes per decode call from the committed ncu capture of this workload,
+    if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(HERE, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(cfg.name)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("kernel_sources_sha256") != kernel_sources_sha():
+        return None
+    return rec.get("traffic_bytes_per_launch")
+
+
+def kernel_sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(HERE, "paged_kv_cache_342_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("decode") or name in ("common.cuh", "tensor_map.cu"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
 
 
 def main():

@@ -237,6 +237,10 @@ int pa_seq_append_slot(pa_alloc_t* a, int64_t seq_id, int64_t* slot, int32_t* co
  * order, their count to *num_cow. */
 int pa_seq_append_slots(pa_alloc_t* a, const int64_t* seq_ids, int n, int64_t* slots,
                         int32_t* cow_pairs, int* num_cow);
+/* Shorten each seq_ids[i] to new_lens[i] (<= its length), e.g. to drop a rejected
+ * draft token; blocks past ceil(new_len/block_size) drop a reference (released in
+ * logical order).  No copy is ever needed.  Ids must be distinct.  All or nothing. */
+int pa_seq_truncate(pa_alloc_t* a, const int64_t* seq_ids, const int64_t* new_lens, int n);
 /* Release seq_id. */
 int pa_seq_free(pa_alloc_t* a, int64_t seq_id);
 int pa_seq_len(const pa_alloc_t* a, int64_t seq_id, int64_t* len);

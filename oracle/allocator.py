@@ -20,7 +20,9 @@ Sources (page title, section):
 Readings where the pages are silent (the C-ABI allocator follows the same ones):
   * free pool order: a LIFO stack whose successive pops return free_order[0],
     free_order[1], ...; a block whose count drops to zero is pushed on top;
-  * a finished sequence releases its blocks in logical order;
+  * a finished sequence releases its blocks in logical order; truncating a sequence
+    (dropping its last tokens, e.g. a rejected draft token) releases the blocks past
+    the new length the same way and never copies;
   * copy-on-write fires when the block the next token goes into has count > 1;
     the writer gets a fresh block, the shared block's count drops by one;
   * a failing call leaves the state unchanged; a batch of appends is all or nothing;
@@ -124,6 +126,28 @@ class BlockManager:
             self.__dict__.clear()
             self.__dict__.update(saved)
             raise
+
+    def truncate(self, seq_ids, new_lens) -> None:
+        """Shorten each listed sequence to its new length (<= current); blocks past
+        ceil(new_len / bs) are released in logical order.  All or nothing."""
+        pairs = list(zip(seq_ids, new_lens))
+        for s, n in pairs:
+            if s not in self.tables:
+                raise AllocError(UNKNOWN_SEQ, str(s))
+        if len({s for s, _ in pairs}) != len(pairs):
+            raise AllocError(INVALID_ARG, "sequence ids repeat")
+        for s, n in pairs:
+            if n < 0 or n > self.lens[s]:
+                raise AllocError(INVALID_ARG, f"cannot truncate {s} to {n}")
+        for s, n in pairs:
+            keep = self._blocks_for(n)
+            table = self.tables[s]
+            for b in table[keep:]:
+                self.ref[b] -= 1
+                if self.ref[b] == 0:
+                    self.free.append(b)
+            del table[keep:]
+            self.lens[s] = n
 
     def free_seq(self, seq_id: int) -> None:
         if seq_id not in self.tables:

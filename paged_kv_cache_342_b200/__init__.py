@@ -70,6 +70,7 @@ _sig("pa_seq_fork", _i32, _p, _i64, _i64)
 _sig("pa_seq_append_slot", _i32, _p, _i64, _I64P, _I32P, _I32P)
 _sig("pa_seq_append_slots", _i32, _p, _p, _i32, _p, _p, ctypes.POINTER(ctypes.c_int))
 _sig("pa_seq_free", _i32, _p, _i64)
+_sig("pa_seq_truncate", _i32, _p, _p, _p, _i32)
 _sig("pa_seq_len", _i32, _p, _i64, _I64P)
 _sig("pa_seq_blocks", _i32, _p, _i64, _p, _i64, _I64P)
 _sig("pa_build_block_tables", _i32, _p, _p, _i32, _p, _i32, _p)
@@ -237,6 +238,14 @@ class BlockAllocator:
         _check(lib.pa_seq_append_slots(self._h, ids.ctypes.data, n, slots.ctypes.data,
                                        pairs.ctypes.data, ctypes.byref(nc)), "pa_seq_append_slots")
         return slots[:n], pairs[:nc.value]
+
+    def truncate(self, seq_ids, new_lens) -> None:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        lens = np.ascontiguousarray(new_lens, dtype=np.int64)
+        if ids.size != lens.size:
+            raise ValueError("seq_ids and new_lens differ in length")
+        _check(lib.pa_seq_truncate(self._h, ids.ctypes.data, lens.ctypes.data, ids.size),
+               "pa_seq_truncate")
 
     def free(self, seq_id: int) -> None:
         _check(lib.pa_seq_free(self._h, seq_id), "pa_seq_free")

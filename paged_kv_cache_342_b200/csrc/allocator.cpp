@@ -212,6 +212,26 @@ int pa_seq_append_slots(pa_alloc_t* a, const int64_t* seq_ids, int n, int64_t* s
   return PA_OK;
 }
 
+int pa_seq_truncate(pa_alloc_t* a, const int64_t* seq_ids, const int64_t* new_lens, int n) {
+  if (!a || n < 0 || (n > 0 && (!seq_ids || !new_lens))) return PA_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)  // validate first: all or nothing
+    if (!a->seqs.count(seq_ids[i])) return PA_ERR_UNKNOWN_SEQ;
+  std::unordered_map<int64_t, int> seen;
+  for (int i = 0; i < n; ++i) {
+    if (new_lens[i] < 0 || new_lens[i] > a->seqs.find(seq_ids[i])->second.len)
+      return PA_ERR_INVALID_ARG;
+    if (seen[seq_ids[i]]++) return PA_ERR_INVALID_ARG;  // ids must be distinct
+  }
+  for (int i = 0; i < n; ++i) {
+    Seq& s = a->seqs.find(seq_ids[i])->second;
+    const size_t keep = static_cast<size_t>(blocks_for(new_lens[i], a->block_size));
+    for (size_t j = keep; j < s.blocks.size(); ++j) a->dec(s.blocks[j]);
+    if (keep < s.blocks.size()) s.blocks.resize(keep);
+    s.len = new_lens[i];
+  }
+  return PA_OK;
+}
+
 int pa_seq_free(pa_alloc_t* a, int64_t seq_id) {
   if (!a) return PA_ERR_INVALID_ARG;
   auto it = a->seqs.find(seq_id);

@@ -4,12 +4,17 @@ Order of a step (the sources are the pages cited in ``include/pa.h``):
   1. the block manager gives every sequence room for one more token
      (``pa_seq_append_slots``): a slot, and a (src, dst) copy where the token's
      block is shared;
-  2. slots, copy pairs, block tables and lengths go to the device in one pinned
-     staging round (the only host-to-device traffic of a step);
+  2. slots, copy pairs, lengths and block tables are packed into one pinned staging
+     buffer and sent to the device in one copy (the only host-to-device traffic of
+     a step);
   3. ``pa_copy_blocks`` makes the copy-on-write copies - before the write, since
      the new token lands in the copy;
   4. ``pa_reshape_and_cache`` writes the new token's K/V into its slot;
   5. ``pa_decode_attention`` attends over every cached token, the new one included.
+
+With ``rolling=True`` each step first rolls the sequences back to the lengths they
+had when bound (``pa_seq_truncate``): every step then decodes the same lengths,
+which is how a long benchmark run stays on one workload.
 
 This module only moves arguments: the work of every step is done by the library.
 """
@@ -22,8 +27,12 @@ from . import (DEFAULT_PARTITION, BlockAllocator, pa_copy_blocks, pa_decode_atte
                pa_decode_workspace_bytes, pa_reshape_and_cache)
 
 
+def _align(n: int, a: int = 256) -> int:
+    return (n + a - 1) // a * a
+
+
 class PagedDecoder:
-    """Device caches + block manager + staging buffers for a fixed set of sequences.
+    """Device caches + block manager + staging for a fixed batch of sequences.
 
     ``k_cache``/``v_cache`` are caller-owned CUDA tensors [NB, Hkv, bs, D].
     ``max_blocks_per_seq`` is the block-table width (capacity per sequence).
@@ -70,72 +79,84 @@ class PagedDecoder:
     def apply_copies(self, pairs: np.ndarray) -> None:
         if len(pairs):
             dev = torch.from_numpy(np.ascontiguousarray(pairs)).to(self.device)
-            pa_copy_blocks(self.k_cache, self.v_cache, dev, pairs, stream=self.stream)
+            pa_copy_blocks(self.k_cache, self.v_cache, dev, pairs, stream=self._torch_stream())
 
     # -- the step ---------------------------------------------------------------
-    def bind(self, seq_ids) -> None:
-        """Fix the batch of sequences the steps run over and allocate staging."""
+    def bind(self, seq_ids, rolling: bool = False) -> None:
+        """Fix the batch the steps run over and allocate the staging buffers."""
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
         self._seq_ids = ids
-        S = ids.size
-        pin = dict(pin_memory=True)
-        self.h_slots = torch.empty(S, dtype=torch.int64, **pin)
-        self.h_pairs = torch.empty((max(S, 1), 2), dtype=torch.int32, **pin)
-        self.h_tables = torch.empty((S, self.max_blocks), dtype=torch.int32, **pin)
-        self.h_lens = torch.empty(S, dtype=torch.int32, **pin)
-        self.d_slots = torch.empty(S, dtype=torch.int64, device=self.device)
-        self.d_pairs = torch.empty((max(S, 1), 2), dtype=torch.int32, device=self.device)
-        self.d_tables = torch.empty((S, self.max_blocks), dtype=torch.int32, device=self.device)
-        self.d_lens = torch.empty(S, dtype=torch.int32, device=self.device)
-        cap = self.max_blocks * self.block_size
+        self.rolling = rolling
+        self._stepped = False
+        self.base_lens = np.array([self.alloc.seq_len(int(s)) for s in ids], np.int64)
+        S, MB = ids.size, self.max_blocks
+        o_slots = 0
+        o_pairs = _align(8 * S)
+        o_lens = o_pairs + _align(8 * max(S, 1))
+        o_tab = o_lens + _align(4 * S)
+        total = o_tab + _align(4 * S * MB)
+        self.h_stage = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+        self.d_stage = torch.empty(total, dtype=torch.uint8, device=self.device)
+
+        def views(buf):
+            return (buf[o_slots:o_slots + 8 * S].view(torch.int64),
+                    buf[o_pairs:o_pairs + 8 * max(S, 1)].view(torch.int32).view(-1, 2),
+                    buf[o_lens:o_lens + 4 * S].view(torch.int32),
+                    buf[o_tab:o_tab + 4 * S * MB].view(torch.int32).view(S, MB))
+
+        self.h_slots, self.h_pairs, self.h_lens, self.h_tables = views(self.h_stage)
+        self.d_slots, self.d_pairs, self.d_lens, self.d_tables = views(self.d_stage)
+        cap = MB * self.block_size
         ws = pa_decode_workspace_bytes(S, self.num_heads, self.head_dim, cap, self.partition_size)
         if ws > self._ws.numel():
             self._ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
 
+    @property
+    def staging_bytes(self) -> int:
+        return self.h_stage.numel()
+
     def prepare(self) -> dict:
-        """Steps 1-3 of the host side: allocate slots, stage and upload metadata.
-        Returns what the kernels need (counts, max length)."""
+        """Host side of a step: slots and copies from the block manager, tables and
+        lengths, all staged and sent to the device in one copy."""
         if self._done is not None:
-            self._done.synchronize()  # staging buffers are free again
+            self._done.synchronize()  # the staging buffer is free again
+        if self.rolling and self._stepped:
+            self.alloc.truncate(self._seq_ids, self.base_lens)
         slots, pairs = self.alloc.append_slots(self._seq_ids, self.h_slots.numpy(),
                                                self.h_pairs.numpy())
+        self._stepped = True
         n_cow = len(pairs)
         _, lens = self.alloc.build_block_tables(self._seq_ids, self.max_blocks,
                                                 self.h_tables.numpy(), self.h_lens.numpy())
         max_len = int(lens.max()) if lens.size else 0
         s = self._torch_stream()
         with torch.cuda.stream(s):
-            self.d_slots.copy_(self.h_slots, non_blocking=True)
-            if n_cow:
-                self.d_pairs[:n_cow].copy_(self.h_pairs[:n_cow], non_blocking=True)
-            self.d_tables.copy_(self.h_tables, non_blocking=True)
-            self.d_lens.copy_(self.h_lens, non_blocking=True)
+            self.d_stage.copy_(self.h_stage, non_blocking=True)
             self._done = torch.cuda.Event()
             self._done.record(s)
         return dict(num_cow=n_cow, max_len=max_len, pairs=self.h_pairs.numpy()[:n_cow])
 
     def launch(self, meta: dict, q, new_k, new_v, out) -> None:
-        """Steps 3-5 on the device."""
+        """Device side of a step: copies, the new token's K/V, attention."""
+        st = self._torch_stream()
         n = meta["num_cow"]
         if n:
-            pa_copy_blocks(self.k_cache, self.v_cache, self.d_pairs[:n], meta["pairs"],
-                           stream=self._stream_arg())
-        pa_reshape_and_cache(new_k, new_v, self.k_cache, self.v_cache, self.d_slots,
-                             stream=self._stream_arg())
+            pa_copy_blocks(self.k_cache, self.v_cache, self.d_pairs[:n], meta["pairs"], stream=st)
+        pa_reshape_and_cache(new_k, new_v, self.k_cache, self.v_cache, self.d_slots, stream=st)
         pa_decode_attention(out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
                             self.scale, self.block_size, self.num_kv_heads, meta["max_len"],
                             self.partition_size, self._ws if self._ws.numel() else None,
-                            stream=self._stream_arg())
+                            stream=st)
 
     def step(self, q, new_k, new_v, out) -> dict:
         meta = self.prepare()
         self.launch(meta, q, new_k, new_v, out)
         return meta
 
-    def _torch_stream(self):
-        if self.stream is None:
-            return torch.cuda.current_stream(self.device)
-        return self.stream
+    def kernel_launches(self, meta: dict) -> int:
+        """Library kernels one step launches (copy, write, partitions, merge)."""
+        parts = max(1, -(-meta["max_len"] // self.partition_size))
+        return (1 if meta["num_cow"] else 0) + 2 + (1 if parts > 1 else 0)
 
-    def _stream_arg(self):
-        return self._torch_stream()
+    def _torch_stream(self):
+        return torch.cuda.current_stream(self.device) if self.stream is None else self.stream

@@ -74,8 +74,15 @@ def test_random_op_sequences(pa, seed):
                 assert slots.tolist() == [r[0] for r in ro]
                 assert [tuple(p) for p in pairs.tolist()] == [(r[1], r[2]) for r in ro if r[1] >= 0]
         elif op < 11:
-            s = live.pop(int(g.integers(0, len(live))))
-            run_both(pa, c, o, "free", s)
+            if g.integers(0, 2):
+                s = live.pop(int(g.integers(0, len(live))))
+                run_both(pa, c, o, "free", s)
+            else:
+                k = int(g.integers(1, 4))
+                ids = [live[int(i)] for i in g.integers(0, len(live), k)]
+                ids = list(dict.fromkeys(ids))
+                lens = [int(g.integers(0, o.lens[i] + 2)) for i in ids]   # may be too long
+                run_both(pa, c, o, "truncate", ids, lens)
         else:
             run_both(pa, c, o, "free", 10_000 + step)      # unknown id
             run_both(pa, c, o, "fork", 10_000 + step, 20_000 + step)

@@ -372,10 +372,15 @@ def random_ops(bm: BlockManager, g: np.random.Generator, n_ops: int, check=None)
             elif op < 9:
                 s = live[int(g.integers(0, len(live)))]
                 log.append(("append", s, bm.append_slot(s)))
-            else:
+            elif g.integers(0, 2):
                 s = live.pop(int(g.integers(0, len(live))))
                 bm.free_seq(s)
                 log.append(("free", s))
+            else:
+                s = live[int(g.integers(0, len(live)))]
+                n = int(g.integers(0, bm.lens[s] + 1))
+                bm.truncate([s], [n])
+                log.append(("truncate", s, n))
         except AllocError as e:
             log.append(("error", e.code))
         if check:
@@ -438,4 +443,30 @@ def test_fork_step_copy_count_prefix_workload():
     pairs = [(r[1], r[2]) for r in res if r[1] >= 0]
     assert len(pairs) == 224
     assert len({d for _, d in pairs}) == 224 and not ({d for _, d in pairs} & {s for s, _ in pairs})
+    _invariants(bm)
+
+
+def test_truncate_then_append_reuses_the_released_block():
+    """Dropping a token that opened a block returns that block; appending again takes
+    it back (LIFO pool) - a rolled-back decode step leaves the state as it was."""
+    bm = BlockManager(8, 4, [5, 2, 7, 0, 1, 3, 4, 6])
+    bm.add(0, 8)
+    before = (bm.stats(), list(bm.free), [list(t) for t in bm.tables.values()])
+    slot, _, _ = bm.append_slot(0)
+    assert slot == 7 * 4
+    bm.truncate([0], [8])
+    after = (bm.stats(), list(bm.free), [list(t) for t in bm.tables.values()])
+    assert before[1:] == after[1:] and before[0]["logical_tokens"] == after[0]["logical_tokens"]
+    with pytest.raises(AllocError):
+        bm.truncate([0], [9])
+
+
+def test_truncate_keeps_shared_blocks_shared():
+    bm = BlockManager(8, 4)
+    bm.add(0, 6)
+    bm.fork(0, 1)
+    bm.truncate([1], [3])            # still inside block 0: nothing released
+    assert bm.ref[0] == 2 and bm.ref[1] == 1 and len(bm.tables[1]) == 1
+    _, src, dst = bm.append_slot(1)  # writing into the shared block copies it
+    assert src == 0 and bm.ref[0] == 1
     _invariants(bm)
