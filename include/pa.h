@@ -52,7 +52,8 @@ typedef enum {
   PA_ERR_SEQ_EXISTS = 4,     /* sequence id already present                         */
   PA_ERR_BAD_INDEX = 5,      /* a kernel met an out-of-range block id / slot / len  */
   PA_ERR_CUDA = 6,           /* a CUDA runtime call or launch failed                */
-  PA_ERR_UNSUPPORTED = 7     /* valid but not built: head_dim / block_size / dtype  */
+  PA_ERR_UNSUPPORTED = 7,    /* valid but not built: head_dim / block_size / dtype  */
+  PA_ERR_TOO_LARGE = 8       /* request exceeds a fixed built-in capacity           */
 } pa_status;
 
 typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
@@ -159,6 +160,37 @@ int pa_decode_attention(void* out, const void* q, const void* k_cache, const voi
                         int head_dim, int max_blocks_per_seq, int64_t num_blocks,
                         int max_seq_len, int partition_size, int dtype, void* workspace,
                         size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_decode_attention_static_ws - pa_decode_attention without a caller-provided
+ * workspace, for callers that are not allowed to allocate device memory: code running
+ * inside a host program that owns and budgets every byte of the GPU's memory (a
+ * serving runtime that reserves the card at start-up, a plug-in loaded into someone
+ * else's process), loops that cannot afford the synchronisation and unbounded latency
+ * of cudaMalloc, and deployments that forbid any allocation after initialisation.
+ * (The pages have no counterpart: this entry point is an interface convenience.)
+ *
+ * Arguments, layouts and results are those of pa_decode_attention minus workspace and
+ * workspace_bytes.  The partition scratch is a library-owned device array of
+ * PA_STATIC_WORKSPACE_BYTES (16 MiB) that every GPU which loads the library holds until
+ * the process exits.  A call whose pa_decode_workspace_bytes(...) exceeds that returns
+ * PA_ERR_TOO_LARGE and does nothing; use pa_decode_attention with your own workspace
+ * for such sizes.  The call allocates nothing (no cudaMalloc / cudaFree).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make that first
+ *     call before any stream capture.
+ *   - Every call on a device shares the one array.  The scratch needs no clearing (each
+ *     call writes every entry it reads), but calls that overlap on the GPU - on
+ *     different streams, or from different threads - race on it and must be ordered
+ *     by the caller.
+ */
+#define PA_STATIC_WORKSPACE_BYTES (16u << 20)
+int pa_decode_attention_static_ws(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  const int32_t* seq_lens, float scale, int block_size,
+                                  int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                                  int max_blocks_per_seq, int64_t num_blocks, int max_seq_len,
+                                  int partition_size, int dtype, pa_stream_t stream);
 
 /*
  * pa_decode_uses_tensor_cores - 1 if pa_decode_attention serves this shape with the

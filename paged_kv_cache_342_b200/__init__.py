@@ -18,8 +18,10 @@ LIB_PATH = os.path.join(_HERE, "libpa.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_NO_FREE_BLOCKS, PA_ERR_UNKNOWN_SEQ = 0, 1, 2, 3
 PA_ERR_SEQ_EXISTS, PA_ERR_BAD_INDEX, PA_ERR_CUDA, PA_ERR_UNSUPPORTED = 4, 5, 6, 7
+PA_ERR_TOO_LARGE = 8
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "NO_FREE_BLOCKS", 3: "UNKNOWN_SEQ",
-                4: "SEQ_EXISTS", 5: "BAD_INDEX", 6: "CUDA", 7: "UNSUPPORTED"}
+                4: "SEQ_EXISTS", 5: "BAD_INDEX", 6: "CUDA", 7: "UNSUPPORTED", 8: "TOO_LARGE"}
+PA_STATIC_WORKSPACE_BYTES = 16 << 20
 PA_F32, PA_BF16, PA_F16 = 0, 1, 2
 DEVERR_SLOT, DEVERR_COPY_BLOCK, DEVERR_TABLE, DEVERR_SEQ_LEN, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 DEFAULT_PARTITION = 512
@@ -60,6 +62,8 @@ _sig("pa_copy_blocks", _i32, _p, _p, _p, _p, _i32, _i32, _i32, _i32, _i64, _i32,
 _sig("pa_decode_workspace_bytes", ctypes.c_size_t, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode_attention", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32, _i32,
      _i32, _i64, _i32, _i32, _i32, _p, ctypes.c_size_t, _p)
+_sig("pa_decode_attention_static_ws", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32,
+     _i32, _i32, _i64, _i32, _i32, _i32, _p)
 _sig("pa_decode_uses_tensor_cores", _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_device_error_read", _i32, ctypes.POINTER(ctypes.c_uint32))
 _sig("pa_last_cuda_error", ctypes.c_char_p)
@@ -170,6 +174,24 @@ def pa_decode_attention(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
         float(scale), block_size, num_kv_heads, S, Hq, D, block_tables.shape[1], NB,
         int(max_seq_len), partition_size, _dtype_code(q), ws_ptr, ws_bytes, _stream(stream)),
         "pa_decode_attention")
+
+
+def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
+                                  block_size, num_kv_heads, max_seq_len,
+                                  partition_size=DEFAULT_PARTITION, stream=None) -> None:
+    """pa_decode_attention with the library's own fixed scratch array instead of a
+    caller workspace: for callers that may not allocate device memory.  Raises
+    PagedAttentionError (TOO_LARGE) when the call needs more than
+    PA_STATIC_WORKSPACE_BYTES of scratch; overlapping calls on one device race."""
+    import torch
+    S, Hq, D = q.shape
+    NB = k_cache.shape[0]
+    _check(lib.pa_decode_attention_static_ws(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), block_size, num_kv_heads, S, Hq, D, block_tables.shape[1], NB,
+        int(max_seq_len), partition_size, _dtype_code(q), _stream(stream)),
+        "pa_decode_attention_static_ws")
 
 
 def pa_decode_uses_tensor_cores(dtype_code, num_heads, num_kv_heads, head_dim, block_size) -> bool:
