@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    # smaller instances of a workload for profiling captures (reported in "config")
+    ap.add_argument("--seqs", type=int, default=None, help="override the batch size")
+    ap.add_argument("--pool-blocks", type=int, default=None, help="override the pool size")
     return ap.parse_args()
 
 
@@ -485,6 +488,12 @@ def main():
         raise SystemExit("--warmup must be at least 3")
     from workloads import CONFIGS, HEADLINE
     cfg = CONFIGS[args.workload or HEADLINE]
+    if args.seqs is not None:
+        if cfg.lens[0] in ("fixed", "prefix"):
+            raise SystemExit("--seqs applies to workloads with drawn lengths")
+        cfg = cfg.with_(num_seqs=args.seqs, name=f"{cfg.name}_s{args.seqs}")
+    if args.pool_blocks is not None:
+        cfg = cfg.with_(num_blocks=args.pool_blocks, name=f"{cfg.name}_nb{args.pool_blocks}")
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

@@ -42,69 +42,101 @@ WsLayout ws_layout(int64_t num_seqs, int64_t num_heads, int64_t head_dim, int64_
   return w;
 }
 
-// Merge: one warp per (sequence, head) row with more than one partition.
+// Merge: combine the partitions of every (sequence, head) row that has more than one:
 //   M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p
-// (m_p in base-2 logits, o_p normalised by its own l_p).  Lanes own head_dim/32
-// consecutive output elements; partitions are walked 4 at a time.
+// (m_p in base-2 logits, o_p normalised by its own l_p).  A CTA of 8 warps serves
+// 8/WPR rows with WPR warps each (WPR grows with the partition count, so long rows
+// are read by up to 8 warps at once); lanes own head_dim/32 consecutive elements,
+// each warp walks partitions wsub, wsub+WPR, ... four at a time, and the row's warps
+// combine their sums in shared memory.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wpr) {
   constexpr int DPL = D / 32;
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= p.num_seqs * p.num_heads) return;
-  const int s = row / p.num_heads;
-  const int L = checked_len(p, s, false);
-  const int nparts = L > 0 ? (L + p.partition_size - 1) / p.partition_size : 1;
-  if (nparts <= 1) return;
-  const float* mrow = p.ws_m + static_cast<int64_t>(row) * p.max_parts;
-  const float* lrow = p.ws_l + static_cast<int64_t>(row) * p.max_parts;
-  const float* orow = p.ws_o + static_cast<int64_t>(row) * p.max_parts * D + lane * DPL;
-  float M = -INFINITY;
-  for (int i = lane; i < nparts; i += 32) M = fmaxf(M, mrow[i]);
-  M = warp_max(M);
-  float den = 0.f;
-  for (int i = lane; i < nparts; i += 32) den += lrow[i] * exp2_safe(mrow[i], M);
-  den = warp_sum(den);
+  __shared__ float sh_acc[8][D];
+  __shared__ float sh_den[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows_per_cta = 8 / wpr;
+  const int wsub = warp % wpr;
+  const int row = blockIdx.x * rows_per_cta + warp / wpr;
+  int nparts = 0;
+  if (row < p.num_seqs * p.num_heads) {
+    const int L = checked_len(p, row / p.num_heads, false);
+    nparts = L > 0 ? (L + p.partition_size - 1) / p.partition_size : 1;
+  }
   float acc[DPL];
 #pragma unroll
   for (int j = 0; j < DPL; ++j) acc[j] = 0.f;
-  int i = 0;
-  for (; i + 4 <= nparts; i += 4) {
-    float w[4], o[4][DPL];
+  float den = 0.f;
+  if (nparts > 1) {
+    const float* mrow = p.ws_m + static_cast<int64_t>(row) * p.max_parts;
+    const float* lrow = p.ws_l + static_cast<int64_t>(row) * p.max_parts;
+    const float* orow = p.ws_o + static_cast<int64_t>(row) * p.max_parts * D + lane * DPL;
+    float M = -INFINITY;
+    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, mrow[i]);
+    M = warp_max(M);
+    int i = wsub;
+    for (; i + 3 * wpr < nparts; i += 4 * wpr) {
+      float w[4], o[4][DPL];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      w[u] = lrow[i + u] * exp2_safe(mrow[i + u], M);
+      for (int u = 0; u < 4; ++u) {
+        const int pi = i + u * wpr;
+        w[u] = lrow[pi] * exp2_safe(mrow[pi], M);
+        const float* src = orow + static_cast<int64_t>(pi) * D;
 #pragma unroll
-      for (int j = 0; j < DPL; j += 2) {
-        const float2 v = *reinterpret_cast<const float2*>(orow + static_cast<int64_t>(i + u) * D + j);
-        o[u][j] = v.x;
-        o[u][j + 1] = v.y;
+        for (int j = 0; j < DPL; j += 2) {
+          const float2 v = *reinterpret_cast<const float2*>(src + j);
+          o[u][j] = v.x;
+          o[u][j + 1] = v.y;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        den += w[u];
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w[u], o[u][j], acc[j]);
       }
     }
+    for (; i < nparts; i += wpr) {
+      const float w = lrow[i] * exp2_safe(mrow[i], M);
+      den += w;
+      const float* src = orow + static_cast<int64_t>(i) * D;
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w[u], o[u][j], acc[j]);
+      for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w, src[j], acc[j]);
+    }
   }
-  for (; i < nparts; ++i) {
-    const float w = lrow[i] * exp2_safe(mrow[i], M);
+  if (wpr > 1) {
 #pragma unroll
-    for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w, orow[static_cast<int64_t>(i) * D + j], acc[j]);
+    for (int j = 0; j < DPL; ++j) sh_acc[warp][lane * DPL + j] = acc[j];
+    if (lane == 0) sh_den[warp] = den;
+    __syncthreads();
+    if (wsub == 0) {
+      for (int w2 = 1; w2 < wpr; ++w2) {
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) acc[j] += sh_acc[warp + w2][lane * DPL + j];
+        den += sh_den[warp + w2];
+      }
+    }
   }
-  T* out = static_cast<T*>(p.out) + static_cast<int64_t>(row) * D + lane * DPL;
-  const float inv = den > 0.f ? 1.f / den : 0.f;
+  if (nparts > 1 && wsub == 0) {
+    T* out = static_cast<T*>(p.out) + static_cast<int64_t>(row) * D + lane * DPL;
+    const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
-  for (int j = 0; j < DPL; ++j) store_elem(out + j, acc[j] * inv);
+    for (int j = 0; j < DPL; ++j) store_elem(out + j, acc[j] * inv);
+  }
 }
 
 template <typename T>
 cudaError_t launch_merge(const DecodeParams& p, cudaStream_t st) {
+  // warps per row: enough that each walks at most ~32 partitions
+  int wpr = 1;
+  while (wpr < 8 && p.max_parts > 32 * wpr) wpr *= 2;
   const int rows = p.num_seqs * p.num_heads;
-  const int grid = (rows + 3) / 4;
+  const int rows_per_cta = 8 / wpr;
+  const int grid = (rows + rows_per_cta - 1) / rows_per_cta;
   switch (p.head_dim) {
-    case 64: merge_kernel<T, 64><<<grid, 128, 0, st>>>(p); break;
-    case 128: merge_kernel<T, 128><<<grid, 128, 0, st>>>(p); break;
-    case 256: merge_kernel<T, 256><<<grid, 128, 0, st>>>(p); break;
+    case 64: merge_kernel<T, 64><<<grid, 256, 0, st>>>(p, wpr); break;
+    case 128: merge_kernel<T, 128><<<grid, 256, 0, st>>>(p, wpr); break;
+    case 256: merge_kernel<T, 256><<<grid, 256, 0, st>>>(p, wpr); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
