@@ -306,21 +306,11 @@ def run_ours(args, cfg):
         toks_d.append([t.to(dev) for t in h])
     out = torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], device=dev)
     stream = torch.cuda.current_stream(dev)
-    ws = dec._ws if dec._ws.numel() else None
 
     def one_step(tokens, ev=None):
         q, nk, nv = tokens
         meta = dec.prepare()
-        n = meta["num_cow"]
-        if n:
-            pa.pa_copy_blocks(kd, vd, dec.d_pairs[:n], meta["pairs"])
-        pa.pa_reshape_and_cache(nk, nv, kd, vd, dec.d_slots)
-        if ev is not None:
-            ev[0].record(stream)
-        pa.pa_decode_attention(out, q, kd, vd, dec.d_tables, dec.d_lens, cfg.scale, bs, Hkv,
-                               meta["max_len"], cfg.partition_size, ws)
-        if ev is not None:
-            ev[1].record(stream)
+        dec.launch(meta, q, nk, nv, out, events=ev)
         return meta
 
     warm_cow = 0
@@ -444,6 +434,7 @@ def run_ours(args, cfg):
                                 "previous one back, so every step decodes these lengths",
                        "parallelism": f"replicas x{world}",
                        "workspace_bytes": int(dec._ws.numel()),
+                       "prefix_group_chunks": int(meta0.get("num_chunks", 0)),
                        "cow_pairs_in_warmup": warm_cow, "cow_pairs_in_timed_steps": cows},
             "roofline": roof,
             "cpu_baseline": cpu,

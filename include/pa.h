@@ -201,6 +201,38 @@ int pa_decode_uses_tensor_cores(int dtype, int num_heads, int num_kv_heads, int 
                                 int block_size);
 
 /*
+ * pa_decode_attention_grouped - pa_decode_attention for a batch in which groups of
+ * sequences share their leading blocks (prompt sharing / parallel samples forked
+ * from one prefix: [GLOSS] prompt sharing and sampling algorithms; [BLOG] "The bonus
+ * contiguous storage can't give you: sharing").  Same result as pa_decode_attention;
+ * the whole partitions a group shares are read once for the group instead of once
+ * per member: a tensor-core tile whose columns are the members' (query, head) pairs.
+ *
+ * Extra arguments (device int32 arrays, as filled by pa_build_prefix_groups and copied
+ * to the device):
+ *   prefix_parts   [num_seqs]  shared partitions of each sequence (0 = not grouped)
+ *   chunk_members  [num_chunks, max_members]  batch positions of a chunk, -1 padded
+ *   chunk_parts    [num_chunks]  shared partitions of the chunk
+ *   max_members    1..16; max_chunk_parts = max(chunk_parts) (sizes the grid).
+ * Contract: all members of a chunk map the chunk's first chunk_parts *
+ * partition_size / block_size logical blocks to the same physical blocks (what
+ * pa_build_prefix_groups guarantees); prefix_parts[i] equals its chunk's parts.
+ * A sequence never has its last token's partition computed by the group, so every
+ * grouped sequence is finished by the merge kernel.  When the shape does not qualify
+ * (f32 cache, block_size not 16/32, max_members * num_heads/num_kv_heads > 16, or a
+ * single partition) the groups are ignored and the plain path runs.
+ */
+int pa_decode_attention_grouped(void* out, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* block_tables,
+                                const int32_t* seq_lens, float scale, int block_size,
+                                int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                                int max_blocks_per_seq, int64_t num_blocks, int max_seq_len,
+                                int partition_size, int dtype, const int32_t* prefix_parts,
+                                const int32_t* chunk_members, const int32_t* chunk_parts,
+                                int num_chunks, int max_members, int max_chunk_parts,
+                                void* workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * pa_device_error_read - synchronise the current device, then return (in *bits) and
  * clear the device error word that the kernels set on out-of-range indices or on
  * a bounded wait that gave up (PA_DEVERR_* bits; 0 = none).
@@ -283,6 +315,19 @@ int pa_seq_blocks(const pa_alloc_t* a, int64_t seq_id, int32_t* out, int64_t cap
  * seq_lens [num_seqs] for the listed sequences, ready to copy to the device. */
 int pa_build_block_tables(const pa_alloc_t* a, const int64_t* seq_ids, int num_seqs,
                           int32_t* tables, int max_blocks_per_seq, int32_t* seq_lens);
+/* Prefix groups for pa_decode_attention_grouped.  Among the listed sequences (batch
+ * positions 0..num_seqs-1), those whose block tables begin with the same physical
+ * block form a group (order of first appearance; at least two members).  Its common
+ * table prefix, in blocks, gives parts = floor(common * block_size / partition_size)
+ * whole partitions that every member shares; groups with parts == 0 are dropped.
+ * Outputs (host buffers): prefix_parts[num_seqs] (the member's parts, 0 if none);
+ * chunk_members[num_chunks * max_members] (each group split in order into chunks of at
+ * most max_members positions, rows padded with -1; capacity num_seqs * max_members);
+ * chunk_parts[num_chunks] (capacity num_seqs); *num_chunks; *max_chunk_parts. */
+int pa_build_prefix_groups(const pa_alloc_t* a, const int64_t* seq_ids, int num_seqs,
+                           int partition_size, int max_members, int32_t* prefix_parts,
+                           int32_t* chunk_members, int32_t* chunk_parts, int* num_chunks,
+                           int* max_chunk_parts);
 int pa_block_refcount(const pa_alloc_t* a, int32_t block, int32_t* refcount);
 /* Free blocks in the order the next pops return them; *n = how many. */
 int pa_alloc_free_list(const pa_alloc_t* a, int32_t* out, int64_t cap, int64_t* n);

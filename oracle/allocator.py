@@ -158,6 +158,46 @@ class BlockManager:
                 self.free.append(b)
         del self.lens[seq_id]
 
+    # -- sharing structure ---------------------------------------------------
+    def prefix_groups(self, seq_ids, partition_size: int, max_members: int):
+        """Batch positions whose block tables begin with the same physical blocks.
+
+        Sequences are grouped by their first block (first appearance order); a group
+        needs at least two members and a common table prefix (in blocks) covering at
+        least one whole partition.  Members are split, in order, into chunks of at most
+        ``max_members``.  Returns (prefix_parts per position, [(members, parts)] chunks)
+        where parts = floor(common_prefix_blocks * block_size / partition_size).
+        """
+        ids = list(seq_ids)
+        by_first, order = {}, []
+        for pos, s in enumerate(ids):
+            t = self.tables[s]
+            if not t:
+                continue
+            if t[0] not in by_first:
+                by_first[t[0]] = []
+                order.append(t[0])
+            by_first[t[0]].append(pos)
+        prefix_parts = [0] * len(ids)
+        chunks = []
+        for first in order:
+            members = by_first[first]
+            if len(members) < 2:
+                continue
+            tabs = [self.tables[ids[m]] for m in members]
+            common = 0
+            while all(common < len(t) for t in tabs) and \
+                    all(t[common] == tabs[0][common] for t in tabs):
+                common += 1
+            parts = common * self.block_size // partition_size
+            if parts == 0:
+                continue
+            for m in members:
+                prefix_parts[m] = parts
+            for i in range(0, len(members), max_members):
+                chunks.append((members[i:i + max_members], parts))
+        return prefix_parts, chunks
+
     # -- views ---------------------------------------------------------------
     def block_tables(self, seq_ids, max_blocks: int):
         rows, lens = [], []

@@ -64,6 +64,8 @@ _sig("pa_decode_attention", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, 
      _i32, _i64, _i32, _i32, _i32, _p, ctypes.c_size_t, _p)
 _sig("pa_decode_attention_static_ws", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32,
      _i32, _i32, _i64, _i32, _i32, _i32, _p)
+_sig("pa_decode_attention_grouped", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32,
+     _i32, _i32, _i64, _i32, _i32, _i32, _p, _p, _p, _i32, _i32, _i32, _p, ctypes.c_size_t, _p)
 _sig("pa_decode_uses_tensor_cores", _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_device_error_read", _i32, ctypes.POINTER(ctypes.c_uint32))
 _sig("pa_last_cuda_error", ctypes.c_char_p)
@@ -79,6 +81,8 @@ _sig("pa_seq_len", _i32, _p, _i64, _I64P)
 _sig("pa_seq_blocks", _i32, _p, _i64, _p, _i64, _I64P)
 _sig("pa_build_block_tables", _i32, _p, _p, _i32, _p, _i32, _p)
 _sig("pa_block_refcount", _i32, _p, _i32, _I32P)
+_sig("pa_build_prefix_groups", _i32, _p, _p, _i32, _i32, _i32, _p, _p, _p,
+     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int))
 _sig("pa_alloc_free_list", _i32, _p, _p, _i64, _I64P)
 _sig("pa_alloc_stats", _i32, _p, ctypes.POINTER(pa_stats_t))
 
@@ -174,6 +178,31 @@ def pa_decode_attention(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
         float(scale), block_size, num_kv_heads, S, Hq, D, block_tables.shape[1], NB,
         int(max_seq_len), partition_size, _dtype_code(q), ws_ptr, ws_bytes, _stream(stream)),
         "pa_decode_attention")
+
+
+def pa_decode_attention_grouped(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
+                                block_size, num_kv_heads, max_seq_len, prefix_parts,
+                                chunk_members, chunk_parts, num_chunks, max_chunk_parts,
+                                partition_size=DEFAULT_PARTITION, workspace=None,
+                                stream=None) -> None:
+    """pa_decode_attention with prefix groups (device int32 tensors prefix_parts [S],
+    chunk_members [>= num_chunks, max_members], chunk_parts [>= num_chunks])."""
+    import torch
+    S, Hq, D = q.shape
+    NB = k_cache.shape[0]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_attention_grouped(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), block_size, num_kv_heads, S, Hq, D, block_tables.shape[1], NB,
+        int(max_seq_len), partition_size, _dtype_code(q),
+        _dev(prefix_parts, "prefix_parts", torch.int32),
+        _dev(chunk_members, "chunk_members", torch.int32),
+        _dev(chunk_parts, "chunk_parts", torch.int32), int(num_chunks),
+        int(chunk_members.shape[1]), int(max_chunk_parts), ws_ptr, ws_bytes, _stream(stream)),
+        "pa_decode_attention_grouped")
 
 
 def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
@@ -292,6 +321,23 @@ class BlockAllocator:
         _check(lib.pa_build_block_tables(self._h, ids.ctypes.data, ids.size, tables.ctypes.data,
                                          max_blocks, lens.ctypes.data), "pa_build_block_tables")
         return tables, lens
+
+    def prefix_groups(self, seq_ids, partition_size: int, max_members: int, prefix_parts=None,
+                      chunk_members=None, chunk_parts=None):
+        """(prefix_parts [n], chunk_members [k, max_members], chunk_parts [k],
+        max_chunk_parts) for pa_decode_attention_grouped; pass preallocated (pinned)
+        arrays of full capacity to fill them in place."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        pp = np.empty(n, np.int32) if prefix_parts is None else prefix_parts
+        cm = np.empty((max(n, 1), max_members), np.int32) if chunk_members is None else chunk_members
+        cp = np.empty(max(n, 1), np.int32) if chunk_parts is None else chunk_parts
+        nc, mp = ctypes.c_int(0), ctypes.c_int(0)
+        _check(lib.pa_build_prefix_groups(self._h, ids.ctypes.data, n, partition_size, max_members,
+                                          pp.ctypes.data, cm.ctypes.data, cp.ctypes.data,
+                                          ctypes.byref(nc), ctypes.byref(mp)),
+               "pa_build_prefix_groups")
+        return pp[:n], cm[:nc.value], cp[:nc.value], mp.value
 
     def refcount(self, block: int) -> int:
         r = ctypes.c_int32()

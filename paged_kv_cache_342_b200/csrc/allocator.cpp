@@ -282,6 +282,61 @@ int pa_build_block_tables(const pa_alloc_t* a, const int64_t* seq_ids, int num_s
   return PA_OK;
 }
 
+int pa_build_prefix_groups(const pa_alloc_t* a, const int64_t* seq_ids, int num_seqs,
+                           int partition_size, int max_members, int32_t* prefix_parts,
+                           int32_t* chunk_members, int32_t* chunk_parts, int* num_chunks,
+                           int* max_chunk_parts) {
+  if (!a || num_seqs < 0 || partition_size <= 0 || max_members < 1 || !num_chunks ||
+      !max_chunk_parts)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs > 0 && (!seq_ids || !prefix_parts || !chunk_members || !chunk_parts))
+    return PA_ERR_INVALID_ARG;
+  std::vector<const Seq*> seqs(static_cast<size_t>(num_seqs));
+  for (int i = 0; i < num_seqs; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
+    seqs[i] = &it->second;
+  }
+  // group positions by first physical block, in order of first appearance
+  std::unordered_map<int32_t, int> group_of;
+  std::vector<std::vector<int>> groups;
+  for (int i = 0; i < num_seqs; ++i) {
+    prefix_parts[i] = 0;
+    if (seqs[i]->blocks.empty()) continue;
+    auto ins = group_of.emplace(seqs[i]->blocks[0], static_cast<int>(groups.size()));
+    if (ins.second) groups.emplace_back();
+    groups[ins.first->second].push_back(i);
+  }
+  int nc = 0, maxp = 0;
+  for (const auto& g : groups) {
+    if (g.size() < 2) continue;
+    const auto& t0 = seqs[g[0]]->blocks;
+    size_t common = t0.size();
+    for (size_t k = 1; k < g.size(); ++k) {
+      const auto& t = seqs[g[k]]->blocks;
+      size_t c = 0;
+      while (c < common && c < t.size() && t[c] == t0[c]) ++c;
+      common = c;
+    }
+    const int parts = static_cast<int>(static_cast<int64_t>(common) * a->block_size / partition_size);
+    if (parts == 0) continue;
+    for (int pos : g) prefix_parts[pos] = parts;
+    for (size_t k = 0; k < g.size(); k += static_cast<size_t>(max_members)) {
+      int32_t* row = chunk_members + static_cast<int64_t>(nc) * max_members;
+      for (int j = 0; j < max_members; ++j) {
+        const size_t idx = k + static_cast<size_t>(j);
+        row[j] = idx < g.size() ? g[idx] : -1;
+      }
+      chunk_parts[nc] = parts;
+      ++nc;
+    }
+    if (parts > maxp) maxp = parts;
+  }
+  *num_chunks = nc;
+  *max_chunk_parts = maxp;
+  return PA_OK;
+}
+
 int pa_block_refcount(const pa_alloc_t* a, int32_t block, int32_t* refcount) {
   if (!a || !refcount || block < 0 || block >= a->num_blocks) return PA_ERR_INVALID_ARG;
   *refcount = a->ref[block];

@@ -29,6 +29,12 @@ struct DecodeParams {
   float* ws_m;  // [S, Hq, P]     partition max (base-2 logits)
   float* ws_l;  // [S, Hq, P]     partition exp-sum
   uint32_t* err;
+  // prefix groups (all null / 0 for the plain call): whole partitions that a group of
+  // sequences shares are computed once per group by the group kernel
+  const int32_t* prefix_parts;   // [S] shared partitions of each sequence (0 = none)
+  const int32_t* chunk_members;  // [num_chunks, max_members] batch positions, -1 padded
+  const int32_t* chunk_parts;    // [num_chunks] shared partitions of each chunk
+  int max_members;
 };
 
 // Device address of the library's error word on the current device.

@@ -17,6 +17,10 @@ cudaError_t launch_decode_simt_bf16(const DecodeParams& p, int gs, cudaStream_t 
 cudaError_t launch_decode_simt_f16(const DecodeParams& p, int gs, cudaStream_t st);
 cudaError_t launch_decode_mma_bf16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_decode_group_bf16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
+                                     cudaStream_t st);
+cudaError_t launch_decode_group_f16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
+                                    cudaStream_t st);
 
 namespace {
 
@@ -158,6 +162,27 @@ bool mma_eligible(int dtype, int group, int head_dim, int block_size) {
          (block_size == 16 || block_size == 32);
 }
 
+// The group kernel is the tensor-core kernel with (member, head) columns.
+bool group_eligible(int dtype, int group, int head_dim, int block_size, int max_members) {
+  return (dtype == PA_BF16 || dtype == PA_F16) && max_members >= 1 &&
+         max_members * group <= 16 && (head_dim == 64 || head_dim == 128 || head_dim == 256) &&
+         (block_size == 16 || block_size == 32);
+}
+
+struct GroupArgs {
+  const int32_t* prefix_parts;
+  const int32_t* chunk_members;
+  const int32_t* chunk_parts;
+  int num_chunks, max_members, max_chunk_parts;
+};
+
+int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                const int32_t* block_tables, const int32_t* seq_lens, float scale, int block_size,
+                int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                int max_blocks_per_seq, int64_t num_blocks, int max_seq_len, int partition_size,
+                int dtype, const GroupArgs* groups, void* workspace, size_t workspace_bytes,
+                pa_stream_t stream);
+
 }  // namespace
 
 }  // namespace pa
@@ -185,6 +210,41 @@ extern "C" int pa_decode_attention(void* out, const void* q, const void* k_cache
                                    int max_blocks_per_seq, int64_t num_blocks, int max_seq_len,
                                    int partition_size, int dtype, void* workspace,
                                    size_t workspace_bytes, pa_stream_t stream) {
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
+                     num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
+                     max_seq_len, partition_size, dtype, nullptr, workspace, workspace_bytes,
+                     stream);
+}
+
+extern "C" int pa_decode_attention_grouped(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* seq_lens, float scale, int block_size,
+    int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
+    int64_t num_blocks, int max_seq_len, int partition_size, int dtype,
+    const int32_t* prefix_parts, const int32_t* chunk_members, const int32_t* chunk_parts,
+    int num_chunks, int max_members, int max_chunk_parts, void* workspace,
+    size_t workspace_bytes, pa_stream_t stream) {
+  if (num_chunks < 0 || max_chunk_parts < 0 || max_members < 1 || max_members > 16)
+    return PA_ERR_INVALID_ARG;
+  if (num_chunks > 65535) return PA_ERR_INVALID_ARG;
+  if (num_chunks > 0 && (!prefix_parts || !chunk_members || !chunk_parts))
+    return PA_ERR_INVALID_ARG;
+  const GroupArgs g{prefix_parts, chunk_members, chunk_parts, num_chunks, max_members,
+                    max_chunk_parts};
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
+                     num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
+                     max_seq_len, partition_size, dtype, &g, workspace, workspace_bytes, stream);
+}
+
+namespace pa {
+namespace {
+
+int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                const int32_t* block_tables, const int32_t* seq_lens, float scale, int block_size,
+                int num_kv_heads, int num_seqs, int num_heads, int head_dim,
+                int max_blocks_per_seq, int64_t num_blocks, int max_seq_len, int partition_size,
+                int dtype, const GroupArgs* groups, void* workspace, size_t workspace_bytes,
+                pa_stream_t stream) {
   if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16) return PA_ERR_INVALID_ARG;
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads ||
       head_dim <= 0 || block_size <= 0 || max_blocks_per_seq < 0 || num_blocks <= 0 ||
@@ -238,6 +298,22 @@ extern "C" int pa_decode_attention(void* out, const void* q, const void* k_cache
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
+  // shared partitions of prefix groups first (only useful when sequences span
+  // several partitions); otherwise the per-sequence kernels do everything
+  if (groups && groups->num_chunks > 0 && groups->max_chunk_parts > 0 && ws.parts > 1 &&
+      group_eligible(dtype, group, head_dim, block_size, groups->max_members)) {
+    p.prefix_parts = groups->prefix_parts;
+    p.chunk_members = groups->chunk_members;
+    p.chunk_parts = groups->chunk_parts;
+    p.max_members = groups->max_members;
+    const int zparts = groups->max_chunk_parts < ws.parts ? groups->max_chunk_parts : ws.parts;
+    e = dtype == PA_BF16 ? launch_decode_group_bf16(p, groups->num_chunks, zparts, st)
+                         : launch_decode_group_f16(p, groups->num_chunks, zparts, st);
+    if (e != cudaSuccess) {
+      note_cuda_error(e);
+      return PA_ERR_CUDA;
+    }
+  }
   if (mma_eligible(dtype, group, head_dim, block_size)) {
     e = dtype == PA_BF16 ? launch_decode_mma_bf16(p, st) : launch_decode_mma_f16(p, st);
   } else {
@@ -261,3 +337,6 @@ extern "C" int pa_decode_attention(void* out, const void* q, const void* k_cache
   }
   return PA_OK;
 }
+
+}  // namespace
+}  // namespace pa

@@ -106,7 +106,11 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return static_cast<uint32_t>((c >> 3) * (BS * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-template <typename T, int D, int BS, int NT, int NW, int NST>
+// GROUP = false: one CTA per (sequence, 8*NT query heads of one kv head, partition).
+// GROUP = true : one CTA per (kv head, chunk of a prefix group, shared partition);
+//   the tile's columns are (member, head) pairs, member = column / group, and the
+//   partition's blocks - identical for every member - are read once for all of them.
+template <typename T, int D, int BS, int NT, int NW, int NST, bool GROUP>
 __global__ void __launch_bounds__(NW * 32)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -116,6 +120,8 @@ __global__ void __launch_bounds__(NW * 32)
   constexpr int TT = C::kTT, KS = C::kKS;
 
   extern __shared__ uint8_t smem_raw[];
+  __shared__ int col_row[C::kHeads];  // q / out row (sequence * Hq + head) of each column
+  __shared__ int col_ok[C::kHeads];   // the column's result is written by this CTA
   // 1024-byte alignment for the swizzle atoms
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -123,19 +129,53 @@ __global__ void __launch_bounds__(NW * 32)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t4 = lane & 3;  // fragment row group / thread in group
-  const int s = blockIdx.y, part = blockIdx.z;
-  const int h0 = blockIdx.x * C::kHeads;
-  const int kvh = h0 / (p.num_heads / p.num_kv_heads);
-
-  const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && part == 0);
+  const int G = p.num_heads / p.num_kv_heads;
   const int ps = p.partition_size;
-  const int nparts = L > 0 ? (L + ps - 1) / ps : 1;
-  if (part >= nparts) return;
-  const int tok_begin = part * ps;
-  const int tok_end = min(L, tok_begin + ps);
+  int kvh, part, nparts, tok_begin, tok_end, table_seq;
+  if constexpr (!GROUP) {
+    const int s = blockIdx.y;
+    const int h0 = blockIdx.x * C::kHeads;
+    part = blockIdx.z;
+    kvh = h0 / G;
+    const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && part == 0);
+    nparts = L > 0 ? (L + ps - 1) / ps : 1;
+    if (part >= nparts || part < group_parts(p, s, L)) return;
+    tok_begin = part * ps;
+    tok_end = min(L, tok_begin + ps);
+    table_seq = s;
+    if (threadIdx.x < C::kHeads) {
+      col_row[threadIdx.x] = s * p.num_heads + h0 + threadIdx.x;
+      col_ok[threadIdx.x] = 1;
+    }
+  } else {
+    const int chunk = blockIdx.y;
+    kvh = blockIdx.x;
+    part = blockIdx.z;
+    if (part >= __ldg(p.chunk_parts + chunk)) return;
+    nparts = 2;  // a grouped partition is always one of several: write partials
+    tok_begin = part * ps;
+    tok_end = tok_begin + ps;
+    if (threadIdx.x < C::kHeads) {
+      const int c = threadIdx.x, mi = c / G;
+      const int m = mi < p.max_members ? __ldg(p.chunk_members + chunk * p.max_members + mi) : -1;
+      const bool member = m >= 0 && m < p.num_seqs;
+      col_row[c] = member ? m * p.num_heads + kvh * G + (c - mi * G) : -1;
+      col_ok[c] = member && part < group_parts(p, m, checked_len(p, m, false));
+    }
+    __syncthreads();
+    // blocks come from the table of the first member that owns this partition
+    table_seq = -1;
+    for (int c = 0; c < C::kHeads; ++c)
+      if (col_ok[c]) {
+        table_seq = col_row[c] / p.num_heads;
+        break;
+      }
+    if (table_seq < 0) return;  // no member needs this partition
+  }
+  __syncthreads();
   const int nblk = tok_end > tok_begin ? (tok_end - tok_begin + BS - 1) / BS : 0;
   const int32_t* table =
-      p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + tok_begin / BS;
+      p.block_tables + static_cast<int64_t>(table_seq) * p.max_blocks_per_seq + tok_begin / BS;
 
   const uint32_t stage0 = base + warp * NST * C::kStageBytes;
   const uint32_t bar0 = base + (C::kSmemBytes - 1024 - NW * NST * 8) + warp * NST * 8;
@@ -146,18 +186,19 @@ __global__ void __launch_bounds__(NW * 32)
   }
   __syncwarp();
 
-  // Q^T as B fragments: qb[nt][ks][0] = q[head n0+g8][16ks + 2t4 .. +1], [1] = +8 dims
+  // Q^T as B fragments: qb[nt][ks][0] = q[column nt*8+g8][16ks + 2t4 .. +1], [1] = +8
+  // dims; a column with no member gets zeros (its result is never written)
   uint32_t qb[NT][KS][2];
-  {
-    const T* qrow = static_cast<const T*>(p.q) + (static_cast<int64_t>(s) * p.num_heads + h0) * D;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+  for (int nt = 0; nt < NT; ++nt) {
+    const int row = col_row[nt * 8 + g8];
+    const T* qp0 = static_cast<const T*>(p.q) + static_cast<int64_t>(row < 0 ? 0 : row) * D;
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        const T* qp = qrow + (nt * 8 + g8) * D + ks * 16 + 2 * t4;
-        qb[nt][ks][0] = __ldg(reinterpret_cast<const unsigned int*>(qp));
-        qb[nt][ks][1] = __ldg(reinterpret_cast<const unsigned int*>(qp + 8));
-      }
+    for (int ks = 0; ks < KS; ++ks) {
+      const T* qp = qp0 + ks * 16 + 2 * t4;
+      qb[nt][ks][0] = row < 0 ? 0u : __ldg(reinterpret_cast<const unsigned int*>(qp));
+      qb[nt][ks][1] = row < 0 ? 0u : __ldg(reinterpret_cast<const unsigned int*>(qp + 8));
+    }
   }
 
   // per thread: heads nt*8 + 2t4 + {0,1}
@@ -376,7 +417,8 @@ __global__ void __launch_bounds__(NW * 32)
       den = fmaf(r[D + 1], f, den);
     }
     const float o = den > 0.f ? num / den : 0.f;
-    const int64_t row = static_cast<int64_t>(s) * p.num_heads + h0 + hh;
+    if (!col_ok[hh]) continue;
+    const int64_t row = col_row[hh];
     if (nparts == 1) {
       store_elem(static_cast<T*>(p.out) + row * D + d, o);
     } else {

@@ -6,8 +6,8 @@
 namespace pa {
 namespace {
 
-template <int D, int BS, int NT>
-cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
+template <int D, int BS, int NT, bool GROUP>
+cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   constexpr int kStage = 2 * BS * D * 2;
   constexpr int NW = kStage <= 16384 ? 4 : (kStage <= 32768 ? 2 : 1);
   constexpr int kRaw = 65536 / (NW * kStage);
@@ -20,41 +20,51 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
   if (!make_cache_tensor_map(&tmk, p.k_cache, rows, D, BS, bf16) ||
       !make_cache_tensor_map(&tmv, p.v_cache, rows, D, BS, bf16))
     return cudaErrorInvalidValue;
-  constexpr auto kern = decode_mma_kernel<__nv_bfloat16, D, BS, NT, NW, NST>;
+  constexpr auto kern = decode_mma_kernel<__nv_bfloat16, D, BS, NT, NW, NST, GROUP>;
   cudaError_t e = ensure_smem_limit<kern>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_heads / C::kHeads, p.num_seqs, p.max_parts);
   kern<<<grid, NW * 32, C::kSmemBytes, st>>>(p, tmk, tmv);
   return cudaGetLastError();
 }
 
-template <int D, int NT>
-cudaError_t by_bs(const DecodeParams& p, cudaStream_t st) {
+template <int D, int NT, bool GROUP>
+cudaError_t by_bs(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   switch (p.block_size) {
-    case 16: return launch<D, 16, NT>(p, st);
-    case 32: return launch<D, 32, NT>(p, st);
+    case 16: return launch<D, 16, NT, GROUP>(p, grid, st);
+    case 32: return launch<D, 32, NT, GROUP>(p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D>
-cudaError_t by_nt(const DecodeParams& p, cudaStream_t st) {
-  switch ((p.num_heads / p.num_kv_heads) / 8) {
-    case 1: return by_bs<D, 1>(p, st);
-    case 2: return by_bs<D, 2>(p, st);
+template <bool GROUP>
+cudaError_t by_shape(const DecodeParams& p, int nt, dim3 grid, cudaStream_t st) {
+  switch (p.head_dim * 4 + nt) {
+    case 64 * 4 + 1: return by_bs<64, 1, GROUP>(p, grid, st);
+    case 64 * 4 + 2: return by_bs<64, 2, GROUP>(p, grid, st);
+    case 128 * 4 + 1: return by_bs<128, 1, GROUP>(p, grid, st);
+    case 128 * 4 + 2: return by_bs<128, 2, GROUP>(p, grid, st);
+    case 256 * 4 + 1: return by_bs<256, 1, GROUP>(p, grid, st);
+    case 256 * 4 + 2: return by_bs<256, 2, GROUP>(p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
+// Per-sequence partitions: 8*NT query heads of one kv head per CTA (NT = group / 8).
 cudaError_t launch_decode_mma_bf16(const DecodeParams& p, cudaStream_t st) {
-  switch (p.head_dim) {
-    case 64: return by_nt<64>(p, st);
-    case 128: return by_nt<128>(p, st);
-    case 256: return by_nt<256>(p, st);
-    default: return cudaErrorInvalidValue;
-  }
+  const int nt = (p.num_heads / p.num_kv_heads) / 8;
+  dim3 grid(p.num_heads / (8 * nt), p.num_seqs, p.max_parts);
+  return by_shape<false>(p, nt, grid, st);
+}
+
+// Shared partitions of prefix groups: columns = max_members * group <= 16.
+cudaError_t launch_decode_group_bf16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
+                                   cudaStream_t st) {
+  const int cols = p.max_members * (p.num_heads / p.num_kv_heads);
+  const int nt = cols <= 8 ? 1 : 2;
+  dim3 grid(p.num_kv_heads, num_chunks, max_chunk_parts);
+  return by_shape<true>(p, nt, grid, st);
 }
 
 }  // namespace pa

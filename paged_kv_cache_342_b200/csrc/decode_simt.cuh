@@ -65,6 +65,18 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int s, bool re
   return L;
 }
 
+// Leading partitions of sequence s that its prefix group's kernel computes (0 when
+// the call has no groups).  Never the partition holding the last token, so every
+// sequence keeps at least one partition of its own and a grouped sequence always
+// goes through the merge.  The per-sequence and group kernels evaluate this same
+// expression, so every partition is written by exactly one of them.
+__device__ __forceinline__ int group_parts(const DecodeParams& p, int s, int L) {
+  if (!p.prefix_parts || L <= 0) return 0;
+  const int g = __ldg(p.prefix_parts + s);
+  const int last = (L - 1) / p.partition_size;
+  return g < 0 ? 0 : (g < last ? g : last);
+}
+
 template <typename T, int D, int BS, int GS, int NW, int NST>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams p) {
   using C = SimtCfg<T, D, BS, GS, NW, NST>;
@@ -83,7 +95,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
   const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && part == 0);
   const int ps = p.partition_size;
   const int nparts = L > 0 ? (L + ps - 1) / ps : 1;
-  if (part >= nparts) return;
+  if (part >= nparts || part < group_parts(p, s, L)) return;
   const int tok_begin = part * ps;
   const int tok_end = min(L, tok_begin + ps);
   const int nblk = tok_end > tok_begin ? (tok_end - tok_begin + BS - 1) / BS : 0;

@@ -16,6 +16,12 @@ With ``rolling=True`` each step first rolls the sequences back to the lengths th
 had when bound (``pa_seq_truncate``): every step then decodes the same lengths,
 which is how a long benchmark run stays on one workload.
 
+Sequences that share leading blocks (forks of one prompt) are found each step by
+``pa_build_prefix_groups``; their shared partitions are then read once per group
+(``pa_decode_attention_grouped``).  ``group_members`` caps a chunk (default: as many
+members as fill one 8-column tensor-core tile, 8 // (num_heads/num_kv_heads); 0
+turns grouping off).
+
 This module only moves arguments: the work of every step is done by the library.
 """
 from __future__ import annotations
@@ -24,7 +30,7 @@ import numpy as np
 import torch
 
 from . import (DEFAULT_PARTITION, BlockAllocator, pa_copy_blocks, pa_decode_attention,
-               pa_decode_workspace_bytes, pa_reshape_and_cache)
+               pa_decode_attention_grouped, pa_decode_workspace_bytes, pa_reshape_and_cache)
 
 
 def _align(n: int, a: int = 256) -> int:
@@ -39,7 +45,8 @@ class PagedDecoder:
     """
 
     def __init__(self, k_cache, v_cache, num_heads: int, scale: float, max_blocks_per_seq: int,
-                 free_order=None, partition_size: int = DEFAULT_PARTITION, stream=None):
+                 free_order=None, partition_size: int = DEFAULT_PARTITION, stream=None,
+                 group_members: int | None = None):
         self.k_cache, self.v_cache = k_cache, v_cache
         self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim = k_cache.shape
         self.num_heads, self.scale = num_heads, scale
@@ -51,6 +58,9 @@ class PagedDecoder:
         self._seq_ids = None
         self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
         self._done = None  # event: the last staging copy has been consumed
+        group = num_heads // self.num_kv_heads
+        self.group_members = (8 // group if group <= 8 else 0) if group_members is None \
+            else group_members
 
     # -- context building ------------------------------------------------------
     def admit(self, seq_id: int, num_tokens: int) -> None:
@@ -89,23 +99,36 @@ class PagedDecoder:
         self.rolling = rolling
         self._stepped = False
         self.base_lens = np.array([self.alloc.seq_len(int(s)) for s in ids], np.int64)
-        S, MB = ids.size, self.max_blocks
-        o_slots = 0
-        o_pairs = _align(8 * S)
-        o_lens = o_pairs + _align(8 * max(S, 1))
-        o_tab = o_lens + _align(4 * S)
-        total = o_tab + _align(4 * S * MB)
+        S, MB, MM = ids.size, self.max_blocks, max(1, self.group_members)
+        S1 = max(S, 1)
+        sizes = [("slots", 8 * S), ("pairs", 8 * S1), ("lens", 4 * S), ("tables", 4 * S * MB),
+                 ("pparts", 4 * S1), ("cmembers", 4 * S1 * MM), ("cparts", 4 * S1)]
+        offs, total = {}, 0
+        for name, n in sizes:
+            offs[name] = total
+            total += _align(n)
         self.h_stage = torch.empty(total, dtype=torch.uint8, pin_memory=True)
         self.d_stage = torch.empty(total, dtype=torch.uint8, device=self.device)
 
         def views(buf):
-            return (buf[o_slots:o_slots + 8 * S].view(torch.int64),
-                    buf[o_pairs:o_pairs + 8 * max(S, 1)].view(torch.int32).view(-1, 2),
-                    buf[o_lens:o_lens + 4 * S].view(torch.int32),
-                    buf[o_tab:o_tab + 4 * S * MB].view(torch.int32).view(S, MB))
+            def sec(name, n, dt):
+                return buf[offs[name]:offs[name] + n].view(dt)
+            return dict(
+                slots=sec("slots", 8 * S, torch.int64),
+                pairs=sec("pairs", 8 * S1, torch.int32).view(-1, 2),
+                lens=sec("lens", 4 * S, torch.int32),
+                tables=sec("tables", 4 * S * MB, torch.int32).view(S, MB),
+                pparts=sec("pparts", 4 * S1, torch.int32),
+                cmembers=sec("cmembers", 4 * S1 * MM, torch.int32).view(S1, MM),
+                cparts=sec("cparts", 4 * S1, torch.int32))
 
-        self.h_slots, self.h_pairs, self.h_lens, self.h_tables = views(self.h_stage)
-        self.d_slots, self.d_pairs, self.d_lens, self.d_tables = views(self.d_stage)
+        h, d = views(self.h_stage), views(self.d_stage)
+        self.h_slots, self.h_pairs, self.h_lens, self.h_tables = (h["slots"], h["pairs"],
+                                                                  h["lens"], h["tables"])
+        self.d_slots, self.d_pairs, self.d_lens, self.d_tables = (d["slots"], d["pairs"],
+                                                                  d["lens"], d["tables"])
+        self.h_groups = (h["pparts"], h["cmembers"], h["cparts"])
+        self.d_groups = (d["pparts"], d["cmembers"], d["cparts"])
         cap = MB * self.block_size
         ws = pa_decode_workspace_bytes(S, self.num_heads, self.head_dim, cap, self.partition_size)
         if ws > self._ws.numel():
@@ -129,24 +152,44 @@ class PagedDecoder:
         _, lens = self.alloc.build_block_tables(self._seq_ids, self.max_blocks,
                                                 self.h_tables.numpy(), self.h_lens.numpy())
         max_len = int(lens.max()) if lens.size else 0
+        num_chunks = max_chunk_parts = 0
+        if self.group_members > 0:
+            hp, hm, hc = self.h_groups
+            _, members, _, max_chunk_parts = self.alloc.prefix_groups(
+                self._seq_ids, self.partition_size, self.group_members, hp.numpy(), hm.numpy(),
+                hc.numpy())
+            num_chunks = len(members)
         s = self._torch_stream()
         with torch.cuda.stream(s):
             self.d_stage.copy_(self.h_stage, non_blocking=True)
             self._done = torch.cuda.Event()
             self._done.record(s)
-        return dict(num_cow=n_cow, max_len=max_len, pairs=self.h_pairs.numpy()[:n_cow])
+        return dict(num_cow=n_cow, max_len=max_len, pairs=self.h_pairs.numpy()[:n_cow],
+                    num_chunks=num_chunks, max_chunk_parts=max_chunk_parts)
 
-    def launch(self, meta: dict, q, new_k, new_v, out) -> None:
-        """Device side of a step: copies, the new token's K/V, attention."""
+    def launch(self, meta: dict, q, new_k, new_v, out, events=None) -> None:
+        """Device side of a step: copies, the new token's K/V, attention.  ``events``
+        (a pair of CUDA events) are recorded around the attention call."""
         st = self._torch_stream()
         n = meta["num_cow"]
         if n:
             pa_copy_blocks(self.k_cache, self.v_cache, self.d_pairs[:n], meta["pairs"], stream=st)
         pa_reshape_and_cache(new_k, new_v, self.k_cache, self.v_cache, self.d_slots, stream=st)
-        pa_decode_attention(out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
-                            self.scale, self.block_size, self.num_kv_heads, meta["max_len"],
-                            self.partition_size, self._ws if self._ws.numel() else None,
-                            stream=st)
+        ws = self._ws if self._ws.numel() else None
+        if events is not None:
+            events[0].record(st)
+        if meta.get("num_chunks", 0):
+            pp, cm, cp = self.d_groups
+            pa_decode_attention_grouped(
+                out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens, self.scale,
+                self.block_size, self.num_kv_heads, meta["max_len"], pp, cm, cp,
+                meta["num_chunks"], meta["max_chunk_parts"], self.partition_size, ws, stream=st)
+        else:
+            pa_decode_attention(out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
+                                self.scale, self.block_size, self.num_kv_heads, meta["max_len"],
+                                self.partition_size, ws, stream=st)
+        if events is not None:
+            events[1].record(st)
 
     def step(self, q, new_k, new_v, out) -> dict:
         meta = self.prepare()
@@ -154,9 +197,13 @@ class PagedDecoder:
         return meta
 
     def kernel_launches(self, meta: dict) -> int:
-        """Library kernels one step launches (copy, write, partitions, merge)."""
+        """Library kernels one step launches (copy, write, group, partitions, merge)."""
         parts = max(1, -(-meta["max_len"] // self.partition_size))
-        return (1 if meta["num_cow"] else 0) + 2 + (1 if parts > 1 else 0)
+        grouped = (meta.get("num_chunks", 0) > 0 and parts > 1
+                   and self.k_cache.dtype != torch.float32
+                   and self.block_size in (16, 32)
+                   and self.group_members * (self.num_heads // self.num_kv_heads) <= 16)
+        return (1 if meta["num_cow"] else 0) + 2 + (1 if grouped else 0) + (1 if parts > 1 else 0)
 
     def _torch_stream(self):
         return torch.cuda.current_stream(self.device) if self.stream is None else self.stream

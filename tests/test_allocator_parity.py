@@ -171,3 +171,65 @@ def test_bad_create_arguments(pa):
         pa.BlockAllocator(4, 4, [0, 1, 1, 2])        # not a permutation
     with pytest.raises(pa.PagedAttentionError):
         pa.BlockAllocator(0, 4)
+
+
+def _compare_groups(c, o, ids, ps, mm):
+    pp, cm, cp, mp = c.prefix_groups(ids, ps, mm)
+    opp, ochunks = o.prefix_groups(ids, ps, mm)
+    assert pp.tolist() == opp
+    assert [(row[row >= 0].tolist(), int(parts)) for row, parts in zip(cm, cp)] == \
+        [(list(m), p) for m, p in ochunks]
+    assert mp == max([p for _, p in ochunks], default=0)
+    return ochunks
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_prefix_groups_random_forks(pa, seed):
+    """Fork forests with appends, copies and frees: both sides find the same groups."""
+    g = np.random.default_rng(100 + seed)
+    bs = int(g.choice([2, 4, 16]))
+    nb = 400
+    c, o = pa.BlockAllocator(nb, bs), BlockManager(nb, bs)
+    live, nid = [], 0
+    for _ in range(60):
+        r = g.integers(0, 10)
+        if r < 3 or not live:
+            n = int(g.integers(0, 6 * bs))
+            c.add(nid, n), o.add(nid, n)
+            live.append(nid)
+            nid += 1
+        elif r < 6:
+            p = live[int(g.integers(0, len(live)))]
+            c.fork(p, nid), o.fork(p, nid)
+            live.append(nid)
+            nid += 1
+        elif r < 9:
+            s = live[int(g.integers(0, len(live)))]
+            for _ in range(int(g.integers(1, 2 * bs))):
+                assert c.append_slot(s) == o.append_slot(s)
+        else:
+            s = live.pop(int(g.integers(0, len(live))))
+            c.free(s), o.free_seq(s)
+    ids = list(g.permutation(live))
+    for ps in (bs, 2 * bs, 4 * bs):
+        for mm in (1, 2, 3, 8):
+            _compare_groups(c, o, ids, ps, mm)
+
+
+def test_prefix_groups_of_the_shared_prefix_workload(pa):
+    from oracle.step import build_context
+    cfg = CONFIGS["prefix_cow_bf16"]
+    inp = make_inputs(cfg, 0, pool=False)
+    o, _, _, _ = build_context(inp, copy_pool=False)
+    c = pa.BlockAllocator(cfg.num_blocks, cfg.block_size, inp.free_order)
+    p = inp.prefix
+    for gi in range(p.groups):
+        c.add(gi * p.samples, p.prefix_len)
+        for i in range(1, p.samples):
+            c.fork(gi * p.samples, gi * p.samples + i)
+    for s in range(cfg.num_seqs):
+        for _ in range(int(p.private_lens[s])):
+            c.append_slot(s)
+    chunks = _compare_groups(c, o, list(range(cfg.num_seqs)), 512, 8)
+    # 1030-token prefix = 64 full blocks shared by all 8 samples -> 2 partitions of 512
+    assert len(chunks) == 32 and all(len(m) == 8 and parts == 2 for m, parts in chunks)

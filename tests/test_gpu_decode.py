@@ -143,3 +143,89 @@ def test_length_beyond_bound_is_skipped_and_reported(pa):
     assert not out[1].any()
     want = oatt.paged_decode_attention(q[:1], k, k, tables[:1], lens[:1], 0.125, bs, Hkv, "f16")
     assert_close(out_f64(out[:1]), want, "f16")
+
+
+# ---------------------------------------------------------------------------
+# prefix groups: shared partitions computed once per group
+# ---------------------------------------------------------------------------
+
+def run_grouped_case(pa, dtype, Hq, Hkv, D, bs, ps, prefix_len, tails, group_sizes, mm,
+                     seed=3):
+    """Groups of sequences forked from one prefix through the block manager, with
+    private tails written into their own blocks; compare the grouped call with the
+    oracle (and with the plain call)."""
+    from oracle.allocator import BlockManager
+    sizes = list(group_sizes)
+    S = sum(sizes)
+    lens = np.array([prefix_len + t for t in tails], np.int64)
+    assert len(lens) == S
+    NB = len(sizes) * (-(-prefix_len // bs)) + int(sum(-(-t // bs) + 1 for t in tails)) + 4
+    bm = BlockManager(NB, bs, np.random.default_rng([seed, 9]).permutation(NB))
+    sid = 0
+    for n in sizes:
+        bm.add(sid, prefix_len)
+        for i in range(1, n):
+            bm.fork(sid, sid + i)
+        sid += n
+    for s in range(S):
+        for _ in range(int(tails[s])):
+            bm.append_slot(s)
+    width = max(len(t) for t in bm.tables.values()) + 1
+    rows, sl = bm.block_tables(range(S), width)
+    tables, sl = np.array(rows, np.int32), np.array(sl, np.int32)
+    k = normal_fill((NB, Hkv, bs, D), dtype, 1.0, seed, 1)
+    v = normal_fill((NB, Hkv, bs, D), dtype, 1.0, seed, 2)
+    q = normal_fill((S, Hq, D), dtype, 1.0, seed, 3)
+    pp, chunks = bm.prefix_groups(range(S), ps, mm)
+    cm = np.full((max(len(chunks), 1), mm), -1, np.int32)
+    cp = np.zeros(max(len(chunks), 1), np.int32)
+    for i, (members, parts) in enumerate(chunks):
+        cm[i, :len(members)] = members
+        cp[i] = parts
+    max_len = int(sl.max())
+    scale = 1 / math.sqrt(D)
+    kd, vd, qd = to_dev(k, dtype), to_dev(v, dtype), to_dev(q, dtype)
+    td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(sl).cuda()
+    wsb = pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+    out = torch.full((S, Hq, D), float("nan"), dtype=TORCH_DT[dtype], device="cuda")
+    pa.pa_decode_attention_grouped(out, qd, kd, vd, td, ld, scale, bs, Hkv, max_len,
+                                   torch.from_numpy(np.array(pp, np.int32)).cuda(),
+                                   torch.from_numpy(cm).cuda(), torch.from_numpy(cp).cuda(),
+                                   len(chunks), max([c[1] for c in chunks], default=0), ps,
+                                   ws if wsb else None)
+    plain = torch.full_like(out, float("nan"))
+    pa.pa_decode_attention(plain, qd, kd, vd, td, ld, scale, bs, Hkv, max_len, ps,
+                           ws if wsb else None)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    want = oatt.paged_decode_attention(q, k, v, tables, sl, scale, bs, Hkv, dtype)
+    return out_f64(out), out_f64(plain), want, chunks
+
+
+GROUP_CASES = [
+    # dtype, Hq, Hkv, D, bs, partition, prefix, tails, group sizes, members per chunk
+    ("bf16", 4, 4, 128, 16, 64, 300, [1, 5, 40, 0, 17, 3, 90, 1], [8], 8),
+    ("f16", 2, 2, 64, 16, 32, 130, [2, 0, 1, 33, 70], [3, 2], 8),       # prefix not whole
+    ("bf16", 4, 2, 128, 32, 64, 256, [1, 9, 64, 2, 3, 1], [6], 4),     # group 2 heads/kv
+    ("bf16", 16, 2, 128, 16, 64, 200, [1, 20, 3], [3], 1),             # GQA 8 + 1 member
+    ("f16", 4, 4, 256, 16, 64, 129, [1] * 11 + [40], [12], 8),         # 2 chunks
+    ("bf16", 2, 2, 128, 16, 64, 64, [0, 0, 5], [3], 8),                 # tails of length 0
+]
+
+
+@pytest.mark.parametrize("case", GROUP_CASES, ids=lambda c: f"{c[0]}-h{c[1]}/{c[2]}-d{c[3]}-b{c[4]}-p{c[5]}-g{c[8]}")
+def test_grouped_matches_oracle_and_plain(pa, case):
+    dtype, Hq, Hkv, D, bs, ps, prefix, tails, sizes, mm = case
+    got, plain, want, chunks = run_grouped_case(pa, dtype, Hq, Hkv, D, bs, ps, prefix, tails,
+                                                sizes, mm)
+    assert_close(got, want, dtype, "grouped")
+    assert_close(plain, want, dtype, "plain")
+    assert np.abs(got - plain).max() <= 2e-2
+
+
+def test_grouped_call_uses_groups(pa):
+    """The shared-prefix case really forms chunks (so the group kernel ran)."""
+    *_, chunks = run_grouped_case(pa, *GROUP_CASES[0])
+    # 300-token prefix at block 16 = 18 full shared blocks = 288 tokens = 4 partitions of 64
+    assert len(chunks) == 1 and chunks[0] == (list(range(8)), 4)
