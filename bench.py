@@ -51,6 +51,9 @@ def parse():
     # smaller instances of a workload for profiling captures (reported in "config")
     ap.add_argument("--seqs", type=int, default=None, help="override the batch size")
     ap.add_argument("--pool-blocks", type=int, default=None, help="override the pool size")
+    # the pages' block-size trade-off: same lengths and slot capacity, other block size
+    ap.add_argument("--block-size", type=int, default=None,
+                    help="override the block size (pool keeps the same number of slots)")
     return ap.parse_args()
 
 
@@ -88,6 +91,37 @@ def unique_context_tokens(dec, cfg, seq_ids) -> int:
             n = min(cfg.block_size, L - j * cfg.block_size)
             fill[b] = max(fill.get(b, 0), n)
     return sum(fill.values())
+
+
+# ---------------------------------------------------------------------------
+# replicas: one process per GPU, no collective on the data path
+# ---------------------------------------------------------------------------
+
+def replica_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 without it)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each rank decodes its own replica of the workload (weak scaling)."""
+    return base_seed + rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's elapsed time: every rank must call this, in the same order."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step: int, steps: int, world: int, elapsed_max_ms: float) -> float:
+    """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
+    return float(bytes_per_step) * steps * world / (elapsed_max_ms * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------------------
@@ -253,9 +287,7 @@ def run_ours(args, cfg):
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = replica_env()
 
     import paged_kv_cache_342_b200 as pa
     from paged_kv_cache_342_b200.runtime import PagedDecoder
@@ -276,7 +308,7 @@ def run_ours(args, cfg):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    seed = args.seed + rank
+    seed = replica_seed(args.seed, rank)
     inp = make_inputs(cfg, seed)
     S, Hq, Hkv, D, bs = cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
     max_len = int((inp.context_lens + 1).max()) + 1
@@ -357,12 +389,8 @@ def run_ours(args, cfg):
     err = pa.pa_device_error_read()
     if err:
         raise RuntimeError(f"device error word {err} after the timed region")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-    total_bytes = float(step_bytes) * args.steps * world
-    value = total_bytes / (elapsed_ms * 1e-3) / 1e9
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    value = job_throughput(step_bytes, args.steps, world, elapsed_ms)
     seqs_per_s = S * world * args.steps / (elapsed_ms * 1e-3)
 
     # ---- end to end through the public API with host buffers ----------------------
@@ -388,12 +416,8 @@ def run_ours(args, cfg):
             e2e_step(k)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        E = float(step_bytes) * args.steps * world / (e_ms * 1e-3) / 1e9
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        E = job_throughput(step_bytes, args.steps, world, e_ms)
         h2d = sum(t.numel() * t.element_size() for t in toks_h[0]) + dec.staging_bytes
         d2h = S * Hq * D * cfg.elem_bytes
         e2e = {"value": round(E, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
@@ -435,6 +459,7 @@ def run_ours(args, cfg):
                        "parallelism": f"replicas x{world}",
                        "workspace_bytes": int(dec._ws.numel()),
                        "prefix_group_chunks": int(meta0.get("num_chunks", 0)),
+                       "pool": pool_summary(dec.alloc.stats()),
                        "cow_pairs_in_warmup": warm_cow, "cow_pairs_in_timed_steps": cows},
             "roofline": roof,
             "cpu_baseline": cpu,
@@ -446,6 +471,14 @@ def run_ours(args, cfg):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def pool_summary(st: dict) -> dict:
+    """Block-manager view of the batch: blocks in use, slots, and the tail waste
+    (unused slots of each sequence's last block) as a share of allocated slots."""
+    return {"used_blocks": st["used_blocks"], "shared_blocks": st["shared_blocks"],
+            "allocated_slots": st["allocated_slots"], "logical_tokens": st["logical_tokens"],
+            "tail_waste_pct": round(100.0 * st["tail_waste_slots"] / max(1, st["allocated_slots"]), 3)}
 
 
 def recorded_traffic(cfg):
@@ -485,6 +518,10 @@ def main():
         cfg = cfg.with_(num_seqs=args.seqs, name=f"{cfg.name}_s{args.seqs}")
     if args.pool_blocks is not None:
         cfg = cfg.with_(num_blocks=args.pool_blocks, name=f"{cfg.name}_nb{args.pool_blocks}")
+    if args.block_size is not None and args.block_size != cfg.block_size:
+        slots = cfg.num_blocks * cfg.block_size
+        cfg = cfg.with_(block_size=args.block_size, num_blocks=slots // args.block_size,
+                        name=f"{cfg.name}_bs{args.block_size}")
     if args.impl == "reference":
         run_reference(args, cfg)
     else:
