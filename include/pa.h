@@ -111,6 +111,27 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_mapping_de
                    pa_stream_t stream);
 
 /*
+ * pa_swap_blocks - copy whole blocks between two caches, e.g. the device pool and a
+ * host swap pool when a sequence is preempted and later resumed ([GLOSS] "pages can
+ * be efficiently swapped or evicted ... spilling to CPU RAM"; [BLOG] "Where it bites":
+ * a full pool swaps blocks out to CPU memory).
+ *   dst_k, dst_v   destination cache [dst_num_blocks, num_kv_heads, block_size, head_dim]
+ *   src_k, src_v   source cache      [src_num_blocks, ...]
+ *   block_mapping  int32 [num_pairs, 2] (src block, dst block), device-reachable
+ *   block_mapping_host  same pairs on the host for validation (nullable)
+ * Each side may be device memory of the current device or page-locked host memory
+ * (cudaHostAlloc / cudaMallocHost / cudaHostRegister; the kernel reaches it through
+ * unified addressing).  Every pointer is checked with cudaPointerGetAttributes before
+ * the launch; pageable or foreign memory gives PA_ERR_INVALID_ARG.  With the host
+ * mapping given, ids must be in range and destinations distinct.  One kernel launch
+ * copies all pairs (K and V); ids outside the pools are skipped (PA_DEVERR_COPY_BLOCK).
+ */
+int pa_swap_blocks(void* dst_k, void* dst_v, int64_t dst_num_blocks, const void* src_k,
+                   const void* src_v, int64_t src_num_blocks, const int32_t* block_mapping,
+                   const int32_t* block_mapping_host, int num_pairs, int num_kv_heads,
+                   int head_dim, int block_size, int dtype, pa_stream_t stream);
+
+/*
  * pa_decode_workspace_bytes - scratch bytes pa_decode_attention needs.
  * P = ceil(max_seq_len / partition_size) partitions per sequence; when P > 1 the
  * workspace holds float32 partial outputs [num_seqs, num_heads, P, head_dim] and
@@ -305,6 +326,17 @@ int pa_seq_append_slots(pa_alloc_t* a, const int64_t* seq_ids, int n, int64_t* s
  * draft token; blocks past ceil(new_len/block_size) drop a reference (released in
  * logical order).  No copy is ever needed.  Ids must be distinct.  All or nothing. */
 int pa_seq_truncate(pa_alloc_t* a, const int64_t* seq_ids, const int64_t* new_lens, int n);
+/* Move sequences from one pool to another (swap-out to a host pool, swap-in back):
+ * each distinct block the moved sequences reference gets one fresh block in `to`
+ * (first-appearance order: sequence order, then logical order), so blocks shared
+ * inside the moved set stay shared; a block also used by sequences staying in `from`
+ * becomes a private copy.  Lengths and logical order are kept; each moved reference in
+ * `from` is dropped in the same order.  pairs_out (capacity cap pairs) receives the
+ * (from_block, to_block) copies to make with pa_swap_blocks, *num_pairs their count.
+ * Ids must be distinct, present in `from`, absent from `to`; block sizes must match.
+ * All or nothing (PA_ERR_NO_FREE_BLOCKS when `to` is short). */
+int pa_seqs_move(pa_alloc_t* from, pa_alloc_t* to, const int64_t* seq_ids, int n,
+                 int32_t* pairs_out, int64_t cap, int64_t* num_pairs);
 /* Release seq_id. */
 int pa_seq_free(pa_alloc_t* a, int64_t seq_id);
 int pa_seq_len(const pa_alloc_t* a, int64_t seq_id, int64_t* len);

@@ -149,6 +149,48 @@ class BlockManager:
             del table[keep:]
             self.lens[s] = n
 
+    def move_to(self, other: "BlockManager", seq_ids):
+        """Move sequences into another pool (e.g. device pool -> host swap pool).
+
+        Every distinct block the moved sequences reference gets one fresh block in
+        ``other`` (taken in order of first appearance: sequence order, then logical
+        order), so sharing inside the moved set is kept; references to blocks shared
+        with sequences that stay behind become private copies.  In this pool each
+        moved reference is dropped in the same order (a block reaching zero goes
+        back on the free stack).  Returns the (this_block, other_block) pairs to copy.
+        All or nothing; ids must be distinct.
+        """
+        ids = list(seq_ids)
+        if len(set(ids)) != len(ids):
+            raise AllocError(INVALID_ARG, "sequence ids repeat")
+        for s in ids:
+            if s not in self.tables:
+                raise AllocError(UNKNOWN_SEQ, str(s))
+            if s in other.tables:
+                raise AllocError(SEQ_EXISTS, str(s))
+        if other.block_size != self.block_size:
+            raise AllocError(INVALID_ARG, "block sizes differ")
+        distinct = []
+        for s in ids:
+            for b in self.tables[s]:
+                if b not in distinct:
+                    distinct.append(b)
+        if len(distinct) > len(other.free):
+            raise AllocError(NO_FREE_BLOCKS, f"need {len(distinct)}, have {len(other.free)}")
+        mapping = {b: other._pop() for b in distinct}
+        for nb in mapping.values():
+            other.ref[nb] = 0                # counted below, one per table entry
+        for s in ids:
+            table = self.tables.pop(s)
+            other.tables[s] = [mapping[b] for b in table]
+            other.lens[s] = self.lens.pop(s)
+            for b in table:
+                other.ref[mapping[b]] += 1
+                self.ref[b] -= 1
+                if self.ref[b] == 0:
+                    self.free.append(b)
+        return [(b, mapping[b]) for b in distinct]
+
     def free_seq(self, seq_id: int) -> None:
         if seq_id not in self.tables:
             raise AllocError(UNKNOWN_SEQ, str(seq_id))

@@ -59,6 +59,7 @@ def _sig(name, res, *args):
 
 _sig("pa_reshape_and_cache", _i32, _p, _p, _p, _p, _p, _i64, _i32, _i32, _i32, _i64, _i32, _p)
 _sig("pa_copy_blocks", _i32, _p, _p, _p, _p, _i32, _i32, _i32, _i32, _i64, _i32, _p)
+_sig("pa_swap_blocks", _i32, _p, _p, _i64, _p, _p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p)
 _sig("pa_decode_workspace_bytes", ctypes.c_size_t, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode_attention", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32, _i32,
      _i32, _i64, _i32, _i32, _i32, _p, ctypes.c_size_t, _p)
@@ -77,6 +78,7 @@ _sig("pa_seq_append_slot", _i32, _p, _i64, _I64P, _I32P, _I32P)
 _sig("pa_seq_append_slots", _i32, _p, _p, _i32, _p, _p, ctypes.POINTER(ctypes.c_int))
 _sig("pa_seq_free", _i32, _p, _i64)
 _sig("pa_seq_truncate", _i32, _p, _p, _p, _i32)
+_sig("pa_seqs_move", _i32, _p, _p, _p, _i32, _p, _i64, _I64P)
 _sig("pa_seq_len", _i32, _p, _i64, _I64P)
 _sig("pa_seq_blocks", _i32, _p, _i64, _p, _i64, _I64P)
 _sig("pa_build_block_tables", _i32, _p, _p, _i32, _p, _i32, _p)
@@ -152,6 +154,33 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, block_mapping_host=None, str
         _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
         _dev(block_mapping, "block_mapping", torch.int32) if n else None, host_ptr, n, Hkv, D, bs,
         NB, _dtype_code(k_cache), _stream(stream)), "pa_copy_blocks")
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, block_mapping_host=None,
+                   stream=None) -> None:
+    """Copy blocks src -> dst between two caches [NB, Hkv, bs, D]; each may be a CUDA
+    tensor or a pinned CPU tensor.  block_mapping int32 [n, 2] (CUDA or pinned)."""
+    import torch
+    n = int(block_mapping.shape[0])
+    if n == 0:
+        return
+    for t, name in ((dst_k, "dst_k"), (dst_v, "dst_v"), (src_k, "src_k"), (src_v, "src_v"),
+                    (block_mapping, "block_mapping")):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if block_mapping.dtype != torch.int32:
+        raise ValueError("block_mapping must be int32")
+    host_ptr = None
+    if block_mapping_host is not None:
+        block_mapping_host = np.ascontiguousarray(block_mapping_host, dtype=np.int32)
+        host_ptr = block_mapping_host.ctypes.data
+    NBd, Hkv, bs, D = dst_k.shape
+    NBs = src_k.shape[0]
+    _check(lib.pa_swap_blocks(dst_k.data_ptr(), dst_v.data_ptr(), NBd, src_k.data_ptr(),
+                              src_v.data_ptr(), NBs, block_mapping.data_ptr(), host_ptr, n, Hkv,
+                              D, bs, _dtype_code(dst_k), _stream(stream)), "pa_swap_blocks")
 
 
 def pa_decode_workspace_bytes(num_seqs, num_heads, head_dim, max_seq_len,
@@ -297,6 +326,17 @@ class BlockAllocator:
             raise ValueError("seq_ids and new_lens differ in length")
         _check(lib.pa_seq_truncate(self._h, ids.ctypes.data, lens.ctypes.data, ids.size),
                "pa_seq_truncate")
+
+    def move_to(self, other: "BlockAllocator", seq_ids) -> np.ndarray:
+        """Move sequences into another pool; returns the (this_block, other_block) copy
+        pairs (int32 [k, 2]) to make with pa_swap_blocks."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        cap = sum(len(self.seq_blocks(int(s))) for s in ids) if ids.size else 0
+        pairs = np.empty((max(cap, 1), 2), np.int32)
+        n = ctypes.c_int64(0)
+        _check(lib.pa_seqs_move(self._h, other._h, ids.ctypes.data, ids.size, pairs.ctypes.data,
+                                cap, ctypes.byref(n)), "pa_seqs_move")
+        return pairs[:n.value]
 
     def free(self, seq_id: int) -> None:
         _check(lib.pa_seq_free(self._h, seq_id), "pa_seq_free")

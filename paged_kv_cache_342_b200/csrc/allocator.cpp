@@ -232,6 +232,51 @@ int pa_seq_truncate(pa_alloc_t* a, const int64_t* seq_ids, const int64_t* new_le
   return PA_OK;
 }
 
+int pa_seqs_move(pa_alloc_t* from, pa_alloc_t* to, const int64_t* seq_ids, int n,
+                 int32_t* pairs_out, int64_t cap, int64_t* num_pairs) {
+  if (!from || !to || from == to || n < 0 || !num_pairs || (n > 0 && !seq_ids))
+    return PA_ERR_INVALID_ARG;
+  if (from->block_size != to->block_size) return PA_ERR_INVALID_ARG;
+  std::unordered_map<int64_t, int> seen;
+  for (int i = 0; i < n; ++i) {
+    if (seen[seq_ids[i]]++) return PA_ERR_INVALID_ARG;  // ids must be distinct
+    if (!from->seqs.count(seq_ids[i])) return PA_ERR_UNKNOWN_SEQ;
+    if (to->seqs.count(seq_ids[i])) return PA_ERR_SEQ_EXISTS;
+  }
+  // distinct blocks of the moved set, in order of first appearance
+  std::vector<int32_t> distinct;
+  std::unordered_map<int32_t, int32_t> index;
+  for (int i = 0; i < n; ++i)
+    for (int32_t b : from->seqs.find(seq_ids[i])->second.blocks)
+      if (index.emplace(b, static_cast<int32_t>(distinct.size())).second) distinct.push_back(b);
+  const int64_t nd = static_cast<int64_t>(distinct.size());
+  if (nd > 0 && (!pairs_out || cap < nd)) return PA_ERR_INVALID_ARG;
+  if (nd > static_cast<int64_t>(to->free_stack.size())) return PA_ERR_NO_FREE_BLOCKS;
+  std::vector<int32_t> fresh(distinct.size());
+  for (size_t k = 0; k < distinct.size(); ++k) {
+    fresh[k] = to->pop();
+    to->ref[fresh[k]] = 0;  // counted below, one per table entry
+    pairs_out[2 * k] = distinct[k];
+    pairs_out[2 * k + 1] = fresh[k];
+  }
+  for (int i = 0; i < n; ++i) {
+    auto it = from->seqs.find(seq_ids[i]);
+    Seq moved;
+    moved.len = it->second.len;
+    moved.blocks.reserve(it->second.blocks.size() + 1);
+    for (int32_t b : it->second.blocks) {
+      const int32_t nb = fresh[static_cast<size_t>(index[b])];
+      moved.blocks.push_back(nb);
+      to->inc(nb);
+      from->dec(b);
+    }
+    from->seqs.erase(it);
+    to->seqs.emplace(seq_ids[i], std::move(moved));
+  }
+  *num_pairs = nd;
+  return PA_OK;
+}
+
 int pa_seq_free(pa_alloc_t* a, int64_t seq_id) {
   if (!a) return PA_ERR_INVALID_ARG;
   auto it = a->seqs.find(seq_id);

@@ -46,28 +46,28 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
 }
 
 // grid: x = chunk of the block, y = pair, z = 0 (K) / 1 (V).  Each CTA copies
-// kPerThread*256 vectors of one block of one tensor.
+// kCopyPerThread*256 vectors of one block of one tensor from the source cache to the
+// destination cache (the same cache for copy-on-write; a device and a host-resident
+// cache for swapping).
 constexpr int kCopyPerThread = 4;
-__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ k_cache,
-                                                          uint4* __restrict__ v_cache,
-                                                          const int32_t* __restrict__ mapping,
-                                                          int64_t vecs_per_block,
-                                                          int64_t num_blocks, uint32_t* err) {
+__global__ void __launch_bounds__(256) copy_blocks_kernel(
+    uint4* __restrict__ dst_k, uint4* __restrict__ dst_v, const uint4* __restrict__ src_k,
+    const uint4* __restrict__ src_v, const int32_t* __restrict__ mapping, int64_t vecs_per_block,
+    int64_t src_blocks, int64_t dst_blocks, uint32_t* err) {
   const int32_t src = __ldg(mapping + 2 * blockIdx.y);
   const int32_t dst = __ldg(mapping + 2 * blockIdx.y + 1);
-  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+  if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) set_error(err, PA_DEVERR_COPY_BLOCK);
     return;
   }
-  uint4* base = blockIdx.z ? v_cache : k_cache;
-  const uint4* s = base + static_cast<int64_t>(src) * vecs_per_block;
-  uint4* d = base + static_cast<int64_t>(dst) * vecs_per_block;
+  const uint4* s = (blockIdx.z ? src_v : src_k) + static_cast<int64_t>(src) * vecs_per_block;
+  uint4* d = (blockIdx.z ? dst_v : dst_k) + static_cast<int64_t>(dst) * vecs_per_block;
   const int64_t first = static_cast<int64_t>(blockIdx.x) * (256 * kCopyPerThread) + threadIdx.x;
   uint4 tmp[kCopyPerThread];
 #pragma unroll
   for (int u = 0; u < kCopyPerThread; ++u) {
     const int64_t i = first + u * 256;
-    if (i < vecs_per_block) tmp[u] = __ldg(s + i);
+    if (i < vecs_per_block) tmp[u] = s[i];
   }
 #pragma unroll
   for (int u = 0; u < kCopyPerThread; ++u) {
@@ -86,6 +86,64 @@ int elem_bytes(int dtype) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The address a kernel on the current device may use for p: device memory of this
+// device, or page-locked host memory (reachable through unified addressing).  Returns
+// nullptr for anything else (pageable host memory, another device's memory).
+const void* device_view(const void* p) {
+  if (!p) return nullptr;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the non-sticky error
+    return nullptr;
+  }
+  if ((at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) && at.device == dev)
+    return at.devicePointer ? at.devicePointer : p;
+  if (at.type == cudaMemoryTypeHost && at.devicePointer) return at.devicePointer;
+  return nullptr;
+}
+
+// Host-side check of a (src, dst) pair list: ids in range, destinations distinct, and
+// (same_cache) no destination that is also a source.
+bool pairs_ok(const int32_t* pairs, int n, int64_t src_blocks, int64_t dst_blocks,
+              bool same_cache) {
+  std::vector<int32_t> dsts(n), srcs(n);
+  for (int i = 0; i < n; ++i) {
+    srcs[i] = pairs[2 * i];
+    dsts[i] = pairs[2 * i + 1];
+    if (srcs[i] < 0 || srcs[i] >= src_blocks || dsts[i] < 0 || dsts[i] >= dst_blocks) return false;
+  }
+  std::sort(dsts.begin(), dsts.end());
+  if (std::adjacent_find(dsts.begin(), dsts.end()) != dsts.end()) return false;
+  if (same_cache) {
+    std::sort(srcs.begin(), srcs.end());
+    for (int32_t d : dsts)
+      if (std::binary_search(srcs.begin(), srcs.end(), d)) return false;
+  }
+  return true;
+}
+
+int launch_copy(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                const int32_t* mapping, int num_pairs, int64_t block_bytes, int64_t src_blocks,
+                int64_t dst_blocks, cudaStream_t stream) {
+  const int64_t vecs = block_bytes / 16;
+  const int64_t chunks = (vecs + 256 * kCopyPerThread - 1) / (256 * kCopyPerThread);
+  if (chunks > 0x7fffffff) return PA_ERR_INVALID_ARG;
+  uint32_t* err = device_error_word();
+  if (!err) {
+    note_cuda_error(cudaGetLastError());
+    return PA_ERR_CUDA;
+  }
+  dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(num_pairs), 2);
+  copy_blocks_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), static_cast<const uint4*>(src_k),
+      static_cast<const uint4*>(src_v), mapping, vecs, src_blocks, dst_blocks, err);
+  const cudaError_t e = cudaGetLastError();
+  note_cuda_error(e);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
 
 int sm_count() {
   int dev = 0, n = 148;
@@ -143,36 +201,37 @@ extern "C" int pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block
   if (num_pairs == 0) return PA_OK;
   if (!k_cache || !v_cache || !block_mapping_dev) return PA_ERR_INVALID_ARG;
   if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
-  if (block_mapping_host) {
-    // every id in range; destinations distinct and never a source
-    for (int i = 0; i < num_pairs; ++i) {
-      const int32_t s = block_mapping_host[2 * i], d = block_mapping_host[2 * i + 1];
-      if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) return PA_ERR_INVALID_ARG;
-    }
-    std::vector<int32_t> dsts(num_pairs), srcs(num_pairs);
-    for (int i = 0; i < num_pairs; ++i) {
-      srcs[i] = block_mapping_host[2 * i];
-      dsts[i] = block_mapping_host[2 * i + 1];
-    }
-    std::sort(dsts.begin(), dsts.end());
-    std::sort(srcs.begin(), srcs.end());
-    if (std::adjacent_find(dsts.begin(), dsts.end()) != dsts.end()) return PA_ERR_INVALID_ARG;
-    for (int32_t d : dsts)
-      if (std::binary_search(srcs.begin(), srcs.end(), d)) return PA_ERR_INVALID_ARG;
-  }
-  const int64_t vecs = block_bytes / 16;
-  const int64_t chunks = (vecs + 256 * kCopyPerThread - 1) / (256 * kCopyPerThread);
-  if (chunks > 0x7fffffff) return PA_ERR_INVALID_ARG;
-  uint32_t* err = device_error_word();
-  if (!err) {
-    note_cuda_error(cudaGetLastError());
-    return PA_ERR_CUDA;
-  }
-  dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(num_pairs), 2);
-  copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping_dev, vecs,
-      num_blocks, err);
-  const cudaError_t e = cudaGetLastError();
-  note_cuda_error(e);
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  if (block_mapping_host && !pairs_ok(block_mapping_host, num_pairs, num_blocks, num_blocks, true))
+    return PA_ERR_INVALID_ARG;
+  return launch_copy(k_cache, v_cache, k_cache, v_cache, block_mapping_dev, num_pairs, block_bytes,
+                     num_blocks, num_blocks, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int pa_swap_blocks(void* dst_k, void* dst_v, int64_t dst_num_blocks,
+                              const void* src_k, const void* src_v, int64_t src_num_blocks,
+                              const int32_t* block_mapping, const int32_t* block_mapping_host,
+                              int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                              int dtype, pa_stream_t stream) {
+  const int eb = elem_bytes(dtype);
+  if (eb == 0 || num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      dst_num_blocks <= 0 || src_num_blocks <= 0 || num_pairs > 65535)
+    return PA_ERR_INVALID_ARG;
+  const int64_t block_bytes = static_cast<int64_t>(num_kv_heads) * block_size * head_dim * eb;
+  if (block_bytes % 16 != 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!aligned16(dst_k) || !aligned16(dst_v) || !aligned16(src_k) || !aligned16(src_v))
+    return PA_ERR_INVALID_ARG;
+  // every pointer the kernel dereferences must be reachable from this device
+  const void* dk = device_view(dst_k);
+  const void* dv = device_view(dst_v);
+  const void* sk = device_view(src_k);
+  const void* sv = device_view(src_v);
+  const void* mp = device_view(block_mapping);
+  if (!dk || !dv || !sk || !sv || !mp) return PA_ERR_INVALID_ARG;
+  if (block_mapping_host &&
+      !pairs_ok(block_mapping_host, num_pairs, src_num_blocks, dst_num_blocks, false))
+    return PA_ERR_INVALID_ARG;
+  return launch_copy(const_cast<void*>(dk), const_cast<void*>(dv), sk, sv,
+                     static_cast<const int32_t*>(mp), num_pairs, block_bytes, src_num_blocks,
+                     dst_num_blocks, static_cast<cudaStream_t>(stream));
 }

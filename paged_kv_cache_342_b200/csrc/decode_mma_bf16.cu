@@ -8,9 +8,12 @@ namespace {
 
 template <int D, int BS, int NT, bool GROUP>
 cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  // about 64 KiB of stages per CTA: warps with two stages each (1-4), then 2-4 stages
   constexpr int kStage = 2 * BS * D * 2;
-  constexpr int NW = kStage <= 16384 ? 4 : (kStage <= 32768 ? 2 : 1);
-  constexpr int kRaw = 65536 / (NW * kStage);
+  constexpr int kBudget = 65536;
+  constexpr int kW = kBudget / (2 * kStage);
+  constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
+  constexpr int kRaw = kBudget / (NW * kStage);
   constexpr int NST = kRaw < 2 ? 2 : (kRaw > 4 ? 4 : kRaw);
   using C = MmaCfg<__nv_bfloat16, D, BS, NT, NW, NST>;
   const uint64_t rows = static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * BS;

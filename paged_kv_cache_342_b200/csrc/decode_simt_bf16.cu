@@ -5,13 +5,15 @@
 namespace pa {
 namespace {
 
-// Stage = one block's K and V runs.  Up to 4 warps; 2-4 stages per warp sized so
-// a CTA holds about 64 KiB of stages (three CTAs per SM at head_dim 128, block 16).
+// Stage = one block's K and V runs.  About 64 KiB of stages per CTA (three CTAs per
+// SM): as many warps as fit with two stages each (1-4), then 2-4 stages per warp.
 template <int D, int BS, int GS>
 cudaError_t launch_auto(const DecodeParams& p, cudaStream_t st) {
   constexpr int kStage = 2 * BS * D * static_cast<int>(sizeof(__nv_bfloat16));
-  constexpr int NW = kStage <= 16384 ? 4 : (kStage <= 32768 ? 2 : 1);
-  constexpr int kRaw = 65536 / (NW * kStage);
+  constexpr int kBudget = 65536;
+  constexpr int kW = kBudget / (2 * kStage);
+  constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
+  constexpr int kRaw = kBudget / (NW * kStage);
   constexpr int NST = kRaw < 2 ? 2 : (kRaw > 4 ? 4 : kRaw);
   return launch_simt<__nv_bfloat16, D, BS, GS, NW, NST>(p, st);
 }

@@ -233,3 +233,123 @@ def test_prefix_groups_of_the_shared_prefix_workload(pa):
     chunks = _compare_groups(c, o, list(range(cfg.num_seqs)), 512, 8)
     # 1030-token prefix = 64 full blocks shared by all 8 samples -> 2 partitions of 512
     assert len(chunks) == 32 and all(len(m) == 8 and parts == 2 for m, parts in chunks)
+
+
+# ---------------------------------------------------------------------------
+# moving sequences between pools (swap out to a host pool and back)
+# ---------------------------------------------------------------------------
+
+def _pools(pa, nb_dev, nb_host, bs, seed):
+    g = np.random.default_rng(seed)
+    od, oh = g.permutation(nb_dev), g.permutation(nb_host)
+    return (pa.BlockAllocator(nb_dev, bs, od), pa.BlockAllocator(nb_host, bs, oh),
+            BlockManager(nb_dev, bs, od), BlockManager(nb_host, bs, oh))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_moves_between_two_pools(pa, seed):
+    g = np.random.default_rng(200 + seed)
+    bs = int(g.choice([2, 4, 16]))
+    cd, ch, od, oh = _pools(pa, 64, 48, bs, seed)
+    where = {}          # seq -> "d" or "h"
+    nid = 0
+    for step in range(250):
+        r = int(g.integers(0, 10))
+        on_dev = [s for s, w in where.items() if w == "d"]
+        on_host = [s for s, w in where.items() if w == "h"]
+        try_ops = []
+        if r < 2 or not on_dev:
+            n = int(g.integers(0, 4 * bs))
+            e1 = e2 = None
+            try:
+                cd.add(nid, n)
+            except pa.PagedAttentionError as e:
+                e1 = e.code
+            try:
+                od.add(nid, n)
+            except AllocError as e:
+                e2 = e.code
+            assert e1 == e2
+            if e1 is None:
+                where[nid] = "d"
+            nid += 1
+        elif r < 4:
+            p = on_dev[int(g.integers(0, len(on_dev)))]
+            cd.fork(p, nid), od.fork(p, nid)
+            where[nid] = "d"
+            nid += 1
+        elif r < 6:
+            s = on_dev[int(g.integers(0, len(on_dev)))]
+            rc, ro = run_both(pa, cd, od, "append_slot", s)
+            assert rc == ro
+        elif r < 8:          # swap out a random subset of the device sequences
+            k = int(g.integers(1, min(4, len(on_dev)) + 1))
+            ids = [int(x) for x in g.choice(on_dev, k, replace=False)]
+            err_c = err_o = None
+            try:
+                pc = cd.move_to(ch, ids)
+            except pa.PagedAttentionError as e:
+                err_c = e.code
+            try:
+                po = od.move_to(oh, ids)
+            except AllocError as e:
+                err_o = e.code
+            assert err_c == err_o
+            if err_c is None:
+                assert [tuple(x) for x in pc.tolist()] == po
+                for s in ids:
+                    where[s] = "h"
+        elif on_host:        # swap back in
+            k = int(g.integers(1, min(3, len(on_host)) + 1))
+            ids = [int(x) for x in g.choice(on_host, k, replace=False)]
+            err_c = err_o = None
+            try:
+                pc = ch.move_to(cd, ids)
+            except pa.PagedAttentionError as e:
+                err_c = e.code
+            try:
+                po = oh.move_to(od, ids)
+            except AllocError as e:
+                err_o = e.code
+            assert err_c == err_o
+            if err_c is None:
+                assert [tuple(x) for x in pc.tolist()] == po
+                for s in ids:
+                    where[s] = "d"
+        same_state(cd, od)
+        same_state(ch, oh)
+
+
+def test_move_keeps_sharing_inside_the_moved_set(pa):
+    cd, ch, od, oh = _pools(pa, 16, 16, 4, 0)
+    for m in (cd, od):
+        m.add(0, 10)          # 3 blocks
+        m.fork(0, 1)
+        m.fork(0, 2)
+    pc = cd.move_to(ch, [0, 1])       # seq 2 stays: shared blocks copied once
+    po = od.move_to(oh, [0, 1])
+    assert [tuple(x) for x in pc.tolist()] == po and len(po) == 3
+    assert ch.seq_blocks(0) == ch.seq_blocks(1)
+    assert all(ch.refcount(b) == 2 for b in ch.seq_blocks(0))
+    assert all(cd.refcount(b) == 1 for b in cd.seq_blocks(2))
+    same_state(cd, od)
+    same_state(ch, oh)
+
+
+def test_full_pool_swap_out_lets_the_batch_continue(pa):
+    """Preemption on the host: the pool runs dry mid-step, the latest sequence is
+    swapped out to the host pool, and the step goes through for the others."""
+    dev, host = pa.BlockAllocator(6, 4), pa.BlockAllocator(8, 4)
+    for s in range(3):
+        dev.add(s, 8)                 # 2 full blocks each: pool empty
+    with pytest.raises(pa.PagedAttentionError) as e:
+        dev.append_slots([0, 1, 2])   # each needs a new block
+    assert e.value.code == "NO_FREE_BLOCKS"
+    assert dev.stats()["free_blocks"] == 0 and dev.seq_len(0) == 8   # unchanged
+    pairs = dev.move_to(host, [2])   # preempt the latest sequence
+    assert len(pairs) == 2 and dev.stats()["free_blocks"] == 2
+    slots, _ = dev.append_slots([0, 1])
+    assert len(slots) == 2 and host.seq_len(2) == 8
+    dev.free(0)                      # a sequence finishes: room to swap back in
+    back = host.move_to(dev, [2])
+    assert len(back) == 2 and dev.seq_len(2) == 8 and host.stats()["num_seqs"] == 0
