@@ -54,6 +54,8 @@ def parse():
     # the pages' block-size trade-off: same lengths and slot capacity, other block size
     ap.add_argument("--block-size", type=int, default=None,
                     help="override the block size (pool keeps the same number of slots)")
+    ap.add_argument("--cache-fp8", action="store_true",
+                    help="store K/V as fp8 e4m3 with per-tensor scales (q/out keep the dtype)")
     return ap.parse_args()
 
 
@@ -61,21 +63,25 @@ def parse():
 # algorithmic bytes (what one step must move at least once)
 # ---------------------------------------------------------------------------
 
-def decode_bytes(cfg, lens, unique_tokens=None) -> int:
+def decode_bytes(cfg, lens, unique_tokens=None, kv_elem_bytes=None) -> int:
     """K/V of every cached token once + q + out + block-table entries + lengths.
-    ``unique_tokens`` (shared-prefix workloads) counts each physical slot once."""
+    ``unique_tokens`` (shared-prefix workloads) counts each physical slot once;
+    ``kv_elem_bytes`` is the cache element size when it differs from q's (fp8)."""
     E = cfg.elem_bytes
+    EKV = E if kv_elem_bytes is None else kv_elem_bytes
     tokens = int(np.sum(lens)) if unique_tokens is None else int(unique_tokens)
-    kv = tokens * cfg.num_kv_heads * cfg.head_dim * 2 * E
+    kv = tokens * cfg.num_kv_heads * cfg.head_dim * 2 * EKV
     qo = 2 * cfg.num_seqs * cfg.num_heads * cfg.head_dim * E
     tab = int(np.sum((np.asarray(lens) + cfg.block_size - 1) // cfg.block_size)) * 4
     return kv + qo + tab + 4 * cfg.num_seqs
 
 
-def cache_op_bytes(cfg, num_tokens, num_pairs) -> int:
+def cache_op_bytes(cfg, num_tokens, num_pairs, kv_elem_bytes=None) -> int:
     E = cfg.elem_bytes
-    row = cfg.num_kv_heads * cfg.head_dim * E
-    reshape = 2 * (2 * num_tokens * row) + 8 * num_tokens       # K and V: read + write
+    EKV = E if kv_elem_bytes is None else kv_elem_bytes
+    row_in = cfg.num_kv_heads * cfg.head_dim * E
+    row = cfg.num_kv_heads * cfg.head_dim * EKV
+    reshape = 2 * num_tokens * (row_in + row) + 8 * num_tokens  # K and V: read + write
     copy = 2 * 2 * num_pairs * cfg.block_size * row              # K and V blocks: read + write
     return reshape + copy
 
@@ -315,9 +321,24 @@ def run_ours(args, cfg):
     max_blocks = (max_len + bs - 1) // bs
     kd = storage_to_torch(inp.k_pool, cfg.dtype).to(dev)
     vd = storage_to_torch(inp.v_pool, cfg.dtype).to(dev)
+    kv_scales, ekv = None, None
+    if args.cache_fp8:
+        # quantize the pool on the device with the library's fp8 write (all slots)
+        kv_scales, ekv = (8.0 * cfg.std / 448.0,) * 2, 1
+        NB = cfg.num_blocks
+        slots_all = torch.arange(NB * bs, dtype=torch.int64, device=dev)
+        k8 = torch.empty(kd.shape, dtype=torch.uint8, device=dev)
+        v8 = torch.empty_like(k8)
+        for src, dst in ((kd, k8), (vd, v8)):
+            rows = src.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous()
+            pa.pa_reshape_and_cache_fp8(rows, rows, dst, dst, slots_all, *kv_scales)
+            del rows
+        kd, vd = k8, v8
+        torch.cuda.synchronize(dev)
     pool_bytes = 2 * kd.numel() * kd.element_size()
     del inp.k_pool, inp.v_pool
-    dec = PagedDecoder(kd, vd, Hq, cfg.scale, max_blocks, inp.free_order, cfg.partition_size)
+    dec = PagedDecoder(kd, vd, Hq, cfg.scale, max_blocks, inp.free_order, cfg.partition_size,
+                       kv_scales=kv_scales)
     if inp.prefix is None:
         for s in range(S):
             dec.admit(s, int(inp.context_lens[s]))
@@ -357,9 +378,9 @@ def run_ours(args, cfg):
     torch.cuda.synchronize(dev)
     lens = np.array([dec.alloc.seq_len(s) for s in range(S)], np.int64)
     uniq = unique_context_tokens(dec, cfg, range(S)) if inp.prefix is not None else None
-    dec_bytes = decode_bytes(cfg, lens, uniq)
-    step_bytes = dec_bytes + cache_op_bytes(cfg, S, 0)
-    logical_dec_bytes = decode_bytes(cfg, lens)
+    dec_bytes = decode_bytes(cfg, lens, uniq, ekv)
+    step_bytes = dec_bytes + cache_op_bytes(cfg, S, 0, ekv)
+    logical_dec_bytes = decode_bytes(cfg, lens, None, ekv)
     launches_per_step = dec.kernel_launches(meta0)
 
     # per-call events on a sample of the steps (the decode call's own duration)
@@ -430,7 +451,8 @@ def run_ours(args, cfg):
     achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-            "kernel": "pa_decode_attention (partition kernel + log-sum-exp merge)",
+            "kernel": ("pa_decode_attention_fp8" if args.cache_fp8 else "pa_decode_attention")
+                      + " (partition kernel + log-sum-exp merge)",
             "bytes_per_launch": int(dec_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 2),
             "launches_timed": len(dec_ms),
             "frac_of_nominal_8000": round(achieved / 8000.0, 4),
@@ -460,7 +482,9 @@ def run_ours(args, cfg):
                        "workspace_bytes": int(dec._ws.numel()),
                        "prefix_group_chunks": int(meta0.get("num_chunks", 0)),
                        "pool": pool_summary(dec.alloc.stats()),
-                       "cow_pairs_in_warmup": warm_cow, "cow_pairs_in_timed_steps": cows},
+                       "cow_pairs_in_warmup": warm_cow, "cow_pairs_in_timed_steps": cows,
+                       "kv_cache": ("fp8 e4m3, per-tensor scales %g" % kv_scales[0])
+                                   if args.cache_fp8 else cfg.dtype},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -25,7 +25,8 @@
  *   - GPU work is enqueued on the caller's stream (a cudaStream_t passed as
  *     pa_stream_t; NULL = legacy default stream) and is asynchronous: no entry
  *     point synchronises, except pa_device_error_read.
- *   - Element types: PA_F32, PA_BF16, PA_F16.  q, out and both caches share one.
+ *   - Element types: PA_F32, PA_BF16, PA_F16.  q, out and both caches share one,
+ *     except in the _fp8 entry points, whose caches hold PA_FP8_E4M3 codes.
  *   - Cache layout (K and V alike): [num_blocks, num_kv_heads, block_size, head_dim];
  *     so each (block, kv head) pair is one contiguous block_size*head_dim run.
  *     Slot s means block s / block_size, offset s % block_size.
@@ -56,7 +57,7 @@ typedef enum {
   PA_ERR_TOO_LARGE = 8       /* request exceeds a fixed built-in capacity           */
 } pa_status;
 
-typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2, PA_FP8_E4M3 = 3 } pa_dtype;
 
 typedef void* pa_stream_t; /* a cudaStream_t */
 
@@ -89,6 +90,20 @@ int pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void
                          const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
                          int head_dim, int block_size, int64_t num_blocks, int dtype,
                          pa_stream_t stream);
+
+/*
+ * pa_reshape_and_cache_fp8 - pa_reshape_and_cache into an fp8 (e4m3) cache ([BLOG]
+ * "Where it bites": a quantized cache stacks with paging; the pages give no format,
+ * so the reading here is one float32 scale per cache tensor).  key/value are
+ * input_dtype (PA_F32, PA_BF16, PA_F16) [num_tokens, num_kv_heads, head_dim]; each
+ * element x is stored as e4m3(float32(x) * (1.0f / scale)), rounded to nearest even,
+ * saturated to +-448.  head_dim must be a multiple of 16.  Slots as in
+ * pa_reshape_and_cache.  Scales must be positive and finite.
+ */
+int pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                             int head_dim, int block_size, int64_t num_blocks, int input_dtype,
+                             float k_scale, float v_scale, pa_stream_t stream);
 
 /*
  * pa_copy_blocks - make the private copies of copy-on-write.
@@ -222,6 +237,20 @@ int pa_decode_uses_tensor_cores(int dtype, int num_heads, int num_kv_heads, int 
                                 int block_size);
 
 /*
+ * pa_decode_attention_fp8 - pa_decode_attention over an fp8 (e4m3) cache written by
+ * pa_reshape_and_cache_fp8: K_t = e4m3(k codes) * k_scale, V_t = e4m3(v codes) *
+ * v_scale.  q and out are dtype (PA_BF16 or PA_F16); head_dim 128 or 256; CUDA-core
+ * kernel for every group size.  The cache is half the bytes of a 16-bit one.
+ */
+int pa_decode_attention_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* seq_lens, float scale,
+                            int block_size, int num_kv_heads, int num_seqs, int num_heads,
+                            int head_dim, int max_blocks_per_seq, int64_t num_blocks,
+                            int max_seq_len, int partition_size, int dtype, float k_scale,
+                            float v_scale, void* workspace, size_t workspace_bytes,
+                            pa_stream_t stream);
+
+/*
  * pa_decode_attention_grouped - pa_decode_attention for a batch in which groups of
  * sequences share their leading blocks (prompt sharing / parallel samples forked
  * from one prefix: [GLOSS] prompt sharing and sampling algorithms; [BLOG] "The bonus
@@ -302,6 +331,10 @@ typedef struct {
   int64_t tail_waste_slots;  /* sum over sequences of blocks*block_size - length */
   int64_t cow_copies;        /* copy-on-write pairs issued so far                */
   int64_t blocks_allocated;  /* blocks taken from the pool so far                */
+  int64_t cached_blocks;     /* blocks registered in the prefix cache            */
+  int64_t evictable_blocks;  /* cached blocks nobody references (reusable)       */
+  int64_t cache_hits;        /* prompt blocks served from the prefix cache       */
+  int64_t cache_evictions;   /* cached blocks evicted to serve a pop             */
 } pa_stats_t;
 
 /* Create a pool; free_order (host int32 [num_blocks], a permutation) or NULL. */
@@ -311,6 +344,17 @@ int pa_alloc_destroy(pa_alloc_t* a);
 
 /* Admit seq_id with num_tokens cached tokens: ceil(num_tokens/block_size) blocks. */
 int pa_seq_add(pa_alloc_t* a, int64_t seq_id, int64_t num_tokens);
+/* Admit seq_id by its prompt's n token ids with automatic prefix caching: every
+ * leading full block whose tokens - and whole prefix - match a cached block reuses
+ * that block (count + 1); the remaining full blocks are fresh and registered in the
+ * cache (the caller must write their K/V before anyone attends over them); a partial
+ * last block is fresh and not registered.  *cached_tokens = tokens covered by reused
+ * blocks (their K/V need not be computed again).  A cached block that nobody
+ * references stays cached but evictable: pops take a free block first, else evict
+ * the least recently released cached block.  A write into a cached block copies it
+ * when shared and uncaches it otherwise. */
+int pa_seq_add_prompt(pa_alloc_t* a, int64_t seq_id, const int32_t* token_ids, int64_t n,
+                      int64_t* cached_tokens);
 /* child shares all of parent's blocks and its length. */
 int pa_seq_fork(pa_alloc_t* a, int64_t parent, int64_t child);
 /* Room for one more token of seq_id: *slot receives its slot; *cow_src/*cow_dst the

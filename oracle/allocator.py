@@ -27,6 +27,23 @@ Readings where the pages are silent (the C-ABI allocator follows the same ones):
     the writer gets a fresh block, the shared block's count drops by one;
   * a failing call leaves the state unchanged; a batch of appends is all or nothing;
   * block-table rows are padded with -1.
+
+Automatic prefix caching ([BLOG] "The bonus contiguous storage can't give you:
+sharing": prefix caching is built on top of copy-on-write; the mechanism is not
+given, so this is the reading taken):
+  * a prompt admitted with its token ids reuses a cached block for every leading
+    full block whose tokens - and whose whole prefix - match an earlier prompt's;
+  * the cache key of a full block is (cache id of the previous block, its tokens);
+    a block registered in the cache gets a fresh cache id, so a key can only match
+    when the entire prefix matches (no hashing, no collisions);
+  * the first block that misses, and every block after it, is a fresh block that is
+    registered (the caller writes its K/V before anyone attends over it); the last
+    partial block is fresh and not registered;
+  * a cached block whose count drops to zero becomes evictable (least recently
+    released first) instead of free; a pop takes a free block if there is one, else
+    evicts the least recently released cached block;
+  * a cached block's content is immutable: a write into it (an append after the
+    sequence was truncated into it) copies it when shared and uncaches it when not.
 """
 from __future__ import annotations
 
@@ -60,13 +77,39 @@ class BlockManager:
         self.lens: dict[int, int] = {}
         self.cow_copies = 0
         self.blocks_allocated = 0
+        # prefix cache
+        self.evictable: list[int] = []        # least recently released first
+        self.cache: dict = {}                 # (parent cache id, tokens) -> block
+        self.cache_of: dict = {}              # block -> (key, cache id)
+        self.next_cache_id = 1
+        self.cache_hits = 0
+        self.cache_evictions = 0
 
     # -- helpers -------------------------------------------------------------
+    def _available(self) -> int:
+        return len(self.free) + len(self.evictable)
+
     def _pop(self) -> int:
-        b = self.free.pop()
+        if self.free:
+            b = self.free.pop()
+        else:
+            b = self.evictable.pop(0)
+            key, _ = self.cache_of.pop(b)
+            del self.cache[key]
+            self.cache_evictions += 1
         self.ref[b] = 1
         self.blocks_allocated += 1
         return b
+
+    def _release(self, b: int) -> None:
+        """One reference to b goes away."""
+        self.ref[b] -= 1
+        if self.ref[b] == 0:
+            (self.evictable if b in self.cache_of else self.free).append(b)
+
+    def _uncache(self, b: int) -> None:
+        key, _ = self.cache_of.pop(b)
+        del self.cache[key]
 
     def _blocks_for(self, n_tokens: int) -> int:
         return (n_tokens + self.block_size - 1) // self.block_size
@@ -79,10 +122,55 @@ class BlockManager:
         if n_tokens < 0:
             raise AllocError(INVALID_ARG, "negative length")
         need = self._blocks_for(n_tokens)
-        if need > len(self.free):
-            raise AllocError(NO_FREE_BLOCKS, f"need {need}, have {len(self.free)}")
+        if need > self._available():
+            raise AllocError(NO_FREE_BLOCKS, f"need {need}, have {self._available()}")
         self.tables[seq_id] = [self._pop() for _ in range(need)]
         self.lens[seq_id] = n_tokens
+
+    def add_prompt(self, seq_id: int, tokens) -> int:
+        """Admit a sequence by its prompt token ids, reusing cached full blocks.
+        Returns the number of leading tokens whose blocks came from the cache."""
+        if seq_id in self.tables:
+            raise AllocError(SEQ_EXISTS, str(seq_id))
+        tokens = [int(t) for t in tokens]
+        bs = self.block_size
+        full = len(tokens) // bs
+        keys, hits, parent = [], [], 0
+        for j in range(full):
+            key = (parent, tuple(tokens[j * bs:(j + 1) * bs]))
+            keys.append(key)
+            if parent is not None and key in self.cache:
+                b = self.cache[key]
+                hits.append(b)
+                parent = self.cache_of[b][1]
+            else:
+                parent = None             # the chain is broken: no later block can match
+        fresh = len(keys) - len(hits) + (1 if len(tokens) % bs else 0)
+        claimable = sum(1 for b in hits if self.ref[b] == 0)
+        if fresh > self._available() - claimable:
+            raise AllocError(NO_FREE_BLOCKS, f"need {fresh}")
+        table = []
+        for b in hits:                    # claim the cached blocks first
+            if self.ref[b] == 0:
+                self.evictable.remove(b)
+            self.ref[b] += 1
+            table.append(b)
+        self.cache_hits += len(hits)
+        parent = self.cache_of[hits[-1]][1] if hits else 0
+        for key in keys[len(hits):]:      # then fresh, registered blocks
+            b = self._pop()
+            key = (parent, key[1])
+            cid = self.next_cache_id
+            self.next_cache_id += 1
+            self.cache[key] = b
+            self.cache_of[b] = (key, cid)
+            parent = cid
+            table.append(b)
+        if len(tokens) % bs:
+            table.append(self._pop())     # the partial last block is never cached
+        self.tables[seq_id] = table
+        self.lens[seq_id] = len(tokens)
+        return len(hits) * bs
 
     def fork(self, parent: int, child: int) -> None:
         """child shares every block of parent (each count + 1)."""
@@ -103,17 +191,19 @@ class BlockManager:
         off = n % self.block_size
         src = dst = -1
         if off == 0:
-            if not self.free:
+            if not self._available():
                 raise AllocError(NO_FREE_BLOCKS, "append")
             table.append(self._pop())
         elif self.ref[table[-1]] > 1:
-            if not self.free:
+            if not self._available():
                 raise AllocError(NO_FREE_BLOCKS, "copy-on-write")
             src = table[-1]
             dst = self._pop()
-            self.ref[src] -= 1
+            self._release(src)
             table[-1] = dst
             self.cow_copies += 1
+        elif table[-1] in self.cache_of:
+            self._uncache(table[-1])     # sole owner writes into a cached block
         self.lens[seq_id] = n + 1
         return table[-1] * self.block_size + off, src, dst
 
@@ -143,9 +233,7 @@ class BlockManager:
             keep = self._blocks_for(n)
             table = self.tables[s]
             for b in table[keep:]:
-                self.ref[b] -= 1
-                if self.ref[b] == 0:
-                    self.free.append(b)
+                self._release(b)
             del table[keep:]
             self.lens[s] = n
 
@@ -175,8 +263,8 @@ class BlockManager:
             for b in self.tables[s]:
                 if b not in distinct:
                     distinct.append(b)
-        if len(distinct) > len(other.free):
-            raise AllocError(NO_FREE_BLOCKS, f"need {len(distinct)}, have {len(other.free)}")
+        if len(distinct) > other._available():
+            raise AllocError(NO_FREE_BLOCKS, f"need {len(distinct)}, have {other._available()}")
         mapping = {b: other._pop() for b in distinct}
         for nb in mapping.values():
             other.ref[nb] = 0                # counted below, one per table entry
@@ -186,18 +274,14 @@ class BlockManager:
             other.lens[s] = self.lens.pop(s)
             for b in table:
                 other.ref[mapping[b]] += 1
-                self.ref[b] -= 1
-                if self.ref[b] == 0:
-                    self.free.append(b)
+                self._release(b)
         return [(b, mapping[b]) for b in distinct]
 
     def free_seq(self, seq_id: int) -> None:
         if seq_id not in self.tables:
             raise AllocError(UNKNOWN_SEQ, str(seq_id))
         for b in self.tables.pop(seq_id):
-            self.ref[b] -= 1
-            if self.ref[b] == 0:
-                self.free.append(b)
+            self._release(b)
         del self.lens[seq_id]
 
     # -- sharing structure ---------------------------------------------------
@@ -257,11 +341,13 @@ class BlockManager:
 
     def stats(self) -> dict:
         bs = self.block_size
-        used = self.num_blocks - len(self.free)
+        used = self.num_blocks - len(self.free) - len(self.evictable)
         return dict(
             num_blocks=self.num_blocks, block_size=bs, free_blocks=len(self.free),
             used_blocks=used, shared_blocks=sum(1 for r in self.ref if r > 1),
             total_refs=sum(self.ref), num_seqs=len(self.tables),
             logical_tokens=sum(self.lens.values()), allocated_slots=used * bs,
             tail_waste_slots=sum(len(t) * bs - self.lens[s] for s, t in self.tables.items()),
-            cow_copies=self.cow_copies, blocks_allocated=self.blocks_allocated)
+            cow_copies=self.cow_copies, blocks_allocated=self.blocks_allocated,
+            cached_blocks=len(self.cache_of), evictable_blocks=len(self.evictable),
+            cache_hits=self.cache_hits, cache_evictions=self.cache_evictions)

@@ -22,7 +22,7 @@ PA_ERR_TOO_LARGE = 8
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "NO_FREE_BLOCKS", 3: "UNKNOWN_SEQ",
                 4: "SEQ_EXISTS", 5: "BAD_INDEX", 6: "CUDA", 7: "UNSUPPORTED", 8: "TOO_LARGE"}
 PA_STATIC_WORKSPACE_BYTES = 16 << 20
-PA_F32, PA_BF16, PA_F16 = 0, 1, 2
+PA_F32, PA_BF16, PA_F16, PA_FP8_E4M3 = 0, 1, 2, 3
 DEVERR_SLOT, DEVERR_COPY_BLOCK, DEVERR_TABLE, DEVERR_SEQ_LEN, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 DEFAULT_PARTITION = 512
 
@@ -48,7 +48,8 @@ class pa_stats_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "num_blocks", "block_size", "free_blocks", "used_blocks", "shared_blocks",
         "total_refs", "num_seqs", "logical_tokens", "allocated_slots", "tail_waste_slots",
-        "cow_copies", "blocks_allocated")]
+        "cow_copies", "blocks_allocated", "cached_blocks", "evictable_blocks", "cache_hits",
+        "cache_evictions")]
 
 
 def _sig(name, res, *args):
@@ -59,6 +60,10 @@ def _sig(name, res, *args):
 
 _sig("pa_reshape_and_cache", _i32, _p, _p, _p, _p, _p, _i64, _i32, _i32, _i32, _i64, _i32, _p)
 _sig("pa_copy_blocks", _i32, _p, _p, _p, _p, _i32, _i32, _i32, _i32, _i64, _i32, _p)
+_sig("pa_reshape_and_cache_fp8", _i32, _p, _p, _p, _p, _p, _i64, _i32, _i32, _i32, _i64, _i32,
+     _f, _f, _p)
+_sig("pa_decode_attention_fp8", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i64, _i32, _i32, _i32, _f, _f, _p, ctypes.c_size_t, _p)
 _sig("pa_swap_blocks", _i32, _p, _p, _i64, _p, _p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p)
 _sig("pa_decode_workspace_bytes", ctypes.c_size_t, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode_attention", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32, _i32,
@@ -74,6 +79,7 @@ _sig("pa_alloc_create", _i32, _i64, _i32, _p, ctypes.POINTER(_p))
 _sig("pa_alloc_destroy", _i32, _p)
 _sig("pa_seq_add", _i32, _p, _i64, _i64)
 _sig("pa_seq_fork", _i32, _p, _i64, _i64)
+_sig("pa_seq_add_prompt", _i32, _p, _i64, _p, _i64, _I64P)
 _sig("pa_seq_append_slot", _i32, _p, _i64, _I64P, _I32P, _I32P)
 _sig("pa_seq_append_slots", _i32, _p, _p, _i32, _p, _p, ctypes.POINTER(ctypes.c_int))
 _sig("pa_seq_free", _i32, _p, _i64)
@@ -106,7 +112,8 @@ def pa_last_cuda_error() -> str:
 
 def _dtype_code(t) -> int:
     import torch
-    codes = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float16: PA_F16}
+    codes = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float16: PA_F16,
+             torch.uint8: PA_FP8_E4M3, torch.float8_e4m3fn: PA_FP8_E4M3}
     if t.dtype not in codes:
         raise ValueError(f"unsupported dtype {t.dtype}")
     return codes[t.dtype]
@@ -138,6 +145,43 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
         _dev(key, "key"), _dev(value, "value"), _dev(k_cache, "k_cache"),
         _dev(v_cache, "v_cache"), _dev(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D,
         bs, NB, _dtype_code(k_cache), _stream(stream)), "pa_reshape_and_cache")
+
+
+def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                             stream=None) -> None:
+    """key/value [T, Hkv, D] (f32/bf16/f16); caches [NB, Hkv, bs, D] of e4m3 codes
+    (a uint8 or float8_e4m3fn CUDA tensor)."""
+    import torch
+    T, Hkv, D = key.shape
+    NB, _, bs, _ = k_cache.shape
+    if k_cache.element_size() != 1:
+        raise ValueError("fp8 caches hold one byte per element")
+    _check(lib.pa_reshape_and_cache_fp8(
+        _dev(key, "key"), _dev(value, "value"), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache"), _dev(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D,
+        bs, NB, _dtype_code(key), float(k_scale), float(v_scale), _stream(stream)),
+        "pa_reshape_and_cache_fp8")
+
+
+def pa_decode_attention_fp8(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
+                            block_size, num_kv_heads, max_seq_len, k_scale, v_scale,
+                            partition_size=DEFAULT_PARTITION, workspace=None,
+                            stream=None) -> None:
+    """pa_decode_attention over e4m3 caches; q/out bf16 or f16."""
+    import torch
+    S, Hq, D = q.shape
+    NB = k_cache.shape[0]
+    if k_cache.element_size() != 1:
+        raise ValueError("fp8 caches hold one byte per element")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_attention_fp8(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), block_size, num_kv_heads, S, Hq, D, block_tables.shape[1], NB,
+        int(max_seq_len), partition_size, _dtype_code(q), float(k_scale), float(v_scale), ws_ptr,
+        ws_bytes, _stream(stream)), "pa_decode_attention_fp8")
 
 
 def pa_copy_blocks(k_cache, v_cache, block_mapping, block_mapping_host=None, stream=None) -> None:
@@ -297,6 +341,15 @@ class BlockAllocator:
 
     def add(self, seq_id: int, num_tokens: int) -> None:
         _check(lib.pa_seq_add(self._h, seq_id, num_tokens), "pa_seq_add")
+
+    def add_prompt(self, seq_id: int, token_ids) -> int:
+        """Admit a sequence by its prompt tokens with prefix caching; returns the number
+        of leading tokens served by cached blocks."""
+        toks = np.ascontiguousarray(token_ids, dtype=np.int32)
+        cached = ctypes.c_int64(0)
+        _check(lib.pa_seq_add_prompt(self._h, seq_id, toks.ctypes.data, toks.size,
+                                     ctypes.byref(cached)), "pa_seq_add_prompt")
+        return cached.value
 
     def fork(self, parent: int, child: int) -> None:
         _check(lib.pa_seq_fork(self._h, parent, child), "pa_seq_fork")

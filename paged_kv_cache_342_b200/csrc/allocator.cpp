@@ -12,10 +12,21 @@
 // Pool order (not fixed by the pages): a LIFO stack; pops return free_order[0],
 // free_order[1], ...; a released block goes on top; a freed sequence releases its
 // blocks in logical order.  Every failing call leaves the state unchanged.
+//
+// Automatic prefix caching (built on the sharing machinery, as the same blog's
+// sharing section says): full prompt blocks are registered under the exact key
+// (cache id of the previous block, the block's token ids); a released cached block
+// becomes evictable (least recently released first) instead of free; a pop takes a
+// free block first, then evicts; a write into a cached block copies it when shared
+// and uncaches it when not.
 #include <cstdint>
 #include <cstring>
+#include <iterator>
+#include <list>
+#include <map>
 #include <new>
 #include <unordered_map>
+#include <utility>
 #include <vector>
 
 #include "../../include/pa.h"
@@ -30,6 +41,8 @@ struct Seq {
 }  // namespace
 
 struct pa_alloc {
+  using CacheKey = std::pair<int64_t, std::vector<int32_t>>;  // (parent cache id, tokens)
+
   int64_t num_blocks = 0;
   int block_size = 0;
   std::vector<int32_t> free_stack;  // back() is the top
@@ -38,10 +51,33 @@ struct pa_alloc {
   int64_t cow_copies = 0;
   int64_t blocks_allocated = 0;
   int64_t shared_blocks = 0;  // maintained incrementally: count of ref > 1
+  // prefix cache
+  std::list<int32_t> evictable;  // cached blocks with ref 0, least recently released first
+  std::vector<std::list<int32_t>::iterator> evict_pos;
+  std::vector<int64_t> cache_id;  // 0 = not cached
+  std::vector<CacheKey> cache_key;
+  std::map<CacheKey, int32_t> cache;
+  int64_t next_cache_id = 1, cache_hits = 0, cache_evictions = 0;
 
+  int64_t available() const {
+    return static_cast<int64_t>(free_stack.size() + evictable.size());
+  }
+  void uncache(int32_t b) {
+    cache.erase(cache_key[b]);
+    cache_key[b] = CacheKey();
+    cache_id[b] = 0;
+  }
   int32_t pop() {
-    int32_t b = free_stack.back();
-    free_stack.pop_back();
+    int32_t b;
+    if (!free_stack.empty()) {
+      b = free_stack.back();
+      free_stack.pop_back();
+    } else {
+      b = evictable.front();
+      evictable.pop_front();
+      uncache(b);
+      ++cache_evictions;
+    }
     ref[b] = 1;
     ++blocks_allocated;
     return b;
@@ -51,7 +87,14 @@ struct pa_alloc {
   }
   void dec(int32_t b) {
     if (ref[b]-- == 2) --shared_blocks;
-    if (ref[b] == 0) free_stack.push_back(b);
+    if (ref[b] == 0) {
+      if (cache_id[b]) {
+        evictable.push_back(b);
+        evict_pos[b] = std::prev(evictable.end());
+      } else {
+        free_stack.push_back(b);
+      }
+    }
   }
 };
 
@@ -80,6 +123,9 @@ int pa_alloc_create(int64_t num_blocks, int block_size, const int32_t* free_orde
   a->num_blocks = num_blocks;
   a->block_size = block_size;
   a->ref.assign(static_cast<size_t>(num_blocks), 0);
+  a->evict_pos.assign(static_cast<size_t>(num_blocks), a->evictable.end());
+  a->cache_id.assign(static_cast<size_t>(num_blocks), 0);
+  a->cache_key.assign(static_cast<size_t>(num_blocks), pa_alloc::CacheKey());
   a->free_stack.resize(static_cast<size_t>(num_blocks));
   if (free_order) {
     std::vector<uint8_t> seen(static_cast<size_t>(num_blocks), 0);
@@ -109,12 +155,62 @@ int pa_seq_add(pa_alloc_t* a, int64_t seq_id, int64_t num_tokens) {
   if (!a || num_tokens < 0) return PA_ERR_INVALID_ARG;
   if (a->seqs.count(seq_id)) return PA_ERR_SEQ_EXISTS;
   int64_t need = blocks_for(num_tokens, a->block_size);
-  if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_NO_FREE_BLOCKS;
+  if (need > a->available()) return PA_ERR_NO_FREE_BLOCKS;
   Seq s;
   s.blocks.reserve(static_cast<size_t>(need + 1));
   for (int64_t i = 0; i < need; ++i) s.blocks.push_back(a->pop());
   s.len = num_tokens;
   a->seqs.emplace(seq_id, std::move(s));
+  return PA_OK;
+}
+
+int pa_seq_add_prompt(pa_alloc_t* a, int64_t seq_id, const int32_t* token_ids, int64_t n,
+                      int64_t* cached_tokens) {
+  if (!a || n < 0 || (n > 0 && !token_ids) || !cached_tokens) return PA_ERR_INVALID_ARG;
+  if (a->seqs.count(seq_id)) return PA_ERR_SEQ_EXISTS;
+  const int bs = a->block_size;
+  const int64_t full = n / bs;
+  // plan: the leading full blocks found in the cache, in order
+  std::vector<int32_t> hits;
+  int64_t parent = 0;
+  for (int64_t j = 0; j < full; ++j) {
+    pa_alloc::CacheKey key(parent, std::vector<int32_t>(token_ids + j * bs, token_ids + (j + 1) * bs));
+    auto it = a->cache.find(key);
+    if (it == a->cache.end()) break;  // the chain is broken: nothing later can match
+    hits.push_back(it->second);
+    parent = a->cache_id[it->second];
+  }
+  const int64_t fresh = full - static_cast<int64_t>(hits.size()) + (n % bs ? 1 : 0);
+  int64_t claimable = 0;
+  for (int32_t b : hits) claimable += a->ref[b] == 0;
+  if (fresh > a->available() - claimable) return PA_ERR_NO_FREE_BLOCKS;
+  Seq s;
+  s.blocks.reserve(static_cast<size_t>(full + 2));
+  for (int32_t b : hits) {  // claim the cached blocks first
+    if (a->ref[b] == 0) {
+      a->evictable.erase(a->evict_pos[b]);
+      a->evict_pos[b] = a->evictable.end();
+      a->ref[b] = 1;
+    } else {
+      a->inc(b);
+    }
+    s.blocks.push_back(b);
+  }
+  a->cache_hits += static_cast<int64_t>(hits.size());
+  for (int64_t j = static_cast<int64_t>(hits.size()); j < full; ++j) {  // fresh, registered
+    const int32_t b = a->pop();
+    pa_alloc::CacheKey key(parent, std::vector<int32_t>(token_ids + j * bs, token_ids + (j + 1) * bs));
+    const int64_t cid = a->next_cache_id++;
+    a->cache.emplace(key, b);
+    a->cache_key[b] = std::move(key);
+    a->cache_id[b] = cid;
+    parent = cid;
+    s.blocks.push_back(b);
+  }
+  if (n % bs) s.blocks.push_back(a->pop());  // the partial last block is never cached
+  s.len = n;
+  a->seqs.emplace(seq_id, std::move(s));
+  *cached_tokens = static_cast<int64_t>(hits.size()) * bs;
   return PA_OK;
 }
 
@@ -145,6 +241,8 @@ static int64_t append_one(pa_alloc* a, Seq& s, int32_t* src, int32_t* dst) {
       *src = last;
       *dst = fresh;
       ++a->cow_copies;
+    } else if (a->cache_id[last]) {
+      a->uncache(last);  // the sole owner writes into a cached block
     }
   }
   ++s.len;
@@ -158,7 +256,7 @@ int pa_seq_append_slot(pa_alloc_t* a, int64_t seq_id, int64_t* slot, int32_t* co
   if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
   Seq& s = it->second;
   bool need = append_needs_block(s, a->block_size, s.blocks.empty() ? 0 : a->ref[s.blocks.back()]);
-  if (need && a->free_stack.empty()) return PA_ERR_NO_FREE_BLOCKS;
+  if (need && a->available() == 0) return PA_ERR_NO_FREE_BLOCKS;
   *slot = append_one(a, s, cow_src, cow_dst);
   return PA_OK;
 }
@@ -196,7 +294,7 @@ int pa_seq_append_slots(pa_alloc_t* a, const int64_t* seq_ids, int n, int64_t* s
     }
     ++len_delta[seq_ids[i]];
   }
-  if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_NO_FREE_BLOCKS;
+  if (need > a->available()) return PA_ERR_NO_FREE_BLOCKS;
   int nc = 0;
   for (int i = 0; i < n; ++i) {
     Seq& s = a->seqs.find(seq_ids[i])->second;
@@ -251,7 +349,7 @@ int pa_seqs_move(pa_alloc_t* from, pa_alloc_t* to, const int64_t* seq_ids, int n
       if (index.emplace(b, static_cast<int32_t>(distinct.size())).second) distinct.push_back(b);
   const int64_t nd = static_cast<int64_t>(distinct.size());
   if (nd > 0 && (!pairs_out || cap < nd)) return PA_ERR_INVALID_ARG;
-  if (nd > static_cast<int64_t>(to->free_stack.size())) return PA_ERR_NO_FREE_BLOCKS;
+  if (nd > to->available()) return PA_ERR_NO_FREE_BLOCKS;
   std::vector<int32_t> fresh(distinct.size());
   for (size_t k = 0; k < distinct.size(); ++k) {
     fresh[k] = to->pop();
@@ -403,7 +501,7 @@ int pa_alloc_stats(const pa_alloc_t* a, pa_stats_t* st) {
   st->num_blocks = a->num_blocks;
   st->block_size = a->block_size;
   st->free_blocks = static_cast<int64_t>(a->free_stack.size());
-  st->used_blocks = a->num_blocks - st->free_blocks;
+  st->used_blocks = a->num_blocks - st->free_blocks - static_cast<int64_t>(a->evictable.size());
   st->shared_blocks = a->shared_blocks;
   st->num_seqs = static_cast<int64_t>(a->seqs.size());
   for (const auto& kv : a->seqs) {
@@ -415,6 +513,10 @@ int pa_alloc_stats(const pa_alloc_t* a, pa_stats_t* st) {
   st->allocated_slots = st->used_blocks * a->block_size;
   st->cow_copies = a->cow_copies;
   st->blocks_allocated = a->blocks_allocated;
+  st->cached_blocks = static_cast<int64_t>(a->cache.size());
+  st->evictable_blocks = static_cast<int64_t>(a->evictable.size());
+  st->cache_hits = a->cache_hits;
+  st->cache_evictions = a->cache_evictions;
   return PA_OK;
 }
 

@@ -10,6 +10,7 @@
 // loops sized to the SM count.  Cache layout [num_blocks, num_kv_heads, block_size,
 // head_dim]; one block of one tensor is num_kv_heads*block_size*head_dim elements.
 #include <algorithm>
+#include <cmath>
 #include <vector>
 
 #include "common.cuh"
@@ -42,6 +43,59 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * nvr + v;
     k_cache[dst] = __ldg(key + i);
     v_cache[dst] = __ldg(value + i);
+  }
+}
+
+// fp8 write: each thread makes one 16-byte vector of e4m3 codes (16 elements of one
+// token row) from the float32 value of each input element times the reciprocal of
+// the tensor's scale, rounded to nearest even and saturated (CUDA's conversion).
+template <typename TQ>
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
+    const TQ* __restrict__ key, const TQ* __restrict__ value, uint4* __restrict__ k_cache,
+    uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int64_t num_tokens,
+    int num_kv_heads, int head_dim, int block_size, int64_t num_slots, float k_inv,
+    float v_inv, uint32_t* err) {
+  constexpr int VQ = ElemTraits<TQ>::kVec;
+  const int nvr = head_dim / 16;  // output vectors per (token, head) row
+  const int64_t per_token = static_cast<int64_t>(num_kv_heads) * nvr;
+  const int64_t total = num_tokens * per_token;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_token;
+    const int64_t r = i - t * per_token;
+    const int h = static_cast<int>(r / nvr);
+    const int v = static_cast<int>(r - static_cast<int64_t>(h) * nvr);
+    const int64_t slot = __ldg(slot_mapping + t);
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      set_error(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t src = (t * num_kv_heads + h) * head_dim + v * 16;
+    const int64_t blk = slot / block_size;
+    const int64_t off = slot - blk * block_size;
+    const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * nvr + v;
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+      const TQ* in = (kv ? value : key) + src;
+      const float inv = kv ? v_inv : k_inv;
+      float f[16];
+#pragma unroll
+      for (int u = 0; u < 16 / VQ; ++u)
+        vec_to_float(__ldg(reinterpret_cast<const uint4*>(in + u * VQ)), f + u * VQ, TQ());
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_fp8x2_storage_t lo =
+            __nv_cvt_float2_to_fp8x2(make_float2(f[4 * j] * inv, f[4 * j + 1] * inv),
+                                     __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi =
+            __nv_cvt_float2_to_fp8x2(make_float2(f[4 * j + 2] * inv, f[4 * j + 3] * inv),
+                                     __NV_SATFINITE, __NV_E4M3);
+        w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+      }
+      (kv ? v_cache : k_cache)[dst] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
@@ -81,6 +135,7 @@ int elem_bytes(int dtype) {
     case PA_F32: return 4;
     case PA_BF16: return 2;
     case PA_F16: return 2;
+    case PA_FP8_E4M3: return 1;
     default: return 0;
   }
 }
@@ -156,6 +211,51 @@ int sm_count() {
 
 using namespace pa;
 
+extern "C" int pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                        void* v_cache, const int64_t* slot_mapping,
+                                        int64_t num_tokens, int num_kv_heads, int head_dim,
+                                        int block_size, int64_t num_blocks, int input_dtype,
+                                        float k_scale, float v_scale, pa_stream_t stream) {
+  if ((input_dtype != PA_F32 && input_dtype != PA_BF16 && input_dtype != PA_F16) ||
+      num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 16 != 0 ||
+      block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  const float k_inv = 1.0f / k_scale, v_inv = 1.0f / v_scale;
+  const int64_t total = num_tokens * num_kv_heads * (head_dim / 16);
+  const int64_t want = (total + 255) / 256;
+  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8));
+  uint32_t* err = device_error_word();
+  if (!err) {
+    note_cuda_error(cudaGetLastError());
+    return PA_ERR_CUDA;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t slots = num_blocks * block_size;
+  auto* kc = static_cast<uint4*>(k_cache);
+  auto* vc = static_cast<uint4*>(v_cache);
+  if (input_dtype == PA_BF16)
+    reshape_and_cache_fp8_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(key), static_cast<const __nv_bfloat16*>(value), kc, vc,
+        slot_mapping, num_tokens, num_kv_heads, head_dim, block_size, slots, k_inv, v_inv, err);
+  else if (input_dtype == PA_F16)
+    reshape_and_cache_fp8_kernel<__half><<<grid, 256, 0, st>>>(
+        static_cast<const __half*>(key), static_cast<const __half*>(value), kc, vc, slot_mapping,
+        num_tokens, num_kv_heads, head_dim, block_size, slots, k_inv, v_inv, err);
+  else
+    reshape_and_cache_fp8_kernel<float><<<grid, 256, 0, st>>>(
+        static_cast<const float*>(key), static_cast<const float*>(value), kc, vc, slot_mapping,
+        num_tokens, num_kv_heads, head_dim, block_size, slots, k_inv, v_inv, err);
+  const cudaError_t e = cudaGetLastError();
+  note_cuda_error(e);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_cache,
                                     void* v_cache, const int64_t* slot_mapping,
                                     int64_t num_tokens, int num_kv_heads, int head_dim,
@@ -166,7 +266,7 @@ extern "C" int pa_reshape_and_cache(const void* key, const void* value, void* k_
       num_blocks <= 0)
     return PA_ERR_INVALID_ARG;
   if ((static_cast<int64_t>(head_dim) * eb) % 16 != 0) return PA_ERR_INVALID_ARG;
-  if (num_tokens == 0) return PA_OK;
+  if (num_tokens == 0) return PA_OK;  // (an fp8 cache copies fp8 rows here, bit for bit)
   if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
   if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID_ARG;

@@ -4,6 +4,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,6 +36,7 @@ struct DecodeParams {
   const int32_t* chunk_members;  // [num_chunks, max_members] batch positions, -1 padded
   const int32_t* chunk_parts;    // [num_chunks] shared partitions of each chunk
   int max_members;
+  float v_scale;  // output multiplier (the fp8 cache's V scale; 1 otherwise)
 };
 
 // Device address of the library's error word on the current device.
@@ -47,6 +49,7 @@ template <typename T> struct ElemTraits;
 template <> struct ElemTraits<float> { static constexpr int kVec = 4; };
 template <> struct ElemTraits<__nv_bfloat16> { static constexpr int kVec = 8; };
 template <> struct ElemTraits<__half> { static constexpr int kVec = 8; };
+template <> struct ElemTraits<__nv_fp8_e4m3> { static constexpr int kVec = 16; };
 
 // 16 bytes of T -> floats (kVec of them)
 __device__ __forceinline__ void vec_to_float(const uint4& v, float* f, float) {
@@ -76,6 +79,22 @@ __device__ __forceinline__ void vec_to_float(const uint4& v, float* f, __half) {
   h2_to_float(v.y, f[2], f[3]);
   h2_to_float(v.z, f[4], f[5]);
   h2_to_float(v.w, f[6], f[7]);
+}
+
+// 16 e4m3 codes -> floats (CUDA's fp8 conversion; exact)
+__device__ __forceinline__ void vec_to_float(const uint4& v, float* f, __nv_fp8_e4m3) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(w[i] >> (16 * j));
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      const float2 ff = __half22float2(*reinterpret_cast<const __half2*>(&h));
+      f[4 * i + 2 * j] = ff.x;
+      f[4 * i + 2 * j + 1] = ff.y;
+    }
+  }
 }
 
 __device__ __forceinline__ void store_elem(float* p, float x) { *p = x; }

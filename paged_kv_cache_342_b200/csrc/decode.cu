@@ -7,6 +7,8 @@
 // attention); "PagedAttention" attention-lab explainer (divagr.pages.dev), "Keep
 // pages in order" and "Measure memory use across requests" (the attention equation
 // is unchanged by paging).
+#include <cmath>
+
 #include "common.cuh"
 #include "decode_simt.cuh"
 
@@ -15,6 +17,7 @@ namespace pa {
 cudaError_t launch_decode_simt_f32(const DecodeParams& p, int gs, cudaStream_t st);
 cudaError_t launch_decode_simt_bf16(const DecodeParams& p, int gs, cudaStream_t st);
 cudaError_t launch_decode_simt_f16(const DecodeParams& p, int gs, cudaStream_t st);
+cudaError_t launch_decode_simt_fp8(const DecodeParams& p, int q_dtype, int gs, cudaStream_t st);
 cudaError_t launch_decode_mma_bf16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_group_bf16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
@@ -180,7 +183,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 const int32_t* block_tables, const int32_t* seq_lens, float scale, int block_size,
                 int num_kv_heads, int num_seqs, int num_heads, int head_dim,
                 int max_blocks_per_seq, int64_t num_blocks, int max_seq_len, int partition_size,
-                int dtype, const GroupArgs* groups, void* workspace, size_t workspace_bytes,
+                int dtype, int cache_dtype, float k_scale, float v_scale,
+                const GroupArgs* groups, void* workspace, size_t workspace_bytes,
                 pa_stream_t stream);
 
 }  // namespace
@@ -212,8 +216,22 @@ extern "C" int pa_decode_attention(void* out, const void* q, const void* k_cache
                                    size_t workspace_bytes, pa_stream_t stream) {
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
                      num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
-                     max_seq_len, partition_size, dtype, nullptr, workspace, workspace_bytes,
-                     stream);
+                     max_seq_len, partition_size, dtype, dtype, 1.f, 1.f, nullptr, workspace,
+                     workspace_bytes, stream);
+}
+
+extern "C" int pa_decode_attention_fp8(void* out, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_tables,
+                                       const int32_t* seq_lens, float scale, int block_size,
+                                       int num_kv_heads, int num_seqs, int num_heads,
+                                       int head_dim, int max_blocks_per_seq, int64_t num_blocks,
+                                       int max_seq_len, int partition_size, int dtype,
+                                       float k_scale, float v_scale, void* workspace,
+                                       size_t workspace_bytes, pa_stream_t stream) {
+  return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
+                     num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
+                     max_seq_len, partition_size, dtype, PA_FP8_E4M3, k_scale, v_scale, nullptr,
+                     workspace, workspace_bytes, stream);
 }
 
 extern "C" int pa_decode_attention_grouped(
@@ -233,7 +251,8 @@ extern "C" int pa_decode_attention_grouped(
                     max_chunk_parts};
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
                      num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
-                     max_seq_len, partition_size, dtype, &g, workspace, workspace_bytes, stream);
+                     max_seq_len, partition_size, dtype, dtype, 1.f, 1.f, &g, workspace,
+                     workspace_bytes, stream);
 }
 
 namespace pa {
@@ -243,9 +262,18 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 const int32_t* block_tables, const int32_t* seq_lens, float scale, int block_size,
                 int num_kv_heads, int num_seqs, int num_heads, int head_dim,
                 int max_blocks_per_seq, int64_t num_blocks, int max_seq_len, int partition_size,
-                int dtype, const GroupArgs* groups, void* workspace, size_t workspace_bytes,
+                int dtype, int cache_dtype, float k_scale, float v_scale,
+                const GroupArgs* groups, void* workspace, size_t workspace_bytes,
                 pa_stream_t stream) {
   if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16) return PA_ERR_INVALID_ARG;
+  const bool fp8 = cache_dtype == PA_FP8_E4M3;
+  if (cache_dtype != dtype && !fp8) return PA_ERR_INVALID_ARG;
+  if (fp8) {
+    if (dtype == PA_F32) return PA_ERR_UNSUPPORTED;
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+      return PA_ERR_INVALID_ARG;
+    if (head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+  }
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads ||
       head_dim <= 0 || block_size <= 0 || max_blocks_per_seq < 0 || num_blocks <= 0 ||
       max_seq_len < 0 || partition_size < 0)
@@ -272,7 +300,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.v_cache = v_cache;
   p.block_tables = block_tables;
   p.seq_lens = seq_lens;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  p.v_scale = v_scale;
   p.num_seqs = num_seqs;
   p.num_heads = num_heads;
   p.num_kv_heads = num_kv_heads;
@@ -300,7 +329,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   cudaError_t e;
   // shared partitions of prefix groups first (only useful when sequences span
   // several partitions); otherwise the per-sequence kernels do everything
-  if (groups && groups->num_chunks > 0 && groups->max_chunk_parts > 0 && ws.parts > 1 &&
+  if (!fp8 && groups && groups->num_chunks > 0 && groups->max_chunk_parts > 0 && ws.parts > 1 &&
       group_eligible(dtype, group, head_dim, block_size, groups->max_members)) {
     p.prefix_parts = groups->prefix_parts;
     p.chunk_members = groups->chunk_members;
@@ -314,7 +343,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
       return PA_ERR_CUDA;
     }
   }
-  if (mma_eligible(dtype, group, head_dim, block_size)) {
+  if (fp8) {
+    e = launch_decode_simt_fp8(p, dtype, simt_heads_per_cta(group, head_dim), st);
+  } else if (mma_eligible(dtype, group, head_dim, block_size)) {
     e = dtype == PA_BF16 ? launch_decode_mma_bf16(p, st) : launch_decode_mma_f16(p, st);
   } else {
     const int gs = simt_heads_per_cta(group, head_dim);

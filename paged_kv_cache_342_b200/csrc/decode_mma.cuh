@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(NW * 32)
       num = fmaf(r[d], f, num);
       den = fmaf(r[D + 1], f, den);
     }
-    const float o = den > 0.f ? num / den : 0.f;
+    const float o = den > 0.f ? num / den * p.v_scale : 0.f;
     if (!col_ok[hh]) continue;
     const int64_t row = col_row[hh];
     if (nparts == 1) {

@@ -37,7 +37,7 @@ constexpr int kRowsPerPass = 4;
 
 template <typename T, int D, int BS, int GS, int NW, int NST>
 struct SimtCfg {
-  static constexpr int kVec = ElemTraits<T>::kVec;
+  static constexpr int kVec = ElemTraits<T>::kVec;  // cache elements per 16-byte vector
   static constexpr int kVecPerRow = D / kVec;
   static constexpr int kVecPerLane = kVecPerRow / kLanesPerRow;
   static constexpr int kEPL = kVecPerLane * kVec;  // = D / 8
@@ -77,9 +77,12 @@ __device__ __forceinline__ int group_parts(const DecodeParams& p, int s, int L) 
   return g < 0 ? 0 : (g < last ? g : last);
 }
 
-template <typename T, int D, int BS, int GS, int NW, int NST>
+// T = cache element type, TQ = query / output type (equal except for fp8 caches).
+template <typename T, typename TQ, int D, int BS, int GS, int NW, int NST>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams p) {
   using C = SimtCfg<T, D, BS, GS, NW, NST>;
+  constexpr int VQ = ElemTraits<TQ>::kVec;  // query elements per 16-byte vector
+  static_assert(C::kVec % VQ == 0, "a cache vector spans whole query vectors");
   constexpr int EPL = C::kEPL;
   constexpr int NVL = C::kVecPerLane;
   constexpr int VEC = C::kVec;
@@ -114,13 +117,17 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
   // q for this lane's elements, pre-scaled into the base-2 logit domain
   float qf[GS][EPL];
   {
-    const T* qb = static_cast<const T*>(p.q) + (static_cast<int64_t>(s) * p.num_heads + h0) * D;
+    const TQ* qb = static_cast<const TQ*>(p.q) + (static_cast<int64_t>(s) * p.num_heads + h0) * D;
 #pragma unroll
     for (int g = 0; g < GS; ++g) {
 #pragma unroll
       for (int k = 0; k < NVL; ++k) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(qb + g * D + (sub + 8 * k) * VEC));
-        vec_to_float(v, &qf[g][k * VEC], T());
+#pragma unroll
+        for (int u = 0; u < VEC / VQ; ++u) {
+          const uint4 v = __ldg(
+              reinterpret_cast<const uint4*>(qb + g * D + (sub + 8 * k) * VEC + u * VQ));
+          vec_to_float(v, &qf[g][k * VEC + u * VQ], TQ());
+        }
       }
 #pragma unroll
       for (int e = 0; e < EPL; ++e) qf[g][e] *= p.scale_log2;
@@ -308,10 +315,10 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
       num = fmaf(r[d], f, num);
       den = fmaf(r[D + 1], f, den);
     }
-    const float o = den > 0.f ? num / den : 0.f;
+    const float o = den > 0.f ? num / den * p.v_scale : 0.f;
     const int64_t row = static_cast<int64_t>(s) * p.num_heads + h0 + g;
     if (nparts == 1) {
-      store_elem(static_cast<T*>(p.out) + row * D + d, o);
+      store_elem(static_cast<TQ*>(p.out) + row * D + d, o);
     } else {
       const int64_t prow = row * p.max_parts + part;
       p.ws_o[prow * D + d] = o;
@@ -324,10 +331,10 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
 }
 
 // Launch one instantiation (sets the dynamic shared-memory limit once).
-template <typename T, int D, int BS, int GS, int NW, int NST>
+template <typename T, typename TQ, int D, int BS, int GS, int NW, int NST>
 cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream) {
   using C = SimtCfg<T, D, BS, GS, NW, NST>;
-  constexpr auto kern = decode_simt_kernel<T, D, BS, GS, NW, NST>;
+  constexpr auto kern = decode_simt_kernel<T, TQ, D, BS, GS, NW, NST>;
   cudaError_t attr = ensure_smem_limit<kern>(C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
   dim3 grid(p.num_heads / GS, p.num_seqs, p.max_parts);

@@ -15,7 +15,7 @@ cudaError_t launch_auto(const DecodeParams& p, cudaStream_t st) {
   constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
   constexpr int kRaw = kBudget / (NW * kStage);
   constexpr int NST = kRaw < 2 ? 2 : (kRaw > 4 ? 4 : kRaw);
-  return launch_simt<__nv_bfloat16, D, BS, GS, NW, NST>(p, st);
+  return launch_simt<__nv_bfloat16, __nv_bfloat16, D, BS, GS, NW, NST>(p, st);
 }
 
 template <int D, int GS>

@@ -22,6 +22,10 @@ Sequences that share leading blocks (forks of one prompt) are found each step by
 members as fill one 8-column tensor-core tile, 8 // (num_heads/num_kv_heads); 0
 turns grouping off).
 
+One-byte caches (uint8 / float8_e4m3fn tensors) are fp8 e4m3 caches with the
+per-tensor ``kv_scales`` (k_scale, v_scale): the step writes with
+``pa_reshape_and_cache_fp8`` and attends with ``pa_decode_attention_fp8``.
+
 This module only moves arguments: the work of every step is done by the library.
 """
 from __future__ import annotations
@@ -30,7 +34,8 @@ import numpy as np
 import torch
 
 from . import (DEFAULT_PARTITION, BlockAllocator, pa_copy_blocks, pa_decode_attention,
-               pa_decode_attention_grouped, pa_decode_workspace_bytes, pa_reshape_and_cache)
+               pa_decode_attention_fp8, pa_decode_attention_grouped, pa_decode_workspace_bytes,
+               pa_reshape_and_cache, pa_reshape_and_cache_fp8)
 
 
 def _align(n: int, a: int = 256) -> int:
@@ -46,7 +51,7 @@ class PagedDecoder:
 
     def __init__(self, k_cache, v_cache, num_heads: int, scale: float, max_blocks_per_seq: int,
                  free_order=None, partition_size: int = DEFAULT_PARTITION, stream=None,
-                 group_members: int | None = None):
+                 group_members: int | None = None, kv_scales=None):
         self.k_cache, self.v_cache = k_cache, v_cache
         self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim = k_cache.shape
         self.num_heads, self.scale = num_heads, scale
@@ -59,8 +64,14 @@ class PagedDecoder:
         self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
         self._done = None  # event: the last staging copy has been consumed
         group = num_heads // self.num_kv_heads
+        self.fp8 = k_cache.element_size() == 1
+        if self.fp8 and kv_scales is None:
+            raise ValueError("an fp8 cache needs kv_scales=(k_scale, v_scale)")
+        self.kv_scales = kv_scales
         self.group_members = (8 // group if group <= 8 else 0) if group_members is None \
             else group_members
+        if self.fp8:
+            self.group_members = 0
 
     # -- context building ------------------------------------------------------
     def admit(self, seq_id: int, num_tokens: int) -> None:
@@ -174,11 +185,20 @@ class PagedDecoder:
         n = meta["num_cow"]
         if n:
             pa_copy_blocks(self.k_cache, self.v_cache, self.d_pairs[:n], meta["pairs"], stream=st)
-        pa_reshape_and_cache(new_k, new_v, self.k_cache, self.v_cache, self.d_slots, stream=st)
+        if self.fp8:
+            pa_reshape_and_cache_fp8(new_k, new_v, self.k_cache, self.v_cache, self.d_slots,
+                                     *self.kv_scales, stream=st)
+        else:
+            pa_reshape_and_cache(new_k, new_v, self.k_cache, self.v_cache, self.d_slots, stream=st)
         ws = self._ws if self._ws.numel() else None
         if events is not None:
             events[0].record(st)
-        if meta.get("num_chunks", 0):
+        if self.fp8:
+            pa_decode_attention_fp8(out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
+                                    self.scale, self.block_size, self.num_kv_heads,
+                                    meta["max_len"], *self.kv_scales, self.partition_size, ws,
+                                    stream=st)
+        elif meta.get("num_chunks", 0):
             pp, cm, cp = self.d_groups
             pa_decode_attention_grouped(
                 out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens, self.scale,
@@ -199,7 +219,7 @@ class PagedDecoder:
     def kernel_launches(self, meta: dict) -> int:
         """Library kernels one step launches (copy, write, group, partitions, merge)."""
         parts = max(1, -(-meta["max_len"] // self.partition_size))
-        grouped = (meta.get("num_chunks", 0) > 0 and parts > 1
+        grouped = (meta.get("num_chunks", 0) > 0 and parts > 1 and not self.fp8
                    and self.k_cache.dtype != torch.float32
                    and self.block_size in (16, 32)
                    and self.group_members * (self.num_heads // self.num_kv_heads) <= 16)

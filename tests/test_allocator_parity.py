@@ -353,3 +353,88 @@ def test_full_pool_swap_out_lets_the_batch_continue(pa):
     dev.free(0)                      # a sequence finishes: room to swap back in
     back = host.move_to(dev, [2])
     assert len(back) == 2 and dev.seq_len(2) == 8 and host.stats()["num_seqs"] == 0
+
+
+# ---------------------------------------------------------------------------
+# automatic prefix caching
+# ---------------------------------------------------------------------------
+
+def _prompt(g, prefixes, bs):
+    """A prompt = one of a few shared prefixes + a random tail (token ids)."""
+    base = prefixes[int(g.integers(0, len(prefixes)))]
+    cut = int(g.integers(0, len(base) + 1))
+    tail = g.integers(0, 50, int(g.integers(0, 3 * bs))).tolist()
+    return base[:cut] + tail
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_prefix_cache_random_ops(pa, seed):
+    g = np.random.default_rng(300 + seed)
+    bs = int(g.choice([2, 4, 8]))
+    nb = int(g.integers(12, 40))
+    order = g.permutation(nb)
+    c, o = pa.BlockAllocator(nb, bs, order), BlockManager(nb, bs, order)
+    prefixes = [g.integers(0, 50, int(g.integers(bs, 6 * bs))).tolist() for _ in range(3)]
+    live, nid = [], 0
+    for step in range(300):
+        r = int(g.integers(0, 12))
+        if r < 4 or not live:
+            toks = _prompt(g, prefixes, bs)
+            rc, ro = run_both(pa, c, o, "add_prompt", nid, toks)
+            assert rc == ro
+            if nid in o.tables:
+                live.append(nid)
+            nid += 1
+        elif r < 6:
+            s = live[int(g.integers(0, len(live)))]
+            rc, ro = run_both(pa, c, o, "append_slot", s)
+            assert rc == ro
+        elif r < 7:
+            p = live[int(g.integers(0, len(live)))]
+            run_both(pa, c, o, "fork", p, nid)
+            if nid in o.tables:
+                live.append(nid)
+            nid += 1
+        elif r < 9:
+            s = live.pop(int(g.integers(0, len(live))))
+            run_both(pa, c, o, "free", s)
+        elif r < 10:
+            s = live[int(g.integers(0, len(live)))]
+            run_both(pa, c, o, "truncate", [s], [int(g.integers(0, o.lens[s] + 1))])
+        else:
+            n = int(g.integers(0, 2 * bs))
+            run_both(pa, c, o, "add", nid, n)
+            if nid in o.tables:
+                live.append(nid)
+            nid += 1
+        same_state(c, o)
+    assert o.cache_hits > 0 and o.cache_evictions > 0      # both paths were exercised
+
+
+def test_identical_system_prompts_are_stored_once(pa):
+    """[GLOSS] prompt sharing: identical system prompts are stored once and mapped into
+    several requests.  Two requests with the same 40-token prompt at block 16: the
+    second reuses both full blocks and only its partial last block is new."""
+    prompt = list(range(100, 140))
+    for m in (pa.BlockAllocator(16, 16), BlockManager(16, 16)):
+        first = m.add_prompt(0, prompt)
+        second = m.add_prompt(1, prompt + [7, 8])
+        t0 = m.seq_blocks(0) if hasattr(m, "seq_blocks") else m.tables[0]
+        t1 = m.seq_blocks(1) if hasattr(m, "seq_blocks") else m.tables[1]
+        assert (first, second) == (0, 32)
+        assert t0[:2] == t1[:2] and t0[2] != t1[2]
+        st = m.stats()
+        assert st["cached_blocks"] == 2 and st["cache_hits"] == 2 and st["used_blocks"] == 4
+
+
+def test_released_cached_blocks_are_reused_before_eviction(pa):
+    for m in (pa.BlockAllocator(4, 4), BlockManager(4, 4)):
+        m.add_prompt(0, list(range(8)))          # 2 cached blocks
+        (m.free_seq if isinstance(m, BlockManager) else m.free)(0)
+        st = m.stats()
+        assert st["evictable_blocks"] == 2 and st["free_blocks"] == 2
+        assert m.add_prompt(1, list(range(8)) + [9]) == 8    # hits both, no eviction
+        assert m.stats()["cache_evictions"] == 0
+        m.add(2, 4)                               # takes the last free block
+        with pytest.raises(Exception):
+            m.add(3, 4)                           # nothing free, nothing evictable

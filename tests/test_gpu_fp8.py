@@ -1,0 +1,156 @@
+"""The fp8 (e4m3) cache: the quantizing write is bit-exact against the oracle's
+codec, and decode over the fp8 cache matches the float64 oracle on the dequantized
+values (per-tensor scales; stored = e4m3(x * (1/scale)), value = code * scale)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.attention as oatt
+from oracle import fp8
+from gpu_util import ATOL, TORCH_DT, assert_close, out_f64, tables_from_order, to_dev
+from oracle.numerics import to_f64
+from workloads import normal_fill
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import paged_kv_cache_342_b200 as m
+    assert torch.cuda.is_available()
+    m.pa_device_error_read()
+    return m
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("D,bs,Hkv", [(128, 16, 4), (64, 8, 2), (256, 32, 2)])
+def test_fp8_write_is_bit_exact(pa, dtype, D, bs, Hkv):
+    NB, T = 24, 29
+    key = normal_fill((T, Hkv, D), dtype, 3.0, 4, 1)
+    val = normal_fill((T, Hkv, D), dtype, 40.0, 4, 2)      # some values saturate
+    ks, vs = 0.0271, 0.05
+    slots = np.random.default_rng(4).choice(NB * bs, T, replace=False).astype(np.int64)
+    slots[3] = -1
+    kc = torch.full((NB, Hkv, bs, D), 0x5A, dtype=torch.uint8, device="cuda")
+    vc = torch.full_like(kc, 0x21)
+    pa.pa_reshape_and_cache_fp8(to_dev(key, dtype), to_dev(val, dtype), kc, vc,
+                                torch.from_numpy(slots).cuda(), ks, vs)
+    want_k = np.full((NB, Hkv, bs, D), 0x5A, np.uint8)
+    want_v = np.full_like(want_k, 0x21)
+    for t, slot in enumerate(slots):
+        if slot < 0:
+            continue
+        b, o = divmod(int(slot), bs)
+        want_k[b, :, o, :] = fp8.quantize(to_f64(key[t], dtype).astype(np.float32), ks)
+        want_v[b, :, o, :] = fp8.quantize(to_f64(val[t], dtype).astype(np.float32), vs)
+    assert np.array_equal(kc.cpu().numpy(), want_k)
+    assert np.array_equal(vc.cpu().numpy(), want_v)
+    assert pa.pa_device_error_read() == 0
+
+
+FP8_CASES = [
+    # q dtype, Hq, Hkv, D, bs, partition, lens
+    ("bf16", 4, 4, 128, 16, 64, (1, 15, 16, 17, 200, 333, 0)),
+    ("f16", 8, 2, 128, 8, 32, (5, 64, 65, 400)),          # group 4
+    ("bf16", 16, 2, 128, 16, 512, (1, 700, 33)),           # group 8 (CUDA cores for fp8)
+    ("f16", 2, 2, 256, 32, 64, (3, 100, 250)),
+    ("bf16", 4, 4, 128, 4, 16, (7, 18, 10)),
+]
+
+
+@pytest.mark.parametrize("case", FP8_CASES, ids=lambda c: f"{c[0]}-h{c[1]}/{c[2]}-d{c[3]}-b{c[4]}")
+def test_fp8_decode_matches_oracle(pa, case):
+    dtype, Hq, Hkv, D, bs, ps, lens = case
+    lens = np.asarray(lens, np.int64)
+    S = lens.size
+    NB = int(sum(-(-int(L) // bs) for L in lens)) + 3
+    g = np.random.default_rng(8)
+    # N(0,1) K/V stored with scale 8/448 (the oracle's codec makes the codes)
+    ks = vs = 8.0 / 448.0
+    kcodes = fp8.quantize(normal_fill((NB, Hkv, bs, D), "f32", 1.0, 8, 1), ks)
+    vcodes = fp8.quantize(normal_fill((NB, Hkv, bs, D), "f32", 1.0, 8, 2), vs)
+    q = normal_fill((S, Hq, D), dtype, 1.0, 8, 3)
+    order = g.permutation(NB).astype(np.int32)
+    tables = tables_from_order(lens, bs, order, int(-(-lens.max() // bs)) + 1)
+    max_len = int(lens.max())
+    out = torch.full((S, Hq, D), float("nan"), dtype=TORCH_DT[dtype], device="cuda")
+    wsb = pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+    scale = 1 / math.sqrt(D)
+    pa.pa_decode_attention_fp8(out, to_dev(q, dtype), torch.from_numpy(kcodes).cuda(),
+                               torch.from_numpy(vcodes).cuda(), torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens.astype(np.int32)).cuda(), scale, bs, Hkv,
+                               max_len, ks, vs, ps, ws if wsb else None)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    want = oatt.paged_decode_attention(to_f64(q, dtype), fp8.dequantize(kcodes, ks),
+                                       fp8.dequantize(vcodes, vs), tables, lens, scale, bs, Hkv,
+                                       "f64")
+    assert_close(out_f64(out), want, dtype, "fp8 cache")
+
+
+def test_fp8_decode_all_codes(pa):
+    """Every finite e4m3 code appears in the cache (magnitudes up to 448 * scale); the
+    output is compared at the tolerance of its own magnitude (bf16 rounding of |out|)."""
+    S, Hq, Hkv, D, bs = 3, 4, 4, 128, 16
+    lens = np.array([256, 100, 37])
+    NB = 24
+    g = np.random.default_rng(9)
+    codes = [g.integers(0, 256, (NB, Hkv, bs, D)).astype(np.uint8) for _ in range(2)]
+    for c in codes:
+        c[(c & 0x7F) == 0x7F] = 0x3F                    # no NaN codes
+    ks, vs = 0.002, 0.004
+    q = normal_fill((S, Hq, D), "bf16", 1.0, 9, 3)
+    tables = tables_from_order(lens, bs, g.permutation(NB).astype(np.int32), 17)
+    out = torch.empty((S, Hq, D), dtype=torch.bfloat16, device="cuda")
+    pa.pa_decode_attention_fp8(out, to_dev(q, "bf16"), torch.from_numpy(codes[0]).cuda(),
+                               torch.from_numpy(codes[1]).cuda(), torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens.astype(np.int32)).cuda(), 1 / math.sqrt(D),
+                               bs, Hkv, 256, ks, vs, 64,
+                               torch.empty(pa.pa_decode_workspace_bytes(S, Hq, D, 256, 64),
+                                           dtype=torch.uint8, device="cuda"))
+    torch.cuda.synchronize()
+    want = oatt.paged_decode_attention(to_f64(q, "bf16"), fp8.dequantize(codes[0], ks),
+                                       fp8.dequantize(codes[1], vs), tables, lens,
+                                       1 / math.sqrt(D), bs, Hkv, "f64")
+    got = out_f64(out)
+    assert np.isfinite(got).all()
+    assert np.all(np.abs(got - want) <= 2e-2 + 2.0 ** -8 * np.abs(want))
+
+
+def test_fp8_decode_step_through_the_runtime(pa):
+    """A whole decode step on an fp8 cache: write the new token (quantized), attend."""
+    from paged_kv_cache_342_b200.runtime import PagedDecoder
+    S, Hq, Hkv, D, bs, NB = 6, 8, 8, 128, 16, 96
+    g = np.random.default_rng(12)
+    lens = g.integers(20, 200, S)
+    ks = vs = 8.0 / 448
+    pool_k = fp8.quantize(normal_fill((NB, Hkv, bs, D), "f32", 1.0, 12, 1), ks)
+    pool_v = fp8.quantize(normal_fill((NB, Hkv, bs, D), "f32", 1.0, 12, 2), vs)
+    kd, vd = torch.from_numpy(pool_k).cuda(), torch.from_numpy(pool_v).cuda()
+    dec = PagedDecoder(kd, vd, Hq, 1 / math.sqrt(D), 16, g.permutation(NB), 64,
+                       kv_scales=(ks, vs))
+    for s in range(S):
+        dec.admit(s, int(lens[s]))
+    dec.bind(range(S))
+    q = normal_fill((S, Hq, D), "bf16", 1.0, 12, 3)
+    nk = normal_fill((S, Hkv, D), "bf16", 1.0, 12, 4)
+    nv = normal_fill((S, Hkv, D), "bf16", 1.0, 12, 5)
+    out = torch.empty((S, Hq, D), dtype=torch.bfloat16, device="cuda")
+    dec.step(to_dev(q, "bf16"), to_dev(nk, "bf16"), to_dev(nv, "bf16"), out)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    tables, sl = dec.h_tables.numpy().copy(), dec.h_lens.numpy().copy()
+    slots = dec.h_slots.numpy().copy()
+    # oracle: quantize the new token into its slot, attend over dequantized values
+    for s, slot in enumerate(slots):
+        b, o = divmod(int(slot), bs)
+        pool_k[b, :, o, :] = fp8.quantize(to_f64(nk[s], "bf16").astype(np.float32), ks)
+        pool_v[b, :, o, :] = fp8.quantize(to_f64(nv[s], "bf16").astype(np.float32), vs)
+    assert np.array_equal(kd.cpu().numpy(), pool_k) and np.array_equal(vd.cpu().numpy(), pool_v)
+    want = oatt.paged_decode_attention(to_f64(q, "bf16"), fp8.dequantize(pool_k, ks),
+                                       fp8.dequantize(pool_v, vs), tables, sl, 1 / math.sqrt(D),
+                                       bs, Hkv, "f64")
+    assert_close(out_f64(out), want, "bf16", "fp8 step")

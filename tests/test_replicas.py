@@ -42,7 +42,7 @@ def _rank_main(rank, world, port, elapsed, out):
 def test_two_replicas_agree_on_the_slowest_rank():
     world, port = 2, _free_port()
     elapsed = [3.0, 5.0]   # ms: rank 1 is slower
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_rank_main, args=(world, port, elapsed, out), nprocs=world,
                            join=True, start_method="spawn")
