@@ -54,6 +54,8 @@ def parse():
     # the pages' block-size trade-off: same lengths and slot capacity, other block size
     ap.add_argument("--block-size", type=int, default=None,
                     help="override the block size (pool keeps the same number of slots)")
+    ap.add_argument("--measure", default="decode", choices=["decode", "swap"],
+                    help="swap: time swapping half the batch to a pinned host pool and back")
     ap.add_argument("--cache-fp8", action="store_true",
                     help="store K/V as fp8 e4m3 with per-tensor scales (q/out keep the dtype)")
     return ap.parse_args()
@@ -530,6 +532,74 @@ def kernel_sources_sha() -> str:
     return h.hexdigest()
 
 
+def run_swap(args, cfg):
+    """Preemption by swapping: half the batch moves to a page-locked host pool and
+    back each step (pa_seqs_move + pa_swap_blocks); reports the copy throughput over
+    the host link, device-timed with CUDA events."""
+    import torch
+
+    import paged_kv_cache_342_b200 as pa
+    from workloads import make_inputs, storage_to_torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(cfg, args.seed)
+    S, bs = cfg.num_seqs, cfg.block_size
+    kd = storage_to_torch(inp.k_pool, cfg.dtype).to(dev)
+    vd = storage_to_torch(inp.v_pool, cfg.dtype).to(dev)
+    dev_pool = pa.BlockAllocator(cfg.num_blocks, bs, inp.free_order)
+    for s_ in range(S):
+        dev_pool.add(s_, int(inp.context_lens[s_]))
+    victims = list(range(S // 2, S))
+    need = sum(len(dev_pool.seq_blocks(v)) for v in victims)
+    host_pool = pa.BlockAllocator(need, bs)
+    kh = torch.empty((need,) + tuple(kd.shape[1:]), dtype=kd.dtype).pin_memory()
+    vh = torch.empty_like(kh).pin_memory()
+    block_bytes = kd[0].numel() * kd.element_size()
+    stream = torch.cuda.current_stream(dev)
+    mapping = torch.empty((need, 2), dtype=torch.int32, device=dev)
+
+    def swap(src_pool, dst_pool, dk, dv, sk, sv, ev=None):
+        pairs = src_pool.move_to(dst_pool, victims)
+        mapping[:len(pairs)].copy_(torch.from_numpy(pairs))
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_swap_blocks(dk, dv, sk, sv, mapping[:len(pairs)], pairs)
+        if ev is not None:
+            ev[1].record(stream)
+        return len(pairs)
+
+    for _ in range(args.warmup):
+        swap(dev_pool, host_pool, kh, vh, kd, vd)
+        swap(host_pool, dev_pool, kd, vd, kh, vh)
+    torch.cuda.synchronize(dev)
+    steps = min(args.steps, 50)
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(2)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    moved = 0
+    t0.record(stream)
+    for k in range(steps):
+        moved += swap(dev_pool, host_pool, kh, vh, kd, vd, evs[k][0])
+        moved += swap(host_pool, dev_pool, kd, vd, kh, vh, evs[k][1])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if pa.pa_device_error_read():
+        raise RuntimeError("device error word set")
+    out_ms = statistics.mean(e[0][0].elapsed_time(e[0][1]) for e in evs)
+    in_ms = statistics.mean(e[1][0].elapsed_time(e[1][1]) for e in evs)
+    per_dir = need * block_bytes * 2          # K and V blocks one way
+    line = {"metric": "swap to host and back: pa_swap_blocks GB/s over the host link",
+            "value": round(2 * per_dir / ((out_ms + in_ms) * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "n_gpus": 1, "steps": steps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": cfg.dtype, "data": "synthetic",
+            "swap_out_GBs": round(per_dir / (out_ms * 1e-3) / 1e9, 2),
+            "swap_in_GBs": round(per_dir / (in_ms * 1e-3) / 1e9, 2),
+            "ms_per_round_trip_including_block_manager": round(t0.elapsed_time(t1) / steps, 3),
+            "config": {"workload": cfg.name, "swapped_sequences": len(victims),
+                       "blocks_each_way": need, "bytes_each_way": per_dir}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.warmup < 3:
@@ -548,6 +618,8 @@ def main():
                         name=f"{cfg.name}_bs{args.block_size}")
     if args.impl == "reference":
         run_reference(args, cfg)
+    elif args.measure == "swap":
+        run_swap(args, cfg)
     else:
         run_ours(args, cfg)
 
