@@ -216,6 +216,57 @@ class PagedDecoder:
         self.launch(meta, q, new_k, new_v, out)
         return meta
 
+    # -- steps fed from host memory ----------------------------------------------
+    def step_host(self, q_h, new_k_h, new_v_h, out_h):
+        """One step whose inputs come from, and whose result goes back to, page-locked
+        host tensors.  Copies run on their own streams and overlap the neighbouring
+        steps' kernels: two device buffer sets alternate, and events order the
+        input copy -> kernels -> output copy of each step.  Returns the event after
+        which ``out_h`` holds this step's result (do not reuse ``out_h`` before)."""
+        if not hasattr(self, "_io"):
+            self._io_init(q_h, new_k_h, out_h)
+        io = self._io[self._io_next]
+        self._io_next ^= 1
+        comp = self._torch_stream()
+        h2d, d2h = self._h2d_stream, self._d2h_stream
+        h2d.wait_event(io["compute_done"])          # the kernels two steps ago used them
+        with torch.cuda.stream(h2d):
+            for dst, src in zip(io["inputs"], (q_h, new_k_h, new_v_h)):
+                dst.copy_(src, non_blocking=True)
+            io["h2d_done"].record(h2d)
+        comp.wait_event(io["h2d_done"])
+        comp.wait_event(io["d2h_done"])             # the output buffer was read back
+        meta = self.prepare()
+        self.launch(meta, *io["inputs"], io["out"])
+        io["compute_done"].record(comp)
+        d2h.wait_event(io["compute_done"])
+        with torch.cuda.stream(d2h):
+            out_h.copy_(io["out"], non_blocking=True)
+            io["d2h_done"].record(d2h)
+        return io["d2h_done"]
+
+    def drain_host_io(self) -> None:
+        """Make the compute stream wait for every outstanding host-I/O copy."""
+        if hasattr(self, "_io"):
+            comp = self._torch_stream()
+            for io in self._io:
+                comp.wait_event(io["d2h_done"])
+
+    def _io_init(self, q_h, kv_h, out_h) -> None:
+        dev = self.device
+        self._h2d_stream = torch.cuda.Stream(device=dev)
+        self._d2h_stream = torch.cuda.Stream(device=dev)
+        self._io, self._io_next = [], 0
+        for _ in range(2):
+            io = {"inputs": [torch.empty(q_h.shape, dtype=q_h.dtype, device=dev),
+                             torch.empty(kv_h.shape, dtype=kv_h.dtype, device=dev),
+                             torch.empty(kv_h.shape, dtype=kv_h.dtype, device=dev)],
+                  "out": torch.empty(out_h.shape, dtype=out_h.dtype, device=dev)}
+            for name in ("h2d_done", "compute_done", "d2h_done"):
+                io[name] = torch.cuda.Event()
+                io[name].record(self._torch_stream())   # start out completed
+            self._io.append(io)
+
     def kernel_launches(self, meta: dict) -> int:
         """Library kernels one step launches (copy, write, group, partitions, merge)."""
         parts = max(1, -(-meta["max_len"] // self.partition_size))
