@@ -67,6 +67,8 @@ typedef void* pa_stream_t; /* a cudaStream_t */
 #define PA_DEVERR_TABLE 4u       /* decode: block-table entry outside [0, num_blocks)*/
 #define PA_DEVERR_SEQ_LEN 8u     /* decode: seq_len < 0, > max_seq_len or > table    */
 #define PA_DEVERR_TIMEOUT 16u    /* a bounded wait on an async copy gave up          */
+#define PA_DEVERR_GROUP 32u      /* grouped decode: a sequence's own partitions start
+                                    below first_part (those partitions were skipped)  */
 
 /* ------------------------------------------------------------------------- */
 /* GPU entry points                                                           */
@@ -239,8 +241,10 @@ int pa_decode_uses_tensor_cores(int dtype, int num_heads, int num_kv_heads, int 
 /*
  * pa_decode_attention_fp8 - pa_decode_attention over an fp8 (e4m3) cache written by
  * pa_reshape_and_cache_fp8: K_t = e4m3(k codes) * k_scale, V_t = e4m3(v codes) *
- * v_scale.  q and out are dtype (PA_BF16 or PA_F16); head_dim 128 or 256; CUDA-core
- * kernel for every group size.  The cache is half the bytes of a 16-bit one.
+ * v_scale.  q and out are dtype (PA_BF16 or PA_F16); head_dim 128 or 256.  Groups of
+ * 8 or 16 query heads per kv head with block_size 16/32 run on tensor cores (the codes
+ * are converted exactly to f16 tiles in shared memory, q to f16, P is f16); other
+ * shapes on CUDA cores.  The cache is half the bytes of a 16-bit one.
  */
 int pa_decode_attention_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, const int32_t* seq_lens, float scale,
@@ -268,7 +272,12 @@ int pa_decode_attention_fp8(void* out, const void* q, const void* k_cache, const
  * partition_size / block_size logical blocks to the same physical blocks (what
  * pa_build_prefix_groups guarantees); prefix_parts[i] equals its chunk's parts.
  * A sequence never has its last token's partition computed by the group, so every
- * grouped sequence is finished by the merge kernel.  When the shape does not qualify
+ * grouped sequence is finished by the merge kernel.  first_part: the lowest partition
+ * any sequence computes itself, min over s of min(prefix_parts[s], (seq_lens[s]-1) /
+ * partition_size) (0 when any sequence has no group); the per-sequence kernel's grid
+ * starts there, so the partitions every group covers launch no CTAs at all.  A
+ * sequence whose own partitions start lower is reported (PA_DEVERR_GROUP) and those
+ * partitions are left out.  When the shape does not qualify
  * (f32 cache, block_size not 16/32, max_members * num_heads/num_kv_heads > 16, or a
  * single partition) the groups are ignored and the plain path runs.
  */
@@ -280,7 +289,8 @@ int pa_decode_attention_grouped(void* out, const void* q, const void* k_cache,
                                 int partition_size, int dtype, const int32_t* prefix_parts,
                                 const int32_t* chunk_members, const int32_t* chunk_parts,
                                 int num_chunks, int max_members, int max_chunk_parts,
-                                void* workspace, size_t workspace_bytes, pa_stream_t stream);
+                                int first_part, void* workspace, size_t workspace_bytes,
+                                pa_stream_t stream);
 
 /*
  * pa_device_error_read - synchronise the current device, then return (in *bits) and

@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "NO_FREE_BLOCKS", 3: "UNKNOWN_SEQ"
 PA_STATIC_WORKSPACE_BYTES = 16 << 20
 PA_F32, PA_BF16, PA_F16, PA_FP8_E4M3 = 0, 1, 2, 3
 DEVERR_SLOT, DEVERR_COPY_BLOCK, DEVERR_TABLE, DEVERR_SEQ_LEN, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
+DEVERR_GROUP = 32
 DEFAULT_PARTITION = 512
 
 
@@ -71,7 +72,8 @@ _sig("pa_decode_attention", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, 
 _sig("pa_decode_attention_static_ws", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32,
      _i32, _i32, _i64, _i32, _i32, _i32, _p)
 _sig("pa_decode_attention_grouped", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32,
-     _i32, _i32, _i64, _i32, _i32, _i32, _p, _p, _p, _i32, _i32, _i32, _p, ctypes.c_size_t, _p)
+     _i32, _i32, _i64, _i32, _i32, _i32, _p, _p, _p, _i32, _i32, _i32, _i32, _p,
+     ctypes.c_size_t, _p)
 _sig("pa_decode_uses_tensor_cores", _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_device_error_read", _i32, ctypes.POINTER(ctypes.c_uint32))
 _sig("pa_last_cuda_error", ctypes.c_char_p)
@@ -257,9 +259,10 @@ def pa_decode_attention_grouped(out, q, k_cache, v_cache, block_tables, seq_lens
                                 block_size, num_kv_heads, max_seq_len, prefix_parts,
                                 chunk_members, chunk_parts, num_chunks, max_chunk_parts,
                                 partition_size=DEFAULT_PARTITION, workspace=None,
-                                stream=None) -> None:
+                                stream=None, first_part=0) -> None:
     """pa_decode_attention with prefix groups (device int32 tensors prefix_parts [S],
-    chunk_members [>= num_chunks, max_members], chunk_parts [>= num_chunks])."""
+    chunk_members [>= num_chunks, max_members], chunk_parts [>= num_chunks]);
+    first_part as documented in pa.h (0 is always safe)."""
     import torch
     S, Hq, D = q.shape
     NB = k_cache.shape[0]
@@ -274,8 +277,8 @@ def pa_decode_attention_grouped(out, q, k_cache, v_cache, block_tables, seq_lens
         _dev(prefix_parts, "prefix_parts", torch.int32),
         _dev(chunk_members, "chunk_members", torch.int32),
         _dev(chunk_parts, "chunk_parts", torch.int32), int(num_chunks),
-        int(chunk_members.shape[1]), int(max_chunk_parts), ws_ptr, ws_bytes, _stream(stream)),
-        "pa_decode_attention_grouped")
+        int(chunk_members.shape[1]), int(max_chunk_parts), int(first_part), ws_ptr, ws_bytes,
+        _stream(stream)), "pa_decode_attention_grouped")
 
 
 def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, seq_lens, scale,

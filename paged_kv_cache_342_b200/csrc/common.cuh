@@ -37,6 +37,7 @@ struct DecodeParams {
   const int32_t* chunk_parts;    // [num_chunks] shared partitions of each chunk
   int max_members;
   float v_scale;  // output multiplier (the fp8 cache's V scale; 1 otherwise)
+  int part_base;  // partition index of grid z = 0 in the per-sequence kernels
 };
 
 // Device address of the library's error word on the current device.

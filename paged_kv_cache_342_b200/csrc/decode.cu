@@ -18,6 +18,7 @@ cudaError_t launch_decode_simt_f32(const DecodeParams& p, int gs, cudaStream_t s
 cudaError_t launch_decode_simt_bf16(const DecodeParams& p, int gs, cudaStream_t st);
 cudaError_t launch_decode_simt_f16(const DecodeParams& p, int gs, cudaStream_t st);
 cudaError_t launch_decode_simt_fp8(const DecodeParams& p, int q_dtype, int gs, cudaStream_t st);
+cudaError_t launch_decode_mma_fp8(const DecodeParams& p, int q_dtype, cudaStream_t st);
 cudaError_t launch_decode_mma_bf16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_group_bf16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
@@ -176,7 +177,7 @@ struct GroupArgs {
   const int32_t* prefix_parts;
   const int32_t* chunk_members;
   const int32_t* chunk_parts;
-  int num_chunks, max_members, max_chunk_parts;
+  int num_chunks, max_members, max_chunk_parts, first_part;
 };
 
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -240,15 +241,16 @@ extern "C" int pa_decode_attention_grouped(
     int num_kv_heads, int num_seqs, int num_heads, int head_dim, int max_blocks_per_seq,
     int64_t num_blocks, int max_seq_len, int partition_size, int dtype,
     const int32_t* prefix_parts, const int32_t* chunk_members, const int32_t* chunk_parts,
-    int num_chunks, int max_members, int max_chunk_parts, void* workspace,
+    int num_chunks, int max_members, int max_chunk_parts, int first_part, void* workspace,
     size_t workspace_bytes, pa_stream_t stream) {
-  if (num_chunks < 0 || max_chunk_parts < 0 || max_members < 1 || max_members > 16)
+  if (num_chunks < 0 || max_chunk_parts < 0 || max_members < 1 || max_members > 16 ||
+      first_part < 0)
     return PA_ERR_INVALID_ARG;
   if (num_chunks > 65535) return PA_ERR_INVALID_ARG;
   if (num_chunks > 0 && (!prefix_parts || !chunk_members || !chunk_parts))
     return PA_ERR_INVALID_ARG;
   const GroupArgs g{prefix_parts, chunk_members, chunk_parts, num_chunks, max_members,
-                    max_chunk_parts};
+                    max_chunk_parts, first_part};
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
                      num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
                      max_seq_len, partition_size, dtype, dtype, 1.f, 1.f, &g, workspace,
@@ -335,6 +337,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.chunk_members = groups->chunk_members;
     p.chunk_parts = groups->chunk_parts;
     p.max_members = groups->max_members;
+    // partitions below first_part belong to the groups for every sequence
+    p.part_base = groups->first_part < ws.parts - 1 ? groups->first_part : ws.parts - 1;
     const int zparts = groups->max_chunk_parts < ws.parts ? groups->max_chunk_parts : ws.parts;
     e = dtype == PA_BF16 ? launch_decode_group_bf16(p, groups->num_chunks, zparts, st)
                          : launch_decode_group_f16(p, groups->num_chunks, zparts, st);
@@ -343,7 +347,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
       return PA_ERR_CUDA;
     }
   }
-  if (fp8) {
+  if (fp8 && group % 8 == 0 && group <= 16 && (block_size == 16 || block_size == 32)) {
+    e = launch_decode_mma_fp8(p, dtype, st);
+  } else if (fp8) {
     e = launch_decode_simt_fp8(p, dtype, simt_heads_per_cta(group, head_dim), st);
   } else if (mma_eligible(dtype, group, head_dim, block_size)) {
     e = dtype == PA_BF16 ? launch_decode_mma_bf16(p, st) : launch_decode_mma_f16(p, st);

@@ -20,6 +20,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "decode_simt.cuh"  // checked_len
 
@@ -82,22 +84,42 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-template <typename T, int D, int BS, int NT, int NW, int NST>
+// FP8: the cache holds e4m3 codes; TMA lands them as 128-element x BS-row slabs and
+// the consuming warp converts them (exactly) into 16-bit tiles of its own.
+template <typename T, int D, int BS, int NT, int NW, int NST, bool FP8 = false>
 struct MmaCfg {
-  static constexpr int kHalves = D / 64;         // 128-byte column slabs per row
+  static constexpr int kHalves = D / 64;         // 128-byte column slabs per 16-bit row
   static constexpr int kSlabBytes = BS * 128;    // one slab of one tile
-  static constexpr int kTileBytes = kHalves * kSlabBytes;  // = BS * D * 2
-  static constexpr int kStageBytes = 2 * kTileBytes;       // K tile + V tile
+  static constexpr int kTileBytes = kHalves * kSlabBytes;  // 16-bit tile = BS * D * 2
+  static constexpr int kF8Slabs = D / 128;       // 128-byte slabs per fp8 row
+  static constexpr int kF8Tile = BS * D;         // fp8 tile bytes
+  static constexpr int kStageBytes = FP8 ? 2 * kF8Tile : 2 * kTileBytes;  // K + V as stored
+  static constexpr int kConvBytes = FP8 ? 2 * kTileBytes : 0;  // per-warp 16-bit K + V
   static constexpr int kTT = BS / 16;            // 16-token row tiles per block
   static constexpr int kKS = D / 16;             // k-steps of q.K / m-tiles of V^T
   static constexpr int kHeads = 8 * NT;
-  static constexpr int kStageArea = NW * NST * kStageBytes;
+  static constexpr int kStageArea = NW * NST * kStageBytes + NW * kConvBytes;
   static constexpr int kRedBytes = NW * kHeads * (D + 2) * 4;
   static constexpr int kSmemBytes =
       1024 + (kStageArea > kRedBytes ? kStageArea : kRedBytes) + NW * NST * 8;
-  static_assert(sizeof(T) == 2, "tensor-core path takes 16-bit caches");
+  static_assert(sizeof(T) == 2, "tensor-core path computes in 16-bit types");
   static_assert(BS % 16 == 0 && kSlabBytes % 1024 == 0, "slabs must stay 1024-byte aligned");
+  static_assert(!FP8 || D % 128 == 0, "fp8 tiles are whole 128-byte slabs");
 };
+
+// q (TQ pair) -> MMA operand pair (T): exact when the types agree
+template <typename T, typename TQ>
+__device__ __forceinline__ uint32_t q_pair(const TQ* qp) {
+  const uint32_t w = __ldg(reinterpret_cast<const unsigned int*>(qp));
+  if constexpr (std::is_same<T, TQ>::value) {
+    return w;
+  } else {
+    float lo, hi;
+    if constexpr (std::is_same<TQ, __nv_bfloat16>::value) bf16x2_to_float(w, lo, hi);
+    else h2_to_float(w, lo, hi);
+    return MmaOps<T>::pack(lo, hi);
+  }
+}
 
 // byte offset of (row r, 16-byte chunk c of the full row) inside a tile stored as
 // D/64 slabs of [BS rows][128 bytes] with the 128-byte swizzle (chunk ^= row % 8)
@@ -110,11 +132,13 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 // GROUP = true : one CTA per (kv head, chunk of a prefix group, shared partition);
 //   the tile's columns are (member, head) pairs, member = column / group, and the
 //   partition's blocks - identical for every member - are read once for all of them.
-template <typename T, int D, int BS, int NT, int NW, int NST, bool GROUP>
+// T = MMA operand type, TQ = query / output type, FP8 = e4m3 cache converted to T.
+template <typename T, typename TQ, int D, int BS, int NT, int NW, int NST, bool GROUP,
+          bool FP8>
 __global__ void __launch_bounds__(NW * 32)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
-  using C = MmaCfg<T, D, BS, NT, NW, NST>;
+  using C = MmaCfg<T, D, BS, NT, NW, NST, FP8>;
   using Ops = MmaOps<T>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int TT = C::kTT, KS = C::kKS;
@@ -135,11 +159,14 @@ __global__ void __launch_bounds__(NW * 32)
   if constexpr (!GROUP) {
     const int s = blockIdx.y;
     const int h0 = blockIdx.x * C::kHeads;
-    part = blockIdx.z;
+    part = p.part_base + blockIdx.z;
     kvh = h0 / G;
-    const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && part == 0);
+    const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0);
     nparts = L > 0 ? (L + ps - 1) / ps : 1;
-    if (part >= nparts || part < group_parts(p, s, L)) return;
+    const int own = group_parts(p, s, L);
+    if (blockIdx.z == 0 && own < p.part_base && threadIdx.x == 0 && blockIdx.x == 0)
+      set_error(p.err, PA_DEVERR_GROUP);
+    if (part >= nparts || part < own) return;
     tok_begin = part * ps;
     tok_end = min(L, tok_begin + ps);
     table_seq = s;
@@ -178,6 +205,8 @@ __global__ void __launch_bounds__(NW * 32)
       p.block_tables + static_cast<int64_t>(table_seq) * p.max_blocks_per_seq + tok_begin / BS;
 
   const uint32_t stage0 = base + warp * NST * C::kStageBytes;
+  // FP8: this warp's 16-bit K and V tiles (the stages hold the fp8 codes)
+  const uint32_t conv0 = base + NW * NST * C::kStageBytes + warp * C::kConvBytes;
   const uint32_t bar0 = base + (C::kSmemBytes - 1024 - NW * NST * 8) + warp * NST * 8;
   if (lane == 0) {
 #pragma unroll
@@ -192,12 +221,12 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int row = col_row[nt * 8 + g8];
-    const T* qp0 = static_cast<const T*>(p.q) + static_cast<int64_t>(row < 0 ? 0 : row) * D;
+    const TQ* qp0 = static_cast<const TQ*>(p.q) + static_cast<int64_t>(row < 0 ? 0 : row) * D;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
-      const T* qp = qp0 + ks * 16 + 2 * t4;
-      qb[nt][ks][0] = row < 0 ? 0u : __ldg(reinterpret_cast<const unsigned int*>(qp));
-      qb[nt][ks][1] = row < 0 ? 0u : __ldg(reinterpret_cast<const unsigned int*>(qp + 8));
+      const TQ* qp = qp0 + ks * 16 + 2 * t4;
+      qb[nt][ks][0] = row < 0 ? 0u : q_pair<T, TQ>(qp);
+      qb[nt][ks][1] = row < 0 ? 0u : q_pair<T, TQ>(qp + 8);
     }
   }
 
@@ -236,10 +265,18 @@ __global__ void __launch_bounds__(NW * 32)
         const uint32_t dst = stage0 + st * C::kStageBytes;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(bar, C::kStageBytes);
+        if constexpr (FP8) {
 #pragma unroll
-        for (int h = 0; h < C::kHalves; ++h) {
-          tma_load_2d(dst + h * C::kSlabBytes, &tmk, 64 * h, row0, bar);
-          tma_load_2d(dst + C::kTileBytes + h * C::kSlabBytes, &tmv, 64 * h, row0, bar);
+          for (int h = 0; h < C::kF8Slabs; ++h) {
+            tma_load_2d(dst + h * C::kSlabBytes, &tmk, 128 * h, row0, bar);
+            tma_load_2d(dst + C::kF8Tile + h * C::kSlabBytes, &tmv, 128 * h, row0, bar);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {
+            tma_load_2d(dst + h * C::kSlabBytes, &tmk, 64 * h, row0, bar);
+            tma_load_2d(dst + C::kTileBytes + h * C::kSlabBytes, &tmv, 64 * h, row0, bar);
+          }
         }
       } else {
         set_error(p.err, PA_DEVERR_TABLE);
@@ -261,9 +298,38 @@ __global__ void __launch_bounds__(NW * 32)
       break;
     }
     if (!((bad >> st) & 1u)) {
-      const uint32_t kt = stage0 + st * C::kStageBytes;
-      const uint32_t vt = kt + C::kTileBytes;
+      uint32_t kt = stage0 + st * C::kStageBytes;
+      uint32_t vt = kt + C::kTileBytes;
       const int valid = min(BS, tok_end - (tok_begin + (warp + k * NW) * BS));
+      if constexpr (FP8) {
+        // e4m3 -> 16-bit, exactly: 16 codes (one swizzled 16-byte chunk of a 128-byte
+        // slab row) become two 16-byte chunks of the 16-bit tile
+        const uint8_t* src = smem + (kt - base);
+        uint8_t* dst = smem + (conv0 - base);
+        constexpr int kChunks = BS * (D / 16);
+#pragma unroll 2
+        for (int i = lane; i < 2 * kChunks; i += 32) {
+          const int tv = i >= kChunks, j = i - tv * kChunks;
+          const int r = j / (D / 16), c = j % (D / 16);
+          const uint4 codes = *reinterpret_cast<const uint4*>(
+              src + tv * C::kF8Tile + (c >> 3) * C::kSlabBytes + r * 128 +
+              (((c & 7) ^ (r & 7)) << 4));
+          const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+          uint32_t h[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                static_cast<__nv_fp8x2_storage_t>(w[u >> 1] >> (16 * (u & 1))), __NV_E4M3);
+            h[u] = static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+          }
+          uint8_t* o = dst + tv * C::kTileBytes;
+          *reinterpret_cast<uint4*>(o + swz<BS>(r, 2 * c)) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(o + swz<BS>(r, 2 * c + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+        __syncwarp();
+        kt = conv0;
+        vt = conv0 + C::kTileBytes;
+      }
       if (valid < BS) {
         // zero the V rows past the end: 16 bytes per lane per step
         uint8_t* vg = smem + (vt - base);
@@ -420,7 +486,7 @@ __global__ void __launch_bounds__(NW * 32)
     if (!col_ok[hh]) continue;
     const int64_t row = col_row[hh];
     if (nparts == 1) {
-      store_elem(static_cast<T*>(p.out) + row * D + d, o);
+      store_elem(static_cast<TQ*>(p.out) + row * D + d, o);
     } else {
       const int64_t prow = row * p.max_parts + part;
       p.ws_o[prow * D + d] = o;

@@ -15,15 +15,17 @@ cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
   constexpr int kRaw = kBudget / (NW * kStage);
   constexpr int NST = kRaw < 2 ? 2 : (kRaw > 4 ? 4 : kRaw);
-  using C = MmaCfg<__half, D, BS, NT, NW, NST>;
+  using C = MmaCfg<__half, D, BS, NT, NW, NST, false>;
   const uint64_t rows = static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * BS;
   if (rows > 0x7fffffffull) return cudaErrorInvalidValue;  // int32 row coordinates
   CUtensorMap tmk, tmv;
   const bool bf16 = false;
-  if (!make_cache_tensor_map(&tmk, p.k_cache, rows, D, BS, bf16) ||
-      !make_cache_tensor_map(&tmv, p.v_cache, rows, D, BS, bf16))
+  const CUtensorMapDataType dt =
+      bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if (!make_cache_tensor_map(&tmk, p.k_cache, rows, D, BS, dt, 2) ||
+      !make_cache_tensor_map(&tmv, p.v_cache, rows, D, BS, dt, 2))
     return cudaErrorInvalidValue;
-  constexpr auto kern = decode_mma_kernel<__half, D, BS, NT, NW, NST, GROUP>;
+  constexpr auto kern = decode_mma_kernel<__half, __half, D, BS, NT, NW, NST, GROUP, false>;
   cudaError_t e = ensure_smem_limit<kern>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, NW * 32, C::kSmemBytes, st>>>(p, tmk, tmv);
@@ -57,7 +59,7 @@ cudaError_t by_shape(const DecodeParams& p, int nt, dim3 grid, cudaStream_t st) 
 // Per-sequence partitions: 8*NT query heads of one kv head per CTA (NT = group / 8).
 cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st) {
   const int nt = (p.num_heads / p.num_kv_heads) / 8;
-  dim3 grid(p.num_heads / (8 * nt), p.num_seqs, p.max_parts);
+  dim3 grid(p.num_heads / (8 * nt), p.num_seqs, p.max_parts - p.part_base);
   return by_shape<false>(p, nt, grid, st);
 }
 

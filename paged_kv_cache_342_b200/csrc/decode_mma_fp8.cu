@@ -1,0 +1,62 @@
+// Tensor-core decode partition kernels for fp8 (e4m3) caches with grouped-query
+// heads: the codes arrive by TMA and are converted exactly to f16 tiles in shared
+// memory; q (bf16 or f16) becomes f16 operands, P is f16, accumulators float32.
+#include "decode_mma.cuh"
+#include "tensor_map.cuh"
+
+namespace pa {
+namespace {
+
+template <typename TQ, int D, int BS, int NT>
+cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
+  // about 64 KiB per CTA: per warp NST fp8 stages plus one 16-bit K+V tile pair
+  constexpr int kStage = 2 * BS * D;      // fp8 K + V
+  constexpr int kConv = 2 * BS * D * 2;   // 16-bit K + V
+  constexpr int kBudget = 65536;
+  constexpr int kW = kBudget / (2 * kStage + kConv);
+  constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
+  constexpr int kRaw = (kBudget / NW - kConv) / kStage;
+  constexpr int NST = kRaw < 2 ? 2 : (kRaw > 4 ? 4 : kRaw);
+  using C = MmaCfg<__half, D, BS, NT, NW, NST, true>;
+  const uint64_t rows = static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * BS;
+  if (rows > 0x7fffffffull) return cudaErrorInvalidValue;  // int32 row coordinates
+  CUtensorMap tmk, tmv;
+  if (!make_cache_tensor_map(&tmk, p.k_cache, rows, D, BS, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
+      !make_cache_tensor_map(&tmv, p.v_cache, rows, D, BS, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
+    return cudaErrorInvalidValue;
+  constexpr auto kern = decode_mma_kernel<__half, TQ, D, BS, NT, NW, NST, false, true>;
+  cudaError_t e = ensure_smem_limit<kern>(C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.num_heads / C::kHeads, p.num_seqs, p.max_parts - p.part_base);
+  kern<<<grid, NW * 32, C::kSmemBytes, st>>>(p, tmk, tmv);
+  return cudaGetLastError();
+}
+
+template <typename TQ, int D, int NT>
+cudaError_t by_bs(const DecodeParams& p, cudaStream_t st) {
+  switch (p.block_size) {
+    case 16: return launch<TQ, D, 16, NT>(p, st);
+    case 32: return launch<TQ, D, 32, NT>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename TQ>
+cudaError_t by_shape(const DecodeParams& p, cudaStream_t st) {
+  const int nt = (p.num_heads / p.num_kv_heads) / 8;
+  switch (p.head_dim * 4 + nt) {
+    case 128 * 4 + 1: return by_bs<TQ, 128, 1>(p, st);
+    case 128 * 4 + 2: return by_bs<TQ, 128, 2>(p, st);
+    case 256 * 4 + 1: return by_bs<TQ, 256, 1>(p, st);
+    case 256 * 4 + 2: return by_bs<TQ, 256, 2>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_mma_fp8(const DecodeParams& p, int q_dtype, cudaStream_t st) {
+  return q_dtype == PA_BF16 ? by_shape<__nv_bfloat16>(p, st) : by_shape<__half>(p, st);
+}
+
+}  // namespace pa

@@ -91,14 +91,17 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane >> 3, sub = lane & 7;
-  const int s = blockIdx.y, part = blockIdx.z;
+  const int s = blockIdx.y, part = p.part_base + blockIdx.z;
   const int h0 = blockIdx.x * GS;
   const int kvh = h0 / (p.num_heads / p.num_kv_heads);
 
-  const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && part == 0);
+  const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0);
   const int ps = p.partition_size;
   const int nparts = L > 0 ? (L + ps - 1) / ps : 1;
-  if (part >= nparts || part < group_parts(p, s, L)) return;
+  const int own = group_parts(p, s, L);
+  if (blockIdx.z == 0 && own < p.part_base && threadIdx.x == 0 && blockIdx.x == 0)
+    set_error(p.err, PA_DEVERR_GROUP);
+  if (part >= nparts || part < own) return;
   const int tok_begin = part * ps;
   const int tok_end = min(L, tok_begin + ps);
   const int nblk = tok_end > tok_begin ? (tok_end - tok_begin + BS - 1) / BS : 0;
@@ -337,7 +340,7 @@ cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream) {
   constexpr auto kern = decode_simt_kernel<T, TQ, D, BS, GS, NW, NST>;
   cudaError_t attr = ensure_smem_limit<kern>(C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
-  dim3 grid(p.num_heads / GS, p.num_seqs, p.max_parts);
+  dim3 grid(p.num_heads / GS, p.num_seqs, p.max_parts - p.part_base);
   kern<<<grid, NW * 32, C::kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }

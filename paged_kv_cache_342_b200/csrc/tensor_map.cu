@@ -24,15 +24,15 @@ EncodeTiledFn encoder() {
 }  // namespace
 
 bool make_cache_tensor_map(CUtensorMap* map, const void* base, uint64_t rows, int head_dim,
-                           int block_size, bool bf16) {
+                           int block_size, CUtensorMapDataType dtype, int elem_bytes) {
   EncodeTiledFn enc = encoder();
-  if (!enc) return false;
+  if (!enc || elem_bytes <= 0 || 128 % elem_bytes) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), rows};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(block_size)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * elem_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes),
+                             static_cast<cuuint32_t>(block_size)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;

@@ -8,10 +8,10 @@
 
 namespace pa {
 
-// A cache tensor [rows = num_blocks*num_kv_heads*block_size, head_dim] of 16-bit
-// elements, loaded in boxes of 64 elements x block_size rows with the 128-byte
-// swizzle.  Returns false if the encoder is unavailable or rejects the shape.
+// A cache tensor [rows = num_blocks*num_kv_heads*block_size, head_dim] of
+// elem_bytes-byte elements, loaded in boxes of 128 bytes x block_size rows with the
+// 128-byte swizzle.  Returns false if the encoder is unavailable or rejects the shape.
 bool make_cache_tensor_map(CUtensorMap* map, const void* base, uint64_t rows, int head_dim,
-                           int block_size, bool bf16);
+                           int block_size, CUtensorMapDataType dtype, int elem_bytes);
 
 }  // namespace pa

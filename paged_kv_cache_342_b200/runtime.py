@@ -163,20 +163,25 @@ class PagedDecoder:
         _, lens = self.alloc.build_block_tables(self._seq_ids, self.max_blocks,
                                                 self.h_tables.numpy(), self.h_lens.numpy())
         max_len = int(lens.max()) if lens.size else 0
-        num_chunks = max_chunk_parts = 0
+        num_chunks = max_chunk_parts = first_part = 0
         if self.group_members > 0:
             hp, hm, hc = self.h_groups
-            _, members, _, max_chunk_parts = self.alloc.prefix_groups(
+            pp, members, _, max_chunk_parts = self.alloc.prefix_groups(
                 self._seq_ids, self.partition_size, self.group_members, hp.numpy(), hm.numpy(),
                 hc.numpy())
             num_chunks = len(members)
+            if num_chunks and lens.size:
+                # the lowest partition any sequence computes itself
+                own = np.minimum(pp, np.maximum(lens.astype(np.int64) - 1, 0) // self.partition_size)
+                first_part = int(own.min())
         s = self._torch_stream()
         with torch.cuda.stream(s):
             self.d_stage.copy_(self.h_stage, non_blocking=True)
             self._done = torch.cuda.Event()
             self._done.record(s)
         return dict(num_cow=n_cow, max_len=max_len, pairs=self.h_pairs.numpy()[:n_cow],
-                    num_chunks=num_chunks, max_chunk_parts=max_chunk_parts)
+                    num_chunks=num_chunks, max_chunk_parts=max_chunk_parts,
+                    first_part=first_part)
 
     def launch(self, meta: dict, q, new_k, new_v, out, events=None) -> None:
         """Device side of a step: copies, the new token's K/V, attention.  ``events``
@@ -203,7 +208,8 @@ class PagedDecoder:
             pa_decode_attention_grouped(
                 out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens, self.scale,
                 self.block_size, self.num_kv_heads, meta["max_len"], pp, cm, cp,
-                meta["num_chunks"], meta["max_chunk_parts"], self.partition_size, ws, stream=st)
+                meta["num_chunks"], meta["max_chunk_parts"], self.partition_size, ws, stream=st,
+                first_part=meta["first_part"])
         else:
             pa_decode_attention(out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
                                 self.scale, self.block_size, self.num_kv_heads, meta["max_len"],

@@ -189,11 +189,13 @@ def run_grouped_case(pa, dtype, Hq, Hkv, D, bs, ps, prefix_len, tails, group_siz
     wsb = pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps)
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
     out = torch.full((S, Hq, D), float("nan"), dtype=TORCH_DT[dtype], device="cuda")
+    own = [min(p_, (int(L) - 1) // ps) if L > 0 else 0 for p_, L in zip(pp, sl)]
+    first = min(own) if chunks else 0
     pa.pa_decode_attention_grouped(out, qd, kd, vd, td, ld, scale, bs, Hkv, max_len,
                                    torch.from_numpy(np.array(pp, np.int32)).cuda(),
                                    torch.from_numpy(cm).cuda(), torch.from_numpy(cp).cuda(),
                                    len(chunks), max([c[1] for c in chunks], default=0), ps,
-                                   ws if wsb else None)
+                                   ws if wsb else None, first_part=first)
     plain = torch.full_like(out, float("nan"))
     pa.pa_decode_attention(plain, qd, kd, vd, td, ld, scale, bs, Hkv, max_len, ps,
                            ws if wsb else None)
@@ -229,3 +231,29 @@ def test_grouped_call_uses_groups(pa):
     *_, chunks = run_grouped_case(pa, *GROUP_CASES[0])
     # 300-token prefix at block 16 = 18 full shared blocks = 288 tokens = 4 partitions of 64
     assert len(chunks) == 1 and chunks[0] == (list(range(8)), 4)
+
+
+def test_grouped_first_part_too_high_is_reported(pa):
+    """A first_part above a sequence's own first partition leaves a hole: reported."""
+    dtype, Hq, Hkv, D, bs, ps = "bf16", 4, 4, 128, 16, 64
+    from oracle.allocator import BlockManager
+    bm = BlockManager(64, bs)
+    bm.add(0, 300)
+    bm.fork(0, 1)
+    bm.add(2, 100)                     # no group: computes from partition 0
+    rows, sl = bm.block_tables([0, 1, 2], 24)
+    pp, chunks = bm.prefix_groups([0, 1, 2], ps, 8)
+    k = to_dev(normal_fill((64, Hkv, bs, D), dtype, 1.0, 2, 1), dtype)
+    q = to_dev(normal_fill((3, Hq, D), dtype, 1.0, 2, 2), dtype)
+    cm = np.full((1, 8), -1, np.int32)
+    cm[0, :2] = chunks[0][0]
+    out = torch.empty((3, Hq, D), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(pa.pa_decode_workspace_bytes(3, Hq, D, 300, ps), dtype=torch.uint8,
+                     device="cuda")
+    pa.pa_decode_attention_grouped(out, q, k, k, torch.tensor(rows, dtype=torch.int32).cuda(),
+                                   torch.tensor(sl, dtype=torch.int32).cuda(), 0.1, bs, Hkv, 300,
+                                   torch.tensor(pp, dtype=torch.int32).cuda(),
+                                   torch.from_numpy(cm).cuda(),
+                                   torch.tensor([chunks[0][1]], dtype=torch.int32).cuda(), 1,
+                                   chunks[0][1], ps, ws, first_part=2)
+    assert pa.pa_device_error_read() == pa.DEVERR_GROUP

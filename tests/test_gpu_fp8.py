@@ -54,7 +54,10 @@ FP8_CASES = [
     # q dtype, Hq, Hkv, D, bs, partition, lens
     ("bf16", 4, 4, 128, 16, 64, (1, 15, 16, 17, 200, 333, 0)),
     ("f16", 8, 2, 128, 8, 32, (5, 64, 65, 400)),          # group 4
-    ("bf16", 16, 2, 128, 16, 512, (1, 700, 33)),           # group 8 (CUDA cores for fp8)
+    ("bf16", 16, 2, 128, 16, 512, (1, 700, 33)),           # group 8: tensor cores
+    ("f16", 16, 2, 128, 32, 128, (1, 300, 64, 0)),         # tensor cores, block 32
+    ("bf16", 32, 2, 256, 16, 64, (5, 200, 129)),           # group 16, head_dim 256
+    ("f16", 8, 2, 128, 16, 64, (9, 90)),                   # group 4: CUDA cores
     ("f16", 2, 2, 256, 32, 64, (3, 100, 250)),
     ("bf16", 4, 4, 128, 4, 16, (7, 18, 10)),
 ]
