@@ -8,6 +8,7 @@
 // pages in order" and "Measure memory use across requests" (the attention equation
 // is unchanged by paging).
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "decode_simt.cuh"
@@ -173,6 +174,28 @@ bool group_eligible(int dtype, int group, int head_dim, int block_size, int max_
          (block_size == 16 || block_size == 32);
 }
 
+// A side stream per device for the group kernel, so that it runs beside the
+// per-sequence kernel (they write disjoint partitions); fork and join through events.
+struct SideStream {
+  std::mutex mu;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+SideStream g_side[64];
+
+cudaError_t side_stream(int dev, SideStream** out) {
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  SideStream& s = g_side[dev];
+  if (!s.stream) {
+    cudaError_t e = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  }
+  *out = &s;
+  return cudaSuccess;
+}
+
 struct GroupArgs {
   const int32_t* prefix_parts;
   const int32_t* chunk_members;
@@ -329,6 +352,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
+  SideStream* joined = nullptr;              // the group kernel to wait for
+  std::unique_lock<std::mutex> side_lock;
   // shared partitions of prefix groups first (only useful when sequences span
   // several partitions); otherwise the per-sequence kernels do everything
   if (!fp8 && groups && groups->num_chunks > 0 && groups->max_chunk_parts > 0 && ws.parts > 1 &&
@@ -340,12 +365,28 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     // partitions below first_part belong to the groups for every sequence
     p.part_base = groups->first_part < ws.parts - 1 ? groups->first_part : ws.parts - 1;
     const int zparts = groups->max_chunk_parts < ws.parts ? groups->max_chunk_parts : ws.parts;
-    e = dtype == PA_BF16 ? launch_decode_group_bf16(p, groups->num_chunks, zparts, st)
-                         : launch_decode_group_f16(p, groups->num_chunks, zparts, st);
+    int dev = 0;
+    SideStream* side = nullptr;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = side_stream(dev, &side);
     if (e != cudaSuccess) {
       note_cuda_error(e);
       return PA_ERR_CUDA;
     }
+    // the group kernel runs on the side stream while the caller's stream goes on to
+    // the per-sequence kernel; the caller's stream waits for it before the merge
+    side_lock = std::unique_lock<std::mutex>(side->mu);
+    e = cudaEventRecord(side->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+    if (e == cudaSuccess)
+      e = dtype == PA_BF16 ? launch_decode_group_bf16(p, groups->num_chunks, zparts, side->stream)
+                           : launch_decode_group_f16(p, groups->num_chunks, zparts, side->stream);
+    if (e == cudaSuccess) e = cudaEventRecord(side->join, side->stream);
+    if (e != cudaSuccess) {
+      note_cuda_error(e);
+      return PA_ERR_CUDA;
+    }
+    joined = side;
   }
   if (fp8 && group % 8 == 0 && group <= 16 && (block_size == 16 || block_size == 32)) {
     e = launch_decode_mma_fp8(p, dtype, st);
@@ -359,6 +400,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
         : dtype == PA_BF16 ? launch_decode_simt_bf16(p, gs, st)
                            : launch_decode_simt_f16(p, gs, st);
   }
+  if (e == cudaSuccess && joined) e = cudaStreamWaitEvent(st, joined->join, 0);
+  if (side_lock.owns_lock()) side_lock.unlock();
   if (e != cudaSuccess) {
     note_cuda_error(e);
     return PA_ERR_CUDA;

@@ -12,7 +12,7 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
   // about 64 KiB per CTA: per warp NST fp8 stages plus one 16-bit K+V tile pair
   constexpr int kStage = 2 * BS * D;      // fp8 K + V
   constexpr int kConv = 2 * BS * D * 2;   // 16-bit K + V
-  constexpr int kBudget = 65536;
+  constexpr int kBudget = 32768;  // small stages: more CTAs per SM hide the conversion latency
   constexpr int kW = kBudget / (2 * kStage + kConv);
   constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
   constexpr int kRaw = (kBudget / NW - kConv) / kStage;

@@ -9,7 +9,7 @@ namespace {
 template <typename TQ, int D, int BS, int GS>
 cudaError_t launch_auto(const DecodeParams& p, cudaStream_t st) {
   constexpr int kStage = 2 * BS * D;  // one byte per element
-  constexpr int kBudget = 65536;
+  constexpr int kBudget = 32768;  // small stages: more CTAs per SM hide the conversion latency
   constexpr int kW = kBudget / (2 * kStage);
   constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
   constexpr int kRaw = kBudget / (NW * kStage);
