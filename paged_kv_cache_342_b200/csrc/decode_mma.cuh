@@ -302,29 +302,36 @@ __global__ void __launch_bounds__(NW * 32)
       uint32_t vt = kt + C::kTileBytes;
       const int valid = min(BS, tok_end - (tok_begin + (warp + k * NW) * BS));
       if constexpr (FP8) {
-        // e4m3 -> 16-bit, exactly: 16 codes (one swizzled 16-byte chunk of a 128-byte
-        // slab row) become two 16-byte chunks of the 16-bit tile
-        const uint8_t* src = smem + (kt - base);
+        // e4m3 -> f16, exactly.  Lane = one 16-byte column chunk c of the fp8 rows
+        // (16 codes) in rows r0, r0 + RPP, ...: a quarter warp reads one 128-byte slab
+        // row; each chunk becomes f16 chunks 2c and 2c+1, stored in an order that
+        // puts the two halves of a quarter warp on different banks.
+        constexpr int CPR = D / 16;          // fp8 chunks per row
+        constexpr int RPP = 32 / CPR;        // rows per pass
+        const int c = lane % CPR, r0 = lane / CPR;
+        const int first = (c & 4) ? 1 : 0;   // store order of the two f16 chunks
+        const uint8_t* src = smem + (kt - base) + (c >> 3) * C::kSlabBytes;
         uint8_t* dst = smem + (conv0 - base);
-        constexpr int kChunks = BS * (D / 16);
-#pragma unroll 2
-        for (int i = lane; i < 2 * kChunks; i += 32) {
-          const int tv = i >= kChunks, j = i - tv * kChunks;
-          const int r = j / (D / 16), c = j % (D / 16);
-          const uint4 codes = *reinterpret_cast<const uint4*>(
-              src + tv * C::kF8Tile + (c >> 3) * C::kSlabBytes + r * 128 +
-              (((c & 7) ^ (r & 7)) << 4));
-          const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
-          uint32_t h[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
-                static_cast<__nv_fp8x2_storage_t>(w[u >> 1] >> (16 * (u & 1))), __NV_E4M3);
-            h[u] = static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+        for (int tv = 0; tv < 2; ++tv) {
+#pragma unroll
+          for (int r = r0; r < BS; r += RPP) {
+            const uint4 codes = *reinterpret_cast<const uint4*>(
+                src + tv * C::kF8Tile + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+            const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+            uint32_t h[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                  static_cast<__nv_fp8x2_storage_t>(w[u >> 1] >> (16 * (u & 1))), __NV_E4M3);
+              h[u] = *reinterpret_cast<const uint32_t*>(&hr);
+            }
+            uint8_t* o = dst + tv * C::kTileBytes;
+            const uint4 lo = make_uint4(h[0], h[1], h[2], h[3]);
+            const uint4 hi = make_uint4(h[4], h[5], h[6], h[7]);
+            *reinterpret_cast<uint4*>(o + swz<BS>(r, 2 * c + first)) = first ? hi : lo;
+            *reinterpret_cast<uint4*>(o + swz<BS>(r, 2 * c + 1 - first)) = first ? lo : hi;
           }
-          uint8_t* o = dst + tv * C::kTileBytes;
-          *reinterpret_cast<uint4*>(o + swz<BS>(r, 2 * c)) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(o + swz<BS>(r, 2 * c + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
         }
         __syncwarp();
         kt = conv0;
