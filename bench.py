@@ -56,6 +56,8 @@ def parse():
                     help="override the block size (pool keeps the same number of slots)")
     ap.add_argument("--measure", default="decode", choices=["decode", "swap"],
                     help="swap: time swapping half the batch to a pinned host pool and back")
+    ap.add_argument("--partition-size", type=int, default=None,
+                    help="override the partition size of the decode split")
     ap.add_argument("--cache-fp8", action="store_true",
                     help="store K/V as fp8 e4m3 with per-tensor scales (q/out keep the dtype)")
     return ap.parse_args()
@@ -617,6 +619,8 @@ def main():
         cfg = cfg.with_(num_seqs=args.seqs, name=f"{cfg.name}_s{args.seqs}")
     if args.pool_blocks is not None:
         cfg = cfg.with_(num_blocks=args.pool_blocks, name=f"{cfg.name}_nb{args.pool_blocks}")
+    if args.partition_size is not None and args.partition_size != cfg.partition_size:
+        cfg = cfg.with_(partition_size=args.partition_size, name=f"{cfg.name}_ps{args.partition_size}")
     if args.block_size is not None and args.block_size != cfg.block_size:
         slots = cfg.num_blocks * cfg.block_size
         cfg = cfg.with_(block_size=args.block_size, num_blocks=slots // args.block_size,

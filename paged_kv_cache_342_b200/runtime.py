@@ -62,7 +62,6 @@ class PagedDecoder:
         self.alloc = BlockAllocator(self.num_blocks, self.block_size, free_order)
         self._seq_ids = None
         self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
-        self._done = None  # event: the last staging copy has been consumed
         group = num_heads // self.num_kv_heads
         self.fp8 = k_cache.element_size() == 1
         if self.fp8 and kv_scales is None:
@@ -118,8 +117,15 @@ class PagedDecoder:
         for name, n in sizes:
             offs[name] = total
             total += _align(n)
-        self.h_stage = torch.empty(total, dtype=torch.uint8, pin_memory=True)
-        self.d_stage = torch.empty(total, dtype=torch.uint8, device=self.device)
+        # two staging sets: step k fills set k % 2 while step k - 1's kernels still
+        # read the other one; the copy runs on its own stream
+        self._h_bufs = [torch.empty(total, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+        self._d_bufs = [torch.empty(total, dtype=torch.uint8, device=self.device)
+                        for _ in range(2)]
+        self._copy_stream = torch.cuda.Stream(device=self.device)
+        self._h2d_done = [None, None]       # the set's host buffer may be rewritten
+        self._kernels_done = [None, None]   # the set's device buffer may be overwritten
+        self._set = 1
 
         def views(buf):
             def sec(name, n, dt):
@@ -133,17 +139,24 @@ class PagedDecoder:
                 cmembers=sec("cmembers", 4 * S1 * MM, torch.int32).view(S1, MM),
                 cparts=sec("cparts", 4 * S1, torch.int32))
 
-        h, d = views(self.h_stage), views(self.d_stage)
+        self._views = [(views(self._h_bufs[i]), views(self._d_bufs[i])) for i in range(2)]
+        self._use_set(0)
+        cap = MB * self.block_size
+        ws = pa_decode_workspace_bytes(S, self.num_heads, self.head_dim, cap, self.partition_size)
+        if ws > self._ws.numel():
+            self._ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
+
+    def _use_set(self, i: int) -> None:
+        """Point the h_* / d_* views at staging set i."""
+        self._set = i
+        h, d = self._views[i]
+        self.h_stage, self.d_stage = self._h_bufs[i], self._d_bufs[i]
         self.h_slots, self.h_pairs, self.h_lens, self.h_tables = (h["slots"], h["pairs"],
                                                                   h["lens"], h["tables"])
         self.d_slots, self.d_pairs, self.d_lens, self.d_tables = (d["slots"], d["pairs"],
                                                                   d["lens"], d["tables"])
         self.h_groups = (h["pparts"], h["cmembers"], h["cparts"])
         self.d_groups = (d["pparts"], d["cmembers"], d["cparts"])
-        cap = MB * self.block_size
-        ws = pa_decode_workspace_bytes(S, self.num_heads, self.head_dim, cap, self.partition_size)
-        if ws > self._ws.numel():
-            self._ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
 
     @property
     def staging_bytes(self) -> int:
@@ -151,9 +164,12 @@ class PagedDecoder:
 
     def prepare(self) -> dict:
         """Host side of a step: slots and copies from the block manager, tables and
-        lengths, all staged and sent to the device in one copy."""
-        if self._done is not None:
-            self._done.synchronize()  # the staging buffer is free again
+        lengths, all staged and sent to the device in one copy (on the copy stream;
+        the compute stream waits for it)."""
+        i = self._set ^ 1 if self._stepped else 0
+        if self._h2d_done[i] is not None:
+            self._h2d_done[i].synchronize()  # that set's host buffer is free again
+        self._use_set(i)
         if self.rolling and self._stepped:
             self.alloc.truncate(self._seq_ids, self.base_lens)
         slots, pairs = self.alloc.append_slots(self._seq_ids, self.h_slots.numpy(),
@@ -174,11 +190,15 @@ class PagedDecoder:
                 # the lowest partition any sequence computes itself
                 own = np.minimum(pp, np.maximum(lens.astype(np.int64) - 1, 0) // self.partition_size)
                 first_part = int(own.min())
-        s = self._torch_stream()
-        with torch.cuda.stream(s):
+        comp, cs = self._torch_stream(), self._copy_stream
+        if self._kernels_done[i] is not None:
+            cs.wait_event(self._kernels_done[i])   # kernels two steps back read it
+        with torch.cuda.stream(cs):
             self.d_stage.copy_(self.h_stage, non_blocking=True)
-            self._done = torch.cuda.Event()
-            self._done.record(s)
+            done = torch.cuda.Event()
+            done.record(cs)
+        self._h2d_done[i] = done
+        comp.wait_event(done)
         return dict(num_cow=n_cow, max_len=max_len, pairs=self.h_pairs.numpy()[:n_cow],
                     num_chunks=num_chunks, max_chunk_parts=max_chunk_parts,
                     first_part=first_part)
@@ -216,6 +236,9 @@ class PagedDecoder:
                                 self.partition_size, ws, stream=st)
         if events is not None:
             events[1].record(st)
+        done = torch.cuda.Event()
+        done.record(st)
+        self._kernels_done[self._set] = done
 
     def step(self, q, new_k, new_v, out) -> dict:
         meta = self.prepare()
