@@ -480,7 +480,9 @@ def run_ours(args, cfg):
             "config": {"workload": cfg.name, "description": cfg.description,
                        "num_seqs": S, "num_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
                        "block_size": bs, "num_blocks": cfg.num_blocks,
-                       "partition_size": cfg.partition_size,
+                       "partition_size": dec.partition_size,
+                       "partition_rule": ("pa_decode_partition_size" if cfg.partition_size == 0
+                                          else "fixed"),
                        "mean_seq_len": round(float(lens.mean()), 1),
                        "max_seq_len": int(lens.max()),
                        "l2": "inputs larger than L2 (K/V pool %.2f GB per rank), no flush"

@@ -159,6 +159,28 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int 
                                  int partition_size);
 
 /*
+ * pa_decode_partition_size - a partition size for pa_decode_attention chosen from the
+ * shape of its grid.  Host only; no GPU work.  (The pages fix no partitioning; the
+ * split of long sequences and its size are this library's.)
+ *   cache_dtype   PA_F32 / PA_BF16 / PA_F16, or PA_FP8_E4M3 for the fp8 entry point
+ *   num_seqs, num_heads, num_kv_heads, head_dim, block_size   as for the decode call
+ *   max_seq_len   the max_seq_len the decode call will be given
+ *   num_sms       SMs of the GPU; 0 = ask the current device
+ * Starting at 512 tokens, the size doubles while the partition grid keeps at least
+ * 12 CTAs per SM (four waves of the three ~64 KiB CTAs an SM holds) that have tokens
+ * to read, counting a sequence's partitions as if its length were spread uniformly
+ * up to max_seq_len ((P + 1) / 2 of P partitions working) and stopping once one
+ * partition covers max_seq_len.  Fewer, longer partitions write and merge less
+ * partial state; enough CTAs keep every SM streaming.  The result is a power of two
+ * times 512 (a multiple of every supported block size) and >= 512.  It does not
+ * consider prefix groups, whose shared partitions want partitions shorter than the
+ * shared prefix (pa_decode_attention_grouped).  Returns 0 for invalid arguments or
+ * when num_sms is 0 and no device can be queried.
+ */
+int pa_decode_partition_size(int cache_dtype, int num_seqs, int num_heads, int num_kv_heads,
+                             int head_dim, int block_size, int max_seq_len, int num_sms);
+
+/*
  * pa_decode_attention - single-query (decode) attention over the paged cache.
  * ([BLOG] "The attention kernel has to read scattered blocks"; [LAB] "Keep pages in
  * order" and "Measure memory use across requests": the attention equation is

@@ -67,6 +67,7 @@ _sig("pa_decode_attention_fp8", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i
      _i32, _i64, _i32, _i32, _i32, _f, _f, _p, ctypes.c_size_t, _p)
 _sig("pa_swap_blocks", _i32, _p, _p, _i64, _p, _p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _p)
 _sig("pa_decode_workspace_bytes", ctypes.c_size_t, _i32, _i32, _i32, _i32, _i32)
+_sig("pa_decode_partition_size", _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode_attention", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32, _i32,
      _i32, _i64, _i32, _i32, _i32, _p, ctypes.c_size_t, _p)
 _sig("pa_decode_attention_static_ws", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32, _i32, _i32,
@@ -233,6 +234,13 @@ def pa_decode_workspace_bytes(num_seqs, num_heads, head_dim, max_seq_len,
                               partition_size=DEFAULT_PARTITION) -> int:
     return int(lib.pa_decode_workspace_bytes(num_seqs, num_heads, head_dim, max_seq_len,
                                              partition_size))
+
+
+def pa_decode_partition_size(cache_dtype_code, num_seqs, num_heads, num_kv_heads, head_dim,
+                             block_size, max_seq_len, num_sms=0) -> int:
+    """The library's partition size for this decode grid (0 = invalid arguments)."""
+    return int(lib.pa_decode_partition_size(cache_dtype_code, num_seqs, num_heads, num_kv_heads,
+                                            head_dim, block_size, int(max_seq_len), num_sms))
 
 
 def pa_decode_attention(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,

@@ -167,6 +167,26 @@ bool mma_eligible(int dtype, int group, int head_dim, int block_size) {
          (block_size == 16 || block_size == 32);
 }
 
+bool mma_fp8_eligible(int group, int block_size) {
+  return group % 8 == 0 && group <= 16 && (block_size == 16 || block_size == 32);
+}
+
+// CTAs along the head axis of one sequence's partition grid, for the kernel that
+// serves the shape: one per kv head on the tensor-core paths (all of a group's query
+// heads are the columns of one tile), one per heads_per_cta query heads otherwise.
+int64_t head_ctas(int cache_dtype, int num_heads, int num_kv_heads, int head_dim,
+                  int block_size) {
+  const int group = num_heads / num_kv_heads;
+  const bool tc = cache_dtype == PA_FP8_E4M3 ? mma_fp8_eligible(group, block_size)
+                                             : mma_eligible(cache_dtype, group, head_dim,
+                                                            block_size);
+  return tc ? num_kv_heads : num_heads / simt_heads_per_cta(group, head_dim);
+}
+
+// The partition kernels are sized to about 64 KiB of shared memory per CTA, so three
+// are resident per SM; the automatic partition size aims at four waves of those.
+constexpr int kAutoCtasPerSm = 3 * 4;
+
 // The group kernel is the tensor-core kernel with (member, head) columns.
 bool group_eligible(int dtype, int group, int head_dim, int block_size, int max_members) {
   return (dtype == PA_BF16 || dtype == PA_F16) && max_members >= 1 &&
@@ -221,6 +241,44 @@ extern "C" int pa_decode_uses_tensor_cores(int dtype, int num_heads, int num_kv_
                                            int head_dim, int block_size) {
   if (num_kv_heads <= 0 || num_heads <= 0 || num_heads % num_kv_heads) return 0;
   return mma_eligible(dtype, num_heads / num_kv_heads, head_dim, block_size) ? 1 : 0;
+}
+
+extern "C" int pa_decode_partition_size(int cache_dtype, int num_seqs, int num_heads,
+                                        int num_kv_heads, int head_dim, int block_size,
+                                        int max_seq_len, int num_sms) {
+  if (cache_dtype != PA_F32 && cache_dtype != PA_BF16 && cache_dtype != PA_F16 &&
+      cache_dtype != PA_FP8_E4M3)
+    return 0;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads ||
+      head_dim <= 0 || max_seq_len < 0 || num_sms < 0)
+    return 0;
+  if (block_size != 4 && block_size != 8 && block_size != 16 && block_size != 32) return 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess || num_sms <= 0) {
+      note_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidDevice);
+      return 0;
+    }
+  }
+  const int64_t rows =
+      static_cast<int64_t>(num_seqs) * head_ctas(cache_dtype, num_heads, num_kv_heads,
+                                                 head_dim, block_size);
+  const int64_t target = static_cast<int64_t>(kAutoCtasPerSm) * num_sms;
+  // Double the partition from the default while the grid keeps enough working CTAs.
+  // With P > 1 partitions a sequence of uniformly spread length works in (P + 1) / 2
+  // of them on average; with one partition every CTA works.  The estimate only falls
+  // as the partition grows, so the first size below the target ends the search.
+  int64_t best = kDefaultPartition;
+  for (int64_t ps = kDefaultPartition; ps <= (int64_t{1} << 30); ps *= 2) {
+    const int64_t parts = (max_seq_len + ps - 1) / ps;
+    const int64_t working = parts <= 1 ? rows : rows * (parts + 1) / 2;
+    if (working < target) break;
+    best = ps;
+    if (parts <= 1) break;
+  }
+  return static_cast<int>(best);
 }
 
 extern "C" size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
@@ -388,7 +446,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     }
     joined = side;
   }
-  if (fp8 && group % 8 == 0 && group <= 16 && (block_size == 16 || block_size == 32)) {
+  if (fp8 && mma_fp8_eligible(group, block_size)) {
     e = launch_decode_mma_fp8(p, dtype, st);
   } else if (fp8) {
     e = launch_decode_simt_fp8(p, dtype, simt_heads_per_cta(group, head_dim), st);

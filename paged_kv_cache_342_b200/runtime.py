@@ -33,9 +33,10 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (DEFAULT_PARTITION, BlockAllocator, pa_copy_blocks, pa_decode_attention,
-               pa_decode_attention_fp8, pa_decode_attention_grouped, pa_decode_workspace_bytes,
-               pa_reshape_and_cache, pa_reshape_and_cache_fp8)
+from . import (DEFAULT_PARTITION, BlockAllocator, _dtype_code, pa_copy_blocks,
+               pa_decode_attention, pa_decode_attention_fp8, pa_decode_attention_grouped,
+               pa_decode_partition_size, pa_decode_workspace_bytes, pa_reshape_and_cache,
+               pa_reshape_and_cache_fp8)
 
 
 def _align(n: int, a: int = 256) -> int:
@@ -47,6 +48,9 @@ class PagedDecoder:
 
     ``k_cache``/``v_cache`` are caller-owned CUDA tensors [NB, Hkv, bs, D].
     ``max_blocks_per_seq`` is the block-table width (capacity per sequence).
+    ``partition_size`` 0 takes ``pa_decode_partition_size`` for the bound batch at
+    that capacity (resolved by ``bind``; it ignores prefix groups, so batches of
+    forks do better with an explicit size shorter than their shared prefix).
     """
 
     def __init__(self, k_cache, v_cache, num_heads: int, scale: float, max_blocks_per_seq: int,
@@ -56,7 +60,8 @@ class PagedDecoder:
         self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim = k_cache.shape
         self.num_heads, self.scale = num_heads, scale
         self.max_blocks = max_blocks_per_seq
-        self.partition_size = partition_size
+        self._partition_arg = partition_size
+        self.partition_size = partition_size or DEFAULT_PARTITION
         self.device = k_cache.device
         self.stream = stream
         self.alloc = BlockAllocator(self.num_blocks, self.block_size, free_order)
@@ -142,6 +147,12 @@ class PagedDecoder:
         self._views = [(views(self._h_bufs[i]), views(self._d_bufs[i])) for i in range(2)]
         self._use_set(0)
         cap = MB * self.block_size
+        if self._partition_arg == 0:
+            ps = pa_decode_partition_size(_dtype_code(self.k_cache), S, self.num_heads, self.num_kv_heads,
+                                          self.head_dim, self.block_size, cap)
+            if ps <= 0:
+                raise RuntimeError("pa_decode_partition_size rejected the bound batch")
+            self.partition_size = ps
         ws = pa_decode_workspace_bytes(S, self.num_heads, self.head_dim, cap, self.partition_size)
         if ws > self._ws.numel():
             self._ws = torch.empty(ws, dtype=torch.uint8, device=self.device)

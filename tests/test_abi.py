@@ -64,6 +64,36 @@ def test_tensor_core_path_selection(pa):
     assert not pa.pa_decode_uses_tensor_cores(pa.PA_BF16, 64, 8, 128, 8)     # block 8
 
 
+def test_partition_size_choice(pa):
+    ps = pa.pa_decode_partition_size
+    # 7B-shaped: 64 seqs x 32 CUDA-core CTAs = 2048 >= 12 x 148, so one partition covers
+    # the longest sequence (512 -> 5, 1024 -> 3, 2048 -> 2, 4096 -> 1 partitions)
+    assert ps(pa.PA_BF16, 64, 32, 32, 128, 16, 2050, 148) == 4096
+    # 13B-shaped: 256 x 40 CTAs, longest 4097 tokens
+    assert ps(pa.PA_F16, 256, 40, 40, 128, 16, 4097, 148) == 8192
+    # GQA 8:1 on tensor cores: 8 seqs x 8 kv-head CTAs; at 2048 tokens 65 partitions
+    # give 64 * 33 = 2112 working CTAs (>= 1776), at 4096 only 64 * 17 = 1088
+    assert ps(pa.PA_BF16, 8, 64, 8, 128, 16, 131073, 148) == 2048
+    assert ps(pa.PA_FP8_E4M3, 8, 64, 8, 128, 16, 131073, 148) == 2048
+    # the same shape on CUDA cores (block 8): 8 seqs x 64/4 CTAs = 128 rows
+    assert ps(pa.PA_BF16, 8, 64, 8, 128, 8, 131073, 148) == 4096     # 128 * 17 = 2176
+    # too few CTAs even at the default size: stay at 512
+    assert ps(pa.PA_F32, 1, 8, 8, 64, 4, 100, 148) == 512
+    assert ps(pa.PA_F32, 5, 4, 4, 64, 4, 0, 148) == 512
+    # a single SM wants no split at all
+    assert ps(pa.PA_BF16, 8, 64, 8, 128, 16, 131073, 1) == 262144
+    # more SMs never give a longer partition
+    sizes = [ps(pa.PA_BF16, 16, 32, 8, 128, 16, 65536, n) for n in (1, 16, 74, 148, 296)]
+    assert sizes == sorted(sizes, reverse=True)
+    assert all(s >= 512 and s % 512 == 0 and (s & (s - 1)) == 0 for s in sizes)
+    # invalid arguments
+    assert ps(9, 8, 64, 8, 128, 16, 1000, 148) == 0
+    assert ps(pa.PA_BF16, 8, 64, 6, 128, 16, 1000, 148) == 0
+    assert ps(pa.PA_BF16, 8, 64, 8, 128, 12, 1000, 148) == 0
+    assert ps(pa.PA_BF16, -1, 64, 8, 128, 16, 1000, 148) == 0
+    assert ps(pa.PA_BF16, 8, 64, 8, 128, 16, 1000, -2) == 0
+
+
 FAKE = 1 << 20  # an aligned, never-dereferenced pointer value: every call below fails
                 # its host-side checks before any launch
 

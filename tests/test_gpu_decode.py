@@ -108,6 +108,19 @@ def test_partition_size_does_not_change_the_result(pa, tc):
         assert np.abs(o - outs[0]).max() <= 2e-2
 
 
+@pytest.mark.parametrize("dtype,Hq,Hkv,bs", [("bf16", 16, 2, 16), ("f16", 4, 4, 16),
+                                          ("f32", 8, 2, 8)])
+def test_library_partition_choice_matches_the_oracle(pa, dtype, Hq, Hkv, bs):
+    lens = (3000, 1, 1500, 2049, 700)
+    # the device's own choice, and the choices for smaller machines (longer partitions)
+    sizes = {pa.pa_decode_partition_size(PA_CODE[dtype], len(lens), Hq, Hkv, 128, bs,
+                                         max(lens), n) for n in (0, 1, 2)}
+    assert 0 not in sizes
+    for ps in sorted(sizes):
+        got, want = run_case(pa, dtype, Hq, Hkv, 128, bs, ps, lens, seed=8)
+        assert_close(got, want, dtype, f"partition {ps}")
+
+
 def test_all_empty_sequences_give_zeros(pa):
     got, _ = run_case(pa, "bf16", 4, 4, 128, 16, 512, (0, 0, 0))
     assert np.array_equal(got, np.zeros_like(got))

@@ -104,7 +104,7 @@ class DecodeConfig:
     scale: float
     std: float
     lens: tuple
-    partition_size: int = 512
+    partition_size: int = 512     # 0: the library's choice for the batch
     description: str = ""
 
     @property
@@ -131,13 +131,13 @@ CONFIGS: dict[str, DecodeConfig] = {
     "7b_bf16": DecodeConfig(
         name="7b_bf16", num_seqs=64, num_heads=32, num_kv_heads=32, head_dim=128,
         block_size=16, num_blocks=8192, dtype="bf16", scale=1.0 / math.sqrt(128.0), std=1.0,
-        lens=("uniform", 128, 2048),
+        lens=("uniform", 128, 2048), partition_size=0,
         description="7B-shaped decode, one layer: 32 q = 32 kv heads, head_dim 128, bf16, "
                     "block 16, batch 64, lengths U[128,2048], 8192-block pool"),
     "13b_fp16": DecodeConfig(
         name="13b_fp16", num_seqs=256, num_heads=40, num_kv_heads=40, head_dim=128,
         block_size=16, num_blocks=16384, dtype="f16", scale=1.0 / math.sqrt(128.0), std=1.0,
-        lens=("lognormal", 512.0, 1.0, 16, 4096),
+        lens=("lognormal", 512.0, 1.0, 16, 4096), partition_size=0,
         description="13B-shaped decode, one layer: 40 heads, head_dim 128, fp16, block 16, "
                     "batch 256, lengths lognormal(median 512, sigma 1) clipped to [16,4096]"),
     "gqa_long_bf16": DecodeConfig(
