@@ -36,6 +36,10 @@ namespace {
 struct Seq {
   std::vector<int32_t> blocks;  // logical order
   int64_t len = 0;
+  // scratch of batched calls, valid while mark equals the allocator's epoch
+  uint64_t mark = 0;
+  int64_t sim_len = 0;
+  int32_t sim_last = -1;
 };
 
 }  // namespace
@@ -58,6 +62,23 @@ struct pa_alloc {
   std::vector<CacheKey> cache_key;
   std::map<CacheKey, int32_t> cache;
   int64_t next_cache_id = 1, cache_hits = 0, cache_evictions = 0;
+  // scratch of batched calls: each call takes a new epoch, so per-sequence and
+  // per-block marks from earlier calls read as unset without clearing anything
+  uint64_t epoch = 0;
+  std::vector<uint64_t> block_mark;
+  std::vector<int32_t> block_val;
+  std::vector<Seq*> batch;
+
+  // Looks every id up once; false if one is unknown.
+  bool resolve(const int64_t* ids, int n) {
+    batch.resize(static_cast<size_t>(n));
+    for (int i = 0; i < n; ++i) {
+      auto it = seqs.find(ids[i]);
+      if (it == seqs.end()) return false;
+      batch[static_cast<size_t>(i)] = &it->second;
+    }
+    return true;
+  }
 
   int64_t available() const {
     return static_cast<int64_t>(free_stack.size() + evictable.size());
@@ -102,6 +123,16 @@ namespace {
 
 inline int64_t blocks_for(int64_t n, int bs) { return (n + bs - 1) / bs; }
 
+// Length of the common prefix of two block lists of at least n entries: whole
+// 16-entry chunks by memcmp, then entry by entry inside the first differing chunk.
+inline size_t common_prefix(const int32_t* x, const int32_t* y, size_t n) {
+  constexpr size_t kChunk = 16;
+  size_t c = 0;
+  while (c + kChunk <= n && std::memcmp(x + c, y + c, kChunk * sizeof(int32_t)) == 0) c += kChunk;
+  while (c < n && x[c] == y[c]) ++c;
+  return c;
+}
+
 // Blocks one append to `s` takes from the pool, given the (possibly simulated)
 // reference count of its last block.
 inline bool append_needs_block(const Seq& s, int bs, int32_t last_ref) {
@@ -123,6 +154,8 @@ int pa_alloc_create(int64_t num_blocks, int block_size, const int32_t* free_orde
   a->num_blocks = num_blocks;
   a->block_size = block_size;
   a->ref.assign(static_cast<size_t>(num_blocks), 0);
+  a->block_mark.assign(static_cast<size_t>(num_blocks), 0);
+  a->block_val.assign(static_cast<size_t>(num_blocks), 0);
   a->evict_pos.assign(static_cast<size_t>(num_blocks), a->evictable.end());
   a->cache_id.assign(static_cast<size_t>(num_blocks), 0);
   a->cache_key.assign(static_cast<size_t>(num_blocks), pa_alloc::CacheKey());
@@ -266,40 +299,38 @@ int pa_seq_append_slots(pa_alloc_t* a, const int64_t* seq_ids, int n, int64_t* s
   if (!a || n < 0 || (n > 0 && (!seq_ids || !slots || !cow_pairs)) || !num_cow)
     return PA_ERR_INVALID_ARG;
   // Dry run: count the blocks the batch takes, simulating lengths and the
-  // reference counts that earlier copies in the batch drop.
-  std::unordered_map<int64_t, int64_t> len_delta;
-  std::unordered_map<int32_t, int32_t> ref_drop;
-  std::unordered_map<int64_t, int32_t> last_block;  // seqs whose last block changed
+  // reference counts that earlier copies in the batch drop (block_val).
+  if (!a->resolve(seq_ids, n)) return PA_ERR_UNKNOWN_SEQ;
+  const uint64_t ep = ++a->epoch;
   int64_t need = 0;
   const int bs = a->block_size;
   for (int i = 0; i < n; ++i) {
-    auto it = a->seqs.find(seq_ids[i]);
-    if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
-    const Seq& s = it->second;
-    int64_t len = s.len + len_delta[seq_ids[i]];
-    if (len % bs == 0) {
+    Seq& s = *a->batch[static_cast<size_t>(i)];
+    if (s.mark != ep) {
+      s.mark = ep;
+      s.sim_len = s.len;
+      s.sim_last = s.blocks.empty() ? -1 : s.blocks.back();
+    }
+    if (s.sim_len % bs == 0) {
       ++need;
-      last_block[seq_ids[i]] = -1;  // a fresh, private block
-    } else {
-      auto lb = last_block.find(seq_ids[i]);
-      int32_t last = (lb != last_block.end()) ? lb->second : s.blocks.back();
-      if (last >= 0) {
-        int32_t r = a->ref[last] - ref_drop[last];
-        if (r > 1) {
-          ++need;
-          ++ref_drop[last];
-          last_block[seq_ids[i]] = -1;
-        }
+      s.sim_last = -1;  // a fresh, private block
+    } else if (s.sim_last >= 0) {
+      const int32_t last = s.sim_last;
+      const int32_t drop = a->block_mark[last] == ep ? a->block_val[last] : 0;
+      if (a->ref[last] - drop > 1) {
+        ++need;
+        a->block_mark[last] = ep;
+        a->block_val[last] = drop + 1;
+        s.sim_last = -1;
       }
     }
-    ++len_delta[seq_ids[i]];
+    ++s.sim_len;
   }
   if (need > a->available()) return PA_ERR_NO_FREE_BLOCKS;
   int nc = 0;
   for (int i = 0; i < n; ++i) {
-    Seq& s = a->seqs.find(seq_ids[i])->second;
     int32_t src, dst;
-    slots[i] = append_one(a, s, &src, &dst);
+    slots[i] = append_one(a, *a->batch[static_cast<size_t>(i)], &src, &dst);
     if (src >= 0) {
       cow_pairs[2 * nc] = src;
       cow_pairs[2 * nc + 1] = dst;
@@ -312,16 +343,17 @@ int pa_seq_append_slots(pa_alloc_t* a, const int64_t* seq_ids, int n, int64_t* s
 
 int pa_seq_truncate(pa_alloc_t* a, const int64_t* seq_ids, const int64_t* new_lens, int n) {
   if (!a || n < 0 || (n > 0 && (!seq_ids || !new_lens))) return PA_ERR_INVALID_ARG;
-  for (int i = 0; i < n; ++i)  // validate first: all or nothing
-    if (!a->seqs.count(seq_ids[i])) return PA_ERR_UNKNOWN_SEQ;
-  std::unordered_map<int64_t, int> seen;
+  // validate first: all or nothing
+  if (!a->resolve(seq_ids, n)) return PA_ERR_UNKNOWN_SEQ;
+  const uint64_t ep = ++a->epoch;
   for (int i = 0; i < n; ++i) {
-    if (new_lens[i] < 0 || new_lens[i] > a->seqs.find(seq_ids[i])->second.len)
-      return PA_ERR_INVALID_ARG;
-    if (seen[seq_ids[i]]++) return PA_ERR_INVALID_ARG;  // ids must be distinct
+    Seq& s = *a->batch[static_cast<size_t>(i)];
+    if (new_lens[i] < 0 || new_lens[i] > s.len) return PA_ERR_INVALID_ARG;
+    if (s.mark == ep) return PA_ERR_INVALID_ARG;  // ids must be distinct
+    s.mark = ep;
   }
   for (int i = 0; i < n; ++i) {
-    Seq& s = a->seqs.find(seq_ids[i])->second;
+    Seq& s = *a->batch[static_cast<size_t>(i)];
     const size_t keep = static_cast<size_t>(blocks_for(new_lens[i], a->block_size));
     for (size_t j = keep; j < s.blocks.size(); ++j) a->dec(s.blocks[j]);
     if (keep < s.blocks.size()) s.blocks.resize(keep);
@@ -407,15 +439,15 @@ int pa_build_block_tables(const pa_alloc_t* a, const int64_t* seq_ids, int num_s
                           int32_t* tables, int max_blocks_per_seq, int32_t* seq_lens) {
   if (!a || num_seqs < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARG;
   if (num_seqs > 0 && (!seq_ids || !tables || !seq_lens)) return PA_ERR_INVALID_ARG;
+  pa_alloc* m = const_cast<pa_alloc*>(a);  // scratch only; the pool is not changed
+  if (!m->resolve(seq_ids, num_seqs)) return PA_ERR_UNKNOWN_SEQ;
   for (int i = 0; i < num_seqs; ++i) {  // validate first: all or nothing
-    auto it = a->seqs.find(seq_ids[i]);
-    if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
-    if (static_cast<int64_t>(it->second.blocks.size()) > max_blocks_per_seq ||
-        it->second.len > INT32_MAX)
+    const Seq& s = *m->batch[static_cast<size_t>(i)];
+    if (static_cast<int64_t>(s.blocks.size()) > max_blocks_per_seq || s.len > INT32_MAX)
       return PA_ERR_INVALID_ARG;
   }
   for (int i = 0; i < num_seqs; ++i) {
-    const Seq& s = a->seqs.find(seq_ids[i])->second;
+    const Seq& s = *m->batch[static_cast<size_t>(i)];
     int32_t* row = tables + static_cast<int64_t>(i) * max_blocks_per_seq;
     size_t nb = s.blocks.size();
     if (nb) std::memcpy(row, s.blocks.data(), nb * sizeof(int32_t));
@@ -434,41 +466,51 @@ int pa_build_prefix_groups(const pa_alloc_t* a, const int64_t* seq_ids, int num_
     return PA_ERR_INVALID_ARG;
   if (num_seqs > 0 && (!seq_ids || !prefix_parts || !chunk_members || !chunk_parts))
     return PA_ERR_INVALID_ARG;
-  std::vector<const Seq*> seqs(static_cast<size_t>(num_seqs));
-  for (int i = 0; i < num_seqs; ++i) {
-    auto it = a->seqs.find(seq_ids[i]);
-    if (it == a->seqs.end()) return PA_ERR_UNKNOWN_SEQ;
-    seqs[i] = &it->second;
-  }
-  // group positions by first physical block, in order of first appearance
-  std::unordered_map<int32_t, int> group_of;
-  std::vector<std::vector<int>> groups;
+  pa_alloc* m = const_cast<pa_alloc*>(a);  // scratch only; the pool is not changed
+  if (!m->resolve(seq_ids, num_seqs)) return PA_ERR_UNKNOWN_SEQ;
+  const std::vector<Seq*>& seqs = m->batch;
+  // group positions by first physical block, in order of first appearance: block_val
+  // holds a block's group while block_mark is this call's epoch
+  const uint64_t ep = ++m->epoch;
+  std::vector<int> gid(static_cast<size_t>(num_seqs), -1);
+  std::vector<int> count;
   for (int i = 0; i < num_seqs; ++i) {
     prefix_parts[i] = 0;
     if (seqs[i]->blocks.empty()) continue;
-    auto ins = group_of.emplace(seqs[i]->blocks[0], static_cast<int>(groups.size()));
-    if (ins.second) groups.emplace_back();
-    groups[ins.first->second].push_back(i);
+    const int32_t b0 = seqs[i]->blocks[0];
+    if (m->block_mark[b0] != ep) {
+      m->block_mark[b0] = ep;
+      m->block_val[b0] = static_cast<int32_t>(count.size());
+      count.push_back(0);
+    }
+    gid[i] = m->block_val[b0];
+    ++count[static_cast<size_t>(gid[i])];
   }
+  // members of each group contiguous, in position order (a counting sort)
+  std::vector<int> start(count.size() + 1, 0);
+  for (size_t g = 0; g < count.size(); ++g) start[g + 1] = start[g] + count[g];
+  std::vector<int> fill(start.begin(), start.end() - 1), flat(static_cast<size_t>(start.back()));
+  for (int i = 0; i < num_seqs; ++i)
+    if (gid[i] >= 0) flat[static_cast<size_t>(fill[static_cast<size_t>(gid[i])]++)] = i;
   int nc = 0, maxp = 0;
-  for (const auto& g : groups) {
-    if (g.size() < 2) continue;
-    const auto& t0 = seqs[g[0]]->blocks;
+  for (size_t gi = 0; gi < count.size(); ++gi) {
+    const int* g = flat.data() + start[gi];
+    const size_t size = static_cast<size_t>(count[gi]);
+    if (size < 2) continue;
+    const auto& t0 = seqs[static_cast<size_t>(g[0])]->blocks;
     size_t common = t0.size();
-    for (size_t k = 1; k < g.size(); ++k) {
-      const auto& t = seqs[g[k]]->blocks;
-      size_t c = 0;
-      while (c < common && c < t.size() && t[c] == t0[c]) ++c;
-      common = c;
+    for (size_t k = 1; k < size && common > 0; ++k) {
+      const auto& t = seqs[static_cast<size_t>(g[k])]->blocks;
+      common = common_prefix(t0.data(), t.data(), common < t.size() ? common : t.size());
     }
     const int parts = static_cast<int>(static_cast<int64_t>(common) * a->block_size / partition_size);
     if (parts == 0) continue;
-    for (int pos : g) prefix_parts[pos] = parts;
-    for (size_t k = 0; k < g.size(); k += static_cast<size_t>(max_members)) {
+    for (size_t k = 0; k < size; ++k) prefix_parts[g[k]] = parts;
+    for (size_t k = 0; k < size; k += static_cast<size_t>(max_members)) {
       int32_t* row = chunk_members + static_cast<int64_t>(nc) * max_members;
       for (int j = 0; j < max_members; ++j) {
         const size_t idx = k + static_cast<size_t>(j);
-        row[j] = idx < g.size() ? g[idx] : -1;
+        row[j] = idx < size ? g[idx] : -1;
       }
       chunk_parts[nc] = parts;
       ++nc;
