@@ -344,7 +344,7 @@ def run_ours(args, cfg):
     pool_bytes = 2 * kd.numel() * kd.element_size()
     del inp.k_pool, inp.v_pool
     dec = PagedDecoder(kd, vd, Hq, cfg.scale, max_blocks, inp.free_order, cfg.partition_size,
-                       kv_scales=kv_scales)
+                       kv_scales=kv_scales, query_dtype=TORCH_DTYPES[cfg.dtype])
     if inp.prefix is None:
         for s in range(S):
             dec.admit(s, int(inp.context_lens[s]))
@@ -368,9 +368,7 @@ def run_ours(args, cfg):
 
     def one_step(tokens, ev=None):
         q, nk, nv = tokens
-        meta = dec.prepare()
-        dec.launch(meta, q, nk, nv, out, events=ev)
-        return meta
+        return dec.step(q, nk, nv, out, events=ev)
 
     warm_cow = 0
     for i in range(args.warmup):
@@ -485,12 +483,14 @@ def run_ours(args, cfg):
                                           else "fixed"),
                        "mean_seq_len": round(float(lens.mean()), 1),
                        "max_seq_len": int(lens.max()),
-                       "l2": "inputs larger than L2 (K/V pool %.2f GB per rank), no flush"
-                             % (pool_bytes / 1e9),
+                       "l2": ("inputs larger than L2 (K/V pool %.2f GB per rank), no flush"
+                              % (pool_bytes / 1e9)) if pool_bytes > L2_BYTES else
+                             ("K/V pool of %.1f KB fits in L2: a parity-size workload, "
+                              "no flush" % (pool_bytes / 1e3)),
                        "steps": "each step appends one token per sequence and rolls the "
                                 "previous one back, so every step decodes these lengths",
                        "parallelism": f"replicas x{world}",
-                       "workspace_bytes": int(dec._ws.numel()),
+                       "workspace_bytes": int(dec.workspace_bytes),
                        "prefix_group_chunks": int(meta0.get("num_chunks", 0)),
                        "pool": pool_summary(dec.alloc.stats()),
                        "cow_pairs_in_warmup": warm_cow, "cow_pairs_in_timed_steps": cows,
@@ -506,6 +506,9 @@ def run_ours(args, cfg):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+L2_BYTES = 126 * 1000 * 1000  # B200 L2
 
 
 def pool_summary(st: dict) -> dict:

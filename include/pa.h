@@ -19,9 +19,11 @@
  *     nothing (argument errors are found before any launch) or, for PA_ERR_CUDA,
  *     that a launch failed.
  *   - Tensor arguments of the GPU entry points are DEVICE pointers owned by the
- *     caller, contiguous, 16-byte aligned, in the layouts stated below.  The
- *     library never allocates, frees or keeps device memory; scratch space is
- *     passed in by the caller (see pa_decode_workspace_bytes).
+ *     caller, contiguous, 16-byte aligned, in the layouts stated below.  The kernel
+ *     entry points never allocate, free or keep device memory; scratch space is
+ *     passed in by the caller (see pa_decode_workspace_bytes).  The decode-step
+ *     runtime (pa_decoder_*) is the exception: it owns the staging and scratch
+ *     buffers it allocates when a batch is bound, and frees them when destroyed.
  *   - GPU work is enqueued on the caller's stream (a cudaStream_t passed as
  *     pa_stream_t; NULL = legacy default stream) and is asynchronous: no entry
  *     point synchronises, except pa_device_error_read.
@@ -440,6 +442,118 @@ int pa_block_refcount(const pa_alloc_t* a, int32_t block, int32_t* refcount);
 /* Free blocks in the order the next pops return them; *n = how many. */
 int pa_alloc_free_list(const pa_alloc_t* a, int32_t* out, int64_t cap, int64_t* n);
 int pa_alloc_stats(const pa_alloc_t* a, pa_stats_t* stats);
+
+/* ------------------------------------------------------------------------- */
+/* Decode-step runtime                                                        */
+/* ------------------------------------------------------------------------- */
+/*
+ * A pa_decoder runs decode steps of a bound batch of sequences, host side included,
+ * in native code.  One step, in the order of [BLOG] "PagedAttention: paging, borrowed
+ * from the operating system" and "The bonus contiguous storage can't give you:
+ * sharing":
+ *   1. (rolling batches) every sequence is truncated back to its length at bind time,
+ *      so that a long run keeps decoding the same lengths;
+ *   2. pa_seq_append_slots gives every sequence room for one more token: its slot,
+ *      and a copy-on-write pair where that token's block is shared;
+ *   3. slots, pairs, lengths and block tables (pa_build_block_tables) and, for
+ *      batches that share prefixes, the prefix groups (pa_build_prefix_groups) are
+ *      written into one of two page-locked staging sets and sent to the device with
+ *      one copy on the decoder's copy stream; the caller's stream waits for it;
+ *   4. pa_copy_blocks makes the copies (before the write: the token lands in the copy);
+ *   5. pa_reshape_and_cache (or _fp8) writes the new tokens' K/V into their slots;
+ *   6. pa_decode_attention (or _fp8, or _grouped when prefix groups exist) attends over
+ *      every cached token, the new one included.
+ * Steps 4-6 are enqueued on the caller's stream; the call returns without waiting
+ * for the GPU.  Step k fills staging set k % 2 while the kernels of step k - 1 may
+ * still read the other set; the host waits only before rewriting a set whose copy
+ * has not finished.
+ *
+ * The decoder borrows the allocator (which must outlive it and must not be used
+ * from another thread during a call) and the caches; it owns its streams, events and
+ * the buffers pa_decoder_bind allocates: the staging sets (pa_decoder_query), the
+ * decode workspace for the bound batch at full table capacity, and, for host-fed
+ * steps, two device sets of q / new K / new V / out.  Nothing is allocated inside a
+ * step except the first host-fed step after a bind to a new batch size.  Not
+ * thread-safe.  Every call makes the decoder's device (current at create) current
+ * for its duration.  A step that fails after step 2 leaves the sequences one token
+ * longer.
+ */
+typedef struct pa_decoder pa_decoder_t;
+
+typedef struct {
+  size_t struct_size;      /* sizeof(pa_decoder_config_t)                          */
+  void* k_cache;           /* device caches, layout above, caller-owned            */
+  void* v_cache;
+  int64_t num_blocks;      /* >= the allocator's pool                              */
+  int num_kv_heads;
+  int block_size;          /* the allocator's block size                           */
+  int head_dim;
+  int num_heads;           /* query heads, a multiple of num_kv_heads              */
+  int dtype;               /* q, new K/V rows, out: PA_F32 / PA_BF16 / PA_F16      */
+  int cache_dtype;         /* dtype, or PA_FP8_E4M3 with dtype PA_BF16 / PA_F16    */
+  float scale;             /* logit scale                                          */
+  float k_scale, v_scale;  /* fp8 per-tensor scales (ignored for 16/32-bit caches) */
+  int max_blocks_per_seq;  /* block-table width: capacity per sequence in blocks   */
+  int partition_size;      /* 0 = pa_decode_partition_size for the bound batch at
+                              full table capacity; else a multiple of block_size   */
+  int group_members;       /* prefix-group chunk size 0..16 (0 = no groups;
+                              always 0 for fp8 caches)                              */
+} pa_decoder_config_t;
+
+typedef struct {
+  size_t struct_size;      /* set by the caller: sizeof(pa_step_info_t)            */
+  int num_cow;             /* copy-on-write pairs of the step                      */
+  int max_seq_len;         /* longest sequence after the append                    */
+  int partition_size;
+  int num_chunks;          /* prefix-group chunks (0 = plain decode)               */
+  int max_chunk_parts;
+  int first_part;
+  int kernels;             /* library kernels the step launched                    */
+  /* Host views of the step's staging set (page-locked; valid until the step after
+   * next): slots int64 [S], cow_pairs int32 [num_cow, 2], block_tables int32
+   * [S, max_blocks_per_seq], seq_lens int32 [S]; S = the bound batch size. */
+  const int64_t* slots;
+  const int32_t* cow_pairs;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+} pa_step_info_t;
+
+/* Checks the configuration (struct_size, pointers, sizes, dtypes) before any CUDA
+ * call; then creates the decoder's streams and events on the current device. */
+int pa_decoder_create(const pa_decoder_config_t* cfg, pa_alloc_t* alloc,
+                      pa_decoder_t** out);
+/* Waits for the decoder's work in flight, then frees everything it owns. */
+int pa_decoder_destroy(pa_decoder_t* d);
+/* Fix the batch (distinct ids present in the allocator, each shorter than the table
+ * capacity) and allocate its buffers; rolling != 0 makes every step first roll the
+ * sequences back to their current lengths.  Waits for the decoder's work in flight. */
+int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int rolling);
+/* One step with DEVICE inputs: q [S, num_heads, head_dim], new_k / new_v
+ * [S, num_kv_heads, head_dim] (row i is seq_ids[i]'s new token), out [S, num_heads,
+ * head_dim], all dtype.  ev_begin / ev_end (cudaEvent_t or NULL) are recorded on the
+ * stream around the attention call.  info (or NULL) receives the step's facts. */
+int pa_decoder_step(pa_decoder_t* d, const void* q, const void* new_k, const void* new_v,
+                    void* out, pa_stream_t stream, void* ev_begin, void* ev_end,
+                    pa_step_info_t* info);
+/* One step with HOST inputs and output (page-locked for the copies to overlap):
+ * q, new_k, new_v are copied to the device on the decoder's input stream, the step
+ * runs on `stream`, and out is copied back on its output stream.  Two device I/O
+ * sets alternate, so a step's copies overlap the neighbouring steps' kernels.  The
+ * call returns at once; *ticket (or NULL) names the step for pa_decoder_wait.  The
+ * caller must not rewrite q / new_k / new_v or read out before that wait. */
+int pa_decoder_step_host(pa_decoder_t* d, const void* q, const void* new_k,
+                         const void* new_v, void* out, pa_stream_t stream, int64_t* ticket,
+                         pa_step_info_t* info);
+/* Block until the host-fed step `ticket` has written its output (and finished reading
+ * its inputs). */
+int pa_decoder_wait(pa_decoder_t* d, int64_t ticket);
+/* Make `stream` wait for every outstanding read-back of host-fed steps. */
+int pa_decoder_drain(pa_decoder_t* d, pa_stream_t stream);
+/* Facts of the bound batch: the partition size in use, the workspace bytes and the
+ * bytes of one staging set (the host-to-device copy of a step).  NULL outputs are
+ * skipped. */
+int pa_decoder_query(const pa_decoder_t* d, int* partition_size, size_t* workspace_bytes,
+                     size_t* staging_bytes);
 
 #ifdef __cplusplus
 }

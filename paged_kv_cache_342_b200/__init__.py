@@ -53,6 +53,21 @@ class pa_stats_t(ctypes.Structure):
         "cache_evictions")]
 
 
+class pa_decoder_config_t(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_size_t), ("k_cache", _p), ("v_cache", _p),
+                ("num_blocks", _i64), ("num_kv_heads", _i32), ("block_size", _i32),
+                ("head_dim", _i32), ("num_heads", _i32), ("dtype", _i32), ("cache_dtype", _i32),
+                ("scale", _f), ("k_scale", _f), ("v_scale", _f), ("max_blocks_per_seq", _i32),
+                ("partition_size", _i32), ("group_members", _i32)]
+
+
+class pa_step_info_t(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_size_t), ("num_cow", _i32), ("max_seq_len", _i32),
+                ("partition_size", _i32), ("num_chunks", _i32), ("max_chunk_parts", _i32),
+                ("first_part", _i32), ("kernels", _i32), ("slots", _I64P),
+                ("cow_pairs", _I32P), ("block_tables", _I32P), ("seq_lens", _I32P)]
+
+
 def _sig(name, res, *args):
     fn = getattr(lib, name)
     fn.restype = res
@@ -96,6 +111,16 @@ _sig("pa_build_prefix_groups", _i32, _p, _p, _i32, _i32, _i32, _p, _p, _p,
      ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int))
 _sig("pa_alloc_free_list", _i32, _p, _p, _i64, _I64P)
 _sig("pa_alloc_stats", _i32, _p, ctypes.POINTER(pa_stats_t))
+_sig("pa_decoder_create", _i32, ctypes.POINTER(pa_decoder_config_t), _p, ctypes.POINTER(_p))
+_sig("pa_decoder_destroy", _i32, _p)
+_sig("pa_decoder_bind", _i32, _p, _p, _i32, _i32)
+_sig("pa_decoder_step", _i32, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.POINTER(pa_step_info_t))
+_sig("pa_decoder_step_host", _i32, _p, _p, _p, _p, _p, _p, _I64P,
+     ctypes.POINTER(pa_step_info_t))
+_sig("pa_decoder_wait", _i32, _p, _i64)
+_sig("pa_decoder_drain", _i32, _p, _p)
+_sig("pa_decoder_query", _i32, _p, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_size_t),
+     ctypes.POINTER(ctypes.c_size_t))
 
 
 def _check(status: int, where: str) -> None:

@@ -1,12 +1,14 @@
-"""One decode step of the paged KV-cache path, driven through the C ABI.
+"""One decode step of the paged KV-cache path, driven through the native step runtime
+(``pa_decoder_*`` in ``include/pa.h``).
 
-Order of a step (the sources are the pages cited in ``include/pa.h``):
+Order of a step (the sources are the pages cited in ``include/pa.h``), all of it in
+the library's C++ and CUDA code:
   1. the block manager gives every sequence room for one more token
      (``pa_seq_append_slots``): a slot, and a (src, dst) copy where the token's
      block is shared;
-  2. slots, copy pairs, lengths and block tables are packed into one pinned staging
-     buffer and sent to the device in one copy (the only host-to-device traffic of
-     a step);
+  2. slots, copy pairs, lengths, block tables and prefix groups are written into one
+     of two page-locked staging sets and sent to the device in one copy (the only
+     host-to-device traffic of a step), on the decoder's own copy stream;
   3. ``pa_copy_blocks`` makes the copy-on-write copies - before the write, since
      the new token lands in the copy;
   4. ``pa_reshape_and_cache`` writes the new token's K/V into its slot;
@@ -23,59 +25,140 @@ members as fill one 8-column tensor-core tile, 8 // (num_heads/num_kv_heads); 0
 turns grouping off).
 
 One-byte caches (uint8 / float8_e4m3fn tensors) are fp8 e4m3 caches with the
-per-tensor ``kv_scales`` (k_scale, v_scale): the step writes with
-``pa_reshape_and_cache_fp8`` and attends with ``pa_decode_attention_fp8``.
+per-tensor ``kv_scales`` (k_scale, v_scale) and a 16-bit ``query_dtype`` for q, the
+new K/V rows and out: the step writes with ``pa_reshape_and_cache_fp8`` and attends
+with ``pa_decode_attention_fp8``.
 
 This module only moves arguments: the work of every step is done by the library.
 """
 from __future__ import annotations
 
+import ctypes
+
 import numpy as np
 import torch
 
-from . import (DEFAULT_PARTITION, BlockAllocator, _dtype_code, pa_copy_blocks,
-               pa_decode_attention, pa_decode_attention_fp8, pa_decode_attention_grouped,
-               pa_decode_partition_size, pa_decode_workspace_bytes, pa_reshape_and_cache,
-               pa_reshape_and_cache_fp8)
+from . import (DEFAULT_PARTITION, BlockAllocator, _check, _dtype_code, lib, pa_copy_blocks,
+               pa_decoder_config_t, pa_step_info_t)
 
 
-def _align(n: int, a: int = 256) -> int:
-    return (n + a - 1) // a * a
+class StepInfo:
+    """Facts of one step, from the library's ``pa_step_info_t``.  ``slots``,
+    ``tables``, ``lens`` and ``pairs`` are numpy views of the step's page-locked
+    staging set, valid until the step after the next (copy them to keep them)."""
+
+    __slots__ = ("num_cow", "max_len", "partition_size", "num_chunks", "max_chunk_parts",
+                 "first_part", "kernels", "_info", "_S", "_MB")
+
+    def __init__(self, info: pa_step_info_t, S: int, MB: int):
+        self.num_cow, self.max_len = info.num_cow, info.max_seq_len
+        self.partition_size, self.num_chunks = info.partition_size, info.num_chunks
+        self.max_chunk_parts, self.first_part = info.max_chunk_parts, info.first_part
+        self.kernels = info.kernels
+        self._info, self._S, self._MB = info, S, MB
+
+    @property
+    def slots(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self._info.slots, (self._S,))
+
+    @property
+    def lens(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self._info.seq_lens, (self._S,))
+
+    @property
+    def tables(self) -> np.ndarray:
+        return np.ctypeslib.as_array(self._info.block_tables, (self._S, self._MB))
+
+    @property
+    def pairs(self) -> np.ndarray:
+        if self.num_cow == 0:
+            return np.zeros((0, 2), np.int32)
+        return np.ctypeslib.as_array(self._info.cow_pairs, (self.num_cow, 2))
+
+    # dict-style access to the scalar facts and the pairs
+    _KEYS = {"num_cow": "num_cow", "max_len": "max_len", "num_chunks": "num_chunks",
+             "max_chunk_parts": "max_chunk_parts", "first_part": "first_part",
+             "kernels": "kernels", "pairs": "pairs", "partition_size": "partition_size"}
+
+    def __getitem__(self, key):
+        return getattr(self, self._KEYS[key])
+
+    def get(self, key, default=None):
+        return getattr(self, self._KEYS[key]) if key in self._KEYS else default
+
+
+class HostStep:
+    """Completion handle of a host-fed step: ``synchronize()`` blocks until the step's
+    output is in its host buffer (and its inputs have been read)."""
+
+    __slots__ = ("_dec", "ticket")
+
+    def __init__(self, dec, ticket: int):
+        self._dec, self.ticket = dec, ticket
+
+    def synchronize(self) -> None:
+        _check(lib.pa_decoder_wait(self._dec, self.ticket), "pa_decoder_wait")
 
 
 class PagedDecoder:
-    """Device caches + block manager + staging for a fixed batch of sequences.
+    """Device caches + block manager + the library's step runtime for a fixed batch.
 
     ``k_cache``/``v_cache`` are caller-owned CUDA tensors [NB, Hkv, bs, D].
     ``max_blocks_per_seq`` is the block-table width (capacity per sequence).
     ``partition_size`` 0 takes ``pa_decode_partition_size`` for the bound batch at
-    that capacity (resolved by ``bind``; it ignores prefix groups, so batches of
-    forks do better with an explicit size shorter than their shared prefix).
+    that capacity (it ignores prefix groups, so batches of forks do better with an
+    explicit size shorter than their shared prefix).
     """
 
     def __init__(self, k_cache, v_cache, num_heads: int, scale: float, max_blocks_per_seq: int,
                  free_order=None, partition_size: int = DEFAULT_PARTITION, stream=None,
-                 group_members: int | None = None, kv_scales=None):
+                 group_members: int | None = None, kv_scales=None, query_dtype=None):
         self.k_cache, self.v_cache = k_cache, v_cache
         self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim = k_cache.shape
         self.num_heads, self.scale = num_heads, scale
         self.max_blocks = max_blocks_per_seq
-        self._partition_arg = partition_size
-        self.partition_size = partition_size or DEFAULT_PARTITION
+        self.partition_size = partition_size
         self.device = k_cache.device
         self.stream = stream
         self.alloc = BlockAllocator(self.num_blocks, self.block_size, free_order)
-        self._seq_ids = None
-        self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
         group = num_heads // self.num_kv_heads
         self.fp8 = k_cache.element_size() == 1
-        if self.fp8 and kv_scales is None:
-            raise ValueError("an fp8 cache needs kv_scales=(k_scale, v_scale)")
+        if self.fp8 and (kv_scales is None or query_dtype is None):
+            raise ValueError("an fp8 cache needs kv_scales=(k_scale, v_scale) and query_dtype")
         self.kv_scales = kv_scales
         self.group_members = (8 // group if group <= 8 else 0) if group_members is None \
             else group_members
         if self.fp8:
             self.group_members = 0
+        self.workspace_bytes = self.staging_bytes = 0
+        self._S = 0
+        cfg = pa_decoder_config_t()
+        cfg.struct_size = ctypes.sizeof(pa_decoder_config_t)
+        cfg.k_cache, cfg.v_cache = k_cache.data_ptr(), v_cache.data_ptr()
+        cfg.num_blocks, cfg.num_kv_heads = self.num_blocks, self.num_kv_heads
+        cfg.block_size, cfg.head_dim, cfg.num_heads = self.block_size, self.head_dim, num_heads
+        cfg.cache_dtype = _dtype_code(k_cache)
+        cfg.dtype = (_dtype_code(torch.empty(0, dtype=query_dtype)) if self.fp8
+                     else cfg.cache_dtype)
+        cfg.scale = float(scale)
+        cfg.k_scale, cfg.v_scale = (float(x) for x in (kv_scales or (1.0, 1.0)))
+        cfg.max_blocks_per_seq, cfg.partition_size = max_blocks_per_seq, partition_size
+        cfg.group_members = self.group_members
+        self._cfg = cfg
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            _check(lib.pa_decoder_create(ctypes.byref(cfg), self.alloc._h, ctypes.byref(h)),
+                   "pa_decoder_create")
+        self._h = h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            try:
+                lib.pa_decoder_destroy(h)
+            except Exception:  # interpreter shutdown: the library may be gone already
+                pass
+            self._h = None
 
     # -- context building ------------------------------------------------------
     def admit(self, seq_id: int, num_tokens: int) -> None:
@@ -108,213 +191,76 @@ class PagedDecoder:
 
     # -- the step ---------------------------------------------------------------
     def bind(self, seq_ids, rolling: bool = False) -> None:
-        """Fix the batch the steps run over and allocate the staging buffers."""
+        """Fix the batch the steps run over; the library allocates its buffers."""
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
-        self._seq_ids = ids
-        self.rolling = rolling
-        self._stepped = False
-        self.base_lens = np.array([self.alloc.seq_len(int(s)) for s in ids], np.int64)
-        S, MB, MM = ids.size, self.max_blocks, max(1, self.group_members)
-        S1 = max(S, 1)
-        sizes = [("slots", 8 * S), ("pairs", 8 * S1), ("lens", 4 * S), ("tables", 4 * S * MB),
-                 ("pparts", 4 * S1), ("cmembers", 4 * S1 * MM), ("cparts", 4 * S1)]
-        offs, total = {}, 0
-        for name, n in sizes:
-            offs[name] = total
-            total += _align(n)
-        # two staging sets: step k fills set k % 2 while step k - 1's kernels still
-        # read the other one; the copy runs on its own stream
-        self._h_bufs = [torch.empty(total, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
-        self._d_bufs = [torch.empty(total, dtype=torch.uint8, device=self.device)
-                        for _ in range(2)]
-        self._copy_stream = torch.cuda.Stream(device=self.device)
-        self._h2d_done = [None, None]       # the set's host buffer may be rewritten
-        self._kernels_done = [None, None]   # the set's device buffer may be overwritten
-        self._set = 1
+        _check(lib.pa_decoder_bind(self._h, ids.ctypes.data, ids.size, int(rolling)),
+               "pa_decoder_bind")
+        self._S = ids.size
+        ps, ws, st = ctypes.c_int(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+        _check(lib.pa_decoder_query(self._h, ctypes.byref(ps), ctypes.byref(ws), ctypes.byref(st)),
+               "pa_decoder_query")
+        self.partition_size = ps.value
+        self.workspace_bytes, self.staging_bytes = ws.value, st.value
 
-        def views(buf):
-            def sec(name, n, dt):
-                return buf[offs[name]:offs[name] + n].view(dt)
-            return dict(
-                slots=sec("slots", 8 * S, torch.int64),
-                pairs=sec("pairs", 8 * S1, torch.int32).view(-1, 2),
-                lens=sec("lens", 4 * S, torch.int32),
-                tables=sec("tables", 4 * S * MB, torch.int32).view(S, MB),
-                pparts=sec("pparts", 4 * S1, torch.int32),
-                cmembers=sec("cmembers", 4 * S1 * MM, torch.int32).view(S1, MM),
-                cparts=sec("cparts", 4 * S1, torch.int32))
-
-        self._views = [(views(self._h_bufs[i]), views(self._d_bufs[i])) for i in range(2)]
-        self._use_set(0)
-        cap = MB * self.block_size
-        if self._partition_arg == 0:
-            ps = pa_decode_partition_size(_dtype_code(self.k_cache), S, self.num_heads, self.num_kv_heads,
-                                          self.head_dim, self.block_size, cap)
-            if ps <= 0:
-                raise RuntimeError("pa_decode_partition_size rejected the bound batch")
-            self.partition_size = ps
-        ws = pa_decode_workspace_bytes(S, self.num_heads, self.head_dim, cap, self.partition_size)
-        if ws > self._ws.numel():
-            self._ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
-
-    def _use_set(self, i: int) -> None:
-        """Point the h_* / d_* views at staging set i."""
-        self._set = i
-        h, d = self._views[i]
-        self.h_stage, self.d_stage = self._h_bufs[i], self._d_bufs[i]
-        self.h_slots, self.h_pairs, self.h_lens, self.h_tables = (h["slots"], h["pairs"],
-                                                                  h["lens"], h["tables"])
-        self.d_slots, self.d_pairs, self.d_lens, self.d_tables = (d["slots"], d["pairs"],
-                                                                  d["lens"], d["tables"])
-        self.h_groups = (h["pparts"], h["cmembers"], h["cparts"])
-        self.d_groups = (d["pparts"], d["cmembers"], d["cparts"])
-
-    @property
-    def staging_bytes(self) -> int:
-        return self.h_stage.numel()
-
-    def prepare(self) -> dict:
-        """Host side of a step: slots and copies from the block manager, tables and
-        lengths, all staged and sent to the device in one copy (on the copy stream;
-        the compute stream waits for it)."""
-        i = self._set ^ 1 if self._stepped else 0
-        if self._h2d_done[i] is not None:
-            self._h2d_done[i].synchronize()  # that set's host buffer is free again
-        self._use_set(i)
-        if self.rolling and self._stepped:
-            self.alloc.truncate(self._seq_ids, self.base_lens)
-        slots, pairs = self.alloc.append_slots(self._seq_ids, self.h_slots.numpy(),
-                                               self.h_pairs.numpy())
-        self._stepped = True
-        n_cow = len(pairs)
-        _, lens = self.alloc.build_block_tables(self._seq_ids, self.max_blocks,
-                                                self.h_tables.numpy(), self.h_lens.numpy())
-        max_len = int(lens.max()) if lens.size else 0
-        num_chunks = max_chunk_parts = first_part = 0
-        if self.group_members > 0:
-            hp, hm, hc = self.h_groups
-            pp, members, _, max_chunk_parts = self.alloc.prefix_groups(
-                self._seq_ids, self.partition_size, self.group_members, hp.numpy(), hm.numpy(),
-                hc.numpy())
-            num_chunks = len(members)
-            if num_chunks and lens.size:
-                # the lowest partition any sequence computes itself
-                own = np.minimum(pp, np.maximum(lens.astype(np.int64) - 1, 0) // self.partition_size)
-                first_part = int(own.min())
-        comp, cs = self._torch_stream(), self._copy_stream
-        if self._kernels_done[i] is not None:
-            cs.wait_event(self._kernels_done[i])   # kernels two steps back read it
-        with torch.cuda.stream(cs):
-            self.d_stage.copy_(self.h_stage, non_blocking=True)
-            done = torch.cuda.Event()
-            done.record(cs)
-        self._h2d_done[i] = done
-        comp.wait_event(done)
-        return dict(num_cow=n_cow, max_len=max_len, pairs=self.h_pairs.numpy()[:n_cow],
-                    num_chunks=num_chunks, max_chunk_parts=max_chunk_parts,
-                    first_part=first_part)
-
-    def launch(self, meta: dict, q, new_k, new_v, out, events=None) -> None:
-        """Device side of a step: copies, the new token's K/V, attention.  ``events``
-        (a pair of CUDA events) are recorded around the attention call."""
-        st = self._torch_stream()
-        n = meta["num_cow"]
-        if n:
-            pa_copy_blocks(self.k_cache, self.v_cache, self.d_pairs[:n], meta["pairs"], stream=st)
-        if self.fp8:
-            pa_reshape_and_cache_fp8(new_k, new_v, self.k_cache, self.v_cache, self.d_slots,
-                                     *self.kv_scales, stream=st)
-        else:
-            pa_reshape_and_cache(new_k, new_v, self.k_cache, self.v_cache, self.d_slots, stream=st)
-        ws = self._ws if self._ws.numel() else None
+    def step(self, q, new_k, new_v, out, events=None) -> StepInfo:
+        """One step on device tensors (q/out [S, Hq, D], new_k/new_v [S, Hkv, D]);
+        ``events`` (a pair of CUDA events) are recorded around the attention call."""
+        self._check_io(q, new_k, new_v, out, cuda=True)
+        info = pa_step_info_t()
+        info.struct_size = ctypes.sizeof(pa_step_info_t)
+        e0 = e1 = None
         if events is not None:
-            events[0].record(st)
-        if self.fp8:
-            pa_decode_attention_fp8(out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
-                                    self.scale, self.block_size, self.num_kv_heads,
-                                    meta["max_len"], *self.kv_scales, self.partition_size, ws,
-                                    stream=st)
-        elif meta.get("num_chunks", 0):
-            pp, cm, cp = self.d_groups
-            pa_decode_attention_grouped(
-                out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens, self.scale,
-                self.block_size, self.num_kv_heads, meta["max_len"], pp, cm, cp,
-                meta["num_chunks"], meta["max_chunk_parts"], self.partition_size, ws, stream=st,
-                first_part=meta["first_part"])
-        else:
-            pa_decode_attention(out, q, self.k_cache, self.v_cache, self.d_tables, self.d_lens,
-                                self.scale, self.block_size, self.num_kv_heads, meta["max_len"],
-                                self.partition_size, ws, stream=st)
-        if events is not None:
-            events[1].record(st)
-        done = torch.cuda.Event()
-        done.record(st)
-        self._kernels_done[self._set] = done
-
-    def step(self, q, new_k, new_v, out) -> dict:
-        meta = self.prepare()
-        self.launch(meta, q, new_k, new_v, out)
-        return meta
+            e0, e1 = (_event_handle(e) for e in events)
+        _check(lib.pa_decoder_step(self._h, q.data_ptr(), new_k.data_ptr(), new_v.data_ptr(),
+                                   out.data_ptr(), self._stream_handle(), e0, e1,
+                                   ctypes.byref(info)), "pa_decoder_step")
+        return StepInfo(info, self._S, self.max_blocks)
 
     # -- steps fed from host memory ----------------------------------------------
-    def step_host(self, q_h, new_k_h, new_v_h, out_h):
+    def step_host(self, q_h, new_k_h, new_v_h, out_h) -> HostStep:
         """One step whose inputs come from, and whose result goes back to, page-locked
-        host tensors.  Copies run on their own streams and overlap the neighbouring
-        steps' kernels: two device buffer sets alternate, and events order the
-        input copy -> kernels -> output copy of each step.  Returns the event after
-        which ``out_h`` holds this step's result (do not reuse ``out_h`` before)."""
-        if not hasattr(self, "_io"):
-            self._io_init(q_h, new_k_h, out_h)
-        io = self._io[self._io_next]
-        self._io_next ^= 1
-        comp = self._torch_stream()
-        h2d, d2h = self._h2d_stream, self._d2h_stream
-        h2d.wait_event(io["compute_done"])          # the kernels two steps ago used them
-        with torch.cuda.stream(h2d):
-            for dst, src in zip(io["inputs"], (q_h, new_k_h, new_v_h)):
-                dst.copy_(src, non_blocking=True)
-            io["h2d_done"].record(h2d)
-        comp.wait_event(io["h2d_done"])
-        comp.wait_event(io["d2h_done"])             # the output buffer was read back
-        meta = self.prepare()
-        self.launch(meta, *io["inputs"], io["out"])
-        io["compute_done"].record(comp)
-        d2h.wait_event(io["compute_done"])
-        with torch.cuda.stream(d2h):
-            out_h.copy_(io["out"], non_blocking=True)
-            io["d2h_done"].record(d2h)
-        return io["d2h_done"]
+        host tensors; the copies overlap the neighbouring steps' kernels.  Returns the
+        handle whose ``synchronize()`` waits for ``out_h`` (do not reuse the buffers
+        before)."""
+        self._check_io(q_h, new_k_h, new_v_h, out_h, cuda=False)
+        ticket = ctypes.c_int64(0)
+        _check(lib.pa_decoder_step_host(self._h, q_h.data_ptr(), new_k_h.data_ptr(),
+                                        new_v_h.data_ptr(), out_h.data_ptr(),
+                                        self._stream_handle(), ctypes.byref(ticket), None),
+               "pa_decoder_step_host")
+        return HostStep(self._h, ticket.value)
 
     def drain_host_io(self) -> None:
         """Make the compute stream wait for every outstanding host-I/O copy."""
-        if hasattr(self, "_io"):
-            comp = self._torch_stream()
-            for io in self._io:
-                comp.wait_event(io["d2h_done"])
+        _check(lib.pa_decoder_drain(self._h, self._stream_handle()), "pa_decoder_drain")
 
-    def _io_init(self, q_h, kv_h, out_h) -> None:
-        dev = self.device
-        self._h2d_stream = torch.cuda.Stream(device=dev)
-        self._d2h_stream = torch.cuda.Stream(device=dev)
-        self._io, self._io_next = [], 0
-        for _ in range(2):
-            io = {"inputs": [torch.empty(q_h.shape, dtype=q_h.dtype, device=dev),
-                             torch.empty(kv_h.shape, dtype=kv_h.dtype, device=dev),
-                             torch.empty(kv_h.shape, dtype=kv_h.dtype, device=dev)],
-                  "out": torch.empty(out_h.shape, dtype=out_h.dtype, device=dev)}
-            for name in ("h2d_done", "compute_done", "d2h_done"):
-                io[name] = torch.cuda.Event()
-                io[name].record(self._torch_stream())   # start out completed
-            self._io.append(io)
-
-    def kernel_launches(self, meta: dict) -> int:
+    def kernel_launches(self, meta: StepInfo) -> int:
         """Library kernels one step launches (copy, write, group, partitions, merge)."""
-        parts = max(1, -(-meta["max_len"] // self.partition_size))
-        grouped = (meta.get("num_chunks", 0) > 0 and parts > 1 and not self.fp8
-                   and self.k_cache.dtype != torch.float32
-                   and self.block_size in (16, 32)
-                   and self.group_members * (self.num_heads // self.num_kv_heads) <= 16)
-        return (1 if meta["num_cow"] else 0) + 2 + (1 if grouped else 0) + (1 if parts > 1 else 0)
+        return meta.kernels
+
+    def _check_io(self, q, new_k, new_v, out, cuda: bool) -> None:
+        S, Hq, Hkv, D = self._S, self.num_heads, self.num_kv_heads, self.head_dim
+        want = self._cfg.dtype
+        for t, shape in ((q, (S, Hq, D)), (new_k, (S, Hkv, D)), (new_v, (S, Hkv, D)),
+                         (out, (S, Hq, D))):
+            if (tuple(t.shape) != shape or t.is_cuda != cuda or not t.is_contiguous()
+                    or _dtype_code(t) != want):
+                raise ValueError(f"step tensor {tuple(t.shape)} {t.dtype} "
+                                 f"({'cuda' if t.is_cuda else 'host'}) does not fit the "
+                                 f"bound batch {shape}")
 
     def _torch_stream(self):
         return torch.cuda.current_stream(self.device) if self.stream is None else self.stream
+
+    def _stream_handle(self) -> int:
+        return self._torch_stream().cuda_stream
+
+
+def _event_handle(ev) -> int:
+    """The cudaEvent_t of a torch CUDA event (recorded once if it was never used, so
+    that it exists)."""
+    h = ev.cuda_event
+    if not h:
+        ev.record()
+        h = ev.cuda_event
+    return h

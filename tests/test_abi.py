@@ -94,6 +94,51 @@ def test_partition_size_choice(pa):
     assert ps(pa.PA_BF16, 8, 64, 8, 128, 16, 1000, -2) == 0
 
 
+def _decoder_config(pa, **kw):
+    c = pa.pa_decoder_config_t()
+    c.struct_size = ctypes.sizeof(pa.pa_decoder_config_t)
+    c.k_cache = c.v_cache = 1 << 20
+    c.num_blocks, c.num_kv_heads, c.block_size, c.head_dim, c.num_heads = 64, 4, 16, 128, 8
+    c.dtype = c.cache_dtype = pa.PA_BF16
+    c.scale, c.k_scale, c.v_scale = 0.1, 1.0, 1.0
+    c.max_blocks_per_seq, c.partition_size, c.group_members = 8, 0, 1
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def test_decoder_config_checks(pa):
+    alloc = pa.BlockAllocator(64, 16)
+    h = ctypes.c_void_p()
+    create = lambda c, a=alloc._h: pa.lib.pa_decoder_create(ctypes.byref(c), a, ctypes.byref(h))
+    bad = [dict(struct_size=8), dict(k_cache=0), dict(v_cache=(1 << 20) + 4), dict(num_heads=6),
+           dict(dtype=9), dict(cache_dtype=pa.PA_F16), dict(dtype=pa.PA_F32,
+           cache_dtype=pa.PA_FP8_E4M3), dict(partition_size=520), dict(group_members=17),
+           dict(block_size=8),                                   # not the allocator's
+           dict(num_blocks=32)]                                  # smaller than its pool
+    for kw in bad:
+        assert create(_decoder_config(pa, **kw)) == pa.PA_ERR_INVALID_ARG, kw
+        assert not h.value
+    assert create(_decoder_config(pa), None) == pa.PA_ERR_INVALID_ARG
+    if not _has_gpu():
+        # a valid configuration gets past every host check to the first CUDA call
+        assert create(_decoder_config(pa)) == pa.PA_ERR_CUDA
+        assert create(_decoder_config(pa, cache_dtype=pa.PA_FP8_E4M3)) == pa.PA_ERR_CUDA
+        assert not h.value
+    info = pa.pa_step_info_t()
+    assert pa.lib.pa_decoder_bind(None, None, 0, 0) == pa.PA_ERR_INVALID_ARG
+    assert pa.lib.pa_decoder_step(None, 0, 0, 0, 0, None, None, None,
+                                  ctypes.byref(info)) == pa.PA_ERR_INVALID_ARG
+    assert pa.lib.pa_decoder_wait(None, 1) == pa.PA_ERR_INVALID_ARG
+    assert pa.lib.pa_decoder_query(None, None, None, None) == pa.PA_ERR_INVALID_ARG
+    assert pa.lib.pa_decoder_destroy(None) == pa.PA_ERR_INVALID_ARG
+
+
+def _has_gpu():
+    import torch
+    return torch.cuda.is_available()
+
+
 FAKE = 1 << 20  # an aligned, never-dereferenced pointer value: every call below fails
                 # its host-side checks before any launch
 

@@ -134,7 +134,7 @@ def test_fp8_decode_step_through_the_runtime(pa):
     pool_v = fp8.quantize(normal_fill((NB, Hkv, bs, D), "f32", 1.0, 12, 2), vs)
     kd, vd = torch.from_numpy(pool_k).cuda(), torch.from_numpy(pool_v).cuda()
     dec = PagedDecoder(kd, vd, Hq, 1 / math.sqrt(D), 16, g.permutation(NB), 64,
-                       kv_scales=(ks, vs))
+                       kv_scales=(ks, vs), query_dtype=torch.bfloat16)
     for s in range(S):
         dec.admit(s, int(lens[s]))
     dec.bind(range(S))
@@ -142,11 +142,11 @@ def test_fp8_decode_step_through_the_runtime(pa):
     nk = normal_fill((S, Hkv, D), "bf16", 1.0, 12, 4)
     nv = normal_fill((S, Hkv, D), "bf16", 1.0, 12, 5)
     out = torch.empty((S, Hq, D), dtype=torch.bfloat16, device="cuda")
-    dec.step(to_dev(q, "bf16"), to_dev(nk, "bf16"), to_dev(nv, "bf16"), out)
+    meta = dec.step(to_dev(q, "bf16"), to_dev(nk, "bf16"), to_dev(nv, "bf16"), out)
     torch.cuda.synchronize()
     assert pa.pa_device_error_read() == 0
-    tables, sl = dec.h_tables.numpy().copy(), dec.h_lens.numpy().copy()
-    slots = dec.h_slots.numpy().copy()
+    tables, sl = meta.tables.copy(), meta.lens.copy()
+    slots = meta.slots.copy()
     # oracle: quantize the new token into its slot, attend over dequantized values
     for s, slot in enumerate(slots):
         b, o = divmod(int(slot), bs)

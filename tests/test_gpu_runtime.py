@@ -44,3 +44,54 @@ def test_host_buffer_steps_match_device_steps():
     for i in range(steps):
         events[i].synchronize()
         assert torch.equal(outs_h[i], refs[i].cpu()), f"step {i}"
+
+
+def test_rolling_and_growing_steps_rebind_and_partition_choice():
+    import paged_kv_cache_342_b200 as pa
+    import paged_kv_cache_342_b200.runtime as rt
+    import oracle.attention as oatt
+    from gpu_util import assert_close, out_f64, to_host
+    S, Hq, Hkv, D, bs, NB, MB = 6, 16, 2, 128, 16, 256, 40
+    g = np.random.default_rng(3)
+    kd = to_dev(normal_fill((NB, Hkv, bs, D), "bf16", 1.0, 3, 1), "bf16")
+    vd = to_dev(normal_fill((NB, Hkv, bs, D), "bf16", 1.0, 3, 2), "bf16")
+    dec = rt.PagedDecoder(kd, vd, Hq, 1 / math.sqrt(D), MB, g.permutation(NB), 0)
+    lens0 = g.integers(40, 500, S)
+    for s in range(S):
+        dec.admit(s, int(lens0[s]))
+    dec.bind(range(S), rolling=True)
+    assert dec.partition_size == pa.pa_decode_partition_size(pa.PA_BF16, S, Hq, Hkv, D, bs,
+                                                             MB * bs)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def step(n, events=None):
+        q, k, v = (to_dev(normal_fill(sh, "bf16", 1.0, 60 + n, j), "bf16")
+                   for j, sh in enumerate(((n, Hq, D), (n, Hkv, D), (n, Hkv, D))))
+        out = torch.empty((n, Hq, D), dtype=torch.bfloat16, device="cuda")
+        meta = dec.step(q, k, v, out, events=events)
+        return meta, q, out
+
+    for _ in range(3):                                   # rolling: the same lengths
+        meta, _, _ = step(S, ev)
+        assert np.array_equal(meta.lens, lens0 + 1)
+    torch.cuda.synchronize()
+    assert ev[0].elapsed_time(ev[1]) > 0
+
+    dec.bind([4, 1, 2], rolling=False)                   # a smaller batch, growing
+    for i in range(3):
+        meta, q, out = step(3)
+        assert np.array_equal(meta.lens, lens0[[4, 1, 2]] + 2 + i)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    want = oatt.paged_decode_attention(to_host(q, "bf16"), to_host(kd, "bf16"),
+                                       to_host(vd, "bf16"), meta.tables.copy(),
+                                       meta.lens.copy(), 1 / math.sqrt(D), bs, Hkv, "bf16")
+    assert_close(out_f64(out), want, "bf16", "after rebind")
+
+    dec.bind(range(S), rolling=False)                    # back to the larger batch
+    meta, q, out = step(S)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    assert meta.kernels == 2 + (1 if -(-meta.max_len // dec.partition_size) > 1 else 0)
+    with pytest.raises(ValueError):                      # tensors must fit the batch
+        dec.step(q[:2], q[:2, :Hkv], q[:2, :Hkv], out[:2])

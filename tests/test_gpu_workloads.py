@@ -73,9 +73,9 @@ def test_workload_step(pa, name, fork_step):
     meta = dec.step(to_dev(inp.q, dt), to_dev(inp.new_k, dt), to_dev(inp.new_v, dt), out)
     torch.cuda.synchronize()
     assert pa.pa_device_error_read() == 0
-    slots_c = dec.h_slots.numpy().copy()
-    pairs_c = meta["pairs"].copy()
-    tables_c, lens_c = dec.h_tables.numpy().copy(), dec.h_lens.numpy().copy()
+    slots_c = meta.slots.copy()
+    pairs_c = meta.pairs.copy()
+    tables_c, lens_c = meta.tables.copy(), meta.lens.copy()
 
     # ---- oracle (in place on the host pool: the device has its own copy) -----
     seqs, heads = _sample(cfg, name)
