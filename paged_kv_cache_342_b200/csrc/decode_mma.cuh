@@ -74,6 +74,27 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
+// Four e4m3 codes (bytes 0..3 of w) -> f16x2 (codes 0,1) and f16x2 (codes 2,3), exact,
+// by the hardware convert.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2_cvt(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const __half2_raw l = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xffffu),
+                                                   __NV_E4M3);
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16),
+                                                   __NV_E4M3);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+}
+// Codes (byte0, byte2) -> f16x2 `even`, (byte1, byte3) -> f16x2 `odd`, each value the
+// code's times 2^-8, by bit placement: a code s|eeee|mmm becomes the f16 s|0eeee|mmm0000000
+// (exponent bias 15 instead of 7; subnormals map to f16 subnormals the same way).
+__device__ __forceinline__ uint32_t e4m3_place(uint32_t x) {  // x = [c1 0 c0 0] bytes
+  return (x & 0x80008000u) | ((x >> 1) & 0x3f803f80u);
+}
+__device__ __forceinline__ void e4m3_pairs_to_f16x2_bits(uint32_t w, uint32_t& even,
+                                                         uint32_t& odd) {
+  even = e4m3_place(__byte_perm(w, 0u, 0x2404));
+  odd = e4m3_place(__byte_perm(w, 0u, 0x3414));
+}
 // 2-D tiled TMA load of one box into shared memory, completion on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
@@ -85,7 +106,21 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 
 // FP8: the cache holds e4m3 codes; TMA lands them as 128-element x BS-row slabs and
-// the consuming warp converts them (exactly) into 16-bit tiles of its own.
+// the MMA operands are loaded straight from them with ldmatrix (a pair of codes is
+// one 16-bit ldmatrix element) and converted to f16 in registers, exactly:
+//   - K (A of S^T = K.Q^T): a thread holds 4 consecutive dims of one token; the
+//     k-order of each 16-dim step is permuted (dims 4t..4t+1 and 4t+2..4t+3 play
+//     k = 2t..2t+1 and 2t+8..2t+9), and Q^T's B fragments use the same permutation;
+//   - V (A of O^T += V^T.P^T): the transposing ldmatrix gives a thread 2 tokens x 2
+//     dims; even dims form rows 0-7 of the m16 tile, odd dims rows 8-15, and the
+//     epilogue puts the dims back in order.
+// Conversions: K codes through the hardware e4m3x2 -> f16x2 convert; V codes by
+// bit placement (sign to bit 15, the 7 magnitude bits to bits 13..7 of the f16),
+// which is the code's value times 2^-8 for every finite code (normal and subnormal
+// alike), the 2^8 going into v_scale.  The split keeps both the conversion unit and
+// the integer ALU busy: converting K by bit placement as well made the kernel ALU
+// bound (294 us against 254 us on the long-context GQA shape).  Codes 0x7F / 0xFF (NaN) are not special-cased
+// on that path; a cache holds them only for NaN inputs.
 template <typename T, int D, int BS, int NT, int NW, int NST, bool FP8 = false>
 struct MmaCfg {
   static constexpr int kHalves = D / 64;         // 128-byte column slabs per 16-bit row
@@ -94,11 +129,10 @@ struct MmaCfg {
   static constexpr int kF8Slabs = D / 128;       // 128-byte slabs per fp8 row
   static constexpr int kF8Tile = BS * D;         // fp8 tile bytes
   static constexpr int kStageBytes = FP8 ? 2 * kF8Tile : 2 * kTileBytes;  // K + V as stored
-  static constexpr int kConvBytes = FP8 ? 2 * kTileBytes : 0;  // per-warp 16-bit K + V
   static constexpr int kTT = BS / 16;            // 16-token row tiles per block
   static constexpr int kKS = D / 16;             // k-steps of q.K / m-tiles of V^T
   static constexpr int kHeads = 8 * NT;
-  static constexpr int kStageArea = NW * NST * kStageBytes + NW * kConvBytes;
+  static constexpr int kStageArea = NW * NST * kStageBytes;
   static constexpr int kRedBytes = NW * kHeads * (D + 2) * 4;
   static constexpr int kSmemBytes =
       1024 + (kStageArea > kRedBytes ? kStageArea : kRedBytes) + NW * NST * 8;
@@ -205,8 +239,6 @@ __global__ void __launch_bounds__(NW * 32)
       p.block_tables + static_cast<int64_t>(table_seq) * p.max_blocks_per_seq + tok_begin / BS;
 
   const uint32_t stage0 = base + warp * NST * C::kStageBytes;
-  // FP8: this warp's 16-bit K and V tiles (the stages hold the fp8 codes)
-  const uint32_t conv0 = base + NW * NST * C::kStageBytes + warp * C::kConvBytes;
   const uint32_t bar0 = base + (C::kSmemBytes - 1024 - NW * NST * 8) + warp * NST * 8;
   if (lane == 0) {
 #pragma unroll
@@ -216,7 +248,8 @@ __global__ void __launch_bounds__(NW * 32)
   __syncwarp();
 
   // Q^T as B fragments: qb[nt][ks][0] = q[column nt*8+g8][16ks + 2t4 .. +1], [1] = +8
-  // dims; a column with no member gets zeros (its result is never written)
+  // dims (FP8: dims 16ks + 4t4 .. +1 and +2 .. +3, the K operand's permutation); a
+  // column with no member gets zeros (its result is never written)
   uint32_t qb[NT][KS][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -224,9 +257,9 @@ __global__ void __launch_bounds__(NW * 32)
     const TQ* qp0 = static_cast<const TQ*>(p.q) + static_cast<int64_t>(row < 0 ? 0 : row) * D;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
-      const TQ* qp = qp0 + ks * 16 + 2 * t4;
+      const TQ* qp = qp0 + ks * 16 + (FP8 ? 4 * t4 : 2 * t4);
       qb[nt][ks][0] = row < 0 ? 0u : q_pair<T, TQ>(qp);
-      qb[nt][ks][1] = row < 0 ? 0u : q_pair<T, TQ>(qp + 8);
+      qb[nt][ks][1] = row < 0 ? 0u : q_pair<T, TQ>(qp + (FP8 ? 2 : 8));
     }
   }
 
@@ -298,47 +331,12 @@ __global__ void __launch_bounds__(NW * 32)
       break;
     }
     if (!((bad >> st) & 1u)) {
-      uint32_t kt = stage0 + st * C::kStageBytes;
-      uint32_t vt = kt + C::kTileBytes;
+      const uint32_t kt = stage0 + st * C::kStageBytes;
+      const uint32_t vt = kt + (FP8 ? C::kF8Tile : C::kTileBytes);
       const int valid = min(BS, tok_end - (tok_begin + (warp + k * NW) * BS));
-      if constexpr (FP8) {
-        // e4m3 -> f16, exactly.  Lane = one 16-byte column chunk c of the fp8 rows
-        // (16 codes) in rows r0, r0 + RPP, ...: a quarter warp reads one 128-byte slab
-        // row; each chunk becomes f16 chunks 2c and 2c+1, stored in an order that
-        // puts the two halves of a quarter warp on different banks.
-        constexpr int CPR = D / 16;          // fp8 chunks per row
-        constexpr int RPP = 32 / CPR;        // rows per pass
-        const int c = lane % CPR, r0 = lane / CPR;
-        const int first = (c & 4) ? 1 : 0;   // store order of the two f16 chunks
-        const uint8_t* src = smem + (kt - base) + (c >> 3) * C::kSlabBytes;
-        uint8_t* dst = smem + (conv0 - base);
-#pragma unroll
-        for (int tv = 0; tv < 2; ++tv) {
-#pragma unroll
-          for (int r = r0; r < BS; r += RPP) {
-            const uint4 codes = *reinterpret_cast<const uint4*>(
-                src + tv * C::kF8Tile + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-            const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
-            uint32_t h[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
-                  static_cast<__nv_fp8x2_storage_t>(w[u >> 1] >> (16 * (u & 1))), __NV_E4M3);
-              h[u] = *reinterpret_cast<const uint32_t*>(&hr);
-            }
-            uint8_t* o = dst + tv * C::kTileBytes;
-            const uint4 lo = make_uint4(h[0], h[1], h[2], h[3]);
-            const uint4 hi = make_uint4(h[4], h[5], h[6], h[7]);
-            *reinterpret_cast<uint4*>(o + swz<BS>(r, 2 * c + first)) = first ? hi : lo;
-            *reinterpret_cast<uint4*>(o + swz<BS>(r, 2 * c + 1 - first)) = first ? lo : hi;
-          }
-        }
-        __syncwarp();
-        kt = conv0;
-        vt = conv0 + C::kTileBytes;
-      }
-      if (valid < BS) {
-        // zero the V rows past the end: 16 bytes per lane per step
+      if (!FP8 && valid < BS) {
+        // zero the V rows past the end (0 * NaN would poison the tile; the FP8 path's
+        // V conversion never makes a NaN): 16 bytes per lane per step
         uint8_t* vg = smem + (vt - base);
         const int nchunks = (BS - valid) * (D / 8);
         for (int i = lane; i < nchunks; i += 32) {
@@ -360,12 +358,32 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {
           const int r = tt * 16 + (mi & 1) * 8 + ri;
+          if constexpr (FP8) {
+            // one ldmatrix.x4 = 16 tokens x 32 dims of codes = two k-steps
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            uint32_t a[4];
-            ldsm_x4(kt + swz<BS>(r, 2 * ks + (mi >> 1)), a);
+            for (int kp = 0; kp < KS / 2; ++kp) {
+              uint32_t w[4];
+              ldsm_x4(kt + swz<BS>(r, 2 * kp + (mi >> 1)), w);
+              uint32_t a0[4], a1[4];
+              e4m3x4_to_f16x2x2_cvt(w[0], a0[0], a0[2]);
+              e4m3x4_to_f16x2x2_cvt(w[1], a0[1], a0[3]);
+              e4m3x4_to_f16x2x2_cvt(w[2], a1[0], a1[2]);
+              e4m3x4_to_f16x2x2_cvt(w[3], a1[1], a1[3]);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) Ops::mma(sacc[tt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+              for (int nt = 0; nt < NT; ++nt) {
+                Ops::mma(sacc[tt][nt], a0, qb[nt][2 * kp][0], qb[nt][2 * kp][1]);
+                Ops::mma(sacc[tt][nt], a1, qb[nt][2 * kp + 1][0], qb[nt][2 * kp + 1][1]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              uint32_t a[4];
+              ldsm_x4(kt + swz<BS>(r, 2 * ks + (mi >> 1)), a);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                Ops::mma(sacc[tt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+            }
           }
         }
       }
@@ -421,13 +439,34 @@ __global__ void __launch_bounds__(NW * 32)
         const int mi = lane >> 3, ri = lane & 7;
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {
-          const int r = tt * 16 + (mi >> 1) * 8 + ri;
+          if constexpr (FP8) {
+            // one transposing ldmatrix.x4 = 16 tokens x 32 dims of codes = two m-tiles
+            const int r = tt * 16 + (mi & 1) * 8 + ri;
 #pragma unroll
-          for (int mt = 0; mt < KS; ++mt) {
-            uint32_t a[4];
-            ldsm_x4_trans(vt + swz<BS>(r, 2 * mt + (mi & 1)), a);
+            for (int mp = 0; mp < KS / 2; ++mp) {
+              uint32_t w[4];
+              ldsm_x4_trans(vt + swz<BS>(r, 2 * mp + (mi >> 1)), w);
+              uint32_t a0[4], a1[4];
+              e4m3_pairs_to_f16x2_bits(w[0], a0[0], a0[1]);
+              e4m3_pairs_to_f16x2_bits(w[1], a0[2], a0[3]);
+              e4m3_pairs_to_f16x2_bits(w[2], a1[0], a1[1]);
+              e4m3_pairs_to_f16x2_bits(w[3], a1[2], a1[3]);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) Ops::mma(oacc[mt][nt], a, pb[tt][nt][0], pb[tt][nt][1]);
+              for (int nt = 0; nt < NT; ++nt) {
+                Ops::mma(oacc[2 * mp][nt], a0, pb[tt][nt][0], pb[tt][nt][1]);
+                Ops::mma(oacc[2 * mp + 1][nt], a1, pb[tt][nt][0], pb[tt][nt][1]);
+              }
+            }
+          } else {
+            const int r = tt * 16 + (mi >> 1) * 8 + ri;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+              uint32_t a[4];
+              ldsm_x4_trans(vt + swz<BS>(r, 2 * mt + (mi & 1)), a);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                Ops::mma(oacc[mt][nt], a, pb[tt][nt][0], pb[tt][nt][1]);
+            }
           }
         }
       }
@@ -467,8 +506,9 @@ __global__ void __launch_bounds__(NW * 32)
       float* r = red + (warp * C::kHeads + nt * 8 + 2 * t4 + j) * (D + 2);
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
-        r[mt * 16 + g8] = oacc[mt][nt][j];
-        r[mt * 16 + g8 + 8] = oacc[mt][nt][2 + j];
+        // FP8: rows g8 / g8 + 8 of an m-tile hold dims 2g8 / 2g8 + 1
+        r[mt * 16 + (FP8 ? 2 * g8 : g8)] = oacc[mt][nt][j];
+        r[mt * 16 + (FP8 ? 2 * g8 + 1 : g8 + 8)] = oacc[mt][nt][2 + j];
       }
       if (g8 == 0) {
         r[D] = m[nt][j];
@@ -489,7 +529,8 @@ __global__ void __launch_bounds__(NW * 32)
       num = fmaf(r[d], f, num);
       den = fmaf(r[D + 1], f, den);
     }
-    const float o = den > 0.f ? num / den * p.v_scale : 0.f;
+    // FP8: the V operands carry the code values times 2^-8
+    const float o = den > 0.f ? num / den * (FP8 ? p.v_scale * 256.f : p.v_scale) : 0.f;
     if (!col_ok[hh]) continue;
     const int64_t row = col_row[hh];
     if (nparts == 1) {

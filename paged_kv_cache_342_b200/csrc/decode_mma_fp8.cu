@@ -1,6 +1,7 @@
 // Tensor-core decode partition kernels for fp8 (e4m3) caches with grouped-query
-// heads: the codes arrive by TMA and are converted exactly to f16 tiles in shared
-// memory; q (bf16 or f16) becomes f16 operands, P is f16, accumulators float32.
+// heads: the codes arrive by TMA, ldmatrix loads them as MMA fragments and they are
+// converted exactly to f16 in registers; q (bf16 or f16) becomes f16 operands, P is
+// f16, accumulators float32.
 #include "decode_mma.cuh"
 #include "tensor_map.cuh"
 
@@ -9,13 +10,13 @@ namespace {
 
 template <typename TQ, int D, int BS, int NT>
 cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
-  // about 64 KiB per CTA: per warp NST fp8 stages plus one 16-bit K+V tile pair
+  // about 32 KiB of fp8 stages per CTA: warps with two stages each (1-4), then 2-4
+  // stages; small CTAs, so that several per SM hide the conversion work
   constexpr int kStage = 2 * BS * D;      // fp8 K + V
-  constexpr int kConv = 2 * BS * D * 2;   // 16-bit K + V
-  constexpr int kBudget = 32768;  // small stages: more CTAs per SM hide the conversion latency
-  constexpr int kW = kBudget / (2 * kStage + kConv);
+  constexpr int kBudget = 32768;
+  constexpr int kW = kBudget / (2 * kStage);
   constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
-  constexpr int kRaw = (kBudget / NW - kConv) / kStage;
+  constexpr int kRaw = kBudget / (NW * kStage);
   constexpr int NST = kRaw < 2 ? 2 : (kRaw > 4 ? 4 : kRaw);
   using C = MmaCfg<__half, D, BS, NT, NW, NST, true>;
   const uint64_t rows = static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * BS;
