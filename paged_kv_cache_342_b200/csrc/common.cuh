@@ -98,6 +98,14 @@ __device__ __forceinline__ void vec_to_float(const uint4& v, float* f, __nv_fp8_
   }
 }
 
+// e4m3 -> f16 by bit placement: with x = [c1 0 c0 0] (two codes in the high bytes of
+// the halves), a code s|eeee|mmm becomes the f16 s|0eeee|mmm0000000: exponent bias 15
+// instead of 7, so the f16 is the code's value times 2^-8, exactly, for every finite
+// code (subnormal codes become f16 subnormals the same way).  Integer ALU only.
+__device__ __forceinline__ uint32_t e4m3_place(uint32_t x) {
+  return (x & 0x80008000u) | ((x >> 1) & 0x3f803f80u);
+}
+
 __device__ __forceinline__ void store_elem(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void store_elem(__half* p, float x) { *p = __float2half_rn(x); }

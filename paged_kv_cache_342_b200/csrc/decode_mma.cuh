@@ -85,11 +85,7 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2_cvt(uint32_t w, uint32_t& lo, 
   hi = *reinterpret_cast<const uint32_t*>(&h);
 }
 // Codes (byte0, byte2) -> f16x2 `even`, (byte1, byte3) -> f16x2 `odd`, each value the
-// code's times 2^-8, by bit placement: a code s|eeee|mmm becomes the f16 s|0eeee|mmm0000000
-// (exponent bias 15 instead of 7; subnormals map to f16 subnormals the same way).
-__device__ __forceinline__ uint32_t e4m3_place(uint32_t x) {  // x = [c1 0 c0 0] bytes
-  return (x & 0x80008000u) | ((x >> 1) & 0x3f803f80u);
-}
+// code's times 2^-8 (e4m3_place).
 __device__ __forceinline__ void e4m3_pairs_to_f16x2_bits(uint32_t w, uint32_t& even,
                                                          uint32_t& odd) {
   even = e4m3_place(__byte_perm(w, 0u, 0x2404));
