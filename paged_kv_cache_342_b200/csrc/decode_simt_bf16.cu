@@ -5,17 +5,27 @@
 namespace pa {
 namespace {
 
-// Stage = one block's K and V runs.  About 64 KiB of stages per CTA (three CTAs per
-// SM): as many warps as fit with two stages each (1-4), then 2-4 stages per warp.
-template <int D, int BS, int GS>
-cudaError_t launch_auto(const DecodeParams& p, cudaStream_t st) {
+// Stage = one block's K and V runs.  kBudget bytes of stages per CTA: as many warps
+// as fit with two stages each (1-4), then 2-4 stages per warp.
+template <int D, int BS, int GS, int kBudget>
+cudaError_t launch_budget(const DecodeParams& p, cudaStream_t st) {
   constexpr int kStage = 2 * BS * D * static_cast<int>(sizeof(__nv_bfloat16));
-  constexpr int kBudget = 65536;
   constexpr int kW = kBudget / (2 * kStage);
   constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
   constexpr int kRaw = kBudget / (NW * kStage);
   constexpr int NST = kRaw < 2 ? 2 : (kRaw > 4 ? 4 : kRaw);
   return launch_simt<__nv_bfloat16, __nv_bfloat16, D, BS, GS, NW, NST>(p, st);
+}
+
+// About 64 KiB per CTA (three CTAs per SM) for whole sequences and long partitions.
+// When prefix groups cover every partition but each sequence's last one, the CTAs
+// here read only those short tails (tens to a few hundred tokens): then 32 KiB CTAs,
+// twice as many per SM, overlap their start-up and epilogue better.
+template <int D, int BS, int GS>
+cudaError_t launch_auto(const DecodeParams& p, cudaStream_t st) {
+  if (p.part_base > 0 && p.max_parts - p.part_base == 1)
+    return launch_budget<D, BS, GS, 32768>(p, st);
+  return launch_budget<D, BS, GS, 65536>(p, st);
 }
 
 template <int D, int GS>
