@@ -212,6 +212,20 @@ def hbm_peak():
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
+def host_cpu() -> dict:
+    """The host's logical CPU count and model name (for the CPU baseline)."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"logical_cpus": os.cpu_count(), "model": model}
+
+
 class OracleTimer:
     """The CPU oracle's decode attention on whole sequences (all heads)."""
 
@@ -311,7 +325,15 @@ def run_ours(args, cfg):
         timer = OracleTimer(cfg, make_inputs(cfg, args.seed))
         gbs, sps, desc = timer.budgeted(12.0)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": timer.threads, "kind": "oracle",
-               "sample": desc, "seqs_per_s": round(sps, 3)}
+               "sample": desc, "seqs_per_s": round(sps, 3), "host": host_cpu()}
+        try:  # the same oracle on one core
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(1):
+                gbs1, sps1, desc1 = timer.budgeted(4.0)
+            cpu["single_core"] = {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
+                                  "sample": desc1, "seqs_per_s": round(sps1, 3)}
+        except ImportError:
+            pass
         del timer
 
     torch.cuda.set_device(local)
@@ -462,6 +484,7 @@ def run_ours(args, cfg):
                       + " (partition kernel + log-sum-exp merge)",
             "bytes_per_launch": int(dec_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 2),
             "launches_timed": len(dec_ms),
+            "median_launch_us": round(statistics.median(dec_ms) * 1e3, 2),
             "frac_of_nominal_8000": round(achieved / 8000.0, 4),
             "traffic": recorded_traffic(cfg)}
     if uniq is not None:
