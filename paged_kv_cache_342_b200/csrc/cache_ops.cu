@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ k_cache,
     uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int64_t num_tokens,
     int num_kv_heads, int nvr, int block_size, int64_t num_slots, uint32_t* err) {
+  allow_dependents();  // the decode kernel after this one may start its prologue
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * nvr;
   const int64_t total = num_tokens * per_token;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
     uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int64_t num_tokens,
     int num_kv_heads, int head_dim, int block_size, int64_t num_slots, float k_inv,
     float v_inv, uint32_t* err) {
+  allow_dependents();  // the decode kernel after this one may start its prologue
   constexpr int VQ = ElemTraits<TQ>::kVec;
   const int nvr = head_dim / 16;  // output vectors per (token, head) row
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * nvr;

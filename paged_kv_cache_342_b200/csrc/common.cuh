@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/pa.h"
 
 namespace pa {
@@ -198,6 +200,35 @@ void note_cuda_error(cudaError_t e);
 
 // Raise a kernel's dynamic shared-memory limit once per device.  The kernel is a
 // template argument so every instantiation keeps its own per-device flags.
+// Programmatic dependent launch (sm_90+): a kernel launched with launch_dependent()
+// may be scheduled while the kernel before it on the stream is finishing, once that
+// kernel's CTAs have called allow_dependents() (or exited); its CTAs then block in
+// grid_dependency_wait(), their first statement, until that kernel has completed and
+// its writes are visible, so nothing is ever read early, whatever kernel precedes.
+// What overlaps is the launch and CTA start-up.  Both are no-ops for kernels launched
+// the ordinary way.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <auto Kern>
 cudaError_t ensure_smem_limit(int bytes) {
   static bool done[64] = {};

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
   constexpr int DPL = D / 32;
   __shared__ float sh_acc[8][D];
   __shared__ float sh_den[8];
+  grid_dependency_wait();  // the partials of the partition kernel before this one
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_per_cta = 8 / wpr;
   const int wsub = warp % wpr;
@@ -134,8 +135,18 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
   }
 }
 
+// dependent: launched to overlap the tail of the partition kernel just before it on
+// the stream (not after an event wait, which must hold in full)
+template <typename T, int D>
+cudaError_t launch_merge_d(const DecodeParams& p, int grid, int wpr, bool dependent,
+                           cudaStream_t st) {
+  if (dependent) return launch_dependent(merge_kernel<T, D>, dim3(grid), dim3(256), 0, st, p, wpr);
+  merge_kernel<T, D><<<grid, 256, 0, st>>>(p, wpr);
+  return cudaGetLastError();
+}
+
 template <typename T>
-cudaError_t launch_merge(const DecodeParams& p, cudaStream_t st) {
+cudaError_t launch_merge(const DecodeParams& p, bool dependent, cudaStream_t st) {
   // warps per row: enough that each walks at most ~32 partitions
   int wpr = 1;
   while (wpr < 8 && p.max_parts > 32 * wpr) wpr *= 2;
@@ -143,12 +154,11 @@ cudaError_t launch_merge(const DecodeParams& p, cudaStream_t st) {
   const int rows_per_cta = 8 / wpr;
   const int grid = (rows + rows_per_cta - 1) / rows_per_cta;
   switch (p.head_dim) {
-    case 64: merge_kernel<T, 64><<<grid, 256, 0, st>>>(p, wpr); break;
-    case 128: merge_kernel<T, 128><<<grid, 256, 0, st>>>(p, wpr); break;
-    case 256: merge_kernel<T, 256><<<grid, 256, 0, st>>>(p, wpr); break;
+    case 64: return launch_merge_d<T, 64>(p, grid, wpr, dependent, st);
+    case 128: return launch_merge_d<T, 128>(p, grid, wpr, dependent, st);
+    case 256: return launch_merge_d<T, 256>(p, grid, wpr, dependent, st);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -465,9 +475,10 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     return PA_ERR_CUDA;
   }
   if (ws.parts > 1) {
-    e = dtype == PA_F32    ? launch_merge<float>(p, st)
-        : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, st)
-                           : launch_merge<__half>(p, st);
+    const bool dependent = joined == nullptr;
+    e = dtype == PA_F32    ? launch_merge<float>(p, dependent, st)
+        : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, dependent, st)
+                           : launch_merge<__half>(p, dependent, st);
     if (e != cudaSuccess) {
       note_cuda_error(e);
       return PA_ERR_CUDA;

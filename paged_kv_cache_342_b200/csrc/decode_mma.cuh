@@ -168,6 +168,9 @@ template <typename T, typename TQ, int D, int BS, int NT, int NW, int NST, bool 
 __global__ void __launch_bounds__(NW * 32)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
+  // launched to overlap the end of the kernel before it on the stream (typically the
+  // write of the new tokens' K/V): nothing is read before that kernel is done
+  grid_dependency_wait();
   using C = MmaCfg<T, D, BS, NT, NW, NST, FP8>;
   using Ops = MmaOps<T>;
   constexpr unsigned FULL = 0xffffffffu;
@@ -473,6 +476,7 @@ __global__ void __launch_bounds__(NW * 32)
       ++issued;
     }
   }
+  allow_dependents();  // the merge may launch now; it waits for this grid's writes
   if (aborted) {
     if (lane == 0) set_error(p.err, PA_DEVERR_TIMEOUT);
     for (; k < issued; ++k) mbar_wait_bounded(bar0 + 8 * (k % NST), (k / NST) & 1);

@@ -28,8 +28,11 @@ cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   constexpr auto kern = decode_mma_kernel<__nv_bfloat16, __nv_bfloat16, D, BS, NT, NW, NST, GROUP, false>;
   cudaError_t e = ensure_smem_limit<kern>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, NW * 32, C::kSmemBytes, st>>>(p, tmk, tmv);
-  return cudaGetLastError();
+  if constexpr (GROUP) {
+    kern<<<grid, NW * 32, C::kSmemBytes, st>>>(p, tmk, tmv);
+    return cudaGetLastError();
+  }
+  return launch_dependent(kern, grid, dim3(NW * 32), C::kSmemBytes, st, p, tmk, tmv);
 }
 
 template <int D, int NT, bool GROUP>

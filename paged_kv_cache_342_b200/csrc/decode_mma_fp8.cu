@@ -29,8 +29,7 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
   cudaError_t e = ensure_smem_limit<kern>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_heads / C::kHeads, p.num_seqs, p.max_parts - p.part_base);
-  kern<<<grid, NW * 32, C::kSmemBytes, st>>>(p, tmk, tmv);
-  return cudaGetLastError();
+  return launch_dependent(kern, grid, dim3(NW * 32), C::kSmemBytes, st, p, tmk, tmv);
 }
 
 template <typename TQ, int D, int NT>

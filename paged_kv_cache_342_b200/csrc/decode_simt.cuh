@@ -80,6 +80,9 @@ __device__ __forceinline__ int group_parts(const DecodeParams& p, int s, int L) 
 // T = cache element type, TQ = query / output type (equal except for fp8 caches).
 template <typename T, typename TQ, int D, int BS, int GS, int NW, int NST>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams p) {
+  // launched to overlap the end of the kernel before it on the stream (typically the
+  // write of the new tokens' K/V): nothing is read before that kernel is done
+  grid_dependency_wait();
   using C = SimtCfg<T, D, BS, GS, NW, NST>;
   constexpr int VQ = ElemTraits<TQ>::kVec;  // query elements per 16-byte vector
   static_assert(C::kVec % VQ == 0, "a cache vector spans whole query vectors");
@@ -257,6 +260,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
       ++issued;
     }
   }
+  allow_dependents();  // the merge may launch now; it waits for this grid's writes
   if (aborted) {
     if (lane == 0) set_error(p.err, PA_DEVERR_TIMEOUT);
     // let copies already in flight land before the shared memory is reused
@@ -341,8 +345,7 @@ cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream) {
   cudaError_t attr = ensure_smem_limit<kern>(C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
   dim3 grid(p.num_heads / GS, p.num_seqs, p.max_parts - p.part_base);
-  kern<<<grid, NW * 32, C::kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(kern, grid, dim3(NW * 32), C::kSmemBytes, stream, p);
 }
 
 }  // namespace pa

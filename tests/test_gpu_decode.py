@@ -270,3 +270,43 @@ def test_grouped_first_part_too_high_is_reported(pa):
                                    torch.tensor([chunks[0][1]], dtype=torch.int32).cuda(), 1,
                                    chunks[0][1], ps, ws, first_part=2)
     assert pa.pa_device_error_read() == pa.DEVERR_GROUP
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (16, 2)])
+def test_decode_right_after_a_kernel_that_writes_its_inputs(pa, Hq, Hkv):
+    # the decode kernels are launched to overlap the end of the kernel before them on
+    # the stream; here that kernel writes q and the cache, so an early read would show
+    S, D, bs = 3, 128, 16
+    lens = np.array([700, 33, 1500], np.int32)
+    NB = int(sum(blocks_for(int(L), bs) for L in lens)) + 2
+    order = np.random.default_rng(4).permutation(NB).astype(np.int32)
+    tables = tables_from_order(lens, bs, order, int(max(blocks_for(int(L), bs) for L in lens)))
+    k = to_dev(normal_fill((NB, Hkv, bs, D), "bf16", 1.0, 21, 1), "bf16")
+    v = to_dev(normal_fill((NB, Hkv, bs, D), "bf16", 1.0, 21, 2), "bf16")
+    qs = [to_dev(normal_fill((S, Hq, D), "bf16", 1.0, 21, 3 + i), "bf16") for i in range(6)]
+    t_d, l_d = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    wsb = pa.pa_decode_workspace_bytes(S, Hq, D, int(lens.max()), 256)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+
+    def decode(q, out):
+        pa.pa_decode_attention(out, q, k, v, t_d, l_d, 1 / math.sqrt(D), bs, Hkv,
+                               int(lens.max()), 256, ws)
+
+    refs = []
+    for q in qs:
+        out = torch.empty_like(q)
+        decode(q, out)
+        refs.append(out)
+    torch.cuda.synchronize()
+    q_live = torch.zeros_like(qs[0])
+    outs = []
+    for i, q in enumerate(qs):
+        torch.mul(q, 1.0, out=q_live)          # a kernel writing q just before the decode
+        k.mul_(1.0)                             # and one rewriting the cache in place
+        out = torch.empty_like(q)
+        decode(q_live, out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    for i in range(len(qs)):
+        assert torch.equal(outs[i], refs[i]), f"iteration {i}"
