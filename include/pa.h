@@ -330,6 +330,16 @@ int pa_device_error_read(uint32_t* bits);
  */
 const char* pa_last_cuda_error(void);
 
+/*
+ * pa_selftest_bounded_wait - failure-detection check of the bounded waits.  Launches
+ * one thread that waits, with the same bounded mbarrier wait as the decode kernels, on
+ * an mbarrier that nothing ever completes.  After the bound (about one second of
+ * %globaltimer, or 2^26 polls) the wait gives up, the kernel sets PA_DEVERR_TIMEOUT in
+ * the device error word and returns, and the context stays usable.  Read the result
+ * with pa_device_error_read.  (Not part of the pages' method: a diagnostic.)
+ */
+int pa_selftest_bounded_wait(pa_stream_t stream);
+
 /* ------------------------------------------------------------------------- */
 /* Host block allocator                                                       */
 /* ------------------------------------------------------------------------- */

@@ -93,6 +93,7 @@ _sig("pa_decode_attention_grouped", _i32, _p, _p, _p, _p, _p, _p, _f, _i32, _i32
 _sig("pa_decode_uses_tensor_cores", _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_device_error_read", _i32, ctypes.POINTER(ctypes.c_uint32))
 _sig("pa_last_cuda_error", ctypes.c_char_p)
+_sig("pa_selftest_bounded_wait", _i32, _p)
 _sig("pa_alloc_create", _i32, _i64, _i32, _p, ctypes.POINTER(_p))
 _sig("pa_alloc_destroy", _i32, _p)
 _sig("pa_seq_add", _i32, _p, _i64, _i64)
@@ -335,6 +336,10 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, seq_le
 def pa_decode_uses_tensor_cores(dtype_code, num_heads, num_kv_heads, head_dim, block_size) -> bool:
     return bool(lib.pa_decode_uses_tensor_cores(dtype_code, num_heads, num_kv_heads, head_dim,
                                                 block_size))
+
+
+def pa_selftest_bounded_wait(stream=None) -> None:
+    _check(lib.pa_selftest_bounded_wait(_stream(stream)), "pa_selftest_bounded_wait")
 
 
 def pa_device_error_read() -> int:

@@ -40,7 +40,32 @@ void note_cuda_error(cudaError_t e) {
            text ? text : "?");
 }
 
+// One thread waits, with the decode kernels' bounded wait, on an mbarrier that nothing
+// ever completes: the bound (about one second) must end the wait and report it.
+__global__ void bounded_wait_selftest_kernel(uint32_t* err) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+  mbar_init(b, 1);
+  mbar_init_fence();
+  if (!mbar_wait_bounded(b, 0)) set_error(err, PA_DEVERR_TIMEOUT);
+}
+
 }  // namespace pa
+
+extern "C" int pa_selftest_bounded_wait(pa_stream_t stream) {
+  uint32_t* err = pa::device_error_word();
+  if (!err) {
+    pa::note_cuda_error(cudaGetLastError());
+    return PA_ERR_CUDA;
+  }
+  pa::bounded_wait_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(err);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    pa::note_cuda_error(e);
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
 
 extern "C" const char* pa_last_cuda_error(void) { return pa::g_last_cuda_error; }
 
