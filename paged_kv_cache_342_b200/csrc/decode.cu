@@ -55,14 +55,38 @@ WsLayout ws_layout(int64_t num_seqs, int64_t num_heads, int64_t head_dim, int64_
 //   M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p
 // (m_p in base-2 logits, o_p normalised by its own l_p).  A CTA of 8 warps serves
 // 8/WPR rows with WPR warps each (WPR grows with the partition count, so long rows
-// are read by up to 8 warps at once); lanes own head_dim/32 consecutive elements,
-// each warp walks partitions wsub, wsub+WPR, ... four at a time, and the row's warps
-// combine their sums in shared memory.
+// are read by up to 8 warps at once); lanes own head_dim/32 consecutive elements.
+// Each warp walks partitions wsub, wsub+WPR, ... eight at a time with a running
+// maximum (earlier sums rescaled when it grows), so the partials are read in one pass
+// with eight loads in flight per lane; the row's warps then combine their (max, sum,
+// weighted output) in shared memory.
+template <int DPL>
+__device__ __forceinline__ void load_lane(const float* src, float (&o)[DPL]) {
+  if constexpr (DPL % 4 == 0) {
+#pragma unroll
+    for (int j = 0; j < DPL; j += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src + j);
+      o[j] = v.x;
+      o[j + 1] = v.y;
+      o[j + 2] = v.z;
+      o[j + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < DPL; j += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(src + j);
+      o[j] = v.x;
+      o[j + 1] = v.y;
+    }
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wpr) {
   constexpr int DPL = D / 32;
+  constexpr int U = 8;  // partitions in flight per warp
   __shared__ float sh_acc[8][D];
-  __shared__ float sh_den[8];
+  __shared__ float sh_den[8], sh_max[8];
   grid_dependency_wait();  // the partials of the partition kernel before this one
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_per_cta = 8 / wpr;
@@ -76,54 +100,64 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
   float acc[DPL];
 #pragma unroll
   for (int j = 0; j < DPL; ++j) acc[j] = 0.f;
-  float den = 0.f;
+  float den = 0.f, M = -INFINITY;
   if (nparts > 1) {
     const float* mrow = p.ws_m + static_cast<int64_t>(row) * p.max_parts;
     const float* lrow = p.ws_l + static_cast<int64_t>(row) * p.max_parts;
     const float* orow = p.ws_o + static_cast<int64_t>(row) * p.max_parts * D + lane * DPL;
-    float M = -INFINITY;
-    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, mrow[i]);
-    M = warp_max(M);
-    int i = wsub;
-    for (; i + 3 * wpr < nparts; i += 4 * wpr) {
-      float w[4], o[4][DPL];
+    for (int i = wsub; i < nparts; i += U * wpr) {
+      float mv[U], lv[U], o[U][DPL];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int pi = i + u * wpr;
-        w[u] = lrow[pi] * exp2_safe(mrow[pi], M);
-        const float* src = orow + static_cast<int64_t>(pi) * D;
+        if (pi < nparts) {
+          mv[u] = mrow[pi];
+          lv[u] = lrow[pi];
+          load_lane<DPL>(orow + static_cast<int64_t>(pi) * D, o[u]);
+        } else {
+          mv[u] = -INFINITY;
+          lv[u] = 0.f;
 #pragma unroll
-        for (int j = 0; j < DPL; j += 2) {
-          const float2 v = *reinterpret_cast<const float2*>(src + j);
-          o[u][j] = v.x;
-          o[u][j + 1] = v.y;
+          for (int j = 0; j < DPL; ++j) o[u][j] = 0.f;
         }
       }
+      float mx = M;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        den += w[u];
+      for (int u = 0; u < U; ++u) mx = fmaxf(mx, mv[u]);
+      const float c = exp2_safe(M, mx);
+      den *= c;
 #pragma unroll
-        for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w[u], o[u][j], acc[j]);
+      for (int j = 0; j < DPL; ++j) acc[j] *= c;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float w = lv[u] * exp2_safe(mv[u], mx);
+        den += w;
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w, o[u][j], acc[j]);
       }
-    }
-    for (; i < nparts; i += wpr) {
-      const float w = lrow[i] * exp2_safe(mrow[i], M);
-      den += w;
-      const float* src = orow + static_cast<int64_t>(i) * D;
-#pragma unroll
-      for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w, src[j], acc[j]);
+      M = mx;
     }
   }
   if (wpr > 1) {
 #pragma unroll
     for (int j = 0; j < DPL; ++j) sh_acc[warp][lane * DPL + j] = acc[j];
-    if (lane == 0) sh_den[warp] = den;
+    if (lane == 0) {
+      sh_den[warp] = den;
+      sh_max[warp] = M;
+    }
     __syncthreads();
     if (wsub == 0) {
-      for (int w2 = 1; w2 < wpr; ++w2) {
+      float Mr = M;
+      for (int w2 = 1; w2 < wpr; ++w2) Mr = fmaxf(Mr, sh_max[warp + w2]);
+      const float c0 = exp2_safe(M, Mr);
+      den *= c0;
 #pragma unroll
-        for (int j = 0; j < DPL; ++j) acc[j] += sh_acc[warp + w2][lane * DPL + j];
-        den += sh_den[warp + w2];
+      for (int j = 0; j < DPL; ++j) acc[j] *= c0;
+      for (int w2 = 1; w2 < wpr; ++w2) {
+        const float c = exp2_safe(sh_max[warp + w2], Mr);
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) acc[j] = fmaf(c, sh_acc[warp + w2][lane * DPL + j], acc[j]);
+        den = fmaf(c, sh_den[warp + w2], den);
       }
     }
   }
