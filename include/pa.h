@@ -268,8 +268,12 @@ int pa_decode_uses_tensor_cores(int dtype, int num_heads, int num_kv_heads, int 
  * v_scale.  q and out are dtype (PA_BF16 or PA_F16); head_dim 128 or 256.  Groups of
  * 8 or 16 query heads per kv head with block_size 16/32 run on tensor cores (the codes
  * are loaded as MMA fragments and converted exactly to f16 in registers, q to f16, P
- * is f16); other shapes on CUDA cores.  The cache is half the bytes of a 16-bit one.
- * Codes 0x7F / 0xFF (NaN; written only for NaN inputs) give unspecified outputs.
+ * is f16); other shapes on CUDA cores, where the codes become f16 exactly and the
+ * products are mixed-precision f16 x f16 -> float32 FMAs: q is carried as f16 (a bf16 q
+ * times a power of two per head, exact apart from parts below 2^-24 of the head's
+ * largest element) and the softmax weights of p.V are rounded to f16.  The cache is
+ * half the bytes of a 16-bit one.  Codes 0x7F / 0xFF (NaN; written only for NaN
+ * inputs) give unspecified outputs.
  */
 int pa_decode_attention_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, const int32_t* seq_lens, float scale,

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
 #include <utility>
 
 #include "../../include/pa.h"
@@ -106,6 +107,43 @@ __device__ __forceinline__ void vec_to_float(const uint4& v, float* f, __nv_fp8_
 // code (subnormal codes become f16 subnormals the same way).  Integer ALU only.
 __device__ __forceinline__ uint32_t e4m3_place(uint32_t x) {
   return (x & 0x80008000u) | ((x >> 1) & 0x3f803f80u);
+}
+
+// ---- mixed-precision arithmetic for fp8 caches on CUDA cores -------------------
+// 16 e4m3 codes -> 8 f16x2 words (codes 2i, 2i+1 in word i, low half first), exact.
+__device__ __forceinline__ void e4m3x16_to_f16x2(const uint4& v, uint32_t* h) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>(w[i] >> (16 * j)), __NV_E4M3);
+      h[2 * i + j] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+  }
+}
+// c + a.lo * b.lo + a.hi * b.hi with f16 multiplicands and float32 sums (each step one
+// fused multiply-add of exact f16 products: fma.rn.f32.f16).
+__device__ __forceinline__ float fma_f16x2_f32(uint32_t a2, uint32_t b2, float c) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.f16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.f16 %0, ah, bh, %0;\n\t}"
+      : "+f"(c)
+      : "r"(a2), "r"(b2));
+  return c;
+}
+// c0 += p * v.lo, c1 += p * v.hi (f16 p and v, float32 sums).
+__device__ __forceinline__ void fma_f16_f16x2_f32(uint16_t p, uint32_t v2, float& c0,
+                                                  float& c1) {
+  asm("{\n\t.reg .b16 vl, vh;\n\t"
+      "mov.b32 {vl, vh}, %3;\n\t"
+      "fma.rn.f32.f16 %0, %2, vl, %0;\n\t"
+      "fma.rn.f32.f16 %1, %2, vh, %1;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "h"(p), "r"(v2));
 }
 
 __device__ __forceinline__ void store_elem(float* p, float x) { *p = x; }

@@ -77,6 +77,50 @@ __device__ __forceinline__ int group_parts(const DecodeParams& p, int s, int L) 
   return g < 0 ? 0 : (g < last ? g : last);
 }
 
+// fp8 caches: the query heads h0..h0+GS-1 of sequence s as f16 pairs for this lane's
+// elements (the same elements as the float path: vectors sub, sub+8, ... of VEC),
+// times 2^qe per head (a bf16 q scaled so that its largest magnitude lies in
+// [2^14, 2^15): every bf16 value of the row is then an f16, apart from parts below
+// 2^-24 of that maximum; an f16 q as it is), and sl2 = scale * log2(e) * 2^-qe.
+template <typename TQ, int D, int GS, int EPL, int NVL, int VEC>
+__device__ __forceinline__ void load_q_f16(const DecodeParams& p, int s, int h0, int sub,
+                                           uint32_t (&qh)[GS][EPL / 2], float (&sl2)[GS]) {
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int VQ = ElemTraits<TQ>::kVec;
+  const TQ* qb = static_cast<const TQ*>(p.q) + (static_cast<int64_t>(s) * p.num_heads + h0) * D;
+#pragma unroll
+  for (int g = 0; g < GS; ++g) {
+    float f[EPL];
+#pragma unroll
+    for (int k = 0; k < NVL; ++k)
+#pragma unroll
+      for (int u = 0; u < VEC / VQ; ++u) {
+        const uint4 v =
+            __ldg(reinterpret_cast<const uint4*>(qb + g * D + (sub + 8 * k) * VEC + u * VQ));
+        vec_to_float(v, &f[k * VEC + u * VQ], TQ());
+      }
+    int qe = 0;
+    if constexpr (std::is_same<TQ, __nv_bfloat16>::value) {
+      float mx = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) mx = fmaxf(mx, fabsf(f[e]));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+      int ex = 0;
+      if (mx > 0.f) frexpf(mx, &ex);  // mx in [2^(ex-1), 2^ex)
+      qe = max(-126, min(126, 15 - ex));
+    }
+    const float sc = ldexpf(1.f, qe);
+#pragma unroll
+    for (int e = 0; e < EPL / 2; ++e) {
+      const __half2 h2 = __floats2half2_rn(f[2 * e] * sc, f[2 * e + 1] * sc);
+      qh[g][e] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    sl2[g] = p.scale_log2 * ldexpf(1.f, -qe);
+  }
+}
+
 // T = cache element type, TQ = query / output type (equal except for fp8 caches).
 template <typename T, typename TQ, int D, int BS, int GS, int NW, int NST>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams p) {
@@ -120,9 +164,15 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
   }
   __syncwarp();
 
-  // q for this lane's elements, pre-scaled into the base-2 logit domain
-  float qf[GS][EPL];
-  {
+  // q for this lane's elements, pre-scaled into the base-2 logit domain (fp8 caches:
+  // q as f16 pairs times 2^qe, the scale applied to each score instead)
+  constexpr bool F8 = std::is_same<T, __nv_fp8_e4m3>::value;
+  float qf[F8 ? 1 : GS][F8 ? 1 : EPL];
+  uint32_t qh[F8 ? GS : 1][F8 ? EPL / 2 : 1];
+  float sl2[GS];
+  if constexpr (F8) {
+    load_q_f16<TQ, D, GS, EPL, NVL, VEC>(p, s, h0, sub, qh, sl2);
+  } else {
     const TQ* qb = static_cast<const TQ*>(p.q) + (static_cast<int64_t>(s) * p.num_heads + h0) * D;
 #pragma unroll
     for (int g = 0; g < GS; ++g) {
@@ -137,6 +187,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
       }
 #pragma unroll
       for (int e = 0; e < EPL; ++e) qf[g][e] *= p.scale_log2;
+      sl2[g] = 1.f;
     }
   }
 
@@ -202,21 +253,28 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
 #pragma unroll
       for (int pp = 0; pp < C::kPasses; ++pp) {
         const int t = pp * kRowsPerPass + grp;
-        float kf[EPL];
+        float kf[F8 ? 1 : EPL];
+        uint32_t kh[F8 ? EPL / 2 : 1];
 #pragma unroll
         for (int kk = 0; kk < NVL; ++kk) {
           const uint4 v = *reinterpret_cast<const uint4*>(Ks + t * D + (sub + 8 * kk) * VEC);
-          vec_to_float(v, &kf[kk * VEC], T());
+          if constexpr (F8) e4m3x16_to_f16x2(v, &kh[kk * VEC / 2]);
+          else vec_to_float(v, &kf[kk * VEC], T());
         }
 #pragma unroll
         for (int g = 0; g < GS; ++g) {
           float d = 0.f;
+          if constexpr (F8) {
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) d = fmaf(qf[g][e], kf[e], d);
+            for (int e = 0; e < EPL / 2; ++e) d = fma_f16x2_f32(qh[g][e], kh[e], d);
+          } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) d = fmaf(qf[g][e], kf[e], d);
+          }
           d += __shfl_xor_sync(FULL, d, 1);
           d += __shfl_xor_sync(FULL, d, 2);
           d += __shfl_xor_sync(FULL, d, 4);
-          sc[g][pp] = (t < valid) ? d : -INFINITY;
+          sc[g][pp] = (t < valid) ? d * sl2[g] : -INFINITY;
         }
       }
 #pragma unroll
@@ -231,8 +289,10 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
         for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
 #pragma unroll
         for (int pp = 0; pp < C::kPasses; ++pp) {
-          sc[g][pp] = exp2_safe(sc[g][pp], mn);
-          l[g] += sc[g][pp];
+          float pw = exp2_safe(sc[g][pp], mn);
+          if constexpr (F8) pw = __half2float(__float2half_rn(pw));  // the f16 weight of p.V
+          sc[g][pp] = pw;
+          l[g] += pw;
         }
         m[g] = mn;
       }
@@ -240,16 +300,32 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
       for (int pp = 0; pp < C::kPasses; ++pp) {
         const int t = pp * kRowsPerPass + grp;
         if (t < valid) {
-          float vf[EPL];
+          if constexpr (F8) {
+            uint32_t vh[EPL / 2];
 #pragma unroll
-          for (int kk = 0; kk < NVL; ++kk) {
-            const uint4 v = *reinterpret_cast<const uint4*>(Vs + t * D + (sub + 8 * kk) * VEC);
-            vec_to_float(v, &vf[kk * VEC], T());
-          }
+            for (int kk = 0; kk < NVL; ++kk) {
+              const uint4 v = *reinterpret_cast<const uint4*>(Vs + t * D + (sub + 8 * kk) * VEC);
+              e4m3x16_to_f16x2(v, &vh[kk * VEC / 2]);
+            }
 #pragma unroll
-          for (int g = 0; g < GS; ++g) {
+            for (int g = 0; g < GS; ++g) {
+              const uint16_t pw = __half_as_ushort(__float2half_rn(sc[g][pp]));  // exact
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[g][e] = fmaf(sc[g][pp], vf[e], acc[g][e]);
+              for (int e = 0; e < EPL / 2; ++e)
+                fma_f16_f16x2_f32(pw, vh[e], acc[g][2 * e], acc[g][2 * e + 1]);
+            }
+          } else {
+            float vf[EPL];
+#pragma unroll
+            for (int kk = 0; kk < NVL; ++kk) {
+              const uint4 v = *reinterpret_cast<const uint4*>(Vs + t * D + (sub + 8 * kk) * VEC);
+              vec_to_float(v, &vf[kk * VEC], T());
+            }
+#pragma unroll
+            for (int g = 0; g < GS; ++g) {
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) acc[g][e] = fmaf(sc[g][pp], vf[e], acc[g][e]);
+            }
           }
         }
       }
