@@ -71,6 +71,8 @@ typedef void* pa_stream_t; /* a cudaStream_t */
 #define PA_DEVERR_TIMEOUT 16u    /* a bounded wait on an async copy gave up          */
 #define PA_DEVERR_GROUP 32u      /* grouped decode: a sequence's own partitions start
                                     below first_part (those partitions were skipped)  */
+#define PA_DEVERR_ORDER 64u      /* pa_decode: a seq_order entry outside [0, num_seqs)
+                                    (that grid row was skipped)                       */
 
 /* ------------------------------------------------------------------------- */
 /* GPU entry points                                                           */
@@ -320,6 +322,48 @@ int pa_decode_attention_grouped(void* out, const void* q, const void* k_cache,
                                 int num_chunks, int max_members, int max_chunk_parts,
                                 int first_part, void* workspace, size_t workspace_bytes,
                                 pa_stream_t stream);
+
+/*
+ * pa_decode - the decode call with every option in one argument block: the plain,
+ * fp8 and grouped forms above, and the order in which the partition grid takes the
+ * sequences.  Same results as those entry points.
+ *   struct_size      sizeof(pa_decode_args_t)
+ *   out ... workspace_bytes, stream   as for pa_decode_attention
+ *   cache_dtype      dtype, or PA_FP8_E4M3 (then k_scale / v_scale as for
+ *                    pa_decode_attention_fp8; ignored otherwise)
+ *   seq_order        NULL, or device int32 [num_seqs], a permutation of the batch
+ *                    positions: grid row y of the partition kernels serves sequence
+ *                    seq_order[y].  Giving the longest sequences first lets their
+ *                    long rows start early and the short ones fill the end (the
+ *                    results do not depend on it).  An entry outside [0, num_seqs)
+ *                    skips that row and sets PA_DEVERR_ORDER.
+ *   prefix_parts ... first_part   the prefix-group arguments of
+ *                    pa_decode_attention_grouped; num_chunks = 0 for none (not with an
+ *                    fp8 cache).
+ */
+typedef struct {
+  size_t struct_size;
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  float scale;
+  int block_size, num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq;
+  int64_t num_blocks;
+  int max_seq_len, partition_size, dtype, cache_dtype;
+  float k_scale, v_scale;
+  const int32_t* seq_order;
+  const int32_t* prefix_parts;
+  const int32_t* chunk_members;
+  const int32_t* chunk_parts;
+  int num_chunks, max_members, max_chunk_parts, first_part;
+  void* workspace;
+  size_t workspace_bytes;
+  pa_stream_t stream;
+} pa_decode_args_t;
+int pa_decode(const pa_decode_args_t* args);
 
 /*
  * pa_device_error_read - synchronise the current device, then return (in *bits) and

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "NO_FREE_BLOCKS", 3: "UNKNOWN_SEQ"
 PA_STATIC_WORKSPACE_BYTES = 16 << 20
 PA_F32, PA_BF16, PA_F16, PA_FP8_E4M3 = 0, 1, 2, 3
 DEVERR_SLOT, DEVERR_COPY_BLOCK, DEVERR_TABLE, DEVERR_SEQ_LEN, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
-DEVERR_GROUP = 32
+DEVERR_GROUP, DEVERR_ORDER = 32, 64
 DEFAULT_PARTITION = 512
 
 
@@ -59,6 +59,19 @@ class pa_decoder_config_t(ctypes.Structure):
                 ("head_dim", _i32), ("num_heads", _i32), ("dtype", _i32), ("cache_dtype", _i32),
                 ("scale", _f), ("k_scale", _f), ("v_scale", _f), ("max_blocks_per_seq", _i32),
                 ("partition_size", _i32), ("group_members", _i32)]
+
+
+class pa_decode_args_t(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_size_t), ("out", _p), ("q", _p), ("k_cache", _p),
+                ("v_cache", _p), ("block_tables", _p), ("seq_lens", _p), ("scale", _f),
+                ("block_size", _i32), ("num_kv_heads", _i32), ("num_seqs", _i32),
+                ("num_heads", _i32), ("head_dim", _i32), ("max_blocks_per_seq", _i32),
+                ("num_blocks", _i64), ("max_seq_len", _i32), ("partition_size", _i32),
+                ("dtype", _i32), ("cache_dtype", _i32), ("k_scale", _f), ("v_scale", _f),
+                ("seq_order", _p), ("prefix_parts", _p), ("chunk_members", _p),
+                ("chunk_parts", _p), ("num_chunks", _i32), ("max_members", _i32),
+                ("max_chunk_parts", _i32), ("first_part", _i32), ("workspace", _p),
+                ("workspace_bytes", ctypes.c_size_t), ("stream", _p)]
 
 
 class pa_step_info_t(ctypes.Structure):
@@ -112,6 +125,7 @@ _sig("pa_build_prefix_groups", _i32, _p, _p, _i32, _i32, _i32, _p, _p, _p,
      ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int))
 _sig("pa_alloc_free_list", _i32, _p, _p, _i64, _I64P)
 _sig("pa_alloc_stats", _i32, _p, ctypes.POINTER(pa_stats_t))
+_sig("pa_decode", _i32, ctypes.POINTER(pa_decode_args_t))
 _sig("pa_decoder_create", _i32, ctypes.POINTER(pa_decoder_config_t), _p, ctypes.POINTER(_p))
 _sig("pa_decoder_destroy", _i32, _p)
 _sig("pa_decoder_bind", _i32, _p, _p, _i32, _i32)
@@ -331,6 +345,35 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, seq_le
         float(scale), block_size, num_kv_heads, S, Hq, D, block_tables.shape[1], NB,
         int(max_seq_len), partition_size, _dtype_code(q), _stream(stream)),
         "pa_decode_attention_static_ws")
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
+              num_kv_heads, max_seq_len, partition_size=DEFAULT_PARTITION, workspace=None,
+              seq_order=None, kv_scales=None, stream=None) -> None:
+    """pa_decode_attention (or, for a one-byte cache, pa_decode_attention_fp8 with
+    kv_scales = (k_scale, v_scale)) through the argument block, with an optional
+    int32 CUDA tensor seq_order [S] (the order the grid takes the sequences in)."""
+    import torch
+    S, Hq, D = q.shape
+    a = pa_decode_args_t()
+    a.struct_size = ctypes.sizeof(pa_decode_args_t)
+    a.out, a.q = _dev(out, "out"), _dev(q, "q")
+    a.k_cache, a.v_cache = _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache")
+    a.block_tables = _dev(block_tables, "block_tables", torch.int32)
+    a.seq_lens = _dev(seq_lens, "seq_lens", torch.int32)
+    a.scale, a.block_size, a.num_kv_heads = float(scale), block_size, num_kv_heads
+    a.num_seqs, a.num_heads, a.head_dim = S, Hq, D
+    a.max_blocks_per_seq, a.num_blocks = block_tables.shape[1], k_cache.shape[0]
+    a.max_seq_len, a.partition_size = int(max_seq_len), partition_size
+    a.dtype, a.cache_dtype = _dtype_code(q), _dtype_code(k_cache)
+    a.k_scale, a.v_scale = (float(x) for x in (kv_scales or (1.0, 1.0)))
+    if seq_order is not None:
+        a.seq_order = _dev(seq_order, "seq_order", torch.int32)
+    if workspace is not None:
+        a.workspace = _dev(workspace, "workspace")
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
+    a.stream = _stream(stream)
+    _check(lib.pa_decode(ctypes.byref(a)), "pa_decode")
 
 
 def pa_decode_uses_tensor_cores(dtype_code, num_heads, num_kv_heads, head_dim, block_size) -> bool:

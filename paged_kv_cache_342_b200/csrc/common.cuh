@@ -41,7 +41,21 @@ struct DecodeParams {
   int max_members;
   float v_scale;  // output multiplier (the fp8 cache's V scale; 1 otherwise)
   int part_base;  // partition index of grid z = 0 in the per-sequence kernels
+  // [S] or null: grid row y of the per-sequence kernels serves sequence seq_order[y]
+  // (longest first, so that the long rows start early and the short ones fill the end)
+  const int32_t* seq_order;
 };
+
+// The sequence grid row y serves; -1 (reported) for an order entry out of range.
+__device__ __forceinline__ int row_sequence(const DecodeParams& p, int y, bool report) {
+  if (!p.seq_order) return y;
+  const int s = __ldg(p.seq_order + y);
+  if (s < 0 || s >= p.num_seqs) {
+    if (report && p.err) atomicOr(p.err, PA_DEVERR_ORDER);
+    return -1;
+  }
+  return s;
+}
 
 // Device address of the library's error word on the current device.
 uint32_t* device_error_word();

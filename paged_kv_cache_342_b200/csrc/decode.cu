@@ -272,8 +272,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 int num_kv_heads, int num_seqs, int num_heads, int head_dim,
                 int max_blocks_per_seq, int64_t num_blocks, int max_seq_len, int partition_size,
                 int dtype, int cache_dtype, float k_scale, float v_scale,
-                const GroupArgs* groups, void* workspace, size_t workspace_bytes,
-                pa_stream_t stream);
+                const GroupArgs* groups, const int32_t* seq_order, void* workspace,
+                size_t workspace_bytes, pa_stream_t stream);
 
 }  // namespace
 
@@ -342,7 +342,7 @@ extern "C" int pa_decode_attention(void* out, const void* q, const void* k_cache
                                    size_t workspace_bytes, pa_stream_t stream) {
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
                      num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
-                     max_seq_len, partition_size, dtype, dtype, 1.f, 1.f, nullptr, workspace,
+                     max_seq_len, partition_size, dtype, dtype, 1.f, 1.f, nullptr, nullptr, workspace,
                      workspace_bytes, stream);
 }
 
@@ -357,7 +357,30 @@ extern "C" int pa_decode_attention_fp8(void* out, const void* q, const void* k_c
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
                      num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
                      max_seq_len, partition_size, dtype, PA_FP8_E4M3, k_scale, v_scale, nullptr,
-                     workspace, workspace_bytes, stream);
+                     nullptr, workspace, workspace_bytes, stream);
+}
+
+extern "C" int pa_decode(const pa_decode_args_t* a) {
+  if (!a || a->struct_size != sizeof(pa_decode_args_t)) return PA_ERR_INVALID_ARG;
+  const bool fp8 = a->cache_dtype == PA_FP8_E4M3;
+  if (!fp8 && a->cache_dtype != a->dtype) return PA_ERR_INVALID_ARG;
+  GroupArgs g{};
+  const GroupArgs* gp = nullptr;
+  if (a->num_chunks != 0) {
+    if (fp8 || a->num_chunks < 0 || a->num_chunks > 65535 || a->max_chunk_parts < 0 ||
+        a->max_members < 1 || a->max_members > 16 || a->first_part < 0 ||
+        !a->prefix_parts || !a->chunk_members || !a->chunk_parts)
+      return PA_ERR_INVALID_ARG;
+    g = GroupArgs{a->prefix_parts, a->chunk_members, a->chunk_parts, a->num_chunks,
+                  a->max_members, a->max_chunk_parts, a->first_part};
+    gp = &g;
+  }
+  return decode_impl(a->out, a->q, a->k_cache, a->v_cache, a->block_tables, a->seq_lens,
+                     a->scale, a->block_size, a->num_kv_heads, a->num_seqs, a->num_heads,
+                     a->head_dim, a->max_blocks_per_seq, a->num_blocks, a->max_seq_len,
+                     a->partition_size, a->dtype, a->cache_dtype,
+                     fp8 ? a->k_scale : 1.f, fp8 ? a->v_scale : 1.f, gp, a->seq_order,
+                     a->workspace, a->workspace_bytes, a->stream);
 }
 
 extern "C" int pa_decode_attention_grouped(
@@ -378,7 +401,7 @@ extern "C" int pa_decode_attention_grouped(
                     max_chunk_parts, first_part};
   return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, scale, block_size,
                      num_kv_heads, num_seqs, num_heads, head_dim, max_blocks_per_seq, num_blocks,
-                     max_seq_len, partition_size, dtype, dtype, 1.f, 1.f, &g, workspace,
+                     max_seq_len, partition_size, dtype, dtype, 1.f, 1.f, &g, nullptr, workspace,
                      workspace_bytes, stream);
 }
 
@@ -390,8 +413,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 int num_kv_heads, int num_seqs, int num_heads, int head_dim,
                 int max_blocks_per_seq, int64_t num_blocks, int max_seq_len, int partition_size,
                 int dtype, int cache_dtype, float k_scale, float v_scale,
-                const GroupArgs* groups, void* workspace, size_t workspace_bytes,
-                pa_stream_t stream) {
+                const GroupArgs* groups, const int32_t* seq_order, void* workspace,
+                size_t workspace_bytes, pa_stream_t stream) {
   if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16) return PA_ERR_INVALID_ARG;
   const bool fp8 = cache_dtype == PA_FP8_E4M3;
   if (cache_dtype != dtype && !fp8) return PA_ERR_INVALID_ARG;
@@ -429,6 +452,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.seq_lens = seq_lens;
   p.scale_log2 = scale * k_scale * 1.4426950408889634f;
   p.v_scale = v_scale;
+  p.seq_order = seq_order;
   p.num_seqs = num_seqs;
   p.num_heads = num_heads;
   p.num_kv_heads = num_kv_heads;

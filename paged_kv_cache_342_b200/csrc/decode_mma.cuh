@@ -190,7 +190,9 @@ __global__ void __launch_bounds__(NW * 32)
   const int ps = p.partition_size;
   int kvh, part, nparts, tok_begin, tok_end, table_seq;
   if constexpr (!GROUP) {
-    const int s = blockIdx.y;
+    const int s =
+        row_sequence(p, blockIdx.y, threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0);
+    if (s < 0) return;
     const int h0 = blockIdx.x * C::kHeads;
     part = p.part_base + blockIdx.z;
     kvh = h0 / G;

@@ -138,7 +138,9 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane >> 3, sub = lane & 7;
-  const int s = blockIdx.y, part = p.part_base + blockIdx.z;
+  const int s = row_sequence(p, blockIdx.y, threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0);
+  const int part = p.part_base + blockIdx.z;
+  if (s < 0) return;
   const int h0 = blockIdx.x * GS;
   const int kvh = h0 / (p.num_heads / p.num_kv_heads);
 

@@ -89,7 +89,7 @@ struct pa_decoder {
   int num_seqs = 0, members = 0, partition = 0;
   bool bound = false, rolling = false, stepped = false;
   size_t off_slots = 0, off_pairs = 0, off_lens = 0, off_tables = 0, off_pparts = 0,
-         off_cmembers = 0, off_cparts = 0, stage_bytes = 0;
+         off_cmembers = 0, off_cparts = 0, off_order = 0, stage_bytes = 0;
   StageSet sets[2];
   int cur = 0;
   void* ws = nullptr;
@@ -197,6 +197,10 @@ int prepare(pa_decoder* d, cudaStream_t comp, pa_step_info_t* info) {
   if (rc != PA_OK) return rc;
   int max_len = 0;
   for (int s = 0; s < S; ++s) max_len = std::max(max_len, lens[s]);
+  // the partition grid takes the sequences longest first (ties in batch order)
+  int32_t* order = d->h<int32_t>(st, d->off_order);
+  for (int s = 0; s < S; ++s) order[s] = s;
+  std::stable_sort(order, order + S, [lens](int32_t x, int32_t y) { return lens[x] > lens[y]; });
   const int parts = (max_len + d->partition - 1) / d->partition;
   int num_chunks = 0, max_chunk_parts = 0, first_part = 0;
   if (groups_used(d, parts)) {
@@ -263,25 +267,42 @@ int launch(pa_decoder* d, const pa_step_info_t* info, const void* q, const void*
   if (ev_begin && cudaEventRecord(ev_begin, comp) != cudaSuccess) return PA_ERR_CUDA;
   const int32_t* tables = d->d<int32_t>(st, d->off_tables);
   const int32_t* lens = d->d<int32_t>(st, d->off_lens);
-  if (d->fp8()) {
-    rc = pa_decode_attention_fp8(out, q, c.k_cache, c.v_cache, tables, lens, c.scale,
-                                 c.block_size, c.num_kv_heads, S, c.num_heads, c.head_dim,
-                                 c.max_blocks_per_seq, c.num_blocks, info->max_seq_len,
-                                 d->partition, c.dtype, c.k_scale, c.v_scale, d->ws,
-                                 d->ws_bytes, comp);
-  } else if (info->num_chunks > 0) {
-    rc = pa_decode_attention_grouped(
-        out, q, c.k_cache, c.v_cache, tables, lens, c.scale, c.block_size, c.num_kv_heads, S,
-        c.num_heads, c.head_dim, c.max_blocks_per_seq, c.num_blocks, info->max_seq_len,
-        d->partition, c.dtype, d->d<int32_t>(st, d->off_pparts),
-        d->d<int32_t>(st, d->off_cmembers), d->d<int32_t>(st, d->off_cparts), info->num_chunks,
-        d->members, info->max_chunk_parts, info->first_part, d->ws, d->ws_bytes, comp);
-  } else {
-    rc = pa_decode_attention(out, q, c.k_cache, c.v_cache, tables, lens, c.scale, c.block_size,
-                             c.num_kv_heads, S, c.num_heads, c.head_dim, c.max_blocks_per_seq,
-                             c.num_blocks, info->max_seq_len, d->partition, c.dtype, d->ws,
-                             d->ws_bytes, comp);
+  pa_decode_args_t a{};
+  a.struct_size = sizeof(a);
+  a.out = out;
+  a.q = q;
+  a.k_cache = c.k_cache;
+  a.v_cache = c.v_cache;
+  a.block_tables = tables;
+  a.seq_lens = lens;
+  a.scale = c.scale;
+  a.block_size = c.block_size;
+  a.num_kv_heads = c.num_kv_heads;
+  a.num_seqs = S;
+  a.num_heads = c.num_heads;
+  a.head_dim = c.head_dim;
+  a.max_blocks_per_seq = c.max_blocks_per_seq;
+  a.num_blocks = c.num_blocks;
+  a.max_seq_len = info->max_seq_len;
+  a.partition_size = d->partition;
+  a.dtype = c.dtype;
+  a.cache_dtype = c.cache_dtype;
+  a.k_scale = c.k_scale;
+  a.v_scale = c.v_scale;
+  a.seq_order = d->d<int32_t>(st, d->off_order);
+  if (info->num_chunks > 0) {
+    a.prefix_parts = d->d<int32_t>(st, d->off_pparts);
+    a.chunk_members = d->d<int32_t>(st, d->off_cmembers);
+    a.chunk_parts = d->d<int32_t>(st, d->off_cparts);
+    a.num_chunks = info->num_chunks;
+    a.max_members = d->members;
+    a.max_chunk_parts = info->max_chunk_parts;
+    a.first_part = info->first_part;
   }
+  a.workspace = d->ws;
+  a.workspace_bytes = d->ws_bytes;
+  a.stream = comp;
+  rc = pa_decode(&a);
   if (rc != PA_OK) return rc;
   if (ev_end && cudaEventRecord(ev_end, comp) != cudaSuccess) return PA_ERR_CUDA;
   if (cudaEventRecord(st.kernels_done, comp) != cudaSuccess) return PA_ERR_CUDA;
@@ -400,6 +421,7 @@ int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int r
   d->off_pparts = take(4 * S);
   d->off_cmembers = take(4 * S * MM);
   d->off_cparts = take(4 * S);
+  d->off_order = take(4 * S);
   d->stage_bytes = off;
   cudaError_t e = cudaSuccess;
   for (StageSet& s : d->sets) {

@@ -134,6 +134,27 @@ def test_decoder_config_checks(pa):
     assert pa.lib.pa_decoder_destroy(None) == pa.PA_ERR_INVALID_ARG
 
 
+def test_decode_argument_block(pa):
+    a = pa.pa_decode_args_t()
+    a.struct_size = ctypes.sizeof(pa.pa_decode_args_t)
+    a.out = a.q = a.k_cache = a.v_cache = a.block_tables = a.seq_lens = FAKE
+    a.scale, a.block_size, a.num_kv_heads, a.num_seqs, a.num_heads = 0.1, 16, 4, 0, 8
+    a.head_dim, a.max_blocks_per_seq, a.num_blocks, a.max_seq_len = 128, 8, 64, 100
+    a.partition_size, a.dtype, a.cache_dtype = 512, pa.PA_BF16, pa.PA_BF16
+    # every field read where the library expects it: an empty batch is accepted
+    assert pa.lib.pa_decode(ctypes.byref(a)) == pa.PA_OK
+    for field, bad in (("struct_size", 16), ("cache_dtype", pa.PA_F16), ("head_dim", 96),
+                       ("num_chunks", -1), ("partition_size", 520)):
+        b = pa.pa_decode_args_t.from_buffer_copy(a)
+        setattr(b, field, bad)
+        assert pa.lib.pa_decode(ctypes.byref(b)) in (pa.PA_ERR_INVALID_ARG,
+                                                    pa.PA_ERR_UNSUPPORTED), field
+    c = pa.pa_decode_args_t.from_buffer_copy(a)
+    c.num_chunks = 3                                    # groups without their arrays
+    assert pa.lib.pa_decode(ctypes.byref(c)) == pa.PA_ERR_INVALID_ARG
+    assert pa.lib.pa_decode(None) == pa.PA_ERR_INVALID_ARG
+
+
 def _has_gpu():
     import torch
     return torch.cuda.is_available()

@@ -310,3 +310,42 @@ def test_decode_right_after_a_kernel_that_writes_its_inputs(pa, Hq, Hkv):
     assert pa.pa_device_error_read() == 0
     for i in range(len(qs)):
         assert torch.equal(outs[i], refs[i]), f"iteration {i}"
+
+
+@pytest.mark.parametrize("Hq,Hkv,ps", [(4, 4, 512), (16, 2, 64), (8, 2, 32)])
+def test_sequence_order_does_not_change_the_result(pa, Hq, Hkv, ps):
+    # pa_decode with seq_order: the grid takes the sequences in another order; every
+    # output is bit-identical to the plain call's
+    S, D, bs = 7, 128, 16
+    lens = np.array([300, 5, 1000, 64, 0, 129, 700], np.int64)
+    NB = int(sum(blocks_for(int(L), bs) for L in lens)) + 3
+    order = np.random.default_rng(6).permutation(NB).astype(np.int32)
+    width = int(max(blocks_for(int(L), bs) for L in lens)) + 1
+    tables = tables_from_order(lens, bs, order, width)
+    k = to_dev(normal_fill((NB, Hkv, bs, D), "bf16", 1.0, 41, 1), "bf16")
+    v = to_dev(normal_fill((NB, Hkv, bs, D), "bf16", 1.0, 41, 2), "bf16")
+    q = to_dev(normal_fill((S, Hq, D), "bf16", 1.0, 41, 3), "bf16")
+    t_d = torch.from_numpy(tables).cuda()
+    l_d = torch.from_numpy(lens.astype(np.int32)).cuda()
+    max_len = int(lens.max())
+    wsb = pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+    ref = torch.empty_like(q)
+    pa.pa_decode_attention(ref, q, k, v, t_d, l_d, 1 / math.sqrt(D), bs, Hkv, max_len, ps,
+                           ws if wsb else None)
+    for perm in (np.argsort(-lens, kind="stable"), np.random.default_rng(2).permutation(S)):
+        out = torch.full_like(q, float("nan"))
+        pa.pa_decode(out, q, k, v, t_d, l_d, 1 / math.sqrt(D), bs, Hkv, max_len, ps,
+                     ws if wsb else None, seq_order=torch.from_numpy(perm.astype(np.int32)).cuda())
+        torch.cuda.synchronize()
+        assert pa.pa_device_error_read() == 0
+        assert torch.equal(out, ref)
+    # an entry out of range skips its row and is reported; the other rows are unchanged
+    bad = np.arange(S, dtype=np.int32)
+    bad[3] = S + 5
+    out = torch.full_like(q, float("nan"))
+    pa.pa_decode(out, q, k, v, t_d, l_d, 1 / math.sqrt(D), bs, Hkv, max_len, ps,
+                 ws if wsb else None, seq_order=torch.from_numpy(bad).cuda())
+    assert pa.pa_device_error_read() & pa.DEVERR_ORDER
+    rows = [s for s in range(S) if s != 3]
+    assert torch.equal(out[rows], ref[rows])
