@@ -385,6 +385,8 @@ int pa_decoder_destroy(pa_decoder_t* d) {
 
 int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int rolling) {
   if (!d || num_seqs <= 0 || !seq_ids || num_seqs > 65535) return PA_ERR_INVALID_ARG;
+  DeviceGuard g(d->device);  // the partition choice asks the decoder's device
+  if (!g.ok()) return PA_ERR_CUDA;
   const pa_decoder_config_t& c = d->cfg;
   std::vector<int64_t> ids(seq_ids, seq_ids + num_seqs), lens(static_cast<size_t>(num_seqs));
   std::vector<int64_t> sorted = ids;
@@ -404,8 +406,7 @@ int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int r
   }
   const size_t ws_need = pa_decode_workspace_bytes(num_seqs, c.num_heads, c.head_dim,
                                                    static_cast<int>(cap), partition);
-  DeviceGuard g(d->device);
-  if (!g.ok() || quiesce(d) != cudaSuccess) return PA_ERR_CUDA;
+  if (quiesce(d) != cudaSuccess) return PA_ERR_CUDA;
   free_stage(d);
   d->bound = false;
 
