@@ -520,8 +520,9 @@ int pa_alloc_stats(const pa_alloc_t* a, pa_stats_t* stats);
  *      one copy on the decoder's copy stream; the caller's stream waits for it;
  *   4. pa_copy_blocks makes the copies (before the write: the token lands in the copy);
  *   5. pa_reshape_and_cache (or _fp8) writes the new tokens' K/V into their slots;
- *   6. pa_decode_attention (or _fp8, or _grouped when prefix groups exist) attends over
- *      every cached token, the new one included.
+ *   6. pa_decode (the plain, fp8 or grouped form) attends over every cached token, the
+ *      new one included; without prefix groups the grid takes the sequences longest
+ *      first (an order sorted on the host each step and staged with the rest).
  * Steps 4-6 are enqueued on the caller's stream; the call returns without waiting
  * for the GPU.  Step k fills staging set k % 2 while the kernels of step k - 1 may
  * still read the other set; the host waits only before rewriting a set whose copy
