@@ -129,9 +129,21 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
-def job_throughput(bytes_per_step: int, steps: int, world: int, elapsed_max_ms: float) -> float:
-    """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
-    return float(bytes_per_step) * steps * world / (elapsed_max_ms * 1e-3) / 1e9
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    """The sum over ranks (every rank must call this, in the same order)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_throughput(job_bytes_per_step: float, steps: int, elapsed_max_ms: float) -> float:
+    """Whole-job GB/s: the bytes all ranks move per step (their replicas differ: each
+    draws its own lengths) over the slowest rank's time."""
+    return float(job_bytes_per_step) * steps / (elapsed_max_ms * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------------------
@@ -437,7 +449,8 @@ def run_ours(args, cfg):
     if err:
         raise RuntimeError(f"device error word {err} after the timed region")
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
-    value = job_throughput(step_bytes, args.steps, world, elapsed_ms)
+    job_step_bytes = sum_over_ranks(step_bytes, world, dev)
+    value = job_throughput(job_step_bytes, args.steps, elapsed_ms)
     seqs_per_s = S * world * args.steps / (elapsed_ms * 1e-3)
 
     # ---- a pool that fits in L2: the decode call also timed cold ---------------------
@@ -482,7 +495,7 @@ def run_ours(args, cfg):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        E = job_throughput(step_bytes, args.steps, world, e_ms)
+        E = job_throughput(job_step_bytes, args.steps, e_ms)
         h2d = sum(t.numel() * t.element_size() for t in toks_h[0]) + dec.staging_bytes
         d2h = S * Hq * D * cfg.elem_bytes
         e2e = {"value": round(E, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),

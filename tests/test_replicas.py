@@ -30,7 +30,8 @@ def _rank_main(rank, world, port, elapsed, out):
         w, r, lr = bench.replica_env()
         dist.barrier()
         slowest = bench.max_over_ranks(elapsed[rank], w)
-        value = bench.job_throughput(1_000_000, 10, w, slowest)
+        job_bytes = bench.sum_over_ranks(1_000_000 * (1 + rank), w)   # replicas differ
+        value = bench.job_throughput(job_bytes, 10, slowest)
         seeds = [None] * world
         dist.all_gather_object(seeds, bench.replica_seed(7, r))
         out[rank] = (w, r, lr, slowest, value, tuple(seeds))
@@ -51,11 +52,12 @@ def test_two_replicas_agree_on_the_slowest_rank():
         w, r, lr, slowest, value, seeds = res[rank]
         assert (w, r, lr) == (2, rank, rank)
         assert slowest == 5.0                      # max over ranks, on every rank
-        # 1 MB per step x 10 steps x 2 ranks over 5 ms = 4 GB/s
-        assert value == pytest.approx(4.0)
+        # (1 + 2) MB per step x 10 steps over 5 ms = 6 GB/s
+        assert value == pytest.approx(6.0)
         assert seeds == (7, 8)                     # distinct replicas
 
 
 def test_single_process_needs_no_group():
     assert bench.max_over_ranks(2.5, 1) == 2.5
-    assert bench.job_throughput(2_000_000_000, 3, 1, 1000.0) == pytest.approx(6.0)
+    assert bench.sum_over_ranks(4.0, 1) == 4.0
+    assert bench.job_throughput(2_000_000_000, 3, 1000.0) == pytest.approx(6.0)
