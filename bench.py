@@ -514,7 +514,7 @@ def run_ours(args, cfg):
             "launches_timed": len(dec_ms),
             "median_launch_us": round(statistics.median(dec_ms) * 1e3, 2),
             "frac_of_nominal_8000": round(achieved / 8000.0, 4),
-            "traffic": recorded_traffic(cfg)}
+            "traffic": None if args.cache_fp8 else recorded_traffic(cfg)}  # records: 16-bit caches
     if cold_ms:
         roof["cold_median_launch_us"] = round(statistics.median(cold_ms) * 1e3, 2)
         roof["cold_note"] = "pool smaller than L2: calls after a 2x-L2 buffer write"
