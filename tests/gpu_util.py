@@ -2,7 +2,6 @@
 tolerances the attention outputs are held to (max-abs error against the float64
 oracle: 1e-4 for float32 caches, 2e-2 for bf16/f16 caches with float32
 accumulation)."""
-import math
 
 import numpy as np
 import torch

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle.cache_ops as ocache
-from gpu_util import PA_CODE, to_dev, to_host
+from gpu_util import to_dev, to_host
 from workloads import CONFIGS, make_inputs, normal_fill
 
 pytestmark = pytest.mark.gpu

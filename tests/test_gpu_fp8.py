@@ -9,7 +9,7 @@ import torch
 
 import oracle.attention as oatt
 from oracle import fp8
-from gpu_util import ATOL, TORCH_DT, assert_close, out_f64, tables_from_order, to_dev
+from gpu_util import TORCH_DT, assert_close, out_f64, tables_from_order, to_dev
 from oracle.numerics import to_f64
 from workloads import normal_fill
 

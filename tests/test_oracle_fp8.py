@@ -1,7 +1,6 @@
 """Pins for the oracle's e4m3 codec: textbook code values, exact round trips, brute
 force over all codes, ties, saturation, and torch's own float8_e4m3fn cast."""
 import numpy as np
-import pytest
 import torch
 
 from oracle import fp8
