@@ -591,7 +591,9 @@ def kernel_sources_sha() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(HERE, "paged_kv_cache_342_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.startswith("decode") or name in ("common.cuh", "tensor_map.cu"):
+        # the kernels a decode call runs (the step runtime's host code is not one)
+        if (name.startswith("decode") and not name.startswith("decoder")) or \
+                name in ("common.cuh", "tensor_map.cu"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
