@@ -450,7 +450,7 @@ int pa_seq_add_prompt(pa_alloc_t* a, int64_t seq_id, const int32_t* token_ids, i
                       int64_t* cached_tokens);
 /* child shares all of parent's blocks and its length. */
 int pa_seq_fork(pa_alloc_t* a, int64_t parent, int64_t child);
-/* Room for one more token of seq_id: *slot receives its slot; *cow_src/*cow_dst the
+/* Room for one more token of seq_id: *slot receives its slot; *cow_src and *cow_dst the
  * copy to make first, or -1/-1.  Length grows by one. */
 int pa_seq_append_slot(pa_alloc_t* a, int64_t seq_id, int64_t* slot, int32_t* cow_src,
                        int32_t* cow_dst);

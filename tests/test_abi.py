@@ -222,3 +222,23 @@ def test_importing_without_library_fails_loudly(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import paged_kv_cache_342_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libpa.so is missing" in r.stderr
+
+
+def test_plain_c_program_builds_and_runs(tmp_path):
+    # the header is C99 (no C++ in it) and the host-only calls work from C
+    import shutil
+    import subprocess
+    import paged_kv_cache_342_b200 as m
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_consumer"
+    libdir = os.path.dirname(m.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_consumer.c"), "-L", libdir, "-lpa",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.strip()
+    # pool order 0, 1, ...: seq 7 holds blocks 0, 1; the fork's append copies block 1
+    # into the next free block, 2, at offset 1 (slot 9)
+    assert out == ("rc=0 slot=9 copy=1->2 used=3 shared=1 ps=4096 bad=1"), out
