@@ -115,8 +115,8 @@ __device__ __forceinline__ void vec_to_float(const uint4& v, float* f, __nv_fp8_
   }
 }
 
-// e4m3 -> f16 by bit placement: with x = [c1 0 c0 0] (two codes in the high bytes of
-// the halves), a code s|eeee|mmm becomes the f16 s|0eeee|mmm0000000: exponent bias 15
+// e4m3 -> f16 by bit placement: with x = [c1 * c0 *] (two codes in the high bytes of
+// the halves; the low bytes are ignored), a code s|eeee|mmm becomes the f16 s|0eeee|mmm0000000: exponent bias 15
 // instead of 7, so the f16 is the code's value times 2^-8, exactly, for every finite
 // code (subnormal codes become f16 subnormals the same way).  Integer ALU only.
 __device__ __forceinline__ uint32_t e4m3_place(uint32_t x) {
@@ -242,9 +242,14 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// exp2 of a base-2 logit difference; -inf - -inf (an empty state) gives 0.
+// exp2 of a base-2 logit difference, a <= m in every use (so the result is in [0, 1]),
+// by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz.f32, relative
+// error about 2^-22).  Results below 2^-126 flush to zero: such a weight next to the
+// maximum's weight of 1 changes no float sum.  -inf - -inf (an empty state) gives 0.
 __device__ __forceinline__ float exp2_safe(float a, float m) {
-  return (m == -INFINITY) ? 0.f : exp2f(a - m);
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(a - m));
+  return (m == -INFINITY) ? 0.f : y;
 }
 
 // Record a failing CUDA call for pa_last_cuda_error (thread-local text).

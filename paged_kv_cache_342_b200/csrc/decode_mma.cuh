@@ -86,10 +86,12 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2_cvt(uint32_t w, uint32_t& lo, 
 }
 // Codes (byte0, byte2) -> f16x2 `even`, (byte1, byte3) -> f16x2 `odd`, each value the
 // code's times 2^-8 (e4m3_place).
+// e4m3_place reads codes from the high byte of each 16-bit half: bytes 1 and 3 already
+// sit there, bytes 0 and 2 get there by one shift.
 __device__ __forceinline__ void e4m3_pairs_to_f16x2_bits(uint32_t w, uint32_t& even,
                                                          uint32_t& odd) {
-  even = e4m3_place(__byte_perm(w, 0u, 0x2404));
-  odd = e4m3_place(__byte_perm(w, 0u, 0x3414));
+  even = e4m3_place(w << 8);
+  odd = e4m3_place(w);
 }
 // 2-D tiled TMA load of one box into shared memory, completion on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -518,22 +520,39 @@ __global__ void __launch_bounds__(NW * 32)
       }
     }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < C::kHeads * D; idx += NW * 32) {
-    const int hh = idx / D, d = idx - hh * D;
+  // per head column, once: the max M, the exp-sum and each warp's weight
+  // exp2(m_w - M) * v_scale / sum, so that an output element is NW fused multiply-adds
+  __shared__ float col_w[NW][C::kHeads];
+  __shared__ float col_m[C::kHeads], col_l[C::kHeads];
+  if (threadIdx.x < C::kHeads) {
+    const int hh = threadIdx.x;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) M = fmaxf(M, red[(w * C::kHeads + hh) * (D + 2) + D]);
-    float num = 0.f, den = 0.f;
+    float f[NW], den = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const float* r = red + (w * C::kHeads + hh) * (D + 2);
-      const float f = exp2_safe(r[D], M);
-      num = fmaf(r[d], f, num);
-      den = fmaf(r[D + 1], f, den);
+      f[w] = exp2_safe(r[D], M);
+      den = fmaf(r[D + 1], f[w], den);
     }
     // FP8: the V operands carry the code values times 2^-8
-    const float o = den > 0.f ? num / den * (FP8 ? p.v_scale * 256.f : p.v_scale) : 0.f;
+    const float sc = den > 0.f ? (FP8 ? p.v_scale * 256.f : p.v_scale) / den : 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) col_w[w][hh] = f[w] * sc;
+    col_m[hh] = M;
+    col_l[hh] = den;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < C::kHeads * D; idx += NW * 32) {
+    const int hh = idx / D, d = idx - hh * D;
     if (!col_ok[hh]) continue;
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      o = fmaf(red[(w * C::kHeads + hh) * (D + 2) + d], col_w[w][hh], o);
+    const float den = col_l[hh];
+    if (!(den > 0.f)) o = 0.f;
     const int64_t row = col_row[hh];
     if (nparts == 1) {
       store_elem(static_cast<TQ*>(p.out) + row * D + d, o);
@@ -541,7 +560,7 @@ __global__ void __launch_bounds__(NW * 32)
       const int64_t prow = row * p.max_parts + part;
       p.ws_o[prow * D + d] = o;
       if (d == 0) {
-        p.ws_m[prow] = M;
+        p.ws_m[prow] = col_m[hh];
         p.ws_l[prow] = den;
       }
     }

@@ -25,7 +25,7 @@
 //  * each 8-lane group keeps its own online-softmax state (m, l, acc) over the rows
 //    it sees, per block: scores, block max, one rescale, then p*V.  Groups merge
 //    with shuffles at the end, warps through shared memory.
-//  * logits are kept in base 2 (q pre-scaled by scale*log2 e; exp2f).
+//  * logits are kept in base 2 (q pre-scaled by scale*log2 e; hardware exp2).
 #pragma once
 
 #include "common.cuh"
