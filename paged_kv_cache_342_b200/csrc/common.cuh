@@ -242,10 +242,15 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// exp2 of a base-2 logit difference, a <= m in every use (so the result is in [0, 1]),
-// by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz.f32, relative
-// error about 2^-22).  Results below 2^-126 flush to zero: such a weight next to the
-// maximum's weight of 1 changes no float sum.  -inf - -inf (an empty state) gives 0.
+// Online softmax with a lazy running max: the max m that the weights are taken against
+// moves only when a new logit passes it by more than this (base 2), so weights stay
+// below 2^kLazyMax and most blocks skip the rescale of the accumulators.
+constexpr float kLazyMax = 8.f;
+
+// exp2 of a base-2 logit difference, a - m <= kLazyMax in every use, by the hardware's
+// approximate base-2 exponential (PTX ex2.approx.ftz.f32, relative error about 2^-22).
+// Results below 2^-126 flush to zero: such a weight next to the largest weight (at
+// least 1) changes no float sum.  -inf - -inf (an empty state) gives 0.
 __device__ __forceinline__ float exp2_safe(float a, float m) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(a - m));

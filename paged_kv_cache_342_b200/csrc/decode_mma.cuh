@@ -391,6 +391,12 @@ __global__ void __launch_bounds__(NW * 32)
         }
       }
       // ---- online softmax per head column ----------------------------------
+      // The running max moves only when some column's block max passes it by more
+      // than kLazyMax (base 2): until then the weights exp2(s - m) stay below
+      // 2^kLazyMax, which P's 16-bit type holds with its full precision, and the
+      // accumulators and sums need no rescale for this block.
+      float bmax[NT][2];
+      bool grow = false;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -408,24 +414,41 @@ __global__ void __launch_bounds__(NW * 32)
           mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
           mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
           mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
-          const float mn = fmaxf(m[nt][j], mx);
-          const float corr = exp2_safe(m[nt][j], mn);
-          m[nt][j] = mn;
+          bmax[nt][j] = mx;
+          grow |= mx > m[nt][j] + kLazyMax;
+        }
+      }
+      if (__any_sync(FULL, grow)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float mn = fmaxf(m[nt][j], bmax[nt][j]);
+            const float corr = exp2_safe(m[nt][j], mn);
+            m[nt][j] = mn;
+            l[nt][j] *= corr;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+              oacc[mt][nt][j] *= corr;
+              oacc[mt][nt][2 + j] *= corr;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
           float ls = 0.f;
 #pragma unroll
           for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-              const float pv = exp2_safe(sacc[tt][nt][2 * r + j], mn);
+              const float pv = exp2_safe(sacc[tt][nt][2 * r + j], m[nt][j]);
               sacc[tt][nt][2 * r + j] = pv;
               ls += pv;
             }
-          l[nt][j] = l[nt][j] * corr + ls;
-#pragma unroll
-          for (int mt = 0; mt < KS; ++mt) {
-            oacc[mt][nt][j] *= corr;
-            oacc[mt][nt][2 + j] *= corr;
-          }
+          l[nt][j] += ls;
         }
       }
       // ---- P^T as B fragments (movmatrix.trans of each 8x8 quarter) ----------

@@ -279,24 +279,39 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
           sc[g][pp] = (t < valid) ? d * sl2[g] : -INFINITY;
         }
       }
+      // fp8 caches keep a lazy running max (kLazyMax): the rescale runs only when some
+      // group's block max passes its m by more than kLazyMax.  The others rescale on
+      // every block (their kernels are bound by memory, not by instruction issue).
+      bool grow = !F8;
+      if constexpr (F8) {
+#pragma unroll
+        for (int g = 0; g < GS; ++g)
+#pragma unroll
+          for (int pp = 0; pp < C::kPasses; ++pp) grow |= sc[g][pp] > m[g] + kLazyMax;
+        grow = __any_sync(FULL, grow);
+      }
+      if (grow) {
+#pragma unroll
+        for (int g = 0; g < GS; ++g) {
+          float mn = m[g];
+#pragma unroll
+          for (int pp = 0; pp < C::kPasses; ++pp) mn = fmaxf(mn, sc[g][pp]);
+          const float corr = exp2_safe(m[g], mn);
+          l[g] *= corr;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
+          m[g] = mn;
+        }
+      }
 #pragma unroll
       for (int g = 0; g < GS; ++g) {
-        float mb = sc[g][0];
-#pragma unroll
-        for (int pp = 1; pp < C::kPasses; ++pp) mb = fmaxf(mb, sc[g][pp]);
-        const float mn = fmaxf(m[g], mb);
-        const float corr = exp2_safe(m[g], mn);
-        l[g] *= corr;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
 #pragma unroll
         for (int pp = 0; pp < C::kPasses; ++pp) {
-          float pw = exp2_safe(sc[g][pp], mn);
+          float pw = exp2_safe(sc[g][pp], m[g]);
           if constexpr (F8) pw = __half2float(__float2half_rn(pw));  // the f16 weight of p.V
           sc[g][pp] = pw;
           l[g] += pw;
         }
-        m[g] = mn;
       }
 #pragma unroll
       for (int pp = 0; pp < C::kPasses; ++pp) {
