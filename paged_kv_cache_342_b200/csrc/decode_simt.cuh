@@ -23,8 +23,9 @@
 //    row, so shared loads are conflict-free).  A warp covers 4 rows per pass; the
 //    q.k partial sums meet in 3 xor-shuffles.
 //  * each 8-lane group keeps its own online-softmax state (m, l, acc) over the rows
-//    it sees, per block: scores, block max, one rescale, then p*V.  Groups merge
-//    with shuffles at the end, warps through shared memory.
+//    it sees, per block: scores, block max, one rescale (fp8 caches: only when the
+//    max moves by more than kLazyMax), then p*V.  Groups merge with shuffles at the
+//    end, warps through shared memory.
 //  * logits are kept in base 2 (q pre-scaled by scale*log2 e; hardware exp2).
 #pragma once
 
