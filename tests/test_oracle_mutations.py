@@ -109,3 +109,61 @@ def test_catches_missing_copy_on_write(monkeypatch):
             self.lens[seq_id] = n + 1
             return table[-1] * self.block_size + off, -1, -1
     assert check_prefix_sharing(bm_cls=NoCow) > 0.0
+
+
+# ---- block manager: refcount and table bookkeeping mistakes ------------------------
+
+def _caught_allocator(bm_cls) -> bool:
+    """Random add/fork/append/free/truncate sequences under the allocator invariants
+    (counts = table entries, free and used partition the pool, ceil(L/bs) blocks)."""
+    from test_oracle_pins import _invariants, random_ops
+    g = np.random.default_rng(11)
+    try:
+        for _ in range(5):
+            random_ops(bm_cls(24, 4, g.permutation(24)), g, 200, _invariants)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_unmutated_allocator_passes():
+    assert not _caught_allocator(oalloc.BlockManager)
+
+
+def test_catches_fork_without_reference_counts():
+    class Bad(oalloc.BlockManager):
+        def fork(self, parent, child):
+            if parent not in self.tables:
+                raise oalloc.AllocError(oalloc.UNKNOWN_SEQ, str(parent))
+            self.tables[child] = list(self.tables[parent])
+            self.lens[child] = self.lens[parent]
+    assert _caught_allocator(Bad)
+
+
+def test_catches_free_that_leaks_blocks():
+    class Bad(oalloc.BlockManager):
+        def free_seq(self, seq_id):
+            self.tables.pop(seq_id)
+            del self.lens[seq_id]
+    assert _caught_allocator(Bad)
+
+
+def test_catches_block_taken_one_token_early():
+    class Bad(oalloc.BlockManager):
+        def append_slot(self, seq_id):
+            table, n = self.tables[seq_id], self.lens[seq_id]
+            if n % self.block_size == self.block_size - 1 and self._available():
+                table.append(self._pop())          # the last slot of a block is never used
+                self.lens[seq_id] = n + 1
+                return table[-1] * self.block_size, -1, -1
+            return super().append_slot(seq_id)
+    assert _caught_allocator(Bad)
+
+
+def test_catches_copy_on_write_that_keeps_the_shared_reference():
+    class Bad(oalloc.BlockManager):
+        def _release(self, b):
+            if self.ref[b] > 1:
+                return                             # the writer's reference is never dropped
+            super()._release(b)
+    assert _caught_allocator(Bad)
