@@ -156,8 +156,10 @@ int pa_swap_blocks(void* dst_k, void* dst_v, int64_t dst_num_blocks, const void*
  * pa_decode_workspace_bytes - scratch bytes pa_decode_attention needs.
  * P = ceil(max_seq_len / partition_size) partitions per sequence; when P > 1 the
  * workspace holds float32 partial outputs [num_seqs, num_heads, P, head_dim] and
- * float32 running max / exp-sum [num_seqs, num_heads, P] each.  Returns 0 when
- * P <= 1 (no merge needed) and 0 for invalid sizes.
+ * float32 max / exp-sum pairs [num_seqs, num_heads, P] each (the max is the one the
+ * partition's weights were taken against; it may trail the true maximum logit by up
+ * to 8 in base 2, and the merge uses each pair as a whole).  Returns 0 when P <= 1
+ * (no merge needed) and 0 for invalid sizes.
  */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_seq_len,
                                  int partition_size);
@@ -212,8 +214,9 @@ int pa_decode_partition_size(int cache_dtype, int num_seqs, int num_heads, int n
  * For each sequence s and query head h (kv head g = h / (num_heads/num_kv_heads)):
  *   out[s,h,:] = sum_t softmax_t(scale * q[s,h,:] . K_t) V_t over the seq_lens[s]
  * cached tokens t, K_t/V_t read from block block_tables[s, t / block_size], offset
- * t % block_size, kv head g.  Accumulation is float32; out is rounded to the cache
- * dtype (round-to-nearest-even).  seq_lens[s] == 0 gives zeros.
+ * t % block_size, kv head g.  Accumulation is float32 and the softmax weights come
+ * from the hardware base-2 exponential (relative error about 2^-22); out is rounded to
+ * the cache dtype (round-to-nearest-even).  seq_lens[s] == 0 gives zeros.
  * Supported: head_dim in {64, 128, 256}; block_size in {4, 8, 16, 32}; tensor-core
  * path for num_heads/num_kv_heads a multiple of 8 with bf16/f16, head_dim 64/128/256
  * and block_size 16/32; other shapes use the CUDA-core path.
