@@ -17,9 +17,8 @@ import torch
 import oracle.attention as oatt
 import oracle.cache_ops as ocache
 from oracle.allocator import AllocError, BlockManager
-from oracle.numerics import to_f64
 from oracle.waste import batch_memory, contiguous_reservation, paged_growth
-from workloads import CONFIGS, make_inputs, normal_fill
+from workloads import CONFIGS, make_inputs, normal_fill, storage_to_torch
 
 pytestmark = pytest.mark.filterwarnings("ignore")
 
@@ -57,7 +56,8 @@ def _draw_contiguous(lens, Hq, Hkv, D, dtype, seed):
 def check_against_sdpa(att=oatt, lens=(5, 13, 7, 18, 10), Hq=4, Hkv=4, D=64, bs=4,
                        dtype="f32", seed=0, scale=0.125, reshape=None):
     """Largest |oracle - torch SDPA| over all (seq, head); SDPA runs in float64 on the
-    contiguous K/V (query head h reads kv head h // (Hq/Hkv) via repeat_interleave)."""
+    contiguous K/V (query head h reads kv head h // (Hq/Hkv) via repeat_interleave),
+    widened from the stored bits by torch's casts."""
     Ks, Vs, q = _draw_contiguous(lens, Hq, Hkv, D, dtype, seed)
     nb = sum(-(-L // bs) for L in lens) + 3
     order = np.random.default_rng(seed).permutation(nb).astype(np.int32)
@@ -66,11 +66,13 @@ def check_against_sdpa(att=oatt, lens=(5, 13, 7, 18, 10), Hq=4, Hkv=4, D=64, bs=
     out = att.paged_decode_attention(q, k, v, tables, seq_lens, scale, bs, Hkv, dtype)
     worst = 0.0
     G = Hq // Hkv
+    # the SDPA side widens the stored bits with torch's own casts, not the oracle's
+    wide = lambda a: storage_to_torch(a, dtype).double()
     for s, L in enumerate(lens):
-        Kt = torch.from_numpy(to_f64(Ks[s], dtype)).permute(1, 0, 2)   # [Hkv, L, D]
-        Vt = torch.from_numpy(to_f64(Vs[s], dtype)).permute(1, 0, 2)
+        Kt = wide(Ks[s]).permute(1, 0, 2)                               # [Hkv, L, D]
+        Vt = wide(Vs[s]).permute(1, 0, 2)
         Kt, Vt = Kt.repeat_interleave(G, 0), Vt.repeat_interleave(G, 0)
-        qt = torch.from_numpy(to_f64(q[s], dtype)).unsqueeze(1)        # [Hq, 1, D]
+        qt = wide(q[s]).unsqueeze(1)                                    # [Hq, 1, D]
         ref = torch.nn.functional.scaled_dot_product_attention(
             qt.unsqueeze(0), Kt.unsqueeze(0), Vt.unsqueeze(0), scale=scale)[0, :, 0, :]
         worst = max(worst, float(np.abs(out[s] - ref.numpy()).max()))
@@ -470,3 +472,309 @@ def test_truncate_keeps_shared_blocks_shared():
     _, src, dst = bm.append_slot(1)  # writing into the shared block copies it
     assert src == 0 and bm.ref[0] == 1
     _invariants(bm)
+
+
+# ---------------------------------------------------------------------------
+# widening of stored values: oracle.numerics.to_f64 against the IEEE-754 binary
+# formats decoded from their definition and against torch's own dtype casts
+# ([LAB] "Measure memory use across requests": paging leaves the attention
+# equation unchanged, so the stored bits must widen to exactly their value)
+# ---------------------------------------------------------------------------
+
+def _decode_binary(bits: int, exp_bits: int, man_bits: int) -> float:
+    """Value of an IEEE-754 binary pattern from the format's definition: sign bit,
+    biased exponent, fraction; exponent 0 is subnormal, all ones is inf / NaN."""
+    sign = -1.0 if (bits >> (exp_bits + man_bits)) & 1 else 1.0
+    e = (bits >> man_bits) & ((1 << exp_bits) - 1)
+    f = bits & ((1 << man_bits) - 1)
+    bias = (1 << (exp_bits - 1)) - 1
+    if e == (1 << exp_bits) - 1:
+        return sign * math.inf if f == 0 else math.nan
+    if e == 0:
+        return sign * math.ldexp(f, 1 - bias - man_bits)
+    return sign * math.ldexp((1 << man_bits) + f, e - bias - man_bits)
+
+
+def _same_f64(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Element-wise exact equality of float64 values, NaN equal to NaN, -0 != +0."""
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    both_nan = np.isnan(a) & np.isnan(b)
+    return both_nan | (a.view(np.uint64) == b.view(np.uint64))
+
+
+# hand values: (dtype, bit pattern, value)
+_HAND_VALUES = [
+    ("bf16", 0x3F80, 1.0), ("bf16", 0xC000, -2.0), ("bf16", 0x0001, 2.0 ** -133),
+    ("bf16", 0x0080, 2.0 ** -126), ("bf16", 0x7F7F, (2 - 2.0 ** -7) * 2.0 ** 127),
+    ("bf16", 0x7F80, math.inf), ("bf16", 0xFF80, -math.inf), ("bf16", 0x7FC0, math.nan),
+    ("bf16", 0x8000, -0.0), ("bf16", 0x3E00, 0.125), ("bf16", 0x4049, 3.140625),
+    ("f16", 0x3C00, 1.0), ("f16", 0xC000, -2.0), ("f16", 0x0001, 2.0 ** -24),
+    ("f16", 0x0400, 2.0 ** -14), ("f16", 0x7BFF, 65504.0), ("f16", 0x7C00, math.inf),
+    ("f16", 0xFC00, -math.inf), ("f16", 0x7E00, math.nan), ("f16", 0x8000, -0.0),
+    ("f16", 0x3555, 0.333251953125),
+    ("f32", 0x3F800000, 1.0), ("f32", 0x00000001, 2.0 ** -149),
+    ("f32", 0x7F7FFFFF, (2 - 2.0 ** -23) * 2.0 ** 127), ("f32", 0xFF800000, -math.inf),
+]
+
+
+def _storage_from_bits(bits: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "bf16":
+        return bits.astype(np.uint16)
+    if dtype == "f16":
+        return bits.astype(np.uint16).view(np.float16)
+    return bits.astype(np.uint32).view(np.float32)
+
+
+def check_widening(fn=None, seed=12) -> int:
+    """Number of stored bit patterns whose widened value differs from (a) the format's
+    definition, (b) torch's cast of the same bits, or (c) the hand values.  Covers all
+    65 536 bf16 and f16 patterns and 40 000 float32 patterns (random plus specials)."""
+    if fn is None:
+        from oracle import numerics
+        fn = numerics.to_f64
+    bad = 0
+    all16 = np.arange(1 << 16, dtype=np.uint32)
+    g = np.random.default_rng(seed)
+    f32 = np.concatenate([g.integers(0, 1 << 32, 40000 - 8, dtype=np.uint64).astype(np.uint32),
+                          np.array([0, 0x80000000, 1, 0x807FFFFF, 0x7F800000, 0x7FC00000,
+                                    0x3F800000, 0xBF800000], np.uint32)])
+    for dtype, bits, (eb, mb), tview in (("bf16", all16, (8, 7), torch.bfloat16),
+                                         ("f16", all16, (5, 10), torch.float16),
+                                         ("f32", f32, (8, 23), torch.float32)):
+        got = np.asarray(fn(_storage_from_bits(bits, dtype), dtype), np.float64)
+        if got.shape != bits.shape:
+            return bits.size
+        definition = np.array([_decode_binary(int(b), eb, mb) for b in bits])
+        if dtype == "f32":
+            t = torch.from_numpy(bits.astype(np.uint32).view(np.int32)).view(torch.float32)
+        else:
+            t = torch.from_numpy(bits.astype(np.uint16).view(np.int16)).view(tview)
+        by_torch = t.double().numpy()
+        bad += int((~_same_f64(got, definition)).sum()) + int((~_same_f64(got, by_torch)).sum())
+    for dtype, b, value in _HAND_VALUES:
+        got = np.asarray(fn(_storage_from_bits(np.array([b], np.uint32), dtype), dtype))
+        bad += int(not _same_f64(got, np.array([value]))[0])
+    return bad
+
+
+def test_widening_matches_the_formats_exactly():
+    assert check_widening() == 0
+
+
+def test_format_decoder_matches_hand_values():
+    """The definition decoder above, checked by itself on the hand values."""
+    for dtype, b, value in _HAND_VALUES:
+        eb, mb = {"bf16": (8, 7), "f16": (5, 10), "f32": (8, 23)}[dtype]
+        assert _same_f64(np.array([_decode_binary(b, eb, mb)]), np.array([value]))[0]
+
+
+# ---------------------------------------------------------------------------
+# moving sequences between two pools (swap out / in): the block manager's move
+# ---------------------------------------------------------------------------
+
+class _Contents:
+    """What each sequence has written, and what each physical slot holds.
+
+    Token ids are unique integers.  Writes follow the block manager's slots and
+    copy-on-write pairs; a move copies the blocks its pairs name.  Reading a
+    sequence back through its block table must give exactly the tokens that
+    sequence was given ([BLOG] "The bonus contiguous storage can't give you:
+    sharing": sharing and copy-on-write never change what a sequence reads)."""
+
+    def __init__(self, pools):
+        self.mem = {id(p): np.full((p.num_blocks, p.block_size), -1, np.int64) for p in pools}
+        self.tokens = {}
+        self.next_tok = 0
+
+    def _fresh(self, n):
+        t = list(range(self.next_tok, self.next_tok + n))
+        self.next_tok += n
+        return t
+
+    def add(self, bm, s, n):
+        bm.add(s, n)
+        toks = self._fresh(n)
+        mem = self.mem[id(bm)]
+        for t, tok in enumerate(toks):
+            mem[bm.tables[s][t // bm.block_size], t % bm.block_size] = tok
+        self.tokens[s] = toks
+
+    def fork(self, bm, p, c):
+        bm.fork(p, c)
+        self.tokens[c] = list(self.tokens[p])
+
+    def append(self, bm, s):
+        slot, src, dst = bm.append_slot(s)
+        mem = self.mem[id(bm)]
+        if src >= 0:
+            mem[dst] = mem[src]
+        tok = self._fresh(1)[0]
+        mem[slot // bm.block_size, slot % bm.block_size] = tok
+        self.tokens[s].append(tok)
+
+    def free(self, bm, s):
+        bm.free_seq(s)
+        del self.tokens[s]
+
+    def move(self, src_bm, dst_bm, ids):
+        pairs = src_bm.move_to(dst_bm, ids)
+        ms, md = self.mem[id(src_bm)], self.mem[id(dst_bm)]
+        for a, b in pairs:
+            md[b] = ms[a]
+        return pairs
+
+    def check(self, bm):
+        mem = self.mem[id(bm)]
+        for s, table in bm.tables.items():
+            L = bm.lens[s]
+            read = [int(mem[table[t // bm.block_size], t % bm.block_size]) for t in range(L)]
+            assert read == self.tokens[s], s
+
+
+def check_moves(bm_cls=BlockManager, seed=21, trials=6, n_ops=250):
+    """Random add / fork / append / free / move-out / move-in sequences over two pools.
+    After every op: the invariants on both pools (counts = table entries, free and
+    used partition each pool, ceil(L/bs) blocks), every sequence reads back exactly
+    its own tokens, and each move's pairs are the moved set's distinct blocks in
+    first-appearance order with distinct fresh destinations."""
+    g = np.random.default_rng(seed)
+    for _ in range(trials):
+        bs = int(g.choice([1, 2, 4]))
+        A = bm_cls(40, bs, g.permutation(40))
+        B = bm_cls(30, bs, g.permutation(30))
+        C = _Contents([A, B])
+        where, nid = {}, 0
+        for _ in range(n_ops):
+            r = int(g.integers(0, 10))
+            pool = A if g.integers(0, 3) else B
+            mine = [s for s, p in where.items() if p is pool]
+            try:
+                if r < 2 or not mine:
+                    C.add(pool, nid, int(g.integers(0, 3 * bs + 1)))
+                    where[nid] = pool
+                    nid += 1
+                elif r < 4:
+                    C.fork(pool, mine[int(g.integers(0, len(mine)))], nid)
+                    where[nid] = pool
+                    nid += 1
+                elif r < 6:
+                    C.append(pool, mine[int(g.integers(0, len(mine)))])
+                elif r < 7:
+                    s = mine[int(g.integers(0, len(mine)))]
+                    C.free(pool, s)
+                    del where[s]
+                else:
+                    other = B if pool is A else A
+                    k = int(g.integers(1, min(4, len(mine)) + 1))
+                    ids = [int(x) for x in g.choice(mine, k, replace=False)]
+                    old = {s: list(pool.tables[s]) for s in ids}
+                    free_before = other.free_list()
+                    pairs = C.move(pool, other, ids)
+                    distinct = list(dict.fromkeys(b for s in ids for b in old[s]))
+                    assert [a for a, _ in pairs] == distinct
+                    assert [b for _, b in pairs] == free_before[:len(distinct)]
+                    m = dict(pairs)
+                    for s in ids:
+                        assert other.tables[s] == [m[b] for b in old[s]]
+                        where[s] = other
+            except AllocError:
+                pass
+            for p in (A, B):
+                _invariants(p)
+                C.check(p)
+    return True
+
+
+def test_moves_keep_invariants_and_contents():
+    assert check_moves()
+
+
+def test_move_hand_case_shared_block_becomes_private():
+    """Worked by hand.  Pool A pops 5, 3, 7, 0, ...; pool B pops 2, 0, 1, 3.
+    seq 0 holds 10 tokens at 4 per block: blocks 5, 3, 7 (7 half full).  seqs 1 and 2
+    fork from it (every count 3).  seq 2 appends: block 7 is shared, so it copies
+    7 -> 0 (7 drops to 2).  Moving seqs 0 and 1 to B: their distinct blocks 5, 3, 7
+    get B's 2, 0, 1, shared by both (count 2 each).  In A, seq 2 keeps 5 and 3, now
+    private (count 1), and block 7 reaches zero and goes back on top of A's stack."""
+    A = BlockManager(8, 4, [5, 3, 7, 0, 1, 2, 4, 6])
+    B = BlockManager(4, 4, [2, 0, 1, 3])
+    A.add(0, 10)
+    A.fork(0, 1)
+    A.fork(0, 2)
+    assert A.tables[0] == [5, 3, 7] and A.ref[5] == A.ref[3] == A.ref[7] == 3
+    slot, src, dst = A.append_slot(2)
+    assert (src, dst) == (7, 0) and slot == 0 * 4 + 2 and A.ref[7] == 2
+    pairs = A.move_to(B, [0, 1])
+    assert pairs == [(5, 2), (3, 0), (7, 1)]
+    assert B.tables[0] == B.tables[1] == [2, 0, 1] and B.lens == {0: 10, 1: 10}
+    assert [B.ref[b] for b in (2, 0, 1)] == [2, 2, 2] and B.free_list() == [3]
+    assert A.tables == {2: [5, 3, 0]} and A.lens == {2: 11}
+    assert [A.ref[b] for b in (5, 3, 0, 7)] == [1, 1, 1, 0]
+    assert A.free_list() == [7, 1, 2, 4, 6]
+    _invariants(A)
+    _invariants(B)
+
+
+# ---------------------------------------------------------------------------
+# prefix groups: a fork forest worked by hand
+# ---------------------------------------------------------------------------
+
+def _fork_forest(bm_cls=BlockManager):
+    """Block size 4, a 32-block pool taken in index order.
+      seq 10: 20 tokens (5 full blocks); 11 and 12 fork from it.
+      11 appends 1 token (a fresh sixth block).  12 is truncated to 9 tokens and
+      appends one: its third block was shared, so it copies (tables diverge after
+      2 blocks).  50 forks from 10 at the end.
+      seq 20: 12 tokens (3 full blocks); 21 forks and appends 1 (a fresh block).
+      seq 30: 3 tokens (1 block); 31 forks from it.
+      seq 40: 16 tokens, alone.
+    Batch order [40, 10, 20, 11, 30, 12, 21, 31, 50] (positions 0..8)."""
+    bm = bm_cls(32, 4)
+    bm.add(10, 20)
+    bm.fork(10, 11)
+    bm.fork(10, 12)
+    bm.append_slot(11)
+    bm.truncate([12], [9])
+    bm.append_slot(12)
+    bm.add(20, 12)
+    bm.fork(20, 21)
+    bm.append_slot(21)
+    bm.add(30, 3)
+    bm.fork(30, 31)
+    bm.add(40, 16)
+    bm.fork(10, 50)
+    return bm, [40, 10, 20, 11, 30, 12, 21, 31, 50]
+
+
+# (partition_size, max_members) -> (prefix_parts per position, chunks)
+# group of 10 (positions 1, 3, 5, 8): common prefix 2 blocks = 8 tokens;
+# group of 20 (positions 2, 6): 3 blocks = 12 tokens; group of 30 (4, 7): 1 block
+# = 4 tokens; 40 (position 0) is alone.  parts = floor(common tokens / partition).
+_FOREST_EXPECTED = {
+    (8, 2): ([0, 1, 1, 1, 0, 1, 1, 0, 1], [([1, 3], 1), ([5, 8], 1), ([2, 6], 1)]),
+    (8, 8): ([0, 1, 1, 1, 0, 1, 1, 0, 1], [([1, 3, 5, 8], 1), ([2, 6], 1)]),
+    (4, 3): ([0, 2, 3, 2, 1, 2, 3, 1, 2],
+             [([1, 3, 5], 2), ([8], 2), ([2, 6], 3), ([4, 7], 1)]),
+    (16, 8): ([0] * 9, []),
+}
+
+
+def check_prefix_groups(bm_cls=BlockManager) -> int:
+    """Number of (partition, max_members) cases whose groups differ from the hand
+    values above."""
+    bm, ids = _fork_forest(bm_cls)
+    bad = 0
+    for (ps, mm), (parts, chunks) in _FOREST_EXPECTED.items():
+        got_parts, got_chunks = bm.prefix_groups(ids, ps, mm)
+        got = (list(got_parts), [(list(m), int(p)) for m, p in got_chunks])
+        bad += int(got != (parts, chunks))
+    return bad
+
+
+def test_prefix_groups_of_a_hand_built_fork_forest():
+    bm, _ = _fork_forest()
+    assert bm.tables[10] == [0, 1, 2, 3, 4] and bm.tables[11] == [0, 1, 2, 3, 4, 5]
+    assert bm.tables[12] == [0, 1, 6] and bm.tables[50] == [0, 1, 2, 3, 4]
+    assert bm.tables[20] == [7, 8, 9] and bm.tables[21] == [7, 8, 9, 10]
+    assert bm.tables[30] == bm.tables[31] == [11] and bm.tables[40] == [12, 13, 14, 15]
+    assert check_prefix_groups() == 0
