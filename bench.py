@@ -9,9 +9,16 @@ pa_decode_attention run.  Inputs are synthetic (seeded, see ``workloads``) and
 resident in HBM before the timed region; the K/V pool is far larger than L2, so no
 flush is needed between steps.
 
+Order of a run: set-up; untimed steps for --settle-ms (clocks up); W warm-up steps;
+the timed region of exactly K steps (clocks sampled through NVML during it); the
+decode call's own loop of --roofline-ms with CUDA events on a sample of its calls
+(the roofline); K host-fed steps (e2e); at N=1 the other workloads
+(``per_workload``: the 13B-shaped, long-context GQA, shared-prefix and tiny ones,
+and fp8 caches), each with loops sized by time; then the CPU oracle on the host.
+
 Under torchrun each rank runs its own replica (its own pool, sequences and seed):
 the path has no exchange step, so there is no collective on the data path; the
-ranks meet only at the barriers around the timed region and in the max-reduction
+ranks meet only at the barriers around the timed regions and in the max-reduction
 of the elapsed time.  Rank 0 prints one JSON line.
 
 ``--impl reference`` times the CPU oracle (rank 0 only) on bounded samples of the
@@ -59,6 +66,14 @@ def parse():
                     help="override the partition size of the decode split")
     ap.add_argument("--cache-fp8", action="store_true",
                     help="store K/V as fp8 e4m3 with per-tensor scales (q/out keep the dtype)")
+    ap.add_argument("--settle-ms", type=float, default=500.0,
+                    help="untimed steps before the warm-up, so that clocks settle")
+    ap.add_argument("--roofline-ms", type=float, default=1000.0,
+                    help="length of the loop in which the decode call is event-timed")
+    ap.add_argument("--per-workload-ms", type=float, default=400.0,
+                    help="length of each timed loop of the other workloads")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="measure only the selected workload")
     return ap.parse_args()
 
 
@@ -150,17 +165,73 @@ def job_throughput(job_bytes_per_step: float, steps: int, elapsed_max_ms: float)
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clocks and clock-event reasons sampled during a timed region.
+
+    NVML is polled from a thread about once a millisecond, so that even a region of
+    a few milliseconds gets samples; without NVML, ``nvidia-smi -lms 50`` is the
+    fallback.  Only samples taken between ``__enter__`` and ``__exit__`` count."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
     FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    _nvml = None
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    def __init__(self, index: int, period_s: float = 0.001):
+        self.index, self.period = index, period_s
+        self.samples, self.max_mhz, self.source = [], None, None
+
+    @classmethod
+    def _handle(cls, index: int):
+        try:
+            import pynvml
+            if cls._nvml is None:
+                pynvml.nvmlInit()
+                cls._nvml = pynvml
+            handle = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(index).uuid)
+                handle = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(index)
+            return pynvml, handle
+        except Exception:
+            return None, None
 
     def __enter__(self):
         import threading
-        self.lines, self.first = [], threading.Event()
+        self.stop = threading.Event()
+        nv, h = self._handle(self.index)
+        if nv is not None:
+            self.source = "nvml"
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+
+            def poll():
+                while not self.stop.is_set():
+                    try:
+                        mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        bits = int(get_reasons(h)) if get_reasons else 0
+                        self.samples.append((time.perf_counter(), mhz, bits))
+                    except Exception:
+                        pass
+                    self.stop.wait(self.period)
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+        else:
+            self._start_smi()
+        deadline = time.perf_counter() + 10
+        while not self.samples and time.perf_counter() < deadline and self.source:
+            time.sleep(0.001)          # sampling is running before the timed region
+        self.t0 = time.perf_counter()
+        return self
+
+    def _start_smi(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -168,47 +239,57 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
-            return self
+            return
+        self.source = "nvidia-smi"
 
         def reader():
             for line in self.proc.stdout:
-                if line.strip():
-                    self.lines.append((time.perf_counter(), line.strip()))
-                    self.first.set()
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    mhz, self.max_mhz = float(parts[0]), float(parts[1])
+                except ValueError:
+                    continue
+                bits = 0
+                for (n, b), v in zip(self.REASONS, parts[3:7]):
+                    if v.lower() == "active":
+                        bits |= b
+                self.samples.append((time.perf_counter(), mhz, bits))
         self.thread = threading.Thread(target=reader, daemon=True)
         self.thread.start()
-        self.first.wait(timeout=10)       # sampling is running before the timed region
-        self.t0 = time.perf_counter()
-        return self
 
     def __exit__(self, *a):
         self.t1 = time.perf_counter()
-        if self.proc is not None:
-            self.proc.terminate()
+        self.stop.set()
+        proc = getattr(self, "proc", None)
+        if proc is not None:
+            proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
+                proc.kill()
+        if getattr(self, "thread", None) is not None:
             self.thread.join(timeout=5)
-            self.lines = [l for t, l in self.lines if self.t0 <= t <= self.t1]
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [(m, b) for t, m, b in self.samples if self.t0 <= t <= self.t1]
+        sm = [m for m, _ in inside]
+        reasons = sorted({n for _, b in inside for n, bit in self.REASONS if b & bit})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": self.source}
+
+
+REJECTED_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def clocks_rejected(summary: dict) -> bool:
+    """A region that saw a hardware or thermal slowdown, or SM clocks far below the
+    maximum with no reason given (a leftover clock lock), is measured again."""
+    if any(r in summary.get("reasons", ()) for r in REJECTED_REASONS):
+        return True
+    mhz, mx = summary.get("sm_mhz"), summary.get("sm_max_mhz")
+    return bool(mhz and mx and mhz < 0.7 * mx and not summary.get("reasons"))
 
 
 def hbm_peak():
@@ -280,34 +361,58 @@ class OracleTimer:
         return b_all / t_all / 1e9, n / t_all, desc
 
 
+def workload_config(cfg, lens, world: int, cache_fp8: bool) -> dict:
+    """The workload as both arms state it in their JSON line (static facts only)."""
+    kv_elem = 1 if cache_fp8 else cfg.elem_bytes
+    pool_bytes = 2 * cfg.num_blocks * cfg.num_kv_heads * cfg.block_size * cfg.head_dim * kv_elem
+    return {
+        "workload": cfg.name, "description": cfg.description,
+        "num_seqs": cfg.num_seqs, "num_heads": cfg.num_heads,
+        "num_kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
+        "block_size": cfg.block_size, "num_blocks": cfg.num_blocks,
+        "partition_size": cfg.partition_size or "library choice (pa_decode_partition_size)",
+        "mean_seq_len": round(float(np.mean(lens)), 1), "max_seq_len": int(np.max(lens)),
+        "l2": ("inputs larger than L2 (K/V pool %.2f GB per rank), no flush"
+               % (pool_bytes / 1e9)) if pool_bytes > L2_BYTES else
+              ("K/V pool of %.1f KB fits in L2: a parity-size workload, no flush"
+               % (pool_bytes / 1e3)),
+        "steps": "each step appends one token per sequence and rolls the previous one "
+                 "back, so every step decodes these lengths",
+        "parallelism": f"replicas x{world}",
+        "kv_cache": "fp8 e4m3, per-tensor scales" if cache_fp8 else cfg.dtype,
+    }
+
+
 def run_reference(args, cfg):
     """The oracle as the reference arm: rank 0 only; each step is the oracle on a
-    bounded sample of the workload (two sequences, all heads)."""
+    bounded sample of the workload (whole sequences, all heads), the requested number
+    of warm-up and timed steps."""
     if int(os.environ.get("RANK", "0")) != 0:
         return
-    from workloads import make_inputs
+    from workloads import draw_lengths, make_inputs
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     timer = OracleTimer(cfg, make_inputs(cfg, args.seed))
-    # bounded: about 2 minutes of oracle work at the default step count
-    per_step = 1 if args.steps * 1 > 500 else 2
-    steps = min(args.steps, 200)
+    # bounded: two sequences per step up to 500 steps, one beyond (the oracle takes
+    # about 10-25 ms per 7B-shaped sequence)
+    per_step = 2 if args.steps <= 500 else 1
     t_all, b_all = 0.0, 0
-    warm = min(args.warmup, 3)
-    for i in range(warm + steps):
+    for i in range(args.warmup + args.steps):
         seqs = [(i * per_step + j) % cfg.num_seqs for j in range(per_step)]
         dt, b = timer.run(seqs)
-        if i >= warm:
+        if i >= args.warmup:
             t_all, b_all = t_all + dt, b_all + b
     value = b_all / t_all / 1e9
     sample = (f"per step: oracle decode attention (float64, all {cfg.num_heads} heads) of "
               f"{per_step} of the {cfg.num_seqs} sequences, cycling through the batch; "
-              f"{steps} timed steps (at most 200 of the requested {args.steps})")
+              f"{args.steps} timed steps after {args.warmup} warm-up steps")
+    lens, _ = draw_lengths(cfg, args.seed)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
-        "n_gpus": args.gpus, "steps": steps, "warmup": warm,
-        "ms_per_step": round(1e3 * t_all / steps, 3), "higher_is_better": True,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t_all / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "seqs_per_s": round(per_step * steps / t_all, 4),
-        "config": {"workload": cfg.name, "description": cfg.description},
+        "seqs_per_s": round(per_step * args.steps / t_all, 4),
+        "config": workload_config(cfg, lens, world, args.cache_fp8),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": timer.threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -320,20 +425,382 @@ def run_reference(args, cfg):
 # our arm
 # ---------------------------------------------------------------------------
 
+def _event_pair():
+    import torch
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+class WorkloadRun:
+    """One workload resident on the device, stepped through the library's step runtime.
+
+    ``host_pool``: the K/V pool is the seeded host draw of ``workloads.make_inputs``
+    (the CPU baseline then reads the same values); otherwise it is drawn on the
+    device with the same distribution (``workloads.device_normal_fill``)."""
+
+    RING = 8
+
+    def __init__(self, cfg, seed: int, dev, cache_fp8: bool = False, host_pool: bool = True):
+        import torch
+
+        import paged_kv_cache_342_b200 as pa
+        from paged_kv_cache_342_b200.runtime import PagedDecoder
+        from workloads import (TORCH_DTYPES, device_normal_fill, make_inputs, step_tokens,
+                               storage_to_torch)
+        self.cfg, self.dev, self.pa, self.cache_fp8 = cfg, dev, pa, cache_fp8
+        inp = make_inputs(cfg, seed, pool=host_pool)
+        self.inp = inp
+        S, Hq, Hkv, D, bs = (cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_dim,
+                             cfg.block_size)
+        max_len = int((inp.context_lens + 1).max()) + 1
+        max_blocks = (max_len + bs - 1) // bs
+        if host_pool:
+            kd = storage_to_torch(inp.k_pool, cfg.dtype).to(dev)
+            vd = storage_to_torch(inp.v_pool, cfg.dtype).to(dev)
+        else:
+            shape = (cfg.num_blocks, Hkv, bs, D)
+            kd = device_normal_fill(shape, cfg.dtype, cfg.std, seed, 2, dev)
+            vd = device_normal_fill(shape, cfg.dtype, cfg.std, seed, 3, dev)
+        self.kv_scales, self.ekv = None, None
+        if cache_fp8:
+            # quantize the pool on the device with the library's fp8 write (all slots)
+            self.kv_scales, self.ekv = (8.0 * cfg.std / 448.0,) * 2, 1
+            NB = cfg.num_blocks
+            slots_all = torch.arange(NB * bs, dtype=torch.int64, device=dev)
+            k8 = torch.empty(kd.shape, dtype=torch.uint8, device=dev)
+            v8 = torch.empty_like(k8)
+            for src, dst in ((kd, k8), (vd, v8)):
+                rows = src.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous()
+                pa.pa_reshape_and_cache_fp8(rows, rows, dst, dst, slots_all, *self.kv_scales)
+                del rows
+            kd, vd = k8, v8
+            torch.cuda.synchronize(dev)
+        self.pool_bytes = 2 * kd.numel() * kd.element_size()
+        self.kd, self.vd = kd, vd
+        dec = PagedDecoder(kd, vd, Hq, cfg.scale, max_blocks, inp.free_order,
+                           cfg.partition_size, kv_scales=self.kv_scales,
+                           query_dtype=TORCH_DTYPES[cfg.dtype])
+        if inp.prefix is None:
+            for s in range(S):
+                dec.admit(s, int(inp.context_lens[s]))
+        else:
+            p = inp.prefix
+            dec.apply_copies(dec.admit_shared_prefix(p.groups, p.samples, p.prefix_len,
+                                                     p.private_lens))
+        # every step decodes the same lengths: sequences roll back one token per step
+        dec.bind(range(S), rolling=True)
+        self.dec = dec
+        # a ring of distinct per-step token sets: pinned host copies and device copies
+        self.toks_h, self.toks_d = [], []
+        for i in range(self.RING):
+            q, nk, nv = (inp.q, inp.new_k, inp.new_v) if i == 0 else step_tokens(cfg, seed, i)
+            h = [storage_to_torch(a, cfg.dtype).pin_memory() for a in (q, nk, nv)]
+            self.toks_h.append(h)
+            self.toks_d.append([t.to(dev) for t in h])
+        self.out = torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.k = 0
+        # the workload is stationary: bytes per step computed once
+        self.meta0 = self.step()
+        torch.cuda.synchronize(dev)
+        self.lens = np.array([dec.alloc.seq_len(s) for s in range(S)], np.int64)
+        self.uniq = (unique_context_tokens(dec, cfg, range(S)) if inp.prefix is not None
+                     else None)
+        self.dec_bytes = decode_bytes(cfg, self.lens, self.uniq, self.ekv)
+        self.step_bytes = self.dec_bytes + cache_op_bytes(cfg, S, 0, self.ekv)
+        self.logical_dec_bytes = decode_bytes(cfg, self.lens, None, self.ekv)
+        self.launches_per_step = dec.kernel_launches(self.meta0)
+        if host_pool:
+            pass                      # the host pool stays for the CPU baseline
+        self.check_errors("set-up")
+
+    def step(self, ev=None):
+        q, nk, nv = self.toks_d[self.k % self.RING]
+        self.k += 1
+        return self.dec.step(q, nk, nv, self.out, events=ev)
+
+    def check_errors(self, where: str):
+        err = self.pa.pa_device_error_read()
+        if err:
+            raise RuntimeError(f"device error word {err} ({where})")
+
+    def run_for(self, seconds: float) -> int:
+        """Untimed steps for about ``seconds`` of device time (clocks settle)."""
+        import torch
+        n, t0 = 0, time.perf_counter()
+        while True:
+            for _ in range(10):
+                self.step()
+            n += 10
+            torch.cuda.synchronize(self.dev)
+            if time.perf_counter() - t0 >= seconds:
+                return n
+
+    def steps_for(self, seconds: float, lo: int = 20, hi: int = 20000) -> int:
+        """How many steps take about ``seconds`` (from 10 event-timed steps)."""
+        import torch
+        a, b = _event_pair()
+        a.record(self.stream)
+        for _ in range(10):
+            self.step()
+        b.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        per = a.elapsed_time(b) / 10 * 1e-3
+        return int(min(hi, max(lo, round(seconds / max(per, 1e-7)))))
+
+    def timed(self, steps: int, world: int = 1, dist=None, clock_index: int = 0):
+        """Exactly ``steps`` steps between two events, bracketed by barrier +
+        synchronize; returns (elapsed ms, clocks summary, copy pairs)."""
+        import torch
+        t0, t1 = _event_pair()
+        cows = 0
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(self.dev)
+        with ClockSampler(clock_index) as clk:
+            t0.record(self.stream)
+            for _ in range(steps):
+                cows += self.step()["num_cow"]
+            t1.record(self.stream)
+            torch.cuda.synchronize(self.dev)
+        if world > 1:
+            dist.barrier()
+        self.check_errors("timed region")
+        return t0.elapsed_time(t1), clk.summary(), cows
+
+    def roofline_loop(self, seconds: float, clock_index: int = 0, samples: int = 200):
+        """Steps for about ``seconds``, the decode call event-timed on ``samples`` of
+        them (every k-th step); returns (call ms list, clocks summary)."""
+        import torch
+        n = self.steps_for(seconds, lo=samples)
+        every = max(1, n // samples)
+        evs = [_event_pair() for _ in range(n // every + 1)]
+        torch.cuda.synchronize(self.dev)
+        e = 0
+        with ClockSampler(clock_index) as clk:
+            for i in range(n):
+                ev = None
+                if i % every == 0:
+                    ev, e = evs[e], e + 1
+                self.step(ev)
+            torch.cuda.synchronize(self.dev)
+        self.check_errors("roofline loop")
+        return [a.elapsed_time(b) for a, b in evs[:e]], clk.summary()
+
+    def cold_calls(self, n: int = 50):
+        """Decode calls after a 2x-L2 buffer write each (pools that fit in L2)."""
+        import torch
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=self.dev)
+        evs = [_event_pair() for _ in range(n)]
+        for ev in evs:
+            flush.fill_(1)
+            self.step(ev)
+        torch.cuda.synchronize(self.dev)
+        del flush
+        return [a.elapsed_time(b) for a, b in evs]
+
+    def e2e(self, steps: int, world: int = 1, dist=None, max_over=None):
+        """The public host-buffer step: inputs from pinned memory, the result back to
+        it, copies overlapped with the neighbouring steps' kernels."""
+        import torch
+        from workloads import TORCH_DTYPES
+        cfg = self.cfg
+        S, Hq, D = cfg.num_seqs, cfg.num_heads, cfg.head_dim
+        outs_h = [torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], pin_memory=True)
+                  for _ in range(2)]
+        done = [None, None]
+
+        def e2e_step(k):
+            if done[k % 2] is not None:
+                done[k % 2].synchronize()          # the caller consumed that result
+            done[k % 2] = self.dec.step_host(*self.toks_h[k % self.RING], outs_h[k % 2])
+
+        for k in range(3):
+            e2e_step(k)
+        torch.cuda.synchronize(self.dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = _event_pair()
+        e0.record(self.stream)
+        for k in range(steps):
+            e2e_step(k)
+        self.dec.drain_host_io()
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        self.check_errors("e2e")
+        e_ms = e0.elapsed_time(e1)
+        if max_over is not None:
+            e_ms = max_over(e_ms)
+        h2d = sum(t.numel() * t.element_size() for t in self.toks_h[0]) + self.dec.staging_bytes
+        d2h = S * Hq * D * cfg.elem_bytes
+        return e_ms, int(h2d), int(d2h)
+
+    def roofline(self, dec_ms, clk, peak, peak_kind):
+        cfg = self.cfg
+        avg = statistics.mean(dec_ms)
+        achieved = self.dec_bytes / (avg * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                "kernel": ("pa_decode_attention_fp8" if self.cache_fp8 else
+                           "pa_decode_attention") + " (partition kernels + log-sum-exp merge)",
+                "bytes_per_launch": int(self.dec_bytes), "avg_launch_us": round(avg * 1e3, 2),
+                "launches_timed": len(dec_ms),
+                "median_launch_us": round(statistics.median(dec_ms) * 1e3, 2),
+                "frac_of_nominal_8000": round(achieved / 8000.0, 4),
+                "traffic": recorded_traffic(cfg, self.cache_fp8),
+                "clocks": clk}
+        if clk.get("sm_mhz"):
+            # the call in SM clock cycles at the median clock (comparable across clocks)
+            roof["avg_launch_kcycles_at_median_clock"] = round(avg * clk["sm_mhz"], 1)
+        if self.uniq is not None:
+            roof["bytes_note"] = "unique bytes: each shared physical slot counted once"
+            roof["logical_bytes_per_launch"] = int(self.logical_dec_bytes)
+            roof["logical_achieved"] = round(self.logical_dec_bytes / (avg * 1e-3) / 1e9, 1)
+        return roof
+
+    def close(self):
+        import torch
+        self.dec = None
+        self.kd = self.vd = self.out = None
+        self.toks_d = self.toks_h = None
+        torch.cuda.synchronize(self.dev)
+        torch.cuda.empty_cache()
+
+
+# the other workloads, measured in the same invocation at N=1 (name, fp8 cache, partition)
+PER_WORKLOAD = [
+    ("13b_fp16", False, None),
+    ("gqa_long_bf16", False, None),
+    ("gqa_long_bf16", False, 0),
+    ("prefix_cow_bf16", False, None),
+    ("tiny_fp32", False, None),
+    ("7b_bf16", True, None),
+    ("13b_fp16", True, None),
+    ("gqa_long_bf16", True, None),
+]
+
+
+def per_workload_key(name, fp8, ps) -> str:
+    return name + ("+fp8_cache" if fp8 else "") + ("" if ps is None else "@library_partition")
+
+
+def measure_other(cfg, seed, dev, fp8, peak, peak_kind, seconds: float) -> dict:
+    """One entry of ``per_workload``: settle, a timed loop sized by time, the decode
+    call's roofline loop, and the host-buffer loop."""
+    run = WorkloadRun(cfg, seed, dev, cache_fp8=fp8, host_pool=False)
+    try:
+        run.run_for(0.3)
+        n = run.steps_for(seconds)
+        ms, clk, _ = run.timed(n, clock_index=dev.index or 0)
+        dec_ms, rclk = run.roofline_loop(seconds, clock_index=dev.index or 0)
+        roof = run.roofline(dec_ms, rclk, peak, peak_kind)
+        if run.pool_bytes <= L2_BYTES:
+            roof["cold_median_launch_us"] = round(statistics.median(run.cold_calls()) * 1e3, 2)
+            roof["cold_note"] = "pool smaller than L2: calls after a 2x-L2 buffer write"
+        e_ms, h2d, d2h = run.e2e(n)
+        S = cfg.num_seqs
+        return {
+            "value": round(run.step_bytes * n / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "steps": n, "ms_per_step": round(ms / n, 4),
+            "seqs_per_s": round(S * n / (ms * 1e-3), 1),
+            "partition_size": run.dec.partition_size,
+            "kv_cache": ("fp8 e4m3, per-tensor scales %g" % run.kv_scales[0]) if fp8
+                        else cfg.dtype,
+            "mean_seq_len": round(float(run.lens.mean()), 1), "max_seq_len": int(run.lens.max()),
+            "pool": "K/V drawn on the device (same distribution, seeded)",
+            "roofline": roof,
+            "e2e": {"value": round(run.step_bytes * n / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e_ms / n, 4)},
+            "gpu_launches": run.launches_per_step * n,
+            "clocks": clk,
+        }
+    finally:
+        run.close()
+
+
 def run_ours(args, cfg):
     import torch
     import torch.distributed as dist
 
     world, rank, local = replica_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    max_over = lambda v: max_over_ranks(v, world, dev)
+    peak, peak_kind = hbm_peak()
 
-    import paged_kv_cache_342_b200 as pa
-    from paged_kv_cache_342_b200.runtime import PagedDecoder
-    from workloads import TORCH_DTYPES, make_inputs, step_tokens, storage_to_torch
+    seed = replica_seed(args.seed, rank)
+    run = WorkloadRun(cfg, seed, dev, cache_fp8=args.cache_fp8, host_pool=True)
+    S = cfg.num_seqs
+    # clocks up and the pipeline steady before the warm-up steps
+    t_settle = time.perf_counter()
+    settle_steps = run.run_for(args.settle_ms * 1e-3)
+    settle_ms = (time.perf_counter() - t_settle) * 1e3
+    warm_cow = 0
+    for _ in range(args.warmup):
+        warm_cow += run.step()["num_cow"]
+    torch.cuda.synchronize(dev)
+    run.check_errors("warm-up")
 
-    # CPU baseline first (before any GPU work), rank 0 at N=1 only
+    # ---- the timed region: exactly --steps steps --------------------------------
+    elapsed_ms, clk, cows = run.timed(args.steps, world, dist, local)
+    retried = False
+    if clocks_rejected(clk):       # measured again once, as the timing rules ask
+        retried = True
+        elapsed_ms, clk, cows = run.timed(args.steps, world, dist, local)
+    elapsed_ms = max_over(elapsed_ms)
+    job_step_bytes = sum_over_ranks(run.step_bytes, world, dev)
+    value = job_throughput(job_step_bytes, args.steps, elapsed_ms)
+    seqs_per_s = S * world * args.steps / (elapsed_ms * 1e-3)
+
+    # ---- the decode call's own duration: its own loop of >= --roofline-ms ---------
+    dec_ms, rclk = run.roofline_loop(args.roofline_ms * 1e-3, local)
+    roof = run.roofline(dec_ms, rclk, peak, peak_kind)
+    if run.pool_bytes <= L2_BYTES and rank == 0:
+        roof["cold_median_launch_us"] = round(statistics.median(run.cold_calls()) * 1e3, 2)
+        roof["cold_note"] = "pool smaller than L2: calls after a 2x-L2 buffer write"
+
+    # ---- end to end through the public API with host buffers ----------------------
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = run.e2e(args.steps, world, dist, max_over)
+        E = job_throughput(job_step_bytes, args.steps, e_ms)
+        e2e = {"value": round(E, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms / args.steps, 4),
+               "seqs_per_s": round(S * world * args.steps / (e_ms * 1e-3), 1)}
+
+    config = workload_config(cfg, run.lens, world, args.cache_fp8)
+    run_info = {
+        "partition_size": run.dec.partition_size,
+        "workspace_bytes": int(run.dec.workspace_bytes),
+        "prefix_group_chunks": int(run.meta0.get("num_chunks", 0)),
+        "pool": pool_summary(run.dec.alloc.stats()),
+        "cow_pairs_in_warmup": warm_cow, "cow_pairs_in_timed_steps": cows,
+        "settle_ms": round(settle_ms, 1), "settle_steps": settle_steps,
+        "timed_region_retried_for_clocks": retried,
+        "kv_cache": ("fp8 e4m3, per-tensor scales %g" % run.kv_scales[0])
+                    if args.cache_fp8 else cfg.dtype,
+    }
+    launches = run.launches_per_step * args.steps
+    inp = run.inp
+    run.close()
+
+    # ---- the other workloads (N=1, default run only) --------------------------------
+    per = None
+    if world == 1 and not args.no_per_workload and args.default_shape:
+        per = {}
+        for name, fp8, ps in PER_WORKLOAD:
+            from workloads import CONFIGS
+            c = CONFIGS[name] if ps is None else CONFIGS[name].with_(partition_size=ps)
+            per[per_workload_key(name, fp8, ps)] = measure_other(
+                c, seed, dev, fp8, peak, peak_kind, args.per_workload_ms * 1e-3)
+
+    # ---- CPU baseline: the oracle on the host cores, rank 0 at N=1 only ------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        timer = OracleTimer(cfg, make_inputs(cfg, args.seed))
+        timer = OracleTimer(cfg, inp)
         gbs, sps, desc = timer.budgeted(12.0)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": timer.threads, "kind": "oracle",
                "sample": desc, "seqs_per_s": round(sps, 3), "host": host_cpu()}
@@ -347,180 +814,6 @@ def run_ours(args, cfg):
             pass
         del timer
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
-    seed = replica_seed(args.seed, rank)
-    inp = make_inputs(cfg, seed)
-    S, Hq, Hkv, D, bs = cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_dim, cfg.block_size
-    max_len = int((inp.context_lens + 1).max()) + 1
-    max_blocks = (max_len + bs - 1) // bs
-    kd = storage_to_torch(inp.k_pool, cfg.dtype).to(dev)
-    vd = storage_to_torch(inp.v_pool, cfg.dtype).to(dev)
-    kv_scales, ekv = None, None
-    if args.cache_fp8:
-        # quantize the pool on the device with the library's fp8 write (all slots)
-        kv_scales, ekv = (8.0 * cfg.std / 448.0,) * 2, 1
-        NB = cfg.num_blocks
-        slots_all = torch.arange(NB * bs, dtype=torch.int64, device=dev)
-        k8 = torch.empty(kd.shape, dtype=torch.uint8, device=dev)
-        v8 = torch.empty_like(k8)
-        for src, dst in ((kd, k8), (vd, v8)):
-            rows = src.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous()
-            pa.pa_reshape_and_cache_fp8(rows, rows, dst, dst, slots_all, *kv_scales)
-            del rows
-        kd, vd = k8, v8
-        torch.cuda.synchronize(dev)
-    pool_bytes = 2 * kd.numel() * kd.element_size()
-    del inp.k_pool, inp.v_pool
-    dec = PagedDecoder(kd, vd, Hq, cfg.scale, max_blocks, inp.free_order, cfg.partition_size,
-                       kv_scales=kv_scales, query_dtype=TORCH_DTYPES[cfg.dtype])
-    if inp.prefix is None:
-        for s in range(S):
-            dec.admit(s, int(inp.context_lens[s]))
-    else:
-        p = inp.prefix
-        dec.apply_copies(dec.admit_shared_prefix(p.groups, p.samples, p.prefix_len,
-                                                 p.private_lens))
-    # every step decodes the same lengths: sequences roll back one token per step
-    dec.bind(range(S), rolling=True)
-
-    # a ring of distinct per-step token sets: pinned host copies and device copies
-    ring = 8
-    toks_h, toks_d = [], []
-    for i in range(ring):
-        q, nk, nv = (inp.q, inp.new_k, inp.new_v) if i == 0 else step_tokens(cfg, seed, i)
-        h = [storage_to_torch(a, cfg.dtype).pin_memory() for a in (q, nk, nv)]
-        toks_h.append(h)
-        toks_d.append([t.to(dev) for t in h])
-    out = torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def one_step(tokens, ev=None):
-        q, nk, nv = tokens
-        return dec.step(q, nk, nv, out, events=ev)
-
-    warm_cow = 0
-    for i in range(args.warmup):
-        warm_cow += one_step(toks_d[i % ring])["num_cow"]
-    torch.cuda.synchronize(dev)
-    if pa.pa_device_error_read() != 0:
-        raise RuntimeError("device error word set during warm-up")
-
-    # the workload is stationary from here on: bytes per step computed once
-    meta0 = one_step(toks_d[0])
-    torch.cuda.synchronize(dev)
-    lens = np.array([dec.alloc.seq_len(s) for s in range(S)], np.int64)
-    uniq = unique_context_tokens(dec, cfg, range(S)) if inp.prefix is not None else None
-    dec_bytes = decode_bytes(cfg, lens, uniq, ekv)
-    step_bytes = dec_bytes + cache_op_bytes(cfg, S, 0, ekv)
-    logical_dec_bytes = decode_bytes(cfg, lens, None, ekv)
-    launches_per_step = dec.kernel_launches(meta0)
-
-    # per-call events on a sample of the steps (the decode call's own duration)
-    n_ev = min(args.steps, 200)
-    ev_every = max(1, args.steps // n_ev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(n_ev)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    cows = 0
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
-        t_start.record(stream)
-        e = 0
-        for k in range(args.steps):
-            ev = None
-            if k % ev_every == 0 and e < n_ev:
-                ev, e = evs[e], e + 1
-            cows += one_step(toks_d[k % ring], ev)["num_cow"]
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    dec_ms = [a.elapsed_time(b) for a, b in evs[:e]]
-    err = pa.pa_device_error_read()
-    if err:
-        raise RuntimeError(f"device error word {err} after the timed region")
-    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
-    job_step_bytes = sum_over_ranks(step_bytes, world, dev)
-    value = job_throughput(job_step_bytes, args.steps, elapsed_ms)
-    seqs_per_s = S * world * args.steps / (elapsed_ms * 1e-3)
-
-    # ---- a pool that fits in L2: the decode call also timed cold ---------------------
-    cold_ms = None
-    if pool_bytes <= L2_BYTES and rank == 0:
-        # between calls, write a buffer of twice the L2 size so that nothing of the
-        # pool stays cached (the warm figures above are the steady state)
-        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
-        cevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(50)]
-        for ev in cevs:
-            flush.fill_(1)
-            one_step(toks_d[0], ev)
-        torch.cuda.synchronize(dev)
-        cold_ms = [a.elapsed_time(b) for a, b in cevs]
-        del flush
-
-    # ---- end to end through the public API with host buffers ----------------------
-    e2e = None
-    if not args.no_e2e:
-        # the public host-buffer step: inputs from pinned memory, result back to it,
-        # copies overlapped with the neighbouring steps' kernels
-        outs_h = [torch.empty((S, Hq, D), dtype=TORCH_DTYPES[cfg.dtype], pin_memory=True)
-                  for _ in range(2)]
-        done = [None, None]
-
-        def e2e_step(k):
-            if done[k % 2] is not None:
-                done[k % 2].synchronize()          # the caller consumed that result
-            done[k % 2] = dec.step_host(*toks_h[k % ring], outs_h[k % 2])
-
-        for k in range(3):
-            e2e_step(k)
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for k in range(args.steps):
-            e2e_step(k)
-        dec.drain_host_io()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        E = job_throughput(job_step_bytes, args.steps, e_ms)
-        h2d = sum(t.numel() * t.element_size() for t in toks_h[0]) + dec.staging_bytes
-        d2h = S * Hq * D * cfg.elem_bytes
-        e2e = {"value": round(E, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms / args.steps, 4),
-               "seqs_per_s": round(S * world * args.steps / (e_ms * 1e-3), 1)}
-
-    # ---- roofline of the decode call --------------------------------------------
-    peak, peak_kind = hbm_peak()
-    dec_avg_ms = statistics.mean(dec_ms)
-    achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-            "kernel": ("pa_decode_attention_fp8" if args.cache_fp8 else "pa_decode_attention")
-                      + " (partition kernel + log-sum-exp merge)",
-            "bytes_per_launch": int(dec_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 2),
-            "launches_timed": len(dec_ms),
-            "median_launch_us": round(statistics.median(dec_ms) * 1e3, 2),
-            "frac_of_nominal_8000": round(achieved / 8000.0, 4),
-            "traffic": None if args.cache_fp8 else recorded_traffic(cfg)}  # records: 16-bit caches
-    if cold_ms:
-        roof["cold_median_launch_us"] = round(statistics.median(cold_ms) * 1e3, 2)
-        roof["cold_note"] = "pool smaller than L2: calls after a 2x-L2 buffer write"
-    if uniq is not None:
-        roof["logical_bytes_per_launch"] = int(logical_dec_bytes)
-        roof["logical_achieved"] = round(logical_dec_bytes / (dec_avg_ms * 1e-3) / 1e9, 1)
-
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -528,32 +821,14 @@ def run_ours(args, cfg):
             "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
             "seqs_per_s": round(seqs_per_s, 1),
-            "config": {"workload": cfg.name, "description": cfg.description,
-                       "num_seqs": S, "num_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
-                       "block_size": bs, "num_blocks": cfg.num_blocks,
-                       "partition_size": dec.partition_size,
-                       "partition_rule": ("pa_decode_partition_size" if cfg.partition_size == 0
-                                          else "fixed"),
-                       "mean_seq_len": round(float(lens.mean()), 1),
-                       "max_seq_len": int(lens.max()),
-                       "l2": ("inputs larger than L2 (K/V pool %.2f GB per rank), no flush"
-                              % (pool_bytes / 1e9)) if pool_bytes > L2_BYTES else
-                             ("K/V pool of %.1f KB fits in L2: a parity-size workload, "
-                              "no flush" % (pool_bytes / 1e3)),
-                       "steps": "each step appends one token per sequence and rolls the "
-                                "previous one back, so every step decodes these lengths",
-                       "parallelism": f"replicas x{world}",
-                       "workspace_bytes": int(dec.workspace_bytes),
-                       "prefix_group_chunks": int(meta0.get("num_chunks", 0)),
-                       "pool": pool_summary(dec.alloc.stats()),
-                       "cow_pairs_in_warmup": warm_cow, "cow_pairs_in_timed_steps": cows,
-                       "kv_cache": ("fp8 e4m3, per-tensor scales %g" % kv_scales[0])
-                                   if args.cache_fp8 else cfg.dtype},
+            "config": config,
+            "run_info": run_info,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk.summary(),
+            "gpu_launches": launches,
+            "clocks": clk,
+            "per_workload": per,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -572,13 +847,13 @@ def pool_summary(st: dict) -> dict:
             "tail_waste_pct": round(100.0 * st["tail_waste_slots"] / max(1, st["allocated_slots"]), 3)}
 
 
-def recorded_traffic(cfg):
+def recorded_traffic(cfg, cache_fp8: bool = False):
     """DRAM bytes per decode call from the committed ncu capture of this workload,
     if it was taken on the current kernel sources (else None)."""
     path = os.path.join(HERE, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(cfg.name)
+            rec = json.load(f).get(cfg.name + ("+fp8_cache" if cache_fp8 else ""))
     except (OSError, ValueError):
         return None
     if not rec or rec.get("kernel_sources_sha256") != kernel_sources_sha():
@@ -685,6 +960,9 @@ def main():
         slots = cfg.num_blocks * cfg.block_size
         cfg = cfg.with_(block_size=args.block_size, num_blocks=slots // args.block_size,
                         name=f"{cfg.name}_bs{args.block_size}")
+    args.default_shape = (args.workload in (None, HEADLINE) and args.seqs is None
+                          and args.pool_blocks is None and args.block_size is None
+                          and args.partition_size is None and not args.cache_fp8)
     if args.impl == "reference":
         run_reference(args, cfg)
     elif args.measure == "swap":

@@ -246,6 +246,11 @@ int pa_decode_attention(void* out, const void* q, const void* k_cache, const voi
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make that first
  *     call before any stream capture.
+ *   - With CUDA's default lazy module loading, the array's 16 MiB are reserved on a
+ *     device when the library's device code is first loaded there: at that first
+ *     call at the latest (at context creation under CUDA_MODULE_LOADING=EAGER).  A
+ *     caller that budgets device memory once at start-up should make one call per
+ *     device during its initialisation, so that nothing is reserved later.
  *   - Every call on a device shares the one array.  The scratch needs no clearing (each
  *     call writes every entry it reads), but calls that overlap on the GPU - on
  *     different streams, or from different threads - race on it and must be ordered
@@ -532,14 +537,21 @@ int pa_alloc_stats(const pa_alloc_t* a, pa_stats_t* stats);
  * has not finished.
  *
  * The decoder borrows the allocator (which must outlive it and must not be used
- * from another thread during a call) and the caches; it owns its streams, events and
- * the buffers pa_decoder_bind allocates: the staging sets (pa_decoder_query), the
- * decode workspace for the bound batch at full table capacity, and, for host-fed
- * steps, two device sets of q / new K / new V / out.  Nothing is allocated inside a
- * step except the first host-fed step after a bind to a new batch size.  Not
- * thread-safe.  Every call makes the decoder's device (current at create) current
- * for its duration.  A step that fails after step 2 leaves the sequences one token
- * longer.
+ * from another thread during a call) and the caches.  It owns its streams, events and
+ * the page-locked host halves of the staging sets.  It allocates no device memory:
+ * the caller passes one device buffer to pa_decoder_bind (its size from
+ * pa_decoder_device_bytes), which holds the device halves of the two staging sets,
+ * the decode workspace for the bound batch at full table capacity and the two device
+ * sets of q / new K / new V / out for host-fed steps.  That buffer must stay
+ * allocated, and be used by nothing else, until the decoder is destroyed or bound
+ * again (both wait for the decoder's work in flight first).  Nothing is allocated
+ * inside a step.  Not thread-safe.  Every call makes the decoder's device (current at
+ * create) current for its duration.
+ * Failures: every check that can refuse a step (a sequence at the table's capacity,
+ * an unknown sequence, the pool out of blocks) runs before the block manager commits
+ * the step, and leaves the state unchanged.  A CUDA call that fails after that commit
+ * leaves the sequences one token longer than the device cache; the decoder then
+ * refuses every further step with PA_ERR_CUDA until it is bound again.
  */
 typedef struct pa_decoder pa_decoder_t;
 
@@ -587,10 +599,18 @@ int pa_decoder_create(const pa_decoder_config_t* cfg, pa_alloc_t* alloc,
                       pa_decoder_t** out);
 /* Waits for the decoder's work in flight, then frees everything it owns. */
 int pa_decoder_destroy(pa_decoder_t* d);
+/* Device bytes pa_decoder_bind needs for a batch of num_seqs sequences (staging sets,
+ * workspace and host-I/O sets, each piece 256-byte aligned).  Host only, except that
+ * the automatic partition size reads the device's SM count. */
+int pa_decoder_device_bytes(const pa_decoder_t* d, int num_seqs, size_t* bytes);
 /* Fix the batch (distinct ids present in the allocator, each shorter than the table
- * capacity) and allocate its buffers; rolling != 0 makes every step first roll the
- * sequences back to their current lengths.  Waits for the decoder's work in flight. */
-int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int rolling);
+ * capacity) and lay its buffers out in the caller's device_buffer (256-byte aligned,
+ * at least pa_decoder_device_bytes(num_seqs) bytes: else PA_ERR_INVALID_ARG and
+ * nothing changes); rolling != 0 makes every step first roll the sequences back to
+ * their current lengths.  Waits for the decoder's work in flight, then drops the
+ * previous batch's buffers. */
+int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int rolling,
+                    void* device_buffer, size_t device_bytes);
 /* One step with DEVICE inputs: q [S, num_heads, head_dim], new_k / new_v
  * [S, num_kv_heads, head_dim] (row i is seq_ids[i]'s new token), out [S, num_heads,
  * head_dim], all dtype.  ev_begin / ev_end (cudaEvent_t or NULL) are recorded on the

@@ -128,7 +128,8 @@ _sig("pa_alloc_stats", _i32, _p, ctypes.POINTER(pa_stats_t))
 _sig("pa_decode", _i32, ctypes.POINTER(pa_decode_args_t))
 _sig("pa_decoder_create", _i32, ctypes.POINTER(pa_decoder_config_t), _p, ctypes.POINTER(_p))
 _sig("pa_decoder_destroy", _i32, _p)
-_sig("pa_decoder_bind", _i32, _p, _p, _i32, _i32)
+_sig("pa_decoder_bind", _i32, _p, _p, _i32, _i32, _p, ctypes.c_size_t)
+_sig("pa_decoder_device_bytes", _i32, _p, _i32, ctypes.POINTER(ctypes.c_size_t))
 _sig("pa_decoder_step", _i32, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.POINTER(pa_step_info_t))
 _sig("pa_decoder_step_host", _i32, _p, _p, _p, _p, _p, _p, _I64P,
      ctypes.POINTER(pa_step_info_t))

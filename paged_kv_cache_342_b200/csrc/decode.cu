@@ -8,6 +8,7 @@
 // pages in order" and "Measure memory use across requests" (the attention equation
 // is unchanged by paging).
 #include <cmath>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -240,8 +241,11 @@ bool group_eligible(int dtype, int group, int head_dim, int block_size, int max_
 
 // A side stream per device for the group kernel, so that it runs beside the
 // per-sequence kernel (they write disjoint partitions); fork and join through events.
+// Created on first use under the mutex; `ready` is published only once the stream
+// and both events exist, and a failed creation destroys what it made.
 struct SideStream {
   std::mutex mu;
+  std::atomic<bool> ready{false};
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
 };
@@ -250,11 +254,25 @@ SideStream g_side[64];
 cudaError_t side_stream(int dev, SideStream** out) {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   SideStream& s = g_side[dev];
-  if (!s.stream) {
-    cudaError_t e = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
-    if (e != cudaSuccess) return e;
+  if (!s.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(s.mu);
+    if (!s.ready.load(std::memory_order_relaxed)) {
+      cudaStream_t stream = nullptr;
+      cudaEvent_t fork = nullptr, join = nullptr;
+      cudaError_t e = cudaStreamCreateWithFlags(&stream, cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+      if (e != cudaSuccess) {
+        if (join) cudaEventDestroy(join);
+        if (fork) cudaEventDestroy(fork);
+        if (stream) cudaStreamDestroy(stream);
+        return e;
+      }
+      s.stream = stream;
+      s.fork = fork;
+      s.join = join;
+      s.ready.store(true, std::memory_order_release);
+    }
   }
   *out = &s;
   return cudaSuccess;

@@ -6,13 +6,16 @@
 // from the block manager (a copy first where its block is shared), the token's K/V
 // written into its slot, then attention over every cached token.
 //
-// Buffers of a bound batch (allocated by pa_decoder_bind, never inside a step):
-//   - two staging sets, each one page-locked host buffer and one device buffer of
-//     the same layout (slots, copy pairs, lengths, block tables, prefix groups);
-//     step k fills set k % 2 while the kernels of step k - 1 still read the other,
-//     and one cudaMemcpyAsync on the decoder's copy stream moves the whole set;
+// Buffers of a bound batch (laid out by pa_decoder_bind, never inside a step):
+//   - two staging sets, each one page-locked host buffer (the decoder's own) and one
+//     device buffer of the same layout (slots, copy pairs, lengths, block tables,
+//     prefix groups); step k fills set k % 2 while the kernels of step k - 1 still
+//     read the other, and one cudaMemcpyAsync on the decoder's copy stream moves the
+//     whole set;
 //   - the decode workspace for the bound batch at full table capacity;
 //   - for steps fed from host memory, two device sets of q / new K / new V / out.
+// All device memory comes from one caller-owned buffer (pa_decoder_device_bytes
+// gives its size); the library allocates no device memory.
 // Events order everything across the caller's stream and the decoder's streams;
 // host waits happen only where a host buffer is about to be rewritten.
 #include <cuda_runtime.h>
@@ -88,6 +91,9 @@ struct pa_decoder {
   std::vector<int64_t> ids, base_lens;
   int num_seqs = 0, members = 0, partition = 0;
   bool bound = false, rolling = false, stepped = false;
+  // a CUDA call failed after the block manager had committed a step: the allocator
+  // is ahead of the device cache, so every later step is refused
+  bool broken = false;
   size_t off_slots = 0, off_pairs = 0, off_lens = 0, off_tables = 0, off_pparts = 0,
          off_cmembers = 0, off_cparts = 0, off_order = 0, stage_bytes = 0;
   StageSet sets[2];
@@ -97,7 +103,8 @@ struct pa_decoder {
 
   // host-fed steps
   IoSet io[2];
-  int io_next = 0, io_seqs = -1;
+  int io_next = 0;
+  bool io_fresh = true;  // the I/O sets' events are recorded at the first host-fed step
   int64_t tickets = 0;
   size_t q_bytes = 0, kv_bytes = 0;
 
@@ -129,26 +136,80 @@ cudaError_t quiesce(pa_decoder* d) {
   return e;
 }
 
+// Drops the bound batch's buffers: frees the page-locked staging halves (the
+// decoder's own) and forgets the caller's device buffer.
 void free_stage(pa_decoder* d) {
   for (StageSet& s : d->sets) {
     if (s.host) cudaFreeHost(s.host);
-    if (s.dev) cudaFree(s.dev);
     s.host = nullptr;
     s.dev = nullptr;
     s.h2d_pending = s.kernels_pending = false;
   }
-  if (d->ws) cudaFree(d->ws);
   d->ws = nullptr;
   d->ws_bytes = 0;
+  for (IoSet& s : d->io) s.q = s.k = s.v = s.out = nullptr;
+  d->io_fresh = true;
 }
 
-void free_io(pa_decoder* d) {
-  for (IoSet& s : d->io) {
-    for (void* p : {s.q, s.k, s.v, s.out})
-      if (p) cudaFree(p);
-    s.q = s.k = s.v = s.out = nullptr;
+// Byte layout of a bound batch.  Staging offsets are the same in the host and the
+// device halves; device offsets are into the caller's buffer.  Every piece starts on
+// a 256-byte boundary.
+struct BatchLayout {
+  size_t off_slots, off_pairs, off_lens, off_tables, off_pparts, off_cmembers, off_cparts,
+      off_order, stage_bytes;
+  int partition;
+  size_t ws_bytes, q_bytes, kv_bytes;
+  size_t dev_stage[2], dev_ws, dev_io[2][4], device_bytes;
+};
+
+int plan_batch(const pa_decoder* d, int num_seqs, BatchLayout* L) {
+  const pa_decoder_config_t& c = d->cfg;
+  const int64_t cap = static_cast<int64_t>(c.max_blocks_per_seq) * c.block_size;
+  int partition = c.partition_size;
+  if (partition == 0) {
+    partition = pa_decode_partition_size(c.cache_dtype, num_seqs, c.num_heads, c.num_kv_heads,
+                                         c.head_dim, c.block_size, static_cast<int>(cap), 0);
+    if (partition <= 0) return PA_ERR_CUDA;
   }
-  d->io_seqs = -1;
+  L->partition = partition;
+  L->ws_bytes = pa_decode_workspace_bytes(num_seqs, c.num_heads, c.head_dim,
+                                          static_cast<int>(cap), partition);
+  const size_t S = static_cast<size_t>(num_seqs);
+  const size_t MM = static_cast<size_t>(std::max(1, d->members));
+  size_t off = 0;
+  auto take = [&off](size_t n) {
+    const size_t at = off;
+    off += align256(n);
+    return at;
+  };
+  L->off_slots = take(8 * S);
+  L->off_pairs = take(8 * S);
+  L->off_lens = take(4 * S);
+  L->off_tables = take(4 * S * static_cast<size_t>(c.max_blocks_per_seq));
+  L->off_pparts = take(4 * S);
+  L->off_cmembers = take(4 * S * MM);
+  L->off_cparts = take(4 * S);
+  L->off_order = take(4 * S);
+  L->stage_bytes = off;
+  L->q_bytes = S * c.num_heads * c.head_dim * elem_size(c.dtype);
+  L->kv_bytes = S * c.num_kv_heads * c.head_dim * elem_size(c.dtype);
+  size_t dev = 0;
+  auto place = [&dev](size_t n) {
+    const size_t at = dev;
+    dev += align256(n);
+    return at;
+  };
+  L->dev_stage[0] = place(L->stage_bytes);
+  L->dev_stage[1] = place(L->stage_bytes);
+  L->dev_ws = place(L->ws_bytes);
+  for (auto& io : L->dev_io) {
+    io[0] = place(L->q_bytes);   // q
+    io[1] = place(L->kv_bytes);  // new K
+    io[2] = place(L->kv_bytes);  // new V
+    io[3] = place(L->q_bytes);   // out
+  }
+  L->device_bytes = dev;
+  return PA_OK;
 }
 
 cudaError_t make_event(cudaEvent_t* ev) {
@@ -189,12 +250,28 @@ int prepare(pa_decoder* d, cudaStream_t comp, pa_step_info_t* info) {
   int32_t* pairs = d->h<int32_t>(st, d->off_pairs);
   int32_t* tables = d->h<int32_t>(st, d->off_tables);
   int32_t* lens = d->h<int32_t>(st, d->off_lens);
+  // Everything that can refuse the step is checked before the block manager commits
+  // it: a sequence already at the table's capacity (rolling batches stay at their
+  // bind-time lengths, which bind checked).  After the append only CUDA calls can
+  // fail, and such a failure marks the decoder broken.
+  if (!d->rolling) {
+    const int64_t cap = static_cast<int64_t>(c.max_blocks_per_seq) * c.block_size;
+    for (int s = 0; s < S; ++s) {
+      int64_t len = 0;
+      rc = pa_seq_len(d->alloc, d->ids[static_cast<size_t>(s)], &len);
+      if (rc != PA_OK) return rc;
+      if (len >= cap) return PA_ERR_INVALID_ARG;
+    }
+  }
   rc = pa_seq_append_slots(d->alloc, d->ids.data(), S, slots, pairs, &ncow);
   if (rc != PA_OK) return rc;
   d->cur = i;
   d->stepped = true;
   rc = pa_build_block_tables(d->alloc, d->ids.data(), S, tables, c.max_blocks_per_seq, lens);
-  if (rc != PA_OK) return rc;
+  if (rc != PA_OK) {  // excluded by the checks above
+    d->broken = true;
+    return rc;
+  }
   int max_len = 0;
   for (int s = 0; s < S; ++s) max_len = std::max(max_len, lens[s]);
   // the partition grid takes the sequences longest first (ties in batch order)
@@ -209,7 +286,10 @@ int prepare(pa_decoder* d, cudaStream_t comp, pa_step_info_t* info) {
                                 d->h<int32_t>(st, d->off_cmembers),
                                 d->h<int32_t>(st, d->off_cparts), &num_chunks,
                                 &max_chunk_parts);
-    if (rc != PA_OK) return rc;
+    if (rc != PA_OK) {  // excluded by the checks above
+      d->broken = true;
+      return rc;
+    }
     if (num_chunks > 0) {
       // the lowest partition any sequence computes itself
       first_part = INT32_MAX;
@@ -226,7 +306,10 @@ int prepare(pa_decoder* d, cudaStream_t comp, pa_step_info_t* info) {
   if (e == cudaSuccess) e = cudaEventRecord(st.h2d_done, d->copy_stream);
   if (e == cudaSuccess) st.h2d_pending = true;
   if (e == cudaSuccess) e = cudaStreamWaitEvent(comp, st.h2d_done, 0);
-  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (e != cudaSuccess) {
+    d->broken = true;
+    return PA_ERR_CUDA;
+  }
 
   const bool grouped = num_chunks > 0;
   info->num_cow = ncow;
@@ -370,7 +453,6 @@ int pa_decoder_destroy(pa_decoder_t* d) {
   DeviceGuard g(d->device);
   quiesce(d);
   free_stage(d);
-  free_io(d);
   for (StageSet& s : d->sets)
     for (cudaEvent_t ev : {s.h2d_done, s.kernels_done})
       if (ev) cudaEventDestroy(ev);
@@ -383,9 +465,23 @@ int pa_decoder_destroy(pa_decoder_t* d) {
   return PA_OK;
 }
 
-int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int rolling) {
-  if (!d || num_seqs <= 0 || !seq_ids || num_seqs > 65535) return PA_ERR_INVALID_ARG;
+int pa_decoder_device_bytes(const pa_decoder_t* d, int num_seqs, size_t* bytes) {
+  if (!d || num_seqs <= 0 || num_seqs > 65535 || !bytes) return PA_ERR_INVALID_ARG;
   DeviceGuard g(d->device);  // the partition choice asks the decoder's device
+  if (!g.ok()) return PA_ERR_CUDA;
+  BatchLayout L{};
+  const int rc = plan_batch(d, num_seqs, &L);
+  if (rc != PA_OK) return rc;
+  *bytes = L.device_bytes;
+  return PA_OK;
+}
+
+int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int rolling,
+                    void* device_buffer, size_t device_bytes) {
+  if (!d || num_seqs <= 0 || !seq_ids || num_seqs > 65535) return PA_ERR_INVALID_ARG;
+  if (!device_buffer || (reinterpret_cast<uintptr_t>(device_buffer) & 255u))
+    return PA_ERR_INVALID_ARG;
+  DeviceGuard g(d->device);
   if (!g.ok()) return PA_ERR_CUDA;
   const pa_decoder_config_t& c = d->cfg;
   std::vector<int64_t> ids(seq_ids, seq_ids + num_seqs), lens(static_cast<size_t>(num_seqs));
@@ -398,53 +494,55 @@ int pa_decoder_bind(pa_decoder_t* d, const int64_t* seq_ids, int num_seqs, int r
     if (rc != PA_OK) return rc;
     if (lens[s] >= cap) return PA_ERR_INVALID_ARG;  // no room for the step's token
   }
-  int partition = c.partition_size;
-  if (partition == 0) {
-    partition = pa_decode_partition_size(c.cache_dtype, num_seqs, c.num_heads, c.num_kv_heads,
-                                         c.head_dim, c.block_size, static_cast<int>(cap), 0);
-    if (partition <= 0) return PA_ERR_CUDA;
-  }
-  const size_t ws_need = pa_decode_workspace_bytes(num_seqs, c.num_heads, c.head_dim,
-                                                   static_cast<int>(cap), partition);
+  BatchLayout L{};
+  int rc = plan_batch(d, num_seqs, &L);
+  if (rc != PA_OK) return rc;
+  if (device_bytes < L.device_bytes) return PA_ERR_INVALID_ARG;
   if (quiesce(d) != cudaSuccess) return PA_ERR_CUDA;
   free_stage(d);
   d->bound = false;
 
-  const size_t S = static_cast<size_t>(num_seqs);
-  const size_t MM = static_cast<size_t>(std::max(1, d->members));
-  size_t off = 0;
-  auto take = [&off](size_t n) {
-    const size_t at = off;
-    off += align256(n);
-    return at;
-  };
-  d->off_slots = take(8 * S);
-  d->off_pairs = take(8 * S);
-  d->off_lens = take(4 * S);
-  d->off_tables = take(4 * S * static_cast<size_t>(c.max_blocks_per_seq));
-  d->off_pparts = take(4 * S);
-  d->off_cmembers = take(4 * S * MM);
-  d->off_cparts = take(4 * S);
-  d->off_order = take(4 * S);
-  d->stage_bytes = off;
+  d->off_slots = L.off_slots;
+  d->off_pairs = L.off_pairs;
+  d->off_lens = L.off_lens;
+  d->off_tables = L.off_tables;
+  d->off_pparts = L.off_pparts;
+  d->off_cmembers = L.off_cmembers;
+  d->off_cparts = L.off_cparts;
+  d->off_order = L.off_order;
+  d->stage_bytes = L.stage_bytes;
+  uint8_t* base = static_cast<uint8_t*>(device_buffer);
   cudaError_t e = cudaSuccess;
-  for (StageSet& s : d->sets) {
-    if (e == cudaSuccess) e = cudaHostAlloc(reinterpret_cast<void**>(&s.host), off, cudaHostAllocDefault);
-    if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&s.dev), off);
-    if (e == cudaSuccess) std::memset(s.host, 0, off);
+  for (int i = 0; i < 2; ++i) {
+    StageSet& st = d->sets[i];
+    st.dev = base + L.dev_stage[i];
+    if (e == cudaSuccess)
+      e = cudaHostAlloc(reinterpret_cast<void**>(&st.host), L.stage_bytes, cudaHostAllocDefault);
+    if (e == cudaSuccess) std::memset(st.host, 0, L.stage_bytes);
   }
-  if (e == cudaSuccess && ws_need > 0) e = cudaMalloc(&d->ws, ws_need);
   if (e != cudaSuccess) {
     free_stage(d);
     return PA_ERR_CUDA;
   }
-  d->ws_bytes = ws_need;
+  d->ws = L.ws_bytes ? base + L.dev_ws : nullptr;
+  d->ws_bytes = L.ws_bytes;
+  for (int i = 0; i < 2; ++i) {
+    IoSet& io = d->io[i];
+    io.q = base + L.dev_io[i][0];
+    io.k = base + L.dev_io[i][1];
+    io.v = base + L.dev_io[i][2];
+    io.out = base + L.dev_io[i][3];
+  }
+  d->q_bytes = L.q_bytes;
+  d->kv_bytes = L.kv_bytes;
+  d->io_fresh = true;
   d->ids = std::move(ids);
   d->base_lens = std::move(lens);
   d->num_seqs = num_seqs;
-  d->partition = partition;
+  d->partition = L.partition;
   d->rolling = rolling != 0;
   d->stepped = false;
+  d->broken = false;
   d->cur = 0;
   d->bound = true;
   return PA_OK;
@@ -455,6 +553,7 @@ int pa_decoder_step(pa_decoder_t* d, const void* q, const void* new_k, const voi
                     pa_step_info_t* info) {
   if (!d || !d->bound || !q || !new_k || !new_v || !out) return PA_ERR_INVALID_ARG;
   if (info && info->struct_size != sizeof(pa_step_info_t)) return PA_ERR_INVALID_ARG;
+  if (d->broken) return PA_ERR_CUDA;
   DeviceGuard g(d->device);
   if (!g.ok()) return PA_ERR_CUDA;
   pa_step_info_t local{};
@@ -462,38 +561,27 @@ int pa_decoder_step(pa_decoder_t* d, const void* q, const void* new_k, const voi
   cudaStream_t comp = static_cast<cudaStream_t>(stream);
   int rc = prepare(d, comp, inf);
   if (rc != PA_OK) return rc;
-  return launch(d, inf, q, new_k, new_v, out, comp, static_cast<cudaEvent_t>(ev_begin),
-                static_cast<cudaEvent_t>(ev_end));
+  rc = launch(d, inf, q, new_k, new_v, out, comp, static_cast<cudaEvent_t>(ev_begin),
+              static_cast<cudaEvent_t>(ev_end));
+  if (rc != PA_OK) d->broken = true;
+  return rc;
 }
 
 int pa_decoder_step_host(pa_decoder_t* d, const void* q, const void* new_k, const void* new_v,
                          void* out, pa_stream_t stream, int64_t* ticket, pa_step_info_t* info) {
   if (!d || !d->bound || !q || !new_k || !new_v || !out) return PA_ERR_INVALID_ARG;
   if (info && info->struct_size != sizeof(pa_step_info_t)) return PA_ERR_INVALID_ARG;
+  if (d->broken) return PA_ERR_CUDA;
   DeviceGuard g(d->device);
   if (!g.ok()) return PA_ERR_CUDA;
-  const pa_decoder_config_t& c = d->cfg;
   cudaStream_t comp = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
-  if (d->io_seqs != d->num_seqs) {  // (re)size the device I/O sets for the bound batch
-    if (quiesce(d) != cudaSuccess) return PA_ERR_CUDA;
-    free_io(d);
-    const size_t S = static_cast<size_t>(d->num_seqs);
-    d->q_bytes = S * c.num_heads * c.head_dim * elem_size(c.dtype);
-    d->kv_bytes = S * c.num_kv_heads * c.head_dim * elem_size(c.dtype);
-    for (IoSet& s : d->io) {
-      for (auto pb : {std::make_pair(&s.q, d->q_bytes), std::make_pair(&s.k, d->kv_bytes),
-                      std::make_pair(&s.v, d->kv_bytes), std::make_pair(&s.out, d->q_bytes)})
-        if (e == cudaSuccess) e = cudaMalloc(pb.first, pb.second);
-      // events start out completed
+  if (d->io_fresh) {  // events start out completed
+    for (IoSet& s : d->io)
       for (cudaEvent_t ev : {s.h2d_done, s.compute_done, s.d2h_done})
         if (e == cudaSuccess) e = cudaEventRecord(ev, comp);
-    }
-    if (e != cudaSuccess) {
-      free_io(d);
-      return PA_ERR_CUDA;
-    }
-    d->io_seqs = d->num_seqs;
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    d->io_fresh = false;
     d->io_next = 0;
   }
   IoSet& io = d->io[d->io_next];
@@ -511,14 +599,20 @@ int pa_decoder_step_host(pa_decoder_t* d, const void* q, const void* new_k, cons
   pa_step_info_t local{};
   pa_step_info_t* inf = info ? info : &local;
   int rc = prepare(d, comp, inf);
-  if (rc == PA_OK) rc = launch(d, inf, io.q, io.k, io.v, io.out, comp, nullptr, nullptr);
   if (rc != PA_OK) return rc;
-  e = cudaEventRecord(io.compute_done, comp);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(d->d2h_stream, io.compute_done, 0);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(out, io.out, d->q_bytes, cudaMemcpyDeviceToHost, d->d2h_stream);
-  if (e == cudaSuccess) e = cudaEventRecord(io.d2h_done, d->d2h_stream);
-  if (e != cudaSuccess) return PA_ERR_CUDA;
+  rc = launch(d, inf, io.q, io.k, io.v, io.out, comp, nullptr, nullptr);
+  if (rc == PA_OK) {
+    e = cudaEventRecord(io.compute_done, comp);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(d->d2h_stream, io.compute_done, 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(out, io.out, d->q_bytes, cudaMemcpyDeviceToHost, d->d2h_stream);
+    if (e == cudaSuccess) e = cudaEventRecord(io.d2h_done, d->d2h_stream);
+    if (e != cudaSuccess) rc = PA_ERR_CUDA;
+  }
+  if (rc != PA_OK) {
+    d->broken = true;
+    return rc;
+  }
   d->io_next ^= 1;
   io.ticket = ++d->tickets;
   if (ticket) *ticket = io.ticket;
@@ -538,7 +632,7 @@ int pa_decoder_wait(pa_decoder_t* d, int64_t ticket) {
 
 int pa_decoder_drain(pa_decoder_t* d, pa_stream_t stream) {
   if (!d) return PA_ERR_INVALID_ARG;
-  if (d->io_seqs < 0) return PA_OK;
+  if (!d->bound || d->io_fresh) return PA_OK;
   DeviceGuard g(d->device);
   cudaStream_t comp = static_cast<cudaStream_t>(stream);
   for (IoSet& s : d->io)

@@ -132,6 +132,7 @@ class PagedDecoder:
             self.group_members = 0
         self.workspace_bytes = self.staging_bytes = 0
         self._S = 0
+        self._device_buffer = None
         cfg = pa_decoder_config_t()
         cfg.struct_size = ctypes.sizeof(pa_decoder_config_t)
         cfg.k_cache, cfg.v_cache = k_cache.data_ptr(), v_cache.data_ptr()
@@ -155,10 +156,11 @@ class PagedDecoder:
         h = getattr(self, "_h", None)
         if h is not None and h.value:
             try:
-                lib.pa_decoder_destroy(h)
+                lib.pa_decoder_destroy(h)   # waits for the work that uses the buffer
             except Exception:  # interpreter shutdown: the library may be gone already
                 pass
             self._h = None
+        self._device_buffer = None
 
     # -- context building ------------------------------------------------------
     def admit(self, seq_id: int, num_tokens: int) -> None:
@@ -191,10 +193,20 @@ class PagedDecoder:
 
     # -- the step ---------------------------------------------------------------
     def bind(self, seq_ids, rolling: bool = False) -> None:
-        """Fix the batch the steps run over; the library allocates its buffers."""
+        """Fix the batch the steps run over.  Its device buffers (staging, workspace,
+        host-I/O sets) are one torch allocation of the size the library asks for,
+        held until the next bind or the decoder's end."""
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
-        _check(lib.pa_decoder_bind(self._h, ids.ctypes.data, ids.size, int(rolling)),
-               "pa_decoder_bind")
+        need = ctypes.c_size_t(0)
+        with torch.cuda.device(self.device):
+            _check(lib.pa_decoder_device_bytes(self._h, ids.size, ctypes.byref(need)),
+                   "pa_decoder_device_bytes")
+            buf = torch.empty(need.value, dtype=torch.uint8, device=self.device)
+        # the library waits for the previous batch's work before it lets go of the old
+        # buffer, so that one is released only after the call
+        _check(lib.pa_decoder_bind(self._h, ids.ctypes.data, ids.size, int(rolling),
+                                   buf.data_ptr(), need.value), "pa_decoder_bind")
+        self._device_buffer = buf
         self._S = ids.size
         ps, ws, st = ctypes.c_int(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
         _check(lib.pa_decoder_query(self._h, ctypes.byref(ps), ctypes.byref(ws), ctypes.byref(st)),

@@ -126,7 +126,9 @@ def test_decoder_config_checks(pa):
         assert create(_decoder_config(pa, cache_dtype=pa.PA_FP8_E4M3)) == pa.PA_ERR_CUDA
         assert not h.value
     info = pa.pa_step_info_t()
-    assert pa.lib.pa_decoder_bind(None, None, 0, 0) == pa.PA_ERR_INVALID_ARG
+    assert pa.lib.pa_decoder_bind(None, None, 0, 0, None, 0) == pa.PA_ERR_INVALID_ARG
+    nbytes = ctypes.c_size_t(0)
+    assert pa.lib.pa_decoder_device_bytes(None, 4, ctypes.byref(nbytes)) == pa.PA_ERR_INVALID_ARG
     assert pa.lib.pa_decoder_step(None, 0, 0, 0, 0, None, None, None,
                                   ctypes.byref(info)) == pa.PA_ERR_INVALID_ARG
     assert pa.lib.pa_decoder_wait(None, 1) == pa.PA_ERR_INVALID_ARG

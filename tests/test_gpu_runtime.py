@@ -95,3 +95,50 @@ def test_rolling_and_growing_steps_rebind_and_partition_choice():
     assert meta.kernels == 2 + (1 if -(-meta.max_len // dec.partition_size) > 1 else 0)
     with pytest.raises(ValueError):                      # tensors must fit the batch
         dec.step(q[:2], q[:2, :Hkv], q[:2, :Hkv], out[:2])
+
+
+def test_caller_buffer_and_capacity_refusal_leave_state_unchanged():
+    """The decoder takes its device memory from the caller: a bind with a buffer that
+    is too small (or misaligned) is refused and changes nothing.  A growing batch whose
+    sequence reaches the table's capacity is refused before the block manager commits
+    the step: lengths, tables and the pool stay as they were, and a rebind with more
+    room lets the batch go on."""
+    import ctypes
+
+    import paged_kv_cache_342_b200 as pa
+    import paged_kv_cache_342_b200.runtime as rt
+    S, Hq, Hkv, D, bs, NB, MB = 2, 8, 8, 128, 16, 64, 4        # capacity 64 tokens
+    kd = to_dev(normal_fill((NB, Hkv, bs, D), "bf16", 1.0, 4, 1), "bf16")
+    vd = to_dev(normal_fill((NB, Hkv, bs, D), "bf16", 1.0, 4, 2), "bf16")
+    dec = rt.PagedDecoder(kd, vd, Hq, 1 / math.sqrt(D), MB, None, 32)
+    dec.admit(0, 61)
+    dec.admit(1, 10)
+    need = ctypes.c_size_t(0)
+    assert pa.lib.pa_decoder_device_bytes(dec._h, S, ctypes.byref(need)) == pa.PA_OK
+    small = torch.empty(need.value - 256, dtype=torch.uint8, device="cuda")
+    ids = np.arange(S, dtype=np.int64)
+    assert pa.lib.pa_decoder_bind(dec._h, ids.ctypes.data, S, 0, small.data_ptr(),
+                                  small.numel()) == pa.PA_ERR_INVALID_ARG
+    big = torch.empty(need.value + 512, dtype=torch.uint8, device="cuda")
+    assert pa.lib.pa_decoder_bind(dec._h, ids.ctypes.data, S, 0, big.data_ptr() + 16,
+                                  need.value) == pa.PA_ERR_INVALID_ARG
+    dec.bind(range(S), rolling=False)
+    q = torch.randn(S, Hq, D, device="cuda").bfloat16()
+    kv = torch.randn(S, Hkv, D, device="cuda").bfloat16()
+    out = torch.empty_like(q)
+    for _ in range(3):                                   # 61 -> 64 tokens: at capacity
+        dec.step(q, kv, kv, out)
+    torch.cuda.synchronize()
+    before = (dec.alloc.stats(), dec.alloc.free_list(), dec.alloc.seq_blocks(0),
+              dec.alloc.seq_len(0), dec.alloc.seq_len(1))
+    assert before[3] == 64
+    with pytest.raises(pa.PagedAttentionError) as e:
+        dec.step(q, kv, kv, out)
+    assert e.value.code == "INVALID_ARG"
+    after = (dec.alloc.stats(), dec.alloc.free_list(), dec.alloc.seq_blocks(0),
+             dec.alloc.seq_len(0), dec.alloc.seq_len(1))
+    assert after == before
+    dec.bind([1], rolling=False)                         # the other sequence goes on
+    meta = dec.step(q[:1], kv[:1], kv[:1], out[:1])
+    torch.cuda.synchronize()
+    assert int(meta.lens[0]) == 14 and pa.pa_device_error_read() == 0

@@ -5,9 +5,10 @@ Some callers may not allocate device memory at all - a host program that owns an
 budgets every byte of the GPU, a plug-in inside another process, a loop that cannot
 pay for cudaMalloc.  For them the library keeps its own fixed scratch array.  These
 tests call that entry point through the C ABI and check that it gives the same
-result as pa_decode_attention with a caller workspace, on two calls in a row (the
-array keeps the previous call's contents), for the CUDA-core and the tensor-core
-kernels, and that an oversized request is refused without touching anything.
+result as pa_decode_attention with a caller workspace, bit for bit, on two calls in
+a row (the array keeps the previous call's contents), for the CUDA-core and the
+tensor-core kernels; that a smaller call after a larger one reads none of the stale
+scratch; and that an oversized request is refused without touching anything.
 
 This file is collected last on purpose: a failure here leaves every other test run.
 """
@@ -17,7 +18,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import ATOL, TORCH_DT, out_f64, tables_from_order, to_dev
+from gpu_util import TORCH_DT, out_f64, tables_from_order, to_dev
 from workloads import normal_fill
 
 pytestmark = pytest.mark.gpu
@@ -58,9 +59,57 @@ def test_static_workspace_matches_caller_workspace(pa, dtype, Hq, Hkv, D, bs, ps
         pa.pa_decode_attention_static_ws(got, q, k, v, tables, seq_lens, scale, bs, Hkv,
                                          max_len, ps)
         torch.cuda.synchronize()
-        g, r = out_f64(got), out_f64(ref)
-        assert np.isfinite(g).all()
-        assert np.abs(g - r).max() <= ATOL[dtype], f"call {call}"
+        assert torch.isfinite(got.float()).all()
+        # the same kernels on the same inputs with the same scratch layout: bit for bit
+        assert torch.equal(got, ref), f"call {call}"
+    assert pa.pa_device_error_read() == 0
+
+
+def _case(dtype, Hq, Hkv, D, bs, lens, seed):
+    lens = np.asarray(lens, np.int64)
+    NB = int(sum(-(-int(L) // bs) for L in lens)) + 3
+    k_h = normal_fill((NB, Hkv, bs, D), dtype, 1.0, seed, 1)
+    v_h = normal_fill((NB, Hkv, bs, D), dtype, 1.0, seed, 2)
+    q_h = normal_fill((lens.size, Hq, D), dtype, 1.0, seed, 3)
+    order = np.random.default_rng(seed).permutation(NB).astype(np.int32)
+    width = -(-int(lens.max()) // bs) + 1
+    tables = tables_from_order(lens, bs, order, width)
+    return lens, k_h, v_h, q_h, tables
+
+
+def test_stale_scratch_of_a_larger_call_does_not_leak(pa):
+    """A first call with many partitions fills much of the shared array; a second,
+    smaller call of another shape must not read any of it: its output equals the
+    caller-workspace call bit for bit and the float64 oracle within tolerance."""
+    import oracle.attention as oatt
+    from gpu_util import assert_close
+    dtype, D, bs = "bf16", 128, 16
+    calls = [
+        # 12 x 16 heads x 63 partitions of 32 tokens: about 6.5 MB of partials
+        dict(Hq=16, Hkv=16, lens=[2000, 1999, 1500, 1024, 777, 2016, 1800, 640, 1300,
+                                  2001, 999, 1234], ps=32, seed=31),
+        # 5 sequences x 8 heads (tensor cores, group 8), 512-token partitions
+        dict(Hq=8, Hkv=1, lens=[3000, 1, 513, 1024, 2047], ps=512, seed=32),
+    ]
+    for i, c in enumerate(calls):
+        lens, k_h, v_h, q_h, tables = _case(dtype, c["Hq"], c["Hkv"], D, bs, c["lens"],
+                                            c["seed"])
+        S, Hq, Hkv = lens.size, c["Hq"], c["Hkv"]
+        k, v, q = to_dev(k_h, dtype), to_dev(v_h, dtype), to_dev(q_h, dtype)
+        t = torch.from_numpy(tables).cuda()
+        sl = torch.from_numpy(lens.astype(np.int32)).cuda()
+        max_len, scale = int(lens.max()), 1.0 / math.sqrt(D)
+        wsb = pa.pa_decode_workspace_bytes(S, Hq, D, max_len, c["ps"])
+        assert 0 < wsb <= pa.PA_STATIC_WORKSPACE_BYTES
+        ref = torch.empty((S, Hq, D), dtype=TORCH_DT[dtype], device="cuda")
+        ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        pa.pa_decode_attention(ref, q, k, v, t, sl, scale, bs, Hkv, max_len, c["ps"], ws)
+        got = torch.full_like(ref, float("nan"))
+        pa.pa_decode_attention_static_ws(got, q, k, v, t, sl, scale, bs, Hkv, max_len, c["ps"])
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref), f"call {i}"
+        want = oatt.paged_decode_attention(q_h, k_h, v_h, tables, lens, scale, bs, Hkv, dtype)
+        assert_close(out_f64(got), want, dtype, f"call {i}")
     assert pa.pa_device_error_read() == 0
 
 

@@ -245,6 +245,28 @@ def make_inputs(cfg: DecodeConfig, seed: int = 0, *, fork_step: bool = False,
                         prefix=prefix)
 
 
+def device_normal_fill(shape, dtype: str, std: float, seed: int, stream: int, device):
+    """N(0, std^2) draws made on a CUDA device by torch's generator keyed by (seed,
+    stream), rounded to ``dtype`` (a torch tensor).  Same distribution as
+    ``normal_fill`` but not the same values: for throughput runs of large pools,
+    where drawing gigabytes on the host would dominate the run and the values only
+    need the workload's distribution."""
+    t = _torch()
+    g = t.Generator(device=device)
+    g.manual_seed((seed * 1_000_003 + stream) & ((1 << 63) - 1))
+    out = t.empty(shape, dtype=TORCH_DTYPES[dtype], device=device)
+    flat = out.view(-1)
+    step = 1 << 28                      # bounded float32 scratch per chunk
+    for lo in range(0, flat.numel(), step):
+        n = min(step, flat.numel() - lo)
+        x = t.randn(n, generator=g, device=device, dtype=t.float32)
+        if std != 1.0:
+            x.mul_(std)
+        flat[lo:lo + n].copy_(x)
+        del x
+    return out
+
+
 def step_tokens(cfg: DecodeConfig, seed: int, step: int):
     """q / new K / new V for decode step ``step`` (>= 1) of a multi-step run."""
     S, Hq, Hkv, D = cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_dim
