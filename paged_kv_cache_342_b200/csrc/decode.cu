@@ -21,6 +21,8 @@ cudaError_t launch_decode_simt_bf16(const DecodeParams& p, int gs, cudaStream_t 
 cudaError_t launch_decode_simt_f16(const DecodeParams& p, int gs, cudaStream_t st);
 cudaError_t launch_decode_simt_fp8(const DecodeParams& p, int q_dtype, int gs, cudaStream_t st);
 cudaError_t launch_decode_mma_fp8(const DecodeParams& p, int q_dtype, cudaStream_t st);
+cudaError_t launch_decode_tc_fp8(const DecodeParams& p, int q_dtype, cudaStream_t st);
+bool tc_fp8_eligible(int group, int head_dim, int block_size);
 cudaError_t launch_decode_mma_bf16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_group_bf16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
@@ -532,7 +534,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     }
     joined = side;
   }
-  if (fp8 && mma_fp8_eligible(group, block_size)) {
+  if (fp8 && tc_fp8_eligible(group, head_dim, block_size)) {
+    e = launch_decode_tc_fp8(p, dtype, st);
+  } else if (fp8 && mma_fp8_eligible(group, block_size)) {
     e = launch_decode_mma_fp8(p, dtype, st);
   } else if (fp8) {
     e = launch_decode_simt_fp8(p, dtype, simt_heads_per_cta(group, head_dim), st);

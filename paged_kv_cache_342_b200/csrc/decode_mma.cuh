@@ -93,15 +93,6 @@ __device__ __forceinline__ void e4m3_pairs_to_f16x2_bits(uint32_t w, uint32_t& e
   even = e4m3_place(w << 8);
   odd = e4m3_place(w);
 }
-// 2-D tiled TMA load of one box into shared memory, completion on an mbarrier.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
 
 // FP8: the cache holds e4m3 codes; TMA lands them as 128-element x BS-row slabs and
 // the MMA operands are loaded straight from them with ldmatrix (a pair of codes is

@@ -60,6 +60,13 @@ FP8_CASES = [
     ("f16", 8, 2, 128, 16, 64, (9, 90)),                   # group 4: CUDA cores
     ("f16", 2, 2, 256, 32, 64, (3, 100, 250)),
     ("bf16", 4, 4, 128, 4, 16, (7, 18, 10)),
+    # the tcgen05 kernel (head_dim 128, groups of 8 or 16): 128-token tiles
+    ("bf16", 32, 2, 128, 16, 256, (1, 127, 128, 129, 1000)),   # group 16
+    ("f16", 32, 2, 128, 32, 64, (5, 333, 64, 65)),            # group 16, partitions < a tile
+    ("f16", 16, 2, 128, 16, 384, (383, 384, 385, 1153)),      # partitions of three tiles
+    ("bf16", 32, 4, 128, 16, 512, (1100, 700)),               # 4 kv heads x group 8
+    ("bf16", 16, 2, 128, 16, 4096, (4096, 17)),               # one partition of 32 tiles
+    ("bf16", 16, 2, 128, 32, 2048, (2048, 1)),
 ]
 
 
@@ -157,3 +164,56 @@ def test_fp8_decode_step_through_the_runtime(pa):
                                        fp8.dequantize(pool_v, vs), tables, sl, 1 / math.sqrt(D),
                                        bs, Hkv, "f64")
     assert_close(out_f64(out), want, "bf16", "fp8 step")
+
+
+@pytest.mark.parametrize("Hq,Hkv,bs,ps,qdt", [(16, 2, 16, 512, "bf16"), (32, 2, 32, 64, "f16"),
+                                             (16, 2, 32, 256, "f16")])
+def test_fp8_tensor_cores_never_read_unused_slots(pa, Hq, Hkv, bs, ps, qdt):
+    """Every slot no sequence owns - the tail of each last block and the blocks in no
+    table - holds the NaN code 0x7F: the tiles' rows past the end must not reach O."""
+    lens = np.array([1, 130, 700, 129], np.int64)
+    S, D = lens.size, 128
+    NB = int(sum(-(-int(L) // bs) for L in lens)) + 4
+    ks = vs = 8.0 / 448.0
+    kc = fp8.quantize(normal_fill((NB, Hkv, bs, D), "f32", 1.0, 13, 1), ks)
+    vc = fp8.quantize(normal_fill((NB, Hkv, bs, D), "f32", 1.0, 13, 2), vs)
+    order = np.random.default_rng(13).permutation(NB).astype(np.int32)
+    tables = tables_from_order(lens, bs, order, int(-(-lens.max() // bs)) + 1)
+    used = np.zeros((NB, bs), bool)
+    for srow, L in zip(tables, lens):
+        for t in range(int(L)):
+            used[srow[t // bs], t % bs] = True
+    for c in (kc, vc):
+        c.transpose(0, 2, 1, 3)[~used] = 0x7F
+    q = normal_fill((S, Hq, D), qdt, 1.0, 13, 3)
+    out = torch.full((S, Hq, D), float("nan"), dtype=TORCH_DT[qdt], device="cuda")
+    wsb = pa.pa_decode_workspace_bytes(S, Hq, D, int(lens.max()), ps)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+    pa.pa_decode_attention_fp8(out, to_dev(q, qdt), torch.from_numpy(kc).cuda(),
+                               torch.from_numpy(vc).cuda(), torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens.astype(np.int32)).cuda(), 1 / math.sqrt(D),
+                               bs, Hkv, int(lens.max()), ks, vs, ps, ws if wsb else None)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    want = oatt.paged_decode_attention(to_f64(q, qdt), fp8.dequantize(kc, ks),
+                                       fp8.dequantize(vc, vs), tables, lens, 1 / math.sqrt(D),
+                                       bs, Hkv, "f64")
+    assert_close(out_f64(out), want, qdt, "fp8 cache, NaN in unused slots")
+
+
+def test_fp8_tensor_cores_out_of_range_table_entry(pa):
+    """A table entry outside the pool is skipped (its rows count as absent) and
+    reported; every output stays finite."""
+    S, Hq, Hkv, D, bs, NB = 2, 16, 2, 128, 16, 16
+    kc = fp8.quantize(normal_fill((NB, Hkv, bs, D), "f32", 1.0, 14, 1), 8.0 / 448)
+    q = normal_fill((S, Hq, D), "bf16", 1.0, 14, 2)
+    tables = np.array([[3, 5, NB + 7], [1, -4, 2]], np.int32)
+    lens = np.array([40, 40], np.int32)
+    out = torch.empty((S, Hq, D), dtype=torch.bfloat16, device="cuda")
+    kd = torch.from_numpy(kc).cuda()
+    pa.pa_decode_attention_fp8(out, to_dev(q, "bf16"), kd, kd, torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens).cuda(), 0.1, bs, Hkv, 40, 8.0 / 448,
+                               8.0 / 448, 512, None)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == pa.DEVERR_TABLE
+    assert torch.isfinite(out).all()
