@@ -31,8 +31,8 @@ struct DecodeParams {
   int64_t num_blocks;
   int max_seq_len, partition_size, max_parts;
   float* ws_o;  // [S, Hq, P, D]  normalised partial outputs
-  float* ws_m;  // [S, Hq, P]     partition max (base-2 logits)
-  float* ws_l;  // [S, Hq, P]     partition exp-sum
+  float* ws_m;  // [P, S, Hq]     partition max (base-2 logits), see ml_index
+  float* ws_l;  // [P, S, Hq]     partition exp-sum
   uint32_t* err;
   // prefix groups (all null / 0 for the plain call): whole partitions that a group of
   // sequences shares are computed once per group by the group kernel
@@ -45,7 +45,16 @@ struct DecodeParams {
   // [S] or null: grid row y of the per-sequence kernels serves sequence seq_order[y]
   // (longest first, so that the long rows start early and the short ones fill the end)
   const int32_t* seq_order;
+  // partitions one CTA of the fp8 tensor-core kernel walks (0 or 1: one)
+  int parts_per_cta;
 };
+
+// Index of (query row, partition) in the partition maxima / exp-sums ws_m, ws_l:
+// partition-major [P, S * Hq], so that one partition's values for a run of query
+// heads are contiguous (and can be written with one bulk copy).
+__device__ __forceinline__ int64_t ml_index(const DecodeParams& p, int64_t row, int part) {
+  return static_cast<int64_t>(part) * p.num_seqs * p.num_heads + row;
+}
 
 // The sequence grid row y serves; -1 (reported) for an order entry out of range.
 __device__ __forceinline__ int row_sequence(const DecodeParams& p, int y, bool report) {

@@ -105,8 +105,9 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
   for (int j = 0; j < DPL; ++j) acc[j] = 0.f;
   float den = 0.f, M = -INFINITY;
   if (nparts > 1) {
-    const float* mrow = p.ws_m + static_cast<int64_t>(row) * p.max_parts;
-    const float* lrow = p.ws_l + static_cast<int64_t>(row) * p.max_parts;
+    const int64_t mstride = static_cast<int64_t>(p.num_seqs) * p.num_heads;
+    const float* mrow = p.ws_m + row;  // partition pi at mrow[pi * mstride]
+    const float* lrow = p.ws_l + row;
     const float* orow = p.ws_o + static_cast<int64_t>(row) * p.max_parts * D + lane * DPL;
     for (int i = wsub; i < nparts; i += U * wpr) {
       float mv[U], lv[U], o[U][DPL];
@@ -114,8 +115,8 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
       for (int u = 0; u < U; ++u) {
         const int pi = i + u * wpr;
         if (pi < nparts) {
-          mv[u] = mrow[pi];
-          lv[u] = lrow[pi];
+          mv[u] = mrow[pi * mstride];
+          lv[u] = lrow[pi * mstride];
           load_lane<DPL>(orow + static_cast<int64_t>(pi) * D, o[u]);
         } else {
           mv[u] = -INFINITY;

@@ -574,8 +574,8 @@ __global__ void __launch_bounds__(NW * 32)
       const int64_t prow = row * p.max_parts + part;
       p.ws_o[prow * D + d] = o;
       if (d == 0) {
-        p.ws_m[prow] = col_m[hh];
-        p.ws_l[prow] = den;
+        p.ws_m[ml_index(p, row, part)] = col_m[hh];
+        p.ws_l[ml_index(p, row, part)] = den;
       }
     }
   }

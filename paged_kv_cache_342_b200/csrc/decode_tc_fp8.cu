@@ -1,29 +1,36 @@
 // Decode partition kernel for fp8 (e4m3) caches with grouped-query heads on the 5th-
 // generation tensor cores (tcgen05.mma kind::f8f6f4, accumulators in tensor memory).
 // Same result as the other partition kernels: softmax(scale * q.K) V over the tokens
-// of one partition, as a normalised partial (max, exp-sum, output) or the final row
+// of each partition, as a normalised partial (max, exp-sum, output) or the final row
 // ("How PagedAttention Powers vLLM's KV Cache", hassanahmed.net, "The attention kernel
 // has to read scattered blocks"; "Where it bites": grouped-query attention and a
 // quantized cache stack with paging).
 //
-// One CTA per (sequence, kv head, partition); 6 warps:
-//   warp 0     walks the block table and brings each block's K and V rows in by TMA
-//              (128-byte rows, 128-byte swizzle) into stages of 128 tokens;
-//   warp 1     issues the MMAs (one thread) as soon as their operands are ready:
-//                S [128 tokens x NS] = K [128 x 128 dims] . Qt^T         (K-major A, B)
-//                O [128 dims x 2G]  += V^T [128 dims x 128 tokens] . Pt  (MN-major A, B)
-//   warps 2-5  one thread per token row: read S from tensor memory, online softmax
-//              per head, write P; at the end one thread per dim row reads O.
+// Persistent CTAs (two per SM) walk a round-robin list of work items (sequence, kv
+// head, up to 2048 tokens of consecutive partitions); 8 warps:
+//   warps 0, 3  walk the block table and bring each block's K (warp 0) and V (warp 3)
+//               rows in by TMA (128-byte rows, 128-byte swizzle) into stages of 128
+//               tokens; a K stage is refilled as soon as its S is computed, a V stage
+//               once its p.V is, so K runs ahead and items follow each other without
+//               a pipeline ramp;
+//   warp 1      issues S [128 tokens x NS] = K [128 x 128 dims] . Qt^T   (K-major A, B)
+//   warp 2      issues O [128 dims x 2G] += V^T [128 x 128 tokens] . Pt  (MN-major A, B)
+//   warps 4-7   one thread per token row: read S from tensor memory, online softmax per
+//               head, write P; a partition's output (one thread per dim row) is read
+//               from tensor memory after the next partition's first tile, from the
+//               other of two O accumulators, so it never stalls the pipeline.
 // The codes are never converted: K and V tiles are the MMA operands as TMA lands
 // them.  q (bf16: 2 terms, f16: 3 terms) is carried as exact e4m3 terms t_j of
 // q * 2^qe (qe per head puts the largest |q| in [128, 256)), the terms as separate
-// columns of S, summed per head.  P is split into hi = e4m3(p) and lo =
-// e4m3((p - hi) * 32), again as separate columns of O: o = O_hi + O_lo / 32.  Weights
-// stay in (0, 2^8] under the lazy running max, so both fit e4m3 (|p - hi| <= 8).
-// Tokens past the end (or in blocks whose table entry is out of range) get -inf
-// scores, and their V rows are zeroed in shared memory (0 * NaN would poison O).
-// Every wait is bounded; a CTA that gives up sets PA_DEVERR_TIMEOUT, drains its
-// copies and MMAs (bounded), frees its tensor memory and writes nothing.
+// columns of S, summed per head; the next item's q is prefetched into registers and
+// written to the other of two Q buffers during the current item.  P is split into
+// hi = e4m3(p) and lo = e4m3((p - hi) * 32), again as separate columns of O:
+// o = O_hi + O_lo / 32.  Weights stay in (0, 2^8] under the lazy running max, so both
+// fit e4m3 (|p - hi| <= 8).  Tokens past the end (or in blocks whose table entry is
+// out of range) get -inf scores, and their V rows are zeroed in shared memory
+// (0 * NaN would poison O).  Every wait is bounded; a CTA that gives up sets
+// PA_DEVERR_TIMEOUT, drains its copies and MMAs (bounded), frees its tensor memory
+// and writes nothing more.
 #include <type_traits>
 
 #include "common.cuh"
@@ -34,7 +41,9 @@
 namespace pa {
 namespace {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 256;
+constexpr int kTcCtasPerSm = 2;
+constexpr int kTcMaxItems = 96;  // work items of one CTA (the launch ensures it)
 
 template <typename TQ, int G, int BS, int NST>
 struct TcCfg {
@@ -42,12 +51,16 @@ struct TcCfg {
   static constexpr int NQT = std::is_same<TQ, __half>::value ? 3 : 2;  // q terms
   static constexpr int NS = (G * NQT + 15) / 16 * 16;                   // S columns
   static constexpr int NO = 2 * G;                                      // O columns
-  static constexpr int kTmemNeed = NO + 2 * NS;
-  static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : 128;
+  // tensor memory: O[0], O[1] (NO columns each), then S[0], S[1] (NS each)
+  static constexpr int kTmemNeed = 2 * NO + 2 * NS;
+  static constexpr int kTmemCols = kTmemNeed <= 32    ? 32
+                                   : kTmemNeed <= 64  ? 64
+                                   : kTmemNeed <= 128 ? 128
+                                                      : 256;
   static constexpr int TILE = TM * D;        // one K or V tile, bytes
   static constexpr int STAGE = 2 * TILE;     // K then V
   static constexpr int QOFF = NST * STAGE;
-  static constexpr int QBYTES = (NS * 128 + 1023) / 1024 * 1024;
+  static constexpr int QBYTES = (NS * 128 + 1023) / 1024 * 1024;  // the Q operand
   static constexpr int POFF = QOFF + QBYTES;
   static constexpr int PBYTES = TM * NO;     // one P buffer
   // P as the MN-major (no swizzle) B operand: core matrices of 8 tokens x 16 bytes;
@@ -55,12 +68,17 @@ struct TcCfg {
   // 8-token groups PK_STRIDE apart.  Byte (t, n) = (t/8) PK_STRIDE + (n/16) 128 +
   // (t%8) 16 + n%16.  Every stride is small, so the operand stays inside its buffer.
   static constexpr int PK_STRIDE = 128 * (NO / 16);
-  static constexpr int SMEM = 1024 + POFF + 2 * PBYTES;
+  // one partition's output on its way out by bulk copy: G rows of 128 floats (or of
+  // 128 output elements), then the partition's G maxima and G exp-sums
+  static constexpr int SOFF = POFF + 2 * PBYTES;
+  static constexpr int STBYTES = G * 512 + 2 * G * 4;
+  static constexpr int SMEM = 1024 + SOFF + STBYTES;
+  static_assert(2 * PBYTES >= 256 * 16, "the P buffers hold the balanced list's scratch");
   static constexpr uint32_t IDESC_S = idesc_e4m3(128, NS, false, false);
   static constexpr uint32_t IDESC_O = idesc_e4m3(128, NO, true, true);
   static_assert(G == 8 || G == 16, "head groups of 8 or 16");
   static_assert(BS == 16 || BS == 32, "block size 16 or 32");
-  static_assert(kTmemNeed <= 128, "tensor memory budget");
+  static_assert(kTmemNeed <= 256, "tensor memory budget");
   static_assert(NS <= 48 && NS % 16 == 0 && NO % 16 == 0, "tile widths");
 };
 
@@ -82,423 +100,644 @@ __device__ __forceinline__ bool wg_wait(uint32_t bar, uint32_t parity) {
   const bool ok = mbar_wait_bounded(bar, parity);
   return bar_red_and(1, 128, ok);
 }
+// Bounded wait by lane 0 of a warp, the result shared with the whole warp.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane) {
+  const bool ok = lane == 0 ? mbar_wait_bounded(bar, parity) : true;
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
 
+// Tokens of partition j of a sequence of length L (partition size ps).
+__device__ __forceinline__ int part_tokens(int j, int ps, int L) {
+  const int b = j * ps;
+  return max(0, min(L, b + ps) - b);
+}
+
+// A work item: partitions [pbeg, pend) of sequence s for the query heads of kv head kvh;
+// kind 1 is an empty sequence (its output is zeros), kind 2 has tiles.
+struct TcItem {
+  int s, kvh, L, pbeg, pend, kind;
+};
+// Item idx of the list: chunk z of ppc partitions (outermost), grid row y (sequence
+// seq_order[y], longest first when an order is given), kv head (innermost).  Returns
+// the kind, 0 for nothing to do.  Bad order entries and lengths are reported once per
+// row (by the item of chunk 0, kv head 0).
+__device__ __forceinline__ int tc_item(const DecodeParams& p, int idx, int ppc, TcItem& it) {
+  const int rows = p.num_seqs * p.num_kv_heads;
+  const int z = idx / rows, r = idx - z * rows;
+  const int y = r / p.num_kv_heads;
+  it.kvh = r - y * p.num_kv_heads;
+  const bool report = z == 0 && it.kvh == 0;
+  it.kind = 0;
+  it.s = row_sequence(p, y, report);
+  if (it.s < 0) return 0;
+  it.L = checked_len(p, it.s, report);
+  const int ps = p.partition_size;
+  const int nparts = it.L > 0 ? (it.L + ps - 1) / ps : 1;
+  const int own = group_parts(p, it.s, it.L);
+  it.pbeg = max(own, p.part_base + z * ppc);
+  it.pend = min(nparts, p.part_base + (z + 1) * ppc);
+  if (it.pbeg >= it.pend) return 0;
+  it.kind = it.L > 0 ? 2 : 1;
+  return it.kind;
+}
+
+// Groups of 8 fit two CTAs per SM (shared memory), so registers are held to 128 per
+// thread; groups of 16 need more shared memory and run one CTA per SM.
 template <typename TQ, int G, int BS, int NST>
-__global__ void __launch_bounds__(kTcThreads)
+__global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
     decode_tc_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
-                         const __grid_constant__ CUtensorMap tmv) {
+                         const __grid_constant__ CUtensorMap tmv, int ppc, int num_items,
+                         int balanced) {
   grid_dependency_wait();
   using C = TcCfg<TQ, G, BS, NST>;
-  constexpr int TM = C::TM, NS = C::NS, NO = C::NO, BPT = C::BPT;
+  constexpr int TM = C::TM, NS = C::NS, NO = C::NO, BPT = C::BPT, D = C::D;
   constexpr unsigned FULL = 0xffffffffu;
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full_k[NST], bar_full_v[NST], bar_empty[NST];
+  __shared__ __align__(8) uint64_t bar_full_k[NST], bar_full_v[NST];
+  __shared__ __align__(8) uint64_t bar_k_empty[NST], bar_v_empty[NST];
   __shared__ __align__(8) uint64_t bar_s_full[2], bar_s_empty[2], bar_p_full[2], bar_p_empty[2];
-  __shared__ __align__(8) uint64_t bar_drain;
+  __shared__ __align__(8) uint64_t bar_q_full, bar_drain[2];
   __shared__ uint32_t tmem_base_sm;
   __shared__ float sh_c[G];          // per-head logit factor (base 2, times 2^-qe)
-  __shared__ float sh_red[4][G];     // per-warp maxima / sums of the softmax warpgroup
+  __shared__ float sh_red[4][G];     // per-warp maxima of the softmax warpgroup
+  __shared__ float sh_sum[4][G];     // per-warp exp-sums of the softmax warpgroup
+  __shared__ float sh_den[2][G], sh_m[2][G];  // per O buffer: exp-sums and maxima
+  __shared__ TcItem sh_items[kTcMaxItems];    // this CTA's work, in order
+  __shared__ int sh_nitems;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool report = threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0;
-  const int s = row_sequence(p, blockIdx.y, report);
-  if (s < 0) return;
-  const int kvh = blockIdx.x, h0 = kvh * G;
-  const int part = p.part_base + blockIdx.z;
-  const int L = checked_len(p, s, report);
   const int ps = p.partition_size;
-  const int nparts = L > 0 ? (L + ps - 1) / ps : 1;
-  const int own = group_parts(p, s, L);
-  if (part >= nparts || part < own) return;
-  const int tok_begin = part * ps;
-  const int tok_end = min(L, tok_begin + ps);
-  const int ntok = tok_end > tok_begin ? tok_end - tok_begin : 0;
-  if (ntok == 0) {  // an empty sequence: zeros (a single partition)
-    for (int i = threadIdx.x; i < G * C::D; i += kTcThreads)
-      store_elem(static_cast<TQ*>(p.out) + (static_cast<int64_t>(s) * p.num_heads + h0) * C::D + i,
-                 0.f);
-    return;
-  }
-  const int ntiles = (ntok + TM - 1) / TM;
-  const int nblk = (ntok + BS - 1) / BS;
-  const int32_t* table =
-      p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + tok_begin / BS;
-
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
   auto b32 = [](const uint64_t& b) { return smem_u32(&b); };
 
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 64) {  // the p.V warp has nothing else to do at the start
     for (int i = 0; i < NST; ++i) {
       mbar_init(b32(bar_full_k[i]), 1);
       mbar_init(b32(bar_full_v[i]), 1);
-      mbar_init(b32(bar_empty[i]), 1);
+      mbar_init(b32(bar_k_empty[i]), 1);
+      mbar_init(b32(bar_v_empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b32(bar_s_full[i]), 1);
       mbar_init(b32(bar_s_empty[i]), 128);
       mbar_init(b32(bar_p_full[i]), 128);
       mbar_init(b32(bar_p_empty[i]), 1);
+      mbar_init(b32(bar_drain[i]), 1);
     }
-    mbar_init(b32(bar_drain), 1);
+    mbar_init(b32(bar_q_full), 128);
     mbar_init_fence();
   }
-  if (warp == 1) {
+  if (warp == 3) {
     tmem_alloc(smem_u32(&tmem_base_sm), C::kTmemCols);
     tmem_relinquish();
+  }
+  if (warp == 2 && balanced) {
+    // Balanced split: every (sequence row, kv head) contributes its partitions; the
+    // flat list of all partitions (row-major) is cut into gridDim.x equal ranges and
+    // this CTA takes its range as runs of consecutive partitions.  Per sequence row:
+    // its sequence, length and first / count of partitions, in the P buffers (free
+    // until the first tile).
+    int* rs = reinterpret_cast<int*>(smem + C::POFF);
+    const int S = p.num_seqs, Hkv = p.num_kv_heads;
+    for (int y = lane; y < S; y += 32) {
+      const bool report = blockIdx.x == 0;
+      const int sq = row_sequence(p, y, report);
+      int L = 0, first = 0, cnt = 0;
+      if (sq >= 0) {
+        L = checked_len(p, sq, report);
+        const int nparts = L > 0 ? (L + ps - 1) / ps : 1;
+        first = max(group_parts(p, sq, L), p.part_base);
+        cnt = max(0, nparts - first);
+      }
+      rs[4 * y] = sq;
+      rs[4 * y + 1] = L;
+      rs[4 * y + 2] = first;
+      rs[4 * y + 3] = cnt;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      int64_t total = 0;
+      for (int y = 0; y < S; ++y) total += static_cast<int64_t>(rs[4 * y + 3]) * Hkv;
+      const int64_t lo = total * blockIdx.x / gridDim.x;
+      const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
+      int n = 0;
+      int64_t at = 0;  // flat index of row y's first partition
+      for (int y = 0; y < S && at < hi && n < kTcMaxItems; ++y) {
+        const int cnt = rs[4 * y + 3];
+        const int64_t span = static_cast<int64_t>(cnt) * Hkv;
+        if (at + span > lo) {
+          for (int kv = 0; kv < Hkv && n < kTcMaxItems; ++kv) {
+            const int64_t b = at + static_cast<int64_t>(kv) * cnt;  // this row's first
+            const int64_t from = max(b, lo), to = min(b + cnt, hi);
+            if (from >= to) continue;
+            TcItem it;
+            it.s = rs[4 * y];
+            it.kvh = kv;
+            it.L = rs[4 * y + 1];
+            it.pbeg = rs[4 * y + 2] + static_cast<int>(from - b);
+            it.pend = rs[4 * y + 2] + static_cast<int>(to - b);
+            it.kind = it.L > 0 ? 2 : 1;
+            sh_items[n++] = it;
+          }
+        }
+        at += span;
+      }
+      sh_nitems = n;
+    }
+  } else if (warp == 2) {
+    // Round-robin: list positions blockIdx.x + k * gridDim.x (chunks of ppc
+    // partitions), evaluated 32 at a time and compacted
+    int n = 0;
+    for (int k0 = 0; k0 < kTcMaxItems; k0 += 32) {
+      const int idx = blockIdx.x + (k0 + lane) * gridDim.x;
+      TcItem it;
+      const bool keep = k0 + lane < kTcMaxItems && idx < num_items && tc_item(p, idx, ppc, it) != 0;
+      const uint32_t m = __ballot_sync(FULL, keep);
+      if (keep) sh_items[n + __popc(m & ((1u << lane) - 1u))] = it;
+      n += __popc(m);
+    }
+    if (lane == 0) sh_nitems = n;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tmem_base_sm;
+  const int nitems = sh_nitems;
   bool aborted = false;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    int tab_base = 0;
-    int32_t tab = lane < nblk ? __ldg(table + lane) : -1;
-    int i = 0;
-    for (; i < ntiles; ++i) {
-      const int st = i % NST;
-      if (i >= NST) {
-        bool ok = lane == 0 ? mbar_wait_bounded(b32(bar_empty[st]), ((i / NST) - 1) & 1) : true;
-        if (!__shfl_sync(FULL, ok, 0)) {
-          aborted = true;
-          break;
+  if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------------ producers
+    const bool is_k = warp == 0;
+    uint64_t* full = is_k ? bar_full_k : bar_full_v;
+    uint64_t* empty = is_k ? bar_k_empty : bar_v_empty;
+    const CUtensorMap* map = is_k ? &tmk : &tmv;
+    const uint32_t half = is_k ? 0u : static_cast<uint32_t>(C::TILE);
+    int g = 0;
+    for (int k = 0; k < nitems && !aborted; ++k) {
+      const TcItem it = sh_items[k];
+      if (it.kind != 2) continue;
+      const int32_t* seq_table =
+          p.block_tables + static_cast<int64_t>(it.s) * p.max_blocks_per_seq;
+      for (int j = it.pbeg; j < it.pend && !aborted; ++j) {
+        const int nblk = (part_tokens(j, ps, it.L) + BS - 1) / BS;
+        const int32_t* table = seq_table + j * ps / BS;
+        int tab_base = 0;
+        int32_t tab = lane < nblk ? __ldg(table + lane) : -1;
+        for (int b0 = 0; b0 < nblk; b0 += BPT, ++g) {
+          const int st = g % NST;
+          if (g >= NST && !warp_wait(b32(empty[st]), ((g / NST) - 1) & 1, lane)) {
+            aborted = true;
+            break;
+          }
+          if (b0 - tab_base >= 32) {
+            tab_base += 32;
+            tab = tab_base + lane < nblk ? __ldg(table + tab_base + lane) : -1;
+          }
+          const int32_t blk = __shfl_sync(FULL, tab, (b0 - tab_base + lane) & 31);
+          const bool in_part = lane < BPT && b0 + lane < nblk;
+          const bool ok = in_part && blk >= 0 && blk < p.num_blocks;
+          if (is_k && in_part && !ok) set_error(p.err, PA_DEVERR_TABLE);
+          const uint32_t nok = __popc(__ballot_sync(FULL, ok));
+          if (lane == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(b32(full[st]), nok * BS * 128);
+          }
+          __syncwarp();
+          if (ok)
+            tma_load_2d(base + st * C::STAGE + half + lane * BS * 128, map, 0,
+                        (blk * p.num_kv_heads + it.kvh) * BS, b32(full[st]));
         }
-      }
-      const int b0 = i * BPT;
-      if (b0 - tab_base >= 32) {
-        tab_base += 32;
-        tab = tab_base + lane < nblk ? __ldg(table + tab_base + lane) : -1;
-      }
-      const int b = b0 + lane;
-      const int32_t blk = __shfl_sync(FULL, tab, (b0 - tab_base + lane) & 31);
-      const bool in_part = lane < BPT && b < nblk;
-      const bool ok = in_part && blk >= 0 && blk < p.num_blocks;
-      if (in_part && !ok) set_error(p.err, PA_DEVERR_TABLE);
-      const uint32_t nok = __popc(__ballot_sync(FULL, ok));
-      const uint32_t kst = base + st * C::STAGE;
-      if (lane == 0) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(b32(bar_full_k[st]), nok * BS * 128);
-        mbar_arrive_expect_tx(b32(bar_full_v[st]), nok * BS * 128);
-      }
-      __syncwarp();
-      if (ok) {
-        const int row0 = (blk * p.num_kv_heads + kvh) * BS;
-        tma_load_2d(kst + lane * BS * 128, &tmk, 0, row0, b32(bar_full_k[st]));
-        tma_load_2d(kst + C::TILE + lane * BS * 128, &tmv, 0, row0, b32(bar_full_v[st]));
       }
     }
     if (aborted && lane == 0) {
       // the last NST issued tiles may still be landing: wait for them (bounded)
-      for (int j = (i > NST ? i - NST : 0); j < i; ++j) {
-        mbar_wait_bounded(b32(bar_full_k[j % NST]), (j / NST) & 1);
-        mbar_wait_bounded(b32(bar_full_v[j % NST]), (j / NST) & 1);
-      }
+      for (int k = (g > NST ? g - NST : 0); k < g; ++k)
+        mbar_wait_bounded(b32(full[k % NST]), (k / NST) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issue
-    named_sync(2, 160);  // q terms are in shared memory
-    tc_fence_after();
-    const uint32_t tO = tbase, tS0 = tbase + NO;
-    const uint32_t qaddr = base + C::QOFF;
-    const uint32_t paddr = base + C::POFF;
-    int ns = 0, npv = 0;
-    uint64_t t0 = global_timer_ns();
-    uint32_t idle = 0;
-    while (npv < ntiles) {
-      bool prog = false;
-      if (ns < ntiles) {
-        const int st = ns % NST;
-        bool ready = lane == 0 && mbar_test(b32(bar_full_k[st]), (ns / NST) & 1) &&
-                     (ns < 2 || mbar_test(b32(bar_s_empty[ns & 1]), ((ns >> 1) - 1) & 1));
-        if (__shfl_sync(FULL, ready, 0)) {
+    // ------------------------------------------------------------------ S = K . Qt^T
+    const uint32_t tS0 = tbase + 2 * NO;
+    int g = 0, kq = 0;
+    for (int k = 0; k < nitems && !aborted; ++k) {
+      const TcItem it = sh_items[k];
+      if (it.kind != 2) continue;
+      if (!warp_wait(b32(bar_q_full), kq & 1, lane)) {  // this item's q terms
+        aborted = true;
+        break;
+      }
+      const uint32_t qaddr = base + C::QOFF;
+      ++kq;
+      for (int j = it.pbeg; j < it.pend && !aborted; ++j) {
+        const int nt = (part_tokens(j, ps, it.L) + TM - 1) / TM;
+        for (int i = 0; i < nt; ++i, ++g) {
+          const int st = g % NST;
+          if (!warp_wait(b32(bar_full_k[st]), (g / NST) & 1, lane) ||
+              (g >= 2 && !warp_wait(b32(bar_s_empty[g & 1]), ((g >> 1) - 1) & 1, lane))) {
+            aborted = true;
+            break;
+          }
           if (lane == 0) {
             tc_fence_after();
             const uint32_t ka = base + st * C::STAGE;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              umma_e4m3(tS0 + (ns & 1) * NS, smem_desc(ka + kk * 32, 16, 1024, kSwizzle128),
+              umma_e4m3(tS0 + (g & 1) * NS, smem_desc(ka + kk * 32, 16, 1024, kSwizzle128),
                         smem_desc(qaddr + kk * 32, 16, 1024, kSwizzle128), C::IDESC_S, kk > 0);
-            umma_commit(b32(bar_s_full[ns & 1]));
+            umma_commit(b32(bar_s_full[g & 1]));
+            umma_commit(b32(bar_k_empty[st]));  // the K stage may be refilled
           }
           __syncwarp();
-          ++ns;
-          prog = true;
         }
       }
-      if (npv < ns) {
-        const int st = npv % NST;
-        bool ready = lane == 0 && mbar_test(b32(bar_p_full[npv & 1]), (npv >> 1) & 1) &&
-                     mbar_test(b32(bar_full_v[st]), (npv / NST) & 1);
-        if (__shfl_sync(FULL, ready, 0)) {
+    }
+    if (aborted && lane == 0 && g > 0) {
+      umma_commit(b32(bar_drain[0]));  // every MMA this thread issued has completed
+      mbar_wait_bounded(b32(bar_drain[0]), 0);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------ O += V^T . Pt
+    const uint32_t paddr = base + C::POFF;
+    int g = 0, pc = 0;
+    for (int k = 0; k < nitems && !aborted; ++k) {
+      const TcItem it = sh_items[k];
+      if (it.kind != 2) continue;
+      for (int j = it.pbeg; j < it.pend && !aborted; ++j, ++pc) {
+        const int nt = (part_tokens(j, ps, it.L) + TM - 1) / TM;
+        const uint32_t tO = tbase + (pc & 1) * NO;
+        for (int i = 0; i < nt; ++i, ++g) {
+          const int st = g % NST;
+          if (!warp_wait(b32(bar_p_full[g & 1]), (g >> 1) & 1, lane) ||
+              !warp_wait(b32(bar_full_v[st]), (g / NST) & 1, lane)) {
+            aborted = true;
+            break;
+          }
           if (lane == 0) {
             tc_fence_after();
             const uint32_t va = base + st * C::STAGE + C::TILE;
-            const uint32_t pa_ = paddr + (npv & 1) * C::PBYTES;
+            const uint32_t pa_ = paddr + (g & 1) * C::PBYTES;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               umma_e4m3(tO, smem_desc(va + kk * 4096, 1024, 1024, kSwizzle128),
                         smem_desc(pa_ + kk * 4 * C::PK_STRIDE, C::PK_STRIDE, 128, kSwizzleNone),
-                        C::IDESC_O, npv > 0 || kk > 0);
-            umma_commit(b32(bar_empty[st]));
-            umma_commit(b32(bar_p_empty[npv & 1]));
+                        C::IDESC_O, i > 0 || kk > 0);
+            umma_commit(b32(bar_v_empty[st]));  // the V stage may be refilled
+            umma_commit(b32(bar_p_empty[g & 1]));
           }
           __syncwarp();
-          ++npv;
-          prog = true;
         }
       }
-      // no progress for about a second: give up (decided by lane 0 for the warp)
-      bool give_up = false;
-      if (prog) {
-        idle = 0;
-        t0 = global_timer_ns();
-      } else {
-        __nanosleep(32);  // leave issue slots to the softmax warp on this scheduler
-        if ((++idle & 255u) == 0) give_up = lane == 0 && global_timer_ns() - t0 > 1000000000ull;
-      }
-      if (__shfl_sync(FULL, give_up, 0)) {
-        aborted = true;
-        break;
-      }
     }
-    if (aborted && lane == 0 && ns + npv > 0) {
-      umma_commit(b32(bar_drain));  // every MMA issued so far has completed
-      mbar_wait_bounded(b32(bar_drain), 0);
+    if (aborted && lane == 0 && g > 0) {
+      umma_commit(b32(bar_drain[1]));
+      mbar_wait_bounded(b32(bar_drain[1]), 0);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------------ softmax warps
-    const int wt = threadIdx.x - 64;  // 0..127
-    // q of the G heads as exact e4m3 terms, K-major rows (term * G + head) of 128
-    // bytes with the 128-byte swizzle; each item is 8 dims of one head
-#pragma unroll
-    for (int it = 0; it < G / 8; ++it) {
-      const int h = wt / 16 + 8 * it, c = wt % 16;
-      const TQ* qp = static_cast<const TQ*>(p.q) +
-                     (static_cast<int64_t>(s) * p.num_heads + h0 + h) * C::D + c * 8;
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(qp));
-      float y[8];
-      vec_to_float(w, y, TQ{});
-      float mx = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) mx = fmaxf(mx, fabsf(y[j]));
-#pragma unroll
-      for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-      // 2^qe puts the largest magnitude in [128, 256)
-      int qe = mx > 0.f ? 7 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127) : 0;
-      qe = qe < -126 ? -126 : (qe > 126 ? 126 : qe);
-      const float sc = __uint_as_float(static_cast<uint32_t>(qe + 127) << 23);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) y[j] *= sc;
-#pragma unroll
-      for (int t = 0; t < C::NQT; ++t) {
-        uint32_t word[2];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint16_t pr = e4m3_pair(y[2 * j], y[2 * j + 1]);
-          float bhi;
-          const float blo = e4m3_pair_back(pr, bhi);
-          y[2 * j] -= blo;  // the remainder, exact in float32
-          y[2 * j + 1] -= bhi;
-          if (j & 1) word[j >> 1] |= static_cast<uint32_t>(pr) << 16;
-          else word[j >> 1] = pr;
-        }
-        const int r = t * G + h;
-        uint8_t* dst = smem + C::QOFF + (r >> 3) * 1024 + (r & 7) * 128 +
-                       ((((c >> 1) ^ (r & 7)) << 4) | ((c & 1) << 3));
-        *reinterpret_cast<uint2*>(dst) = make_uint2(word[0], word[1]);
-      }
-      if (c == 0) sh_c[h] = p.scale_log2 * __uint_as_float(static_cast<uint32_t>(127 - qe) << 23);
-    }
-    for (int i = (G * C::NQT) * 128 / 16 + wt; i < NS * 128 / 16; i += 128)  // padding rows
-      *reinterpret_cast<uint4*>(smem + C::QOFF + i * 16) = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
-    named_sync(2, 160);
-
-    const int wq = warp & 3;       // tensor-memory lane quarter of this warp
-    const int trow = wq * 32 + lane;
+    const int wt = threadIdx.x - 128;  // 0..127
+    const int wq = warp & 3;           // tensor-memory lane quarter of this warp
+    const int trow = wq * 32 + lane;   // token row of a tile, dim row of O
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tO = tbase + lane_off, tS0 = tbase + NO + lane_off;
-    float cf[G], m[G], l[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      cf[h] = sh_c[h];
-      m[h] = -INFINITY;
-      l[h] = 0.f;
-    }
-    int i = 0;
-    for (; i < ntiles; ++i) {
-      const int st = i % NST;
-      const int tok = i * TM + trow;  // token within the partition
-      bool valid = tok < ntok;
-      if (valid) {
-        const int32_t e = __ldg(table + tok / BS);
-        valid = e >= 0 && e < p.num_blocks;
-      }
-      if (!wg_wait(b32(bar_s_full[i & 1]), (i >> 1) & 1)) {
-        aborted = true;
-        break;
-      }
-      tc_fence_after();
-      float sv[NS];
-#pragma unroll
-      for (int c16 = 0; c16 < NS / 16; ++c16) {
-        float v16[16];
-        tmem_ld16(tS0 + (i & 1) * NS + c16 * 16, v16);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) sv[c16 * 16 + j] = v16[j];
-      }
-      tc_fence_before();
-      mbar_arrive(b32(bar_s_empty[i & 1]));
-      float sc[G];
-      bool grow = false;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float a = sv[h];
-#pragma unroll
-        for (int t = 1; t < C::NQT; ++t) a += sv[t * G + h];
-        sc[h] = valid ? a * cf[h] : -INFINITY;
-        grow |= sc[h] > m[h] + kLazyMax;
-      }
-      // the running max moves only when a head's tile max passes it by more than
-      // kLazyMax (base 2); until then the weights stay below 2^kLazyMax
-      if (bar_red_or(1, 128, grow)) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float w = warp_max(sc[h]);
-          if (lane == 0) sh_red[wq][h] = w;
-        }
-        named_sync(1, 128);
-        bool moved = false;
-        float corr[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float tmax =
-              fmaxf(fmaxf(sh_red[0][h], sh_red[1][h]), fmaxf(sh_red[2][h], sh_red[3][h]));
-          const float mn = tmax > m[h] + kLazyMax ? tmax : m[h];
-          corr[h] = exp2_safe(m[h], mn);
-          moved |= mn != m[h];
-          l[h] *= corr[h];
-          m[h] = mn;
-        }
-        if (moved && i > 0) {
-          // rescale O (thread = dim row) once the previous tile's p.V has landed
-          if (!wg_wait(b32(bar_p_empty[(i - 1) & 1]), ((i - 1) >> 1) & 1)) {
-            aborted = true;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int c16 = 0; c16 < NO / 16; ++c16) {
-            float o16[16];
-            tmem_ld16(tO + c16 * 16, o16);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) o16[j] *= corr[(c16 * 16 + j) % G];
-            tmem_st16(tO + c16 * 16, o16);
-          }
-        }
-      }
-      // weights, split into two e4m3 terms (hi, (p - hi) * 32)
-      uint32_t hiw[G / 4], low[G / 4];
-#pragma unroll
-      for (int h = 0; h < G; h += 2) {
-        const float p0 = exp2_safe(sc[h], m[h]), p1 = exp2_safe(sc[h + 1], m[h + 1]);
-        l[h] += p0;
-        l[h + 1] += p1;
-        const uint16_t hp = e4m3_pair(p0, p1);
-        float b1;
-        const float b0 = e4m3_pair_back(hp, b1);
-        const uint16_t lp = e4m3_pair((p0 - b0) * 32.f, (p1 - b1) * 32.f);
-        const int wi = h >> 2, sh = (h & 2) ? 16 : 0;
-        if (sh == 0) {
-          hiw[wi] = hp;
-          low[wi] = lp;
-        } else {
-          hiw[wi] |= static_cast<uint32_t>(hp) << 16;
-          low[wi] |= static_cast<uint32_t>(lp) << 16;
-        }
-      }
-      if (i >= 2 && !wg_wait(b32(bar_p_empty[i & 1]), ((i >> 1) - 1) & 1)) {
-        aborted = true;
-        break;
-      }
-      uint8_t* pb = smem + C::POFF + (i & 1) * C::PBYTES + (trow >> 3) * C::PK_STRIDE +
-                    (trow & 7) * 16;
-      if constexpr (G == 8) {
-        *reinterpret_cast<uint4*>(pb) = make_uint4(hiw[0], hiw[1], low[0], low[1]);
-      } else {
-        *reinterpret_cast<uint4*>(pb) = make_uint4(hiw[0], hiw[1], hiw[2], hiw[3]);
-        *reinterpret_cast<uint4*>(pb + 128) = make_uint4(low[0], low[1], low[2], low[3]);
-      }
-      // rows that carry no token: V zeroed (rows of the last block past the end are
-      // landed by TMA, so wait for it first)
-      if ((i + 1) * TM > ntok && !wg_wait(b32(bar_full_v[st]), (i / NST) & 1)) {
-        aborted = true;
-        break;
-      }
-      if (!valid) {
-        uint4* vrow = reinterpret_cast<uint4*>(smem + st * C::STAGE + C::TILE + trow * 128);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) vrow[j] = make_uint4(0, 0, 0, 0);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(b32(bar_p_full[i & 1]));
-    }
+    const uint32_t tS0 = tbase + 2 * NO + lane_off;
 
-    if (!aborted) {
-      const int last = ntiles - 1;
-      aborted = !wg_wait(b32(bar_p_empty[last & 1]), (last >> 1) & 1);
-    }
-    if (!aborted) {
-      tc_fence_after();
-      // exp-sums over the 128 token rows
+    // q of an item: this thread's 8 dims of heads wt/16 (+ 8) as raw TQ bits
+    struct QRaw {
+      uint4 v[G / 8];
+    };
+    auto load_q = [&](const TcItem& it) {
+      QRaw r;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float w = warp_sum(l[h]);
-        if (lane == 0) sh_red[wq][h] = w;
+      for (int k = 0; k < G / 8; ++k) {
+        const int h = wt / 16 + 8 * k, c = wt % 16;
+        r.v[k] = __ldg(reinterpret_cast<const uint4*>(
+            static_cast<const TQ*>(p.q) +
+            (static_cast<int64_t>(it.s) * p.num_heads + it.kvh * G + h) * D + c * 8));
       }
-      named_sync(1, 128);
-      float den[G];
+      return r;
+    };
+    // ... written into the Q operand as exact e4m3 terms: K-major rows (term * G +
+    // head) of 128 bytes with the 128-byte swizzle; then released to the S warp (the
+    // previous item's S MMAs have all completed by then)
+    auto store_q = [&](const QRaw raw_q) {
+      uint8_t* qb = smem + C::QOFF;
 #pragma unroll
-      for (int h = 0; h < G; ++h) den[h] = sh_red[0][h] + sh_red[1][h] + sh_red[2][h] + sh_red[3][h];
+      for (int k = 0; k < G / 8; ++k) {
+        const int h = wt / 16 + 8 * k, c = wt % 16;
+        float y[8];
+        vec_to_float(raw_q.v[k], y, TQ{});
+        float mx = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(y[e]));
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+        // 2^qe puts the largest magnitude in [128, 256)
+        int qe = mx > 0.f ? 7 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127) : 0;
+        qe = qe < -126 ? -126 : (qe > 126 ? 126 : qe);
+        const float sc = __uint_as_float(static_cast<uint32_t>(qe + 127) << 23);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] *= sc;
+#pragma unroll
+        for (int t = 0; t < C::NQT; ++t) {
+          uint32_t word[2];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint16_t pr = e4m3_pair(y[2 * e], y[2 * e + 1]);
+            float bhi;
+            const float blo = e4m3_pair_back(pr, bhi);
+            y[2 * e] -= blo;  // the remainder, exact in float32
+            y[2 * e + 1] -= bhi;
+            if (e & 1) word[e >> 1] |= static_cast<uint32_t>(pr) << 16;
+            else word[e >> 1] = pr;
+          }
+          const int r = t * G + h;
+          *reinterpret_cast<uint2*>(qb + (r >> 3) * 1024 + (r & 7) * 128 +
+                                    ((((c >> 1) ^ (r & 7)) << 4) | ((c & 1) << 3))) =
+              make_uint2(word[0], word[1]);
+        }
+        if (c == 0) sh_c[h] = p.scale_log2 * __uint_as_float(static_cast<uint32_t>(127 - qe) << 23);
+      }
+      for (int k = (G * C::NQT) * 128 / 16 + wt; k < NS * 128 / 16; k += 128)  // padding rows
+        *reinterpret_cast<uint4*>(qb + k * 16) = make_uint4(0, 0, 0, 0);
+      fence_proxy_async_smem();
+      mbar_arrive(b32(bar_q_full));
+    };
+    // the first item with tiles at list position >= k (nitems if none)
+    auto tile_item_from = [&](int k) {
+      while (k < nitems && sh_items[k].kind != 2) ++k;
+      return k;
+    };
+    // block-table entry of this thread's token in tile i of partition j of item k
+    // (-1 past the partition's end); fetched one tile ahead of its use
+    auto entry = [&](int k, int j, int i) -> int32_t {
+      const TcItem& it = sh_items[k];
+      const int t = i * TM + trow;
+      return t < part_tokens(j, ps, it.L)
+                 ? __ldg(p.block_tables + static_cast<int64_t>(it.s) * p.max_blocks_per_seq +
+                         (j * ps + t) / BS)
+                 : -1;
+    };
+    // a partition's output, read from O buffer ob once its last p.V (tile g_last)
+    // has landed (the partition's exp-sums and maxima are in sh_den / sh_m [ob]); it
+    // goes out through the staging buffer by bulk copies issued by one thread, so no
+    // thread of the warpgroup waits on a global store
+    struct Pending {
+      int s, h0, j, nparts, g_last, ob;
+    };
+    auto epilogue = [&](const Pending& e) -> bool {
+      if (!wg_wait(b32(bar_p_empty[e.g_last & 1]), (e.g_last >> 1) & 1)) return false;
+      tc_fence_after();
       float ov[NO];
 #pragma unroll
       for (int c16 = 0; c16 < NO / 16; ++c16) {
         float o16[16];
-        tmem_ld16(tO + c16 * 16, o16);
+        tmem_ld16(tbase + lane_off + e.ob * NO + c16 * 16, o16);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) ov[c16 * 16 + j] = o16[j];
+        for (int k = 0; k < 16; ++k) ov[c16 * 16 + k] = o16[k];
       }
-      const int d = trow;
+      tc_fence_before();  // O read before a later p.V overwrites it
+      if (wt == 0) bulk_wait_read_all();  // the previous output has left the staging buffer
+      named_sync(1, 128);
+      uint8_t* stg = smem + C::SOFF;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
+        const float den = sh_den[e.ob][h];
         const float o = ov[h] + ov[G + h] * (1.f / 32.f);
-        const float val = den[h] > 0.f ? o * (p.v_scale / den[h]) : 0.f;
-        const int64_t row = static_cast<int64_t>(s) * p.num_heads + h0 + h;
-        if (nparts == 1) {
-          store_elem(static_cast<TQ*>(p.out) + row * C::D + d, val);
+        const float val = den > 0.f ? o * p.v_scale * __frcp_rn(den) : 0.f;
+        if (e.nparts == 1) store_elem(reinterpret_cast<TQ*>(stg) + h * D + trow, val);
+        else reinterpret_cast<float*>(stg)[h * D + trow] = val;
+      }
+      if (e.nparts > 1 && trow < G) {
+        float* ml = reinterpret_cast<float*>(stg + G * 512);
+        ml[trow] = sh_m[e.ob][trow];
+        ml[G + trow] = sh_den[e.ob][trow];
+      }
+      fence_proxy_async_smem();
+      named_sync(1, 128);
+      if (wt == 0) {
+        const uint32_t sa = base + C::SOFF;
+        const int64_t row0 = static_cast<int64_t>(e.s) * p.num_heads + e.h0;
+        if (e.nparts == 1) {
+          bulk_s2g(static_cast<TQ*>(p.out) + row0 * D, sa, G * D * sizeof(TQ));
         } else {
-          const int64_t prow = row * p.max_parts + part;
-          p.ws_o[prow * C::D + d] = val;
-          if (d == h) {
-            p.ws_m[prow] = m[h];
-            p.ws_l[prow] = den[h];
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            bulk_s2g(p.ws_o + ((row0 + h) * p.max_parts + e.j) * D, sa + h * 512, 512);
+          bulk_s2g(p.ws_m + ml_index(p, row0, e.j), sa + G * 512, G * 4);
+          bulk_s2g(p.ws_l + ml_index(p, row0, e.j), sa + G * 512 + G * 4, G * 4);
+        }
+        bulk_commit();
+      }
+      return true;
+    };
+
+    Pending pend{};
+    bool pending = false;
+    int g = 0, pc = 0;
+    QRaw raw_q{};
+    int kcur = tile_item_from(0);
+    int32_t ent = -1;
+    if (kcur < nitems) {
+      raw_q = load_q(sh_items[kcur]);
+      store_q(raw_q);
+      ent = entry(kcur, sh_items[kcur].pbeg, 0);
+    }
+    for (int k = 0; k < nitems && !aborted; ++k) {
+      const TcItem cur = sh_items[k];
+      if (cur.kind == 1) {  // an empty sequence: zeros
+        for (int e = wt; e < G * D; e += 128)
+          store_elem(static_cast<TQ*>(p.out) +
+                         (static_cast<int64_t>(cur.s) * p.num_heads + cur.kvh * G) * D + e,
+                     0.f);
+        continue;
+      }
+      if (cur.kind != 2) continue;
+      // this item's q terms are in the Q operand; prefetch the next item's q, which
+      // replaces them once this item's last S has been computed
+      const int knext = tile_item_from(k + 1);
+      if (knext < nitems) raw_q = load_q(sh_items[knext]);
+      named_sync(1, 128);  // sh_c of this item is complete
+      float cf[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) cf[h] = sh_c[h];
+      const int h0 = cur.kvh * G;
+      const int nparts = (cur.L + ps - 1) / ps;
+
+      for (int j = cur.pbeg; j < cur.pend && !aborted; ++j, ++pc) {
+        const int ntok = part_tokens(j, ps, cur.L);
+        const int nt = (ntok + TM - 1) / TM;
+        const int ob = pc & 1;
+        const uint32_t tO = tbase + lane_off + ob * NO;
+        float m[G], l[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          m[h] = -INFINITY;
+          l[h] = 0.f;
+        }
+        for (int i = 0; i < nt; ++i, ++g) {
+          const int st = g % NST;
+          // the next tile: in this partition, the next one, or the next item's first
+          const int32_t ent_next =
+              i + 1 < nt ? entry(k, j, i + 1)
+                         : (j + 1 < cur.pend ? entry(k, j + 1, 0)
+                                             : (knext < nitems
+                                                    ? entry(knext, sh_items[knext].pbeg, 0)
+                                                    : -1));
+          const bool valid = ent >= 0 && ent < p.num_blocks;
+          ent = ent_next;
+          if (!wg_wait(b32(bar_s_full[g & 1]), (g >> 1) & 1)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          float sv[NS];
+#pragma unroll
+          for (int c16 = 0; c16 < NS / 16; ++c16) {
+            float v16[16];
+            tmem_ld16(tS0 + (g & 1) * NS + c16 * 16, v16);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) sv[c16 * 16 + k] = v16[k];
+          }
+          tc_fence_before();
+          mbar_arrive(b32(bar_s_empty[g & 1]));
+          if (i == nt - 1 && j == cur.pend - 1 && knext < nitems) {
+            named_sync(1, 128);  // every thread has read this item's sh_c
+            store_q(raw_q);      // the last S of this item is done: the next item's q
+          }
+          float sc[G];
+          bool grow = false;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float a = sv[h];
+#pragma unroll
+            for (int t = 1; t < C::NQT; ++t) a += sv[t * G + h];
+            sc[h] = valid ? a * cf[h] : -INFINITY;
+            grow |= sc[h] > m[h] + kLazyMax;
+          }
+          // the running max moves only when a head's tile max passes it by more than
+          // kLazyMax (base 2); until then the weights stay below 2^kLazyMax
+          if (bar_red_or(1, 128, grow)) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float w = warp_max(sc[h]);
+              if (lane == 0) sh_red[wq][h] = w;
+            }
+            named_sync(1, 128);
+            bool moved = false;
+            float corr[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float tmax =
+                  fmaxf(fmaxf(sh_red[0][h], sh_red[1][h]), fmaxf(sh_red[2][h], sh_red[3][h]));
+              const float mn = tmax > m[h] + kLazyMax ? tmax : m[h];
+              corr[h] = exp2_safe(m[h], mn);
+              moved |= mn != m[h];
+              l[h] *= corr[h];
+              m[h] = mn;
+            }
+            if (moved && i > 0) {
+              // rescale O (thread = dim row) once the previous tile's p.V has landed
+              if (!wg_wait(b32(bar_p_empty[(g - 1) & 1]), ((g - 1) >> 1) & 1)) {
+                aborted = true;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int c16 = 0; c16 < NO / 16; ++c16) {
+                float o16[16];
+                tmem_ld16(tO + c16 * 16, o16);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) o16[k] *= corr[(c16 * 16 + k) % G];
+                tmem_st16(tO + c16 * 16, o16);
+              }
+            }
+          }
+          // weights, split into two e4m3 terms (hi, (p - hi) * 32)
+          uint32_t hiw[G / 4], low[G / 4];
+#pragma unroll
+          for (int h = 0; h < G; h += 2) {
+            const float p0 = exp2_safe(sc[h], m[h]), p1 = exp2_safe(sc[h + 1], m[h + 1]);
+            l[h] += p0;
+            l[h + 1] += p1;
+            const uint16_t hp = e4m3_pair(p0, p1);
+            float b1;
+            const float b0 = e4m3_pair_back(hp, b1);
+            const uint16_t lp = e4m3_pair((p0 - b0) * 32.f, (p1 - b1) * 32.f);
+            const int wi = h >> 2;
+            if (h & 2) {
+              hiw[wi] |= static_cast<uint32_t>(hp) << 16;
+              low[wi] |= static_cast<uint32_t>(lp) << 16;
+            } else {
+              hiw[wi] = hp;
+              low[wi] = lp;
+            }
+          }
+          if (g >= 2 && !wg_wait(b32(bar_p_empty[g & 1]), ((g >> 1) - 1) & 1)) {
+            aborted = true;
+            break;
+          }
+          uint8_t* pb = smem + C::POFF + (g & 1) * C::PBYTES + (trow >> 3) * C::PK_STRIDE +
+                        (trow & 7) * 16;
+          if constexpr (G == 8) {
+            *reinterpret_cast<uint4*>(pb) = make_uint4(hiw[0], hiw[1], low[0], low[1]);
+          } else {
+            *reinterpret_cast<uint4*>(pb) = make_uint4(hiw[0], hiw[1], hiw[2], hiw[3]);
+            *reinterpret_cast<uint4*>(pb + 128) = make_uint4(low[0], low[1], low[2], low[3]);
+          }
+          // rows that carry no token: V zeroed (rows of the last block past the end are
+          // landed by TMA, so wait for it first)
+          if ((i + 1) * TM > ntok && !wg_wait(b32(bar_full_v[st]), (g / NST) & 1)) {
+            aborted = true;
+            break;
+          }
+          if (!valid) {
+            uint4* vrow = reinterpret_cast<uint4*>(smem + st * C::STAGE + C::TILE + trow * 128);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) vrow[k] = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(b32(bar_p_full[g & 1]));
+
+          if (i == 0 && pending) {
+            // the previous partition's output, once this partition's first tile is
+            // under way
+            if (!epilogue(pend)) {
+              aborted = true;
+              break;
+            }
+            pending = false;
           }
         }
+        if (aborted) break;
+        // this partition's exp-sums over the 128 token rows; its output is read after
+        // the next partition's first tile
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float w = warp_sum(l[h]);
+          if (lane == 0) sh_sum[wq][h] = w;
+        }
+        named_sync(1, 128);
+        if (trow < G) {
+          sh_den[ob][trow] = sh_sum[0][trow] + sh_sum[1][trow] + sh_sum[2][trow] + sh_sum[3][trow];
+          sh_m[ob][trow] = m[trow];
+        }
+        pend = Pending{cur.s, h0, j, nparts, g - 1, ob};
+        pending = true;
       }
     }
+    if (pending && !aborted) {
+      named_sync(1, 128);  // sh_den / sh_m of the last partition are visible
+      if (!epilogue(pend)) aborted = true;
+    }
+    if (wt == 0) bulk_wait_all();  // the outputs are written before the CTA ends
   }
   allow_dependents();
   if (aborted) set_error(p.err, PA_DEVERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 3) {
     tc_fence_after();
     tmem_dealloc(tbase, C::kTmemCols);
   }
@@ -507,17 +746,44 @@ __global__ void __launch_bounds__(kTcThreads)
 template <typename TQ, int G, int BS, int NST>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st) {
   using C = TcCfg<TQ, G, BS, NST>;
-  const uint64_t rows = static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * BS;
-  if (rows > 0x7fffffffull) return cudaErrorInvalidValue;  // int32 row coordinates
+  const uint64_t cache_rows = static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * BS;
+  if (cache_rows > 0x7fffffffull) return cudaErrorInvalidValue;  // int32 row coordinates
   CUtensorMap tmk, tmv;
-  if (!make_cache_tensor_map(&tmk, p.k_cache, rows, C::D, BS, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
-      !make_cache_tensor_map(&tmv, p.v_cache, rows, C::D, BS, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
+  if (!make_cache_tensor_map(&tmk, p.k_cache, cache_rows, C::D, BS,
+                             CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
+      !make_cache_tensor_map(&tmv, p.v_cache, cache_rows, C::D, BS,
+                             CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
     return cudaErrorInvalidValue;
   constexpr auto kern = decode_tc_fp8_kernel<TQ, G, BS, NST>;
   cudaError_t e = ensure_smem_limit<kern>(C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_kv_heads, p.num_seqs, p.max_parts - p.part_base);
-  return launch_dependent(kern, grid, dim3(kTcThreads), C::SMEM, st, p, tmk, tmv);
+  // Persistent CTAs, kTcCtasPerSm per SM.  With few (sequence, kv head) rows the
+  // partitions are split into equal contiguous ranges (balanced); otherwise the CTAs
+  // walk items of up to 2048 tokens of consecutive partitions round-robin (each
+  // partition is still its own partial either way).
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    sms = 148;
+  const int parts = p.max_parts - p.part_base;
+  const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.num_kv_heads;
+  const int64_t slots = static_cast<int64_t>(kTcCtasPerSm) * sms;
+  const bool balanced = p.num_seqs <= 256 && rows <= kTcMaxItems - 1;
+  const int ppc = p.partition_size >= 2048 ? 1 : 2048 / p.partition_size;
+  const int64_t items = static_cast<int64_t>((parts + ppc - 1) / ppc) * rows;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  int64_t ctas;
+  if (balanced) {
+    const int64_t work = rows * parts;  // an upper bound of the partitions to split
+    ctas = work < slots ? work : slots;
+  } else {
+    // more CTAs when one would otherwise look at more than kTcMaxItems list positions
+    ctas = items < slots ? items : slots;
+    if (ctas * kTcMaxItems < items) ctas = (items + kTcMaxItems - 1) / kTcMaxItems;
+  }
+  if (ctas < 1) ctas = 1;
+  return launch_dependent(kern, dim3(static_cast<unsigned>(ctas)), dim3(kTcThreads), C::SMEM,
+                          st, p, tmk, tmv, ppc, static_cast<int>(items), balanced ? 1 : 0);
 }
 
 constexpr int kTcStages = 3;

@@ -135,3 +135,25 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 }
 
 }  // namespace pa
+
+namespace pa {
+// ---- bulk copies shared -> global (TMA engine), tracked as bulk groups ---------------
+// dst and src 16-byte aligned, bytes a multiple of 16.  The issuing thread is not held
+// up by the memory system: completion is waited for with the wait_group forms.
+__device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// every committed bulk copy of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every committed bulk copy of this thread is complete (its writes performed)
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+}  // namespace pa

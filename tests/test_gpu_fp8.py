@@ -217,3 +217,79 @@ def test_fp8_tensor_cores_out_of_range_table_entry(pa):
     torch.cuda.synchronize()
     assert pa.pa_device_error_read() == pa.DEVERR_TABLE
     assert torch.isfinite(out).all()
+
+
+def _random_codes(shape, seed, stream):
+    """e4m3 codes with magnitudes up to 30 (exponent field <= 11) and random signs;
+    no NaN codes.  Any such byte is a valid cache entry."""
+    g = np.random.default_rng([seed, stream])
+    return (g.integers(0, 0x60, shape) | (g.integers(0, 2, shape) << 7)).astype(np.uint8)
+
+
+def test_fp8_tensor_cores_several_partitions_per_cta(pa):
+    """A grid large enough that each CTA of the tensor-core kernel walks several
+    partitions (152 (sequence, kv head) rows of 8 partitions of 64 tokens: two
+    partitions per CTA under the library's rule), every partition still written as
+    its own partial and merged."""
+    S, Hq, Hkv, D, bs, ps = 19, 64, 8, 128, 16, 64
+    g = np.random.default_rng(15)
+    lens = np.concatenate([[512, 449, 1, 64, 65], g.integers(380, 513, S - 5)]).astype(np.int64)
+    NB = int(sum(-(-int(L) // bs) for L in lens)) + 3
+    kc, vc = _random_codes((NB, Hkv, bs, D), 15, 1), _random_codes((NB, Hkv, bs, D), 15, 2)
+    ks, vs = 1.0 / 64, 1.0 / 32
+    q = normal_fill((S, Hq, D), "bf16", 1.0, 15, 3)
+    tables = tables_from_order(lens, bs, g.permutation(NB).astype(np.int32),
+                               int(-(-lens.max() // bs)) + 1)
+    max_len = int(lens.max())
+    out = torch.full((S, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps), dtype=torch.uint8,
+                     device="cuda")
+    pa.pa_decode_attention_fp8(out, to_dev(q, "bf16"), torch.from_numpy(kc).cuda(),
+                               torch.from_numpy(vc).cuda(), torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens.astype(np.int32)).cuda(), 1 / math.sqrt(D),
+                               bs, Hkv, max_len, ks, vs, ps, ws)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    want = oatt.paged_decode_attention(to_f64(q, "bf16"), fp8.dequantize(kc, ks),
+                                       fp8.dequantize(vc, vs), tables, lens, 1 / math.sqrt(D),
+                                       bs, Hkv, "f64")
+    assert_close(out_f64(out), want, "bf16", "several partitions per CTA")
+
+
+def test_fp8_long_context_gqa_full_size(pa):
+    """The long-context GQA workload at full size on an fp8 cache (random codes, the
+    stated 512-token partitions, the library's launch), sampled against the oracle:
+    two (sequence, kv head) pairs exactly, every output finite."""
+    from workloads import CONFIGS, make_inputs
+    cfg = CONFIGS["gqa_long_bf16"]
+    inp = make_inputs(cfg, 0, pool=False)
+    lens = (inp.context_lens + 1).astype(np.int64)
+    S, Hq, Hkv, D, bs, NB = (cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads, cfg.head_dim,
+                             cfg.block_size, cfg.num_blocks)
+    width = int(-(-lens.max() // bs)) + 1
+    tables = tables_from_order(lens, bs, inp.free_order, width)
+    kc, vc = _random_codes((NB, Hkv, bs, D), 16, 1), _random_codes((NB, Hkv, bs, D), 16, 2)
+    ks, vs = 1.0 / 64, 1.0 / 32
+    max_len, ps = int(lens.max()), cfg.partition_size
+    out = torch.full((S, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps), dtype=torch.uint8,
+                     device="cuda")
+    kd, vd = torch.from_numpy(kc).cuda(), torch.from_numpy(vc).cuda()
+    pa.pa_decode_attention_fp8(out, to_dev(inp.q, "bf16"), kd, vd, torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens.astype(np.int32)).cuda(), cfg.scale, bs, Hkv,
+                               max_len, ks, vs, ps, ws)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    got = out_f64(out)
+    assert np.isfinite(got).all()
+    G = Hq // Hkv
+    for s_, g_ in ((int(np.argmin(lens)), 0), (int(np.argmax(lens)), Hkv - 1)):
+        nb = int(-(-lens[s_] // bs))
+        blocks = tables[s_, :nb]
+        sub_k = fp8.dequantize(kc[blocks, g_:g_ + 1], ks)
+        sub_v = fp8.dequantize(vc[blocks, g_:g_ + 1], vs)
+        want = oatt.paged_decode_attention(
+            to_f64(inp.q[s_:s_ + 1, g_ * G:(g_ + 1) * G], "bf16"), sub_k, sub_v,
+            np.arange(nb, dtype=np.int32)[None, :], lens[s_:s_ + 1], cfg.scale, bs, 1, "f64")
+        assert_close(got[s_:s_ + 1, g_ * G:(g_ + 1) * G], want, "bf16",
+                     f"sequence {s_}, kv head {g_}")
