@@ -30,7 +30,7 @@ struct DecodeParams {
   int num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq;
   int64_t num_blocks;
   int max_seq_len, partition_size, max_parts;
-  float* ws_o;  // [S, Hq, P, D]  normalised partial outputs
+  float* ws_o;  // [P, S, Hq, D]  normalised partial outputs, see o_index
   float* ws_m;  // [P, S, Hq]     partition max (base-2 logits), see ml_index
   float* ws_l;  // [P, S, Hq]     partition exp-sum
   uint32_t* err;
@@ -54,6 +54,11 @@ struct DecodeParams {
 // heads are contiguous (and can be written with one bulk copy).
 __device__ __forceinline__ int64_t ml_index(const DecodeParams& p, int64_t row, int part) {
   return static_cast<int64_t>(part) * p.num_seqs * p.num_heads + row;
+}
+// Offset of the partial output row (query row, partition) in ws_o, partition-major
+// [P, S * Hq, D] like ws_m / ws_l.
+__device__ __forceinline__ int64_t o_index(const DecodeParams& p, int64_t row, int part) {
+  return ml_index(p, row, part) * p.head_dim;
 }
 
 // The sequence grid row y serves; -1 (reported) for an order entry out of range.

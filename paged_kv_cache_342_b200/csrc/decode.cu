@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
     const int64_t mstride = static_cast<int64_t>(p.num_seqs) * p.num_heads;
     const float* mrow = p.ws_m + row;  // partition pi at mrow[pi * mstride]
     const float* lrow = p.ws_l + row;
-    const float* orow = p.ws_o + static_cast<int64_t>(row) * p.max_parts * D + lane * DPL;
+    const float* orow = p.ws_o + static_cast<int64_t>(row) * D + lane * DPL;  // pi: + pi*mstride*D
     for (int i = wsub; i < nparts; i += U * wpr) {
       float mv[U], lv[U], o[U][DPL];
 #pragma unroll
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
         if (pi < nparts) {
           mv[u] = mrow[pi * mstride];
           lv[u] = lrow[pi * mstride];
-          load_lane<DPL>(orow + static_cast<int64_t>(pi) * D, o[u]);
+          load_lane<DPL>(orow + pi * mstride * D, o[u]);
         } else {
           mv[u] = -INFINITY;
           lv[u] = 0.f;

@@ -421,8 +421,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
     if (nparts == 1) {
       store_elem(static_cast<TQ*>(p.out) + row * D + d, o);
     } else {
-      const int64_t prow = row * p.max_parts + part;
-      p.ws_o[prow * D + d] = o;
+      p.ws_o[o_index(p, row, part) + d] = o;
       if (d == 0) {
         p.ws_m[ml_index(p, row, part)] = M;
         p.ws_l[ml_index(p, row, part)] = den;

@@ -163,6 +163,7 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
   __shared__ float sh_red[4][G];     // per-warp maxima of the softmax warpgroup
   __shared__ float sh_sum[4][G];     // per-warp exp-sums of the softmax warpgroup
   __shared__ float sh_den[2][G], sh_m[2][G];  // per O buffer: exp-sums and maxima
+  __shared__ float sh_f[2][G];                // per O buffer: v_scale / exp-sum (0 if none)
   __shared__ TcItem sh_items[kTcMaxItems];    // this CTA's work, in order
   __shared__ int sh_nitems;
 
@@ -502,9 +503,7 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
       uint8_t* stg = smem + C::SOFF;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float den = sh_den[e.ob][h];
-        const float o = ov[h] + ov[G + h] * (1.f / 32.f);
-        const float val = den > 0.f ? o * p.v_scale * __frcp_rn(den) : 0.f;
+        const float val = (ov[h] + ov[G + h] * (1.f / 32.f)) * sh_f[e.ob][h];
         if (e.nparts == 1) store_elem(reinterpret_cast<TQ*>(stg) + h * D + trow, val);
         else reinterpret_cast<float*>(stg)[h * D + trow] = val;
       }
@@ -521,9 +520,7 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
         if (e.nparts == 1) {
           bulk_s2g(static_cast<TQ*>(p.out) + row0 * D, sa, G * D * sizeof(TQ));
         } else {
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-            bulk_s2g(p.ws_o + ((row0 + h) * p.max_parts + e.j) * D, sa + h * 512, 512);
+          bulk_s2g(p.ws_o + o_index(p, row0, e.j), sa, G * 512);  // G contiguous rows
           bulk_s2g(p.ws_m + ml_index(p, row0, e.j), sa + G * 512, G * 4);
           bulk_s2g(p.ws_l + ml_index(p, row0, e.j), sa + G * 512 + G * 4, G * 4);
         }
@@ -720,8 +717,10 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
         }
         named_sync(1, 128);
         if (trow < G) {
-          sh_den[ob][trow] = sh_sum[0][trow] + sh_sum[1][trow] + sh_sum[2][trow] + sh_sum[3][trow];
+          const float den = sh_sum[0][trow] + sh_sum[1][trow] + sh_sum[2][trow] + sh_sum[3][trow];
+          sh_den[ob][trow] = den;
           sh_m[ob][trow] = m[trow];
+          sh_f[ob][trow] = den > 0.f ? p.v_scale / den : 0.f;
         }
         pend = Pending{cur.s, h0, j, nparts, g - 1, ob};
         pending = true;
