@@ -173,18 +173,110 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
   }
 }
 
+// The same merge for partials written sparsely: a partition kernel that runs several
+// consecutive partitions of a row in one CTA combines them itself (by the same rule)
+// and leaves one partial for the range, in its first slot; its other slots hold an
+// empty partial (exp-sum 0).  One warp per row: the lanes read the row's maxima and
+// exp-sums 256 slots at a time (eight per lane in flight), list the slots with a
+// non-zero exp-sum in shared memory, and only those partial outputs are read, eight
+// in flight.  Any mix of full and empty slots gives the dense merge's result.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) merge_sparse_kernel(const DecodeParams p) {
+  constexpr int DPL = D / 32;
+  constexpr int kWin = 256;  // slots examined per window
+  constexpr int U = 8;       // partial outputs in flight per warp
+  __shared__ int sh_slot[4][kWin];
+  __shared__ float sh_mv[4][kWin], sh_lv[4][kWin];
+  grid_dependency_wait();  // the partials of the partition kernel before this one
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + warp;
+  if (row >= p.num_seqs * p.num_heads) return;  // (no block-wide barrier below)
+  const int L = checked_len(p, row / p.num_heads, false);
+  const int nparts = L > 0 ? (L + p.partition_size - 1) / p.partition_size : 1;
+  if (nparts <= 1) return;
+  const int64_t mstride = static_cast<int64_t>(p.num_seqs) * p.num_heads;
+  float acc[DPL];
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) acc[j] = 0.f;
+  float den = 0.f, M = -INFINITY;
+  for (int w0 = 0; w0 < nparts; w0 += kWin) {
+    float mv[kWin / 32], lv[kWin / 32];
+#pragma unroll
+    for (int k = 0; k < kWin / 32; ++k) {
+      const int pi = w0 + k * 32 + lane;
+      mv[k] = pi < nparts ? p.ws_m[pi * mstride + row] : -INFINITY;
+      lv[k] = pi < nparts ? p.ws_l[pi * mstride + row] : 0.f;
+    }
+    int n = 0;
+    float mx = M;
+#pragma unroll
+    for (int k = 0; k < kWin / 32; ++k) {
+      const bool keep = lv[k] > 0.f;
+      const uint32_t b = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const int at = n + __popc(b & ((1u << lane) - 1u));
+        sh_slot[warp][at] = w0 + k * 32 + lane;
+        sh_mv[warp][at] = mv[k];
+        sh_lv[warp][at] = lv[k];
+        mx = fmaxf(mx, mv[k]);
+      }
+      n += __popc(b);
+    }
+    mx = warp_max(mx);
+    const float c = exp2_safe(M, mx);
+    den *= c;
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) acc[j] *= c;
+    M = mx;
+    __syncwarp();
+    for (int b0 = 0; b0 < n; b0 += U) {
+      float o[U][DPL], w[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int at = b0 + u;
+        if (at < n) {
+          w[u] = sh_lv[warp][at] * exp2_safe(sh_mv[warp][at], M);
+          load_lane<DPL>(p.ws_o + (sh_slot[warp][at] * mstride + row) * D + lane * DPL, o[u]);
+        } else {
+          w[u] = 0.f;
+#pragma unroll
+          for (int j = 0; j < DPL; ++j) o[u][j] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        den += w[u];
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w[u], o[u][j], acc[j]);
+      }
+    }
+    __syncwarp();  // the list is read before the next window overwrites it
+  }
+  T* out = static_cast<T*>(p.out) + static_cast<int64_t>(row) * D + lane * DPL;
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) store_elem(out + j, acc[j] * inv);
+}
+
 // dependent: launched to overlap the tail of the partition kernel just before it on
 // the stream (not after an event wait, which must hold in full)
 template <typename T, int D>
 cudaError_t launch_merge_d(const DecodeParams& p, int grid, int wpr, bool dependent,
-                           cudaStream_t st) {
+                           bool sparse, cudaStream_t st) {
+  if (sparse) {
+    const int g4 = (p.num_seqs * p.num_heads + 3) / 4;
+    if (dependent) return launch_dependent(merge_sparse_kernel<T, D>, dim3(g4), dim3(128), 0, st, p);
+    merge_sparse_kernel<T, D><<<g4, 128, 0, st>>>(p);
+    return cudaGetLastError();
+  }
   if (dependent) return launch_dependent(merge_kernel<T, D>, dim3(grid), dim3(256), 0, st, p, wpr);
   merge_kernel<T, D><<<grid, 256, 0, st>>>(p, wpr);
   return cudaGetLastError();
 }
 
+// sparse: the partials come from a kernel that combines consecutive partitions itself
 template <typename T>
-cudaError_t launch_merge(const DecodeParams& p, bool dependent, cudaStream_t st) {
+cudaError_t launch_merge(const DecodeParams& p, bool dependent, bool sparse, cudaStream_t st) {
   // warps per row: enough that each walks at most ~32 partitions
   int wpr = 1;
   while (wpr < 8 && p.max_parts > 32 * wpr) wpr *= 2;
@@ -192,9 +284,9 @@ cudaError_t launch_merge(const DecodeParams& p, bool dependent, cudaStream_t st)
   const int rows_per_cta = 8 / wpr;
   const int grid = (rows + rows_per_cta - 1) / rows_per_cta;
   switch (p.head_dim) {
-    case 64: return launch_merge_d<T, 64>(p, grid, wpr, dependent, st);
-    case 128: return launch_merge_d<T, 128>(p, grid, wpr, dependent, st);
-    case 256: return launch_merge_d<T, 256>(p, grid, wpr, dependent, st);
+    case 64: return launch_merge_d<T, 64>(p, grid, wpr, dependent, sparse, st);
+    case 128: return launch_merge_d<T, 128>(p, grid, wpr, dependent, sparse, st);
+    case 256: return launch_merge_d<T, 256>(p, grid, wpr, dependent, sparse, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -535,7 +627,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     }
     joined = side;
   }
-  if (fp8 && tc_fp8_eligible(group, head_dim, block_size)) {
+  const bool tc = fp8 && tc_fp8_eligible(group, head_dim, block_size);
+  if (tc) {
     e = launch_decode_tc_fp8(p, dtype, st);
   } else if (fp8 && mma_fp8_eligible(group, block_size)) {
     e = launch_decode_mma_fp8(p, dtype, st);
@@ -557,9 +650,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   }
   if (ws.parts > 1) {
     const bool dependent = joined == nullptr;
-    e = dtype == PA_F32    ? launch_merge<float>(p, dependent, st)
-        : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, dependent, st)
-                           : launch_merge<__half>(p, dependent, st);
+    e = dtype == PA_F32    ? launch_merge<float>(p, dependent, tc, st)
+        : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, dependent, tc, st)
+                           : launch_merge<__half>(p, dependent, tc, st);
     if (e != cudaSuccess) {
       note_cuda_error(e);
       return PA_ERR_CUDA;

@@ -163,7 +163,10 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
   __shared__ float sh_red[4][G];     // per-warp maxima of the softmax warpgroup
   __shared__ float sh_sum[4][G];     // per-warp exp-sums of the softmax warpgroup
   __shared__ float sh_den[2][G], sh_m[2][G];  // per O buffer: exp-sums and maxima
-  __shared__ float sh_f[2][G];                // per O buffer: v_scale / exp-sum (0 if none)
+  // an item's partitions combined so far (per head): maximum and exp-sum; the factors
+  // that bring the running output and the newest partition to the common maximum; at
+  // the item's end, v_scale / exp-sum (0 if none)
+  __shared__ float sh_run_m[G], sh_run_l[G], sh_c_old[G], sh_c_new[G], sh_fin[G];
   __shared__ TcItem sh_items[kTcMaxItems];    // this CTA's work, in order
   __shared__ int sh_nitems;
 
@@ -268,6 +271,9 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
   const uint32_t tbase = tmem_base_sm;
   const int nitems = sh_nitems;
   bool aborted = false;
+  // The merge after this kernel may be scheduled once every CTA has got here: its
+  // CTAs then take only what this grid leaves free, and wait for its writes.
+  allow_dependents();
 
   if (warp == 0 || warp == 3) {
     // ------------------------------------------------------------------ producers
@@ -479,50 +485,77 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
                          (j * ps + t) / BS)
                  : -1;
     };
-    // a partition's output, read from O buffer ob once its last p.V (tile g_last)
-    // has landed (the partition's exp-sums and maxima are in sh_den / sh_m [ob]); it
-    // goes out through the staging buffer by bulk copies issued by one thread, so no
-    // thread of the warpgroup waits on a global store
+    // A partition's output, read from O buffer ob once its last p.V (tile g_last)
+    // has landed (the partition's exp-sums and maxima are in sh_den / sh_m [ob]), is
+    // combined with the item's earlier partitions by the log-sum-exp rule: per head,
+    // M = max(m_run, m_j), o_run = o_run 2^(m_run - M) + o_j 2^(m_j - M), and the same
+    // for the exp-sums (thread = dim row; o_run is kept, as float rows, in the staging
+    // buffer the partial leaves from).  After the item's last partition the combined
+    // partial goes out by bulk copies issued by one thread: into the slot of the item's
+    // first partition (the item's other slots get an empty partial: exp-sum 0, maximum
+    // -inf), or, for a sequence of one partition, as the output rows.
+    // bits: 1 = O buffer, 2 = the item's last partition, 4 = a sequence of one partition
     struct Pending {
-      int s, h0, j, nparts, g_last, ob;
+      int s, h0, j, pbeg, g_last, bits;
     };
     auto epilogue = [&](const Pending& e) -> bool {
       if (!wg_wait(b32(bar_p_empty[e.g_last & 1]), (e.g_last >> 1) & 1)) return false;
       tc_fence_after();
+      const int ob = e.bits & 1;
+      const bool first = e.j == e.pbeg, last = (e.bits & 2) != 0, single = (e.bits & 4) != 0;
       float ov[NO];
 #pragma unroll
       for (int c16 = 0; c16 < NO / 16; ++c16) {
         float o16[16];
-        tmem_ld16(tbase + lane_off + e.ob * NO + c16 * 16, o16);
+        tmem_ld16(tbase + lane_off + ob * NO + c16 * 16, o16);
 #pragma unroll
         for (int k = 0; k < 16; ++k) ov[c16 * 16 + k] = o16[k];
       }
       tc_fence_before();  // O read before a later p.V overwrites it
-      if (wt == 0) bulk_wait_read_all();  // the previous output has left the staging buffer
+      if (trow < G) {
+        const float mj = sh_m[ob][trow], lj = sh_den[ob][trow];
+        const float mo = first ? -INFINITY : sh_run_m[trow];
+        const float lo = first ? 0.f : sh_run_l[trow];
+        const float mn = fmaxf(mo, mj);
+        const float co = exp2_safe(mo, mn), cn = exp2_safe(mj, mn);
+        const float ln = lo * co + lj * cn;
+        sh_c_old[trow] = co;
+        sh_c_new[trow] = cn;
+        sh_run_m[trow] = mn;
+        sh_run_l[trow] = ln;
+        if (last) sh_fin[trow] = ln > 0.f ? p.v_scale / ln : 0.f;
+      }
+      const int64_t row0 = static_cast<int64_t>(e.s) * p.num_heads + e.h0;
+      if (!first && wt < 2 * G)  // this partition's slot holds no partial of its own
+        (wt < G ? p.ws_m : p.ws_l)[ml_index(p, row0 + (wt % G), e.j)] = wt < G ? -INFINITY : 0.f;
+      if (first && wt == 0) bulk_wait_read_all();  // the previous output has left staging
       named_sync(1, 128);
       uint8_t* stg = smem + C::SOFF;
+      float* o_run = reinterpret_cast<float*>(stg) + trow;  // head h at o_run[h * D]
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float val = (ov[h] + ov[G + h] * (1.f / 32.f)) * sh_f[e.ob][h];
-        if (e.nparts == 1) store_elem(reinterpret_cast<TQ*>(stg) + h * D + trow, val);
-        else reinterpret_cast<float*>(stg)[h * D + trow] = val;
+        const float oj = (ov[h] + ov[G + h] * (1.f / 32.f)) * sh_c_new[h];
+        const float on = first ? oj : fmaf(o_run[h * D], sh_c_old[h], oj);
+        if (!last) o_run[h * D] = on;
+        else if (single) store_elem(reinterpret_cast<TQ*>(stg) + h * D + trow, on * sh_fin[h]);
+        else o_run[h * D] = on * sh_fin[h];
       }
-      if (e.nparts > 1 && trow < G) {
+      if (!last) return true;
+      if (!single && trow < G) {
         float* ml = reinterpret_cast<float*>(stg + G * 512);
-        ml[trow] = sh_m[e.ob][trow];
-        ml[G + trow] = sh_den[e.ob][trow];
+        ml[trow] = sh_run_m[trow];
+        ml[G + trow] = sh_run_l[trow];
       }
       fence_proxy_async_smem();
       named_sync(1, 128);
       if (wt == 0) {
         const uint32_t sa = base + C::SOFF;
-        const int64_t row0 = static_cast<int64_t>(e.s) * p.num_heads + e.h0;
-        if (e.nparts == 1) {
+        if (single) {
           bulk_s2g(static_cast<TQ*>(p.out) + row0 * D, sa, G * D * sizeof(TQ));
         } else {
-          bulk_s2g(p.ws_o + o_index(p, row0, e.j), sa, G * 512);  // G contiguous rows
-          bulk_s2g(p.ws_m + ml_index(p, row0, e.j), sa + G * 512, G * 4);
-          bulk_s2g(p.ws_l + ml_index(p, row0, e.j), sa + G * 512 + G * 4, G * 4);
+          bulk_s2g(p.ws_o + o_index(p, row0, e.pbeg), sa, G * 512);  // G contiguous rows
+          bulk_s2g(p.ws_m + ml_index(p, row0, e.pbeg), sa + G * 512, G * 4);
+          bulk_s2g(p.ws_l + ml_index(p, row0, e.pbeg), sa + G * 512 + G * 4, G * 4);
         }
         bulk_commit();
       }
@@ -598,10 +631,6 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
           }
           tc_fence_before();
           mbar_arrive(b32(bar_s_empty[g & 1]));
-          if (i == nt - 1 && j == cur.pend - 1 && knext < nitems) {
-            named_sync(1, 128);  // every thread has read this item's sh_c
-            store_q(raw_q);      // the last S of this item is done: the next item's q
-          }
           float sc[G];
           bool grow = false;
 #pragma unroll
@@ -611,6 +640,10 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
             for (int t = 1; t < C::NQT; ++t) a += sv[t * G + h];
             sc[h] = valid ? a * cf[h] : -INFINITY;
             grow |= sc[h] > m[h] + kLazyMax;
+          }
+          if (i == nt - 1 && j == cur.pend - 1 && knext < nitems) {
+            named_sync(1, 128);  // every thread has read this item's sh_c
+            store_q(raw_q);      // the last S of this item is done: the next item's q
           }
           // the running max moves only when a head's tile max passes it by more than
           // kLazyMax (base 2); until then the weights stay below 2^kLazyMax
@@ -717,12 +750,11 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
         }
         named_sync(1, 128);
         if (trow < G) {
-          const float den = sh_sum[0][trow] + sh_sum[1][trow] + sh_sum[2][trow] + sh_sum[3][trow];
-          sh_den[ob][trow] = den;
+          sh_den[ob][trow] = sh_sum[0][trow] + sh_sum[1][trow] + sh_sum[2][trow] + sh_sum[3][trow];
           sh_m[ob][trow] = m[trow];
-          sh_f[ob][trow] = den > 0.f ? p.v_scale / den : 0.f;
         }
-        pend = Pending{cur.s, h0, j, nparts, g - 1, ob};
+        pend = Pending{cur.s, h0, j, cur.pbeg, g - 1,
+                       ob | (j + 1 == cur.pend ? 2 : 0) | (nparts == 1 ? 4 : 0)};
         pending = true;
       }
     }
@@ -732,7 +764,6 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
     }
     if (wt == 0) bulk_wait_all();  // the outputs are written before the CTA ends
   }
-  allow_dependents();
   if (aborted) set_error(p.err, PA_DEVERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
