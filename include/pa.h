@@ -155,11 +155,14 @@ int pa_swap_blocks(void* dst_k, void* dst_v, int64_t dst_num_blocks, const void*
 /*
  * pa_decode_workspace_bytes - scratch bytes pa_decode_attention needs.
  * P = ceil(max_seq_len / partition_size) partitions per sequence; when P > 1 the
- * workspace holds float32 partial outputs [num_seqs, num_heads, P, head_dim] and
- * float32 max / exp-sum pairs [num_seqs, num_heads, P] each (the max is the one the
+ * workspace holds float32 partial outputs [P, num_seqs, num_heads, head_dim] and
+ * float32 maxima and exp-sums [P, num_seqs, num_heads] (the max is the one the
  * partition's weights were taken against; it may trail the true maximum logit by up
- * to 8 in base 2, and the merge uses each pair as a whole).  Returns 0 when P <= 1
- * (no merge needed) and 0 for invalid sizes.
+ * to 8 in base 2, and the merge uses each pair as a whole).  A kernel that computes
+ * several consecutive partitions of a row may combine them itself and leave one
+ * partial in the first one's slot, the others with exp-sum 0.  The contents need no
+ * initialisation and are not kept between calls.  Returns 0 when P <= 1 (no merge
+ * needed) and 0 for invalid sizes.
  */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_seq_len,
                                  int partition_size);

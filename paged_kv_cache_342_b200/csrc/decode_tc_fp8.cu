@@ -795,9 +795,27 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st) {
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     sms = 148;
+  // CTAs resident per SM: two are planned for (one if the kernel's registers or shared
+  // memory did not allow two), from the kernel's attributes and the SM's budgets
+  static const int per_sm = [] {
+    cudaFuncAttributes fa{};
+    int d = 0, smem_sm = 0, reserved = 0, regs_sm = 0;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || cudaGetDevice(&d) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, d) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, d) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, d) != cudaSuccess)
+      return 1;
+    const size_t smem_cta = fa.sharedSizeBytes + C::SMEM + static_cast<size_t>(reserved);
+    const int regs_cta = (fa.numRegs * 32 + 255) / 256 * 256 * (kTcThreads / 32);
+    int n = static_cast<int>(static_cast<size_t>(smem_sm) / smem_cta);
+    if (regs_cta > 0 && regs_sm / regs_cta < n) n = regs_sm / regs_cta;
+    return n < 1 ? 1 : (n > kTcCtasPerSm ? kTcCtasPerSm : n);
+  }();
   const int parts = p.max_parts - p.part_base;
   const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.num_kv_heads;
-  const int64_t slots = static_cast<int64_t>(kTcCtasPerSm) * sms;
+  const int64_t slots = static_cast<int64_t>(per_sm) * sms;
   const bool balanced = p.num_seqs <= 256 && rows <= kTcMaxItems - 1;
   const int ppc = p.partition_size >= 2048 ? 1 : 2048 / p.partition_size;
   const int64_t items = static_cast<int64_t>((parts + ppc - 1) / ppc) * rows;

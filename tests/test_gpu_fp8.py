@@ -228,9 +228,9 @@ def _random_codes(shape, seed, stream):
 
 def test_fp8_tensor_cores_several_partitions_per_cta(pa):
     """A grid large enough that each CTA of the tensor-core kernel walks several
-    partitions (152 (sequence, kv head) rows of 8 partitions of 64 tokens: two
-    partitions per CTA under the library's rule), every partition still written as
-    its own partial and merged."""
+    partitions (152 (sequence, kv head) rows of 8 partitions of 64 tokens: items of
+    consecutive partitions, round-robin), each partition computed on its own and
+    combined with its item's others before the merge."""
     S, Hq, Hkv, D, bs, ps = 19, 64, 8, 128, 16, 64
     g = np.random.default_rng(15)
     lens = np.concatenate([[512, 449, 1, 64, 65], g.integers(380, 513, S - 5)]).astype(np.int64)
@@ -254,6 +254,42 @@ def test_fp8_tensor_cores_several_partitions_per_cta(pa):
                                        fp8.dequantize(vc, vs), tables, lens, 1 / math.sqrt(D),
                                        bs, Hkv, "f64")
     assert_close(out_f64(out), want, "bf16", "several partitions per CTA")
+
+
+def test_fp8_tensor_cores_balanced_split_any_workspace(pa):
+    """Few (sequence, kv head) rows: the tensor-core kernel cuts all partitions into
+    equal ranges (CTAs combine each range's partitions and leave one partial per
+    range; the merge skips the empty slots).  The workspace needs no initialisation:
+    calls on a workspace of 0xff bytes, of zeros, and right after another call give
+    the same bits, and match the oracle."""
+    S, Hq, Hkv, D, bs, ps = 6, 64, 8, 128, 16, 128
+    lens = np.array([3000, 2500, 700, 129, 1, 4096], np.int64)
+    g = np.random.default_rng(21)
+    NB = int(sum(-(-int(L) // bs) for L in lens)) + 3
+    kc, vc = _random_codes((NB, Hkv, bs, D), 21, 1), _random_codes((NB, Hkv, bs, D), 21, 2)
+    ks, vs = 1.0 / 64, 1.0 / 32
+    q = normal_fill((S, Hq, D), "f16", 1.0, 21, 3)
+    tables = tables_from_order(lens, bs, g.permutation(NB).astype(np.int32),
+                               int(-(-lens.max() // bs)) + 1)
+    max_len = int(lens.max())
+    args = (to_dev(q, "f16"), torch.from_numpy(kc).cuda(), torch.from_numpy(vc).cuda(),
+            torch.from_numpy(tables).cuda(), torch.from_numpy(lens.astype(np.int32)).cuda(),
+            1 / math.sqrt(D), bs, Hkv, max_len, ks, vs, ps)
+    nbytes = pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps)
+    outs = []
+    for fill in (0xFF, 0x00, None):
+        ws = (torch.full((nbytes,), fill, dtype=torch.uint8, device="cuda") if fill is not None
+              else ws)  # None: the previous call's workspace as it was left
+        out = torch.full((S, Hq, D), float("nan"), dtype=torch.float16, device="cuda")
+        pa.pa_decode_attention_fp8(out, *args, ws)
+        torch.cuda.synchronize()
+        assert pa.pa_device_error_read() == 0
+        outs.append(out)
+    want = oatt.paged_decode_attention(to_f64(q, "f16"), fp8.dequantize(kc, ks),
+                                       fp8.dequantize(vc, vs), tables, lens, 1 / math.sqrt(D),
+                                       bs, Hkv, "f64")
+    assert_close(out_f64(outs[0]), want, "f16", "balanced split")
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
 def test_fp8_long_context_gqa_full_size(pa):
