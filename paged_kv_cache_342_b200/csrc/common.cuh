@@ -40,6 +40,9 @@ struct DecodeParams {
   const int32_t* chunk_members;  // [num_chunks, max_members] batch positions, -1 padded
   const int32_t* chunk_parts;    // [num_chunks] shared partitions of each chunk
   int max_members;
+  // the one-grid form of a grouped call: chunks, and shared partitions per chunk, in
+  // the grid before the sequences' own partitions
+  int num_chunks, group_zparts;
   float v_scale;  // output multiplier (the fp8 cache's V scale; 1 otherwise)
   int part_base;  // partition index of grid z = 0 in the per-sequence kernels
   // [S] or null: grid row y of the per-sequence kernels serves sequence seq_order[y]

@@ -8,8 +8,6 @@
 // pages in order" and "Measure memory use across requests" (the attention equation
 // is unchanged by paging).
 #include <cmath>
-#include <atomic>
-#include <mutex>
 
 #include "common.cuh"
 #include "decode_simt.cuh"
@@ -25,10 +23,8 @@ cudaError_t launch_decode_tc_fp8(const DecodeParams& p, int q_dtype, cudaStream_
 bool tc_fp8_eligible(int group, int head_dim, int block_size);
 cudaError_t launch_decode_mma_bf16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st);
-cudaError_t launch_decode_group_bf16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
-                                     cudaStream_t st);
-cudaError_t launch_decode_group_f16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
-                                    cudaStream_t st);
+cudaError_t launch_decode_grouped_bf16(const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_decode_grouped_f16(const DecodeParams& p, cudaStream_t st);
 
 namespace {
 
@@ -334,45 +330,6 @@ bool group_eligible(int dtype, int group, int head_dim, int block_size, int max_
          (block_size == 16 || block_size == 32);
 }
 
-// A side stream per device for the group kernel, so that it runs beside the
-// per-sequence kernel (they write disjoint partitions); fork and join through events.
-// Created on first use under the mutex; `ready` is published only once the stream
-// and both events exist, and a failed creation destroys what it made.
-struct SideStream {
-  std::mutex mu;
-  std::atomic<bool> ready{false};
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-};
-SideStream g_side[64];
-
-cudaError_t side_stream(int dev, SideStream** out) {
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  SideStream& s = g_side[dev];
-  if (!s.ready.load(std::memory_order_acquire)) {
-    std::lock_guard<std::mutex> lock(s.mu);
-    if (!s.ready.load(std::memory_order_relaxed)) {
-      cudaStream_t stream = nullptr;
-      cudaEvent_t fork = nullptr, join = nullptr;
-      cudaError_t e = cudaStreamCreateWithFlags(&stream, cudaStreamNonBlocking);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
-      if (e != cudaSuccess) {
-        if (join) cudaEventDestroy(join);
-        if (fork) cudaEventDestroy(fork);
-        if (stream) cudaStreamDestroy(stream);
-        return e;
-      }
-      s.stream = stream;
-      s.fork = fork;
-      s.join = join;
-      s.ready.store(true, std::memory_order_release);
-    }
-  }
-  *out = &s;
-  return cudaSuccess;
-}
-
 struct GroupArgs {
   const int32_t* prefix_parts;
   const int32_t* chunk_members;
@@ -591,44 +548,21 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
-  SideStream* joined = nullptr;              // the group kernel to wait for
-  std::unique_lock<std::mutex> side_lock;
-  // shared partitions of prefix groups first (only useful when sequences span
-  // several partitions); otherwise the per-sequence kernels do everything
+  const bool tc = fp8 && tc_fp8_eligible(group, head_dim, block_size);
   if (!fp8 && groups && groups->num_chunks > 0 && groups->max_chunk_parts > 0 && ws.parts > 1 &&
       group_eligible(dtype, group, head_dim, block_size, groups->max_members)) {
+    // Prefix groups (only useful when sequences span several partitions): one grid of
+    // the groups' shared partitions, then every sequence's own partitions
     p.prefix_parts = groups->prefix_parts;
     p.chunk_members = groups->chunk_members;
     p.chunk_parts = groups->chunk_parts;
     p.max_members = groups->max_members;
+    p.num_chunks = groups->num_chunks;
+    p.group_zparts = groups->max_chunk_parts < ws.parts ? groups->max_chunk_parts : ws.parts;
     // partitions below first_part belong to the groups for every sequence
     p.part_base = groups->first_part < ws.parts - 1 ? groups->first_part : ws.parts - 1;
-    const int zparts = groups->max_chunk_parts < ws.parts ? groups->max_chunk_parts : ws.parts;
-    int dev = 0;
-    SideStream* side = nullptr;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = side_stream(dev, &side);
-    if (e != cudaSuccess) {
-      note_cuda_error(e);
-      return PA_ERR_CUDA;
-    }
-    // the group kernel runs on the side stream while the caller's stream goes on to
-    // the per-sequence kernel; the caller's stream waits for it before the merge
-    side_lock = std::unique_lock<std::mutex>(side->mu);
-    e = cudaEventRecord(side->fork, st);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
-    if (e == cudaSuccess)
-      e = dtype == PA_BF16 ? launch_decode_group_bf16(p, groups->num_chunks, zparts, side->stream)
-                           : launch_decode_group_f16(p, groups->num_chunks, zparts, side->stream);
-    if (e == cudaSuccess) e = cudaEventRecord(side->join, side->stream);
-    if (e != cudaSuccess) {
-      note_cuda_error(e);
-      return PA_ERR_CUDA;
-    }
-    joined = side;
-  }
-  const bool tc = fp8 && tc_fp8_eligible(group, head_dim, block_size);
-  if (tc) {
+    e = dtype == PA_BF16 ? launch_decode_grouped_bf16(p, st) : launch_decode_grouped_f16(p, st);
+  } else if (tc) {
     e = launch_decode_tc_fp8(p, dtype, st);
   } else if (fp8 && mma_fp8_eligible(group, block_size)) {
     e = launch_decode_mma_fp8(p, dtype, st);
@@ -642,17 +576,14 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
         : dtype == PA_BF16 ? launch_decode_simt_bf16(p, gs, st)
                            : launch_decode_simt_f16(p, gs, st);
   }
-  if (e == cudaSuccess && joined) e = cudaStreamWaitEvent(st, joined->join, 0);
-  if (side_lock.owns_lock()) side_lock.unlock();
   if (e != cudaSuccess) {
     note_cuda_error(e);
     return PA_ERR_CUDA;
   }
   if (ws.parts > 1) {
-    const bool dependent = joined == nullptr;
-    e = dtype == PA_F32    ? launch_merge<float>(p, dependent, tc, st)
-        : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, dependent, tc, st)
-                           : launch_merge<__half>(p, dependent, tc, st);
+    e = dtype == PA_F32    ? launch_merge<float>(p, true, tc, st)
+        : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, true, tc, st)
+                           : launch_merge<__half>(p, true, tc, st);
     if (e != cudaSuccess) {
       note_cuda_error(e);
       return PA_ERR_CUDA;

@@ -152,9 +152,15 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 }
 
 // GROUP = false: one CTA per (sequence, 8*NT query heads of one kv head, partition).
-// GROUP = true : one CTA per (kv head, chunk of a prefix group, shared partition);
-//   the tile's columns are (member, head) pairs, member = column / group, and the
-//   partition's blocks - identical for every member - are read once for all of them.
+// GROUP = true : a grouped call in one flat grid of two kinds of work.  First the
+//   prefix groups' shared partitions, one CTA per (kv head, chunk of a group, shared
+//   partition) with kv head fastest: the tile's columns are (member, head) pairs,
+//   member = column / group, and the partition's blocks - identical for every member -
+//   are read once for all of them.  Then every sequence's own partitions, one CTA per
+//   (kv head, grid row - longest first when an order is given -, partition from
+//   part_base on), the columns the group's query heads of that kv head.  So the long
+//   shared partitions start first, the short own ones fill the end, and neither kind
+//   has a last wave of its own.
 // T = MMA operand type, TQ = query / output type, FP8 = e4m3 cache converted to T.
 template <typename T, typename TQ, int D, int BS, int NT, int NW, int NST, bool GROUP,
           bool FP8>
@@ -203,29 +209,58 @@ __global__ void __launch_bounds__(NW * 32)
       col_ok[threadIdx.x] = 1;
     }
   } else {
-    const int chunk = blockIdx.y;
-    kvh = blockIdx.x;
-    part = blockIdx.z;
-    if (part >= __ldg(p.chunk_parts + chunk)) return;
-    nparts = 2;  // a grouped partition is always one of several: write partials
-    tok_begin = part * ps;
-    tok_end = tok_begin + ps;
-    if (threadIdx.x < C::kHeads) {
-      const int c = threadIdx.x, mi = c / G;
-      const int m = mi < p.max_members ? __ldg(p.chunk_members + chunk * p.max_members + mi) : -1;
-      const bool member = m >= 0 && m < p.num_seqs;
-      col_row[c] = member ? m * p.num_heads + kvh * G + (c - mi * G) : -1;
-      col_ok[c] = member && part < group_parts(p, m, checked_len(p, m, false));
-    }
-    __syncthreads();
-    // blocks come from the table of the first member that owns this partition
-    table_seq = -1;
-    for (int c = 0; c < C::kHeads; ++c)
-      if (col_ok[c]) {
-        table_seq = col_row[c] / p.num_heads;
-        break;
+    int chunk = 0;
+    int b = blockIdx.x;
+    const int n_group = p.num_kv_heads * p.num_chunks * p.group_zparts;
+    kvh = b % p.num_kv_heads;
+    const bool own_item = b >= n_group;
+    if (!own_item) {
+      b /= p.num_kv_heads;
+      chunk = b % p.num_chunks;
+      part = b / p.num_chunks;
+    } else {
+      // a sequence's own partition: as the per-sequence kernel, heads of kv head kvh
+      b = (b - n_group) / p.num_kv_heads;
+      const int y = b % p.num_seqs, z = b / p.num_seqs;
+      const bool report = threadIdx.x == 0 && kvh == 0 && z == 0;
+      const int s = row_sequence(p, y, report);
+      if (s < 0) return;
+      part = p.part_base + z;
+      const int L = checked_len(p, s, report);
+      nparts = L > 0 ? (L + ps - 1) / ps : 1;
+      const int own = group_parts(p, s, L);
+      if (report && own < p.part_base) set_error(p.err, PA_DEVERR_GROUP);
+      if (part >= nparts || part < own) return;
+      tok_begin = part * ps;
+      tok_end = min(L, tok_begin + ps);
+      table_seq = s;
+      if (threadIdx.x < C::kHeads) {
+        col_row[threadIdx.x] = threadIdx.x < G ? s * p.num_heads + kvh * G + threadIdx.x : -1;
+        col_ok[threadIdx.x] = threadIdx.x < G ? 1 : 0;
       }
-    if (table_seq < 0) return;  // no member needs this partition
+    }
+    if (!own_item) {
+      if (part >= __ldg(p.chunk_parts + chunk)) return;
+      nparts = 2;  // a grouped partition is always one of several: write partials
+      tok_begin = part * ps;
+      tok_end = tok_begin + ps;
+      if (threadIdx.x < C::kHeads) {
+        const int c = threadIdx.x, mi = c / G;
+        const int m = mi < p.max_members ? __ldg(p.chunk_members + chunk * p.max_members + mi) : -1;
+        const bool member = m >= 0 && m < p.num_seqs;
+        col_row[c] = member ? m * p.num_heads + kvh * G + (c - mi * G) : -1;
+        col_ok[c] = member && part < group_parts(p, m, checked_len(p, m, false));
+      }
+      __syncthreads();
+      // blocks come from the table of the first member that owns this partition
+      table_seq = -1;
+      for (int c = 0; c < C::kHeads; ++c)
+        if (col_ok[c]) {
+          table_seq = col_row[c] / p.num_heads;
+          break;
+        }
+      if (table_seq < 0) return;  // no member needs this partition
+    }
   }
   __syncthreads();
   const int nblk = tok_end > tok_begin ? (tok_end - tok_begin + BS - 1) / BS : 0;

@@ -8,9 +8,11 @@ namespace {
 
 template <int D, int BS, int NT, bool GROUP>
 cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  // about 64 KiB of stages per CTA: warps with two stages each (1-4), then 2-4 stages
+  // about 64 KiB of stages per CTA: warps with two stages each (1-4), then 2-4 stages;
+  // about 16 KiB (one warp) for a grouped call, whose many short own partitions want
+  // small CTAs
   constexpr int kStage = 2 * BS * D * 2;
-  constexpr int kBudget = 65536;
+  constexpr int kBudget = GROUP ? 16384 : 65536;
   constexpr int kW = kBudget / (2 * kStage);
   constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
   constexpr int kRaw = kBudget / (NW * kStage);
@@ -28,10 +30,6 @@ cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   constexpr auto kern = decode_mma_kernel<__half, __half, D, BS, NT, NW, NST, GROUP, false>;
   cudaError_t e = ensure_smem_limit<kern>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  if constexpr (GROUP) {
-    kern<<<grid, NW * 32, C::kSmemBytes, st>>>(p, tmk, tmv);
-    return cudaGetLastError();
-  }
   return launch_dependent(kern, grid, dim3(NW * 32), C::kSmemBytes, st, p, tmk, tmv);
 }
 
@@ -66,13 +64,17 @@ cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st) {
   return by_shape<false>(p, nt, grid, st);
 }
 
-// Shared partitions of prefix groups: columns = max_members * group <= 16.
-cudaError_t launch_decode_group_f16(const DecodeParams& p, int num_chunks, int max_chunk_parts,
-                                   cudaStream_t st) {
+// A grouped call in one grid: the groups' shared partitions (p.num_chunks chunks,
+// p.group_zparts partitions each), then every sequence's own partitions from
+// p.part_base on; launched to overlap the kernel before it on the stream.
+cudaError_t launch_decode_grouped_f16(const DecodeParams& p, cudaStream_t st) {
   const int cols = p.max_members * (p.num_heads / p.num_kv_heads);
   const int nt = cols <= 8 ? 1 : 2;
-  dim3 grid(p.num_kv_heads, num_chunks, max_chunk_parts);
-  return by_shape<true>(p, nt, grid, st);
+  const int64_t n = static_cast<int64_t>(p.num_kv_heads) *
+                    (static_cast<int64_t>(p.num_chunks) * p.group_zparts +
+                     static_cast<int64_t>(p.num_seqs) * (p.max_parts - p.part_base));
+  if (n <= 0 || n > 0x7fffffffLL) return cudaErrorInvalidValue;
+  return by_shape<true>(p, nt, dim3(static_cast<unsigned>(n)), st);
 }
 
 }  // namespace pa
