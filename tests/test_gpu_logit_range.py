@@ -3,8 +3,10 @@ kernels distinguish: slow rises (block maxima a few units above the last max, wh
 lazy running max keeps without rescaling), steady rises that cross the lazy bound every
 other block, a sudden jump of 40 (base 2), a fall, and a flat stretch.  Every query
 head of a kv head shares one direction, so the trajectory is the same for all of them.
-Both kernels (CUDA cores for MHA, tensor cores for groups of 8), bf16 and fp8 caches,
-several partition sizes; compared with the float64 oracle on the stored values."""
+Every kernel (CUDA cores for MHA, tensor cores for groups of 8 and 16, on fp8 caches
+the tcgen05 kernel with its q split into two or three e4m3 terms and its P into two),
+bf16, f16 and fp8 caches, several partition sizes; compared with the float64 oracle on
+the stored values."""
 import math
 
 import numpy as np
@@ -74,6 +76,7 @@ CASES = [
     (16, 2, 128, 16, 64, (700, 333, 1, 97)),    # tensor cores, group 8
     (16, 2, 128, 16, 4096, (700, 333, 1, 97)),
     (16, 2, 128, 32, 128, (700, 161, 40)),      # tensor cores, block 32
+    (32, 2, 128, 16, 256, (700, 333, 1, 97)),   # tensor cores, group 16
 ]
 
 
@@ -98,26 +101,27 @@ def test_logit_trajectory_16bit_cache(pa, case, qdt):
     assert_close(out_f64(out), want, qdt, "logit trajectory")
 
 
+@pytest.mark.parametrize("qdt", ["bf16", "f16"])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"h{c[0]}/{c[1]}-b{c[3]}-p{c[4]}")
-def test_logit_trajectory_fp8_cache(pa, case):
+def test_logit_trajectory_fp8_cache(pa, case, qdt):
     Hq, Hkv, D, bs, ps, lens = case
     k, v, q, tables, scale = build(lens, Hq, Hkv, D, bs, 6)
     k_scale = float(np.abs(k).max()) / 448.0
     v_scale = 4.0 / 448.0
     kc, vc = fp8.quantize(k, k_scale), fp8.quantize(v, v_scale)
-    qs = round_to_storage(q, "bf16")
+    qs = round_to_storage(q, qdt)
     lens = np.asarray(lens, np.int64)
     S, max_len = lens.size, int(lens.max())
-    out = torch.full((S, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = torch.full((S, Hq, D), float("nan"), dtype=TORCH_DT[qdt], device="cuda")
     wsb = pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps)
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
-    pa.pa_decode_attention_fp8(out, to_dev(qs, "bf16"), torch.from_numpy(kc).cuda(),
+    pa.pa_decode_attention_fp8(out, to_dev(qs, qdt), torch.from_numpy(kc).cuda(),
                                torch.from_numpy(vc).cuda(), torch.from_numpy(tables).cuda(),
                                torch.from_numpy(lens.astype(np.int32)).cuda(), scale, bs, Hkv,
                                max_len, k_scale, v_scale, ps, ws if wsb else None)
     torch.cuda.synchronize()
     assert pa.pa_device_error_read() == 0
-    want = oatt.paged_decode_attention(to_f64(qs, "bf16"), fp8.dequantize(kc, k_scale),
+    want = oatt.paged_decode_attention(to_f64(qs, qdt), fp8.dequantize(kc, k_scale),
                                        fp8.dequantize(vc, v_scale), tables, lens, scale, bs,
                                        Hkv, "f64")
-    assert_close(out_f64(out), want, "bf16", "logit trajectory, fp8 cache")
+    assert_close(out_f64(out), want, qdt, "logit trajectory, fp8 cache")
