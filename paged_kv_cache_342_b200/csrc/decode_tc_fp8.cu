@@ -148,7 +148,6 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
     decode_tc_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, int ppc, int num_items,
                          int balanced) {
-  grid_dependency_wait();
   using C = TcCfg<TQ, G, BS, NST>;
   constexpr int TM = C::TM, NS = C::NS, NO = C::NO, BPT = C::BPT, D = C::D;
   constexpr unsigned FULL = 0xffffffffu;
@@ -198,6 +197,9 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
     tmem_alloc(smem_u32(&tmem_base_sm), C::kTmemCols);
     tmem_relinquish();
   }
+  // launched to overlap the end of the kernel before it on the stream: the set-up above
+  // touches no global memory; from here on everything may depend on that kernel
+  grid_dependency_wait();
   if (warp == 2 && balanced) {
     // Balanced split: every (sequence row, kv head) contributes its partitions; the
     // flat list of all partitions (row-major) is cut into gridDim.x equal ranges and
