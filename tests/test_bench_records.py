@@ -45,7 +45,8 @@ def test_kernel_hash_covers_the_decode_kernels_only(tmp_path, monkeypatch):
     assert bench.kernel_sources_sha() != h0
 
 
-@pytest.mark.parametrize("name", ["7b_bf16", "13b_fp16", "gqa_long_bf16", "prefix_cow_bf16"])
+@pytest.mark.parametrize("name", ["7b_bf16", "13b_fp16", "gqa_long_bf16", "prefix_cow_bf16",
+                                  "gqa_long_bf16+fp8_cache"])
 def test_records_are_consistent(name):
     rec = _records()[name]
     assert rec["read_bytes"] + rec["write_bytes"] > 0
