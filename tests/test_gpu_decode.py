@@ -226,6 +226,9 @@ GROUP_CASES = [
     ("bf16", 16, 2, 128, 16, 64, 200, [1, 20, 3], [3], 1),             # GQA 8 + 1 member
     ("f16", 4, 4, 256, 16, 64, 129, [1] * 11 + [40], [12], 8),         # 2 chunks
     ("bf16", 2, 2, 128, 16, 64, 64, [0, 0, 5], [3], 8),                 # tails of length 0
+    # a group beside two sequences of no group (their own prefixes): in the one grid the
+    # group's shared partitions, then every sequence's own partitions from partition 0
+    ("bf16", 8, 8, 128, 16, 64, 200, [3, 50, 0, 7, 130, 9], [4, 1, 1], 8),
 ]
 
 
