@@ -20,7 +20,7 @@ cudaError_t launch_decode_simt_f16(const DecodeParams& p, int gs, cudaStream_t s
 cudaError_t launch_decode_simt_fp8(const DecodeParams& p, int q_dtype, int gs, cudaStream_t st);
 cudaError_t launch_decode_mma_fp8(const DecodeParams& p, int q_dtype, cudaStream_t st);
 cudaError_t launch_decode_tc_fp8(const DecodeParams& p, int q_dtype, cudaStream_t st);
-bool tc_fp8_eligible(int group, int head_dim, int block_size);
+bool tc_fp8_eligible(int group, int head_dim, int block_size, int num_seqs, int num_kv_heads);
 cudaError_t launch_decode_mma_bf16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_grouped_bf16(const DecodeParams& p, cudaStream_t st);
@@ -551,7 +551,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
-  const bool tc = fp8 && tc_fp8_eligible(group, head_dim, block_size);
+  const bool tc = fp8 && tc_fp8_eligible(group, head_dim, block_size, num_seqs, num_kv_heads);
   if (!fp8 && groups && groups->num_chunks > 0 && groups->max_chunk_parts > 0 && ws.parts > 1 &&
       group_eligible(dtype, group, head_dim, block_size, groups->max_members)) {
     // Prefix groups (only useful when sequences span several partitions): one grid of

@@ -6,8 +6,10 @@
 // has to read scattered blocks"; "Where it bites": grouped-query attention and a
 // quantized cache stack with paging).
 //
-// Persistent CTAs (two per SM) walk a round-robin list of work items (sequence, kv
-// head, up to 2048 tokens of consecutive partitions); 8 warps:
+// Persistent CTAs (two per SM) each take an equal contiguous range of the flat list of
+// all partitions (few (sequence, kv head) rows: the shapes where this kernel is the
+// faster one), as work items (sequence, kv head, run of consecutive partitions);
+// 8 warps:
 //   warps 0, 3  walk the block table and bring each block's K (warp 0) and V (warp 3)
 //               rows in by TMA (128-byte rows, 128-byte swizzle) into stages of 128
 //               tokens; a K stage is refilled as soon as its S is computed, a V stage
@@ -43,7 +45,8 @@ namespace {
 
 constexpr int kTcThreads = 256;
 constexpr int kTcCtasPerSm = 2;
-constexpr int kTcMaxItems = 96;  // work items of one CTA (the launch ensures it)
+constexpr int kTcMaxItems = 96;  // work items of one CTA (at most one per row)
+constexpr int kTcMaxSeqs = 256;  // the split's per-row scratch (16 bytes each) in the P buffers
 
 template <typename TQ, int G, int BS, int NST>
 struct TcCfg {
@@ -73,7 +76,7 @@ struct TcCfg {
   static constexpr int SOFF = POFF + 2 * PBYTES;
   static constexpr int STBYTES = G * 512 + 2 * G * 4;
   static constexpr int SMEM = 1024 + SOFF + STBYTES;
-  static_assert(2 * PBYTES >= 256 * 16, "the P buffers hold the balanced list's scratch");
+  static_assert(2 * PBYTES >= kTcMaxSeqs * 16, "the P buffers hold the split's scratch");
   static constexpr uint32_t IDESC_S = idesc_e4m3(128, NS, false, false);
   static constexpr uint32_t IDESC_O = idesc_e4m3(128, NO, true, true);
   static_assert(G == 8 || G == 16, "head groups of 8 or 16");
@@ -117,37 +120,12 @@ __device__ __forceinline__ int part_tokens(int j, int ps, int L) {
 struct TcItem {
   int s, kvh, L, pbeg, pend, kind;
 };
-// Item idx of the list: chunk z of ppc partitions (outermost), grid row y (sequence
-// seq_order[y], longest first when an order is given), kv head (innermost).  Returns
-// the kind, 0 for nothing to do.  Bad order entries and lengths are reported once per
-// row (by the item of chunk 0, kv head 0).
-__device__ __forceinline__ int tc_item(const DecodeParams& p, int idx, int ppc, TcItem& it) {
-  const int rows = p.num_seqs * p.num_kv_heads;
-  const int z = idx / rows, r = idx - z * rows;
-  const int y = r / p.num_kv_heads;
-  it.kvh = r - y * p.num_kv_heads;
-  const bool report = z == 0 && it.kvh == 0;
-  it.kind = 0;
-  it.s = row_sequence(p, y, report);
-  if (it.s < 0) return 0;
-  it.L = checked_len(p, it.s, report);
-  const int ps = p.partition_size;
-  const int nparts = it.L > 0 ? (it.L + ps - 1) / ps : 1;
-  const int own = group_parts(p, it.s, it.L);
-  it.pbeg = max(own, p.part_base + z * ppc);
-  it.pend = min(nparts, p.part_base + (z + 1) * ppc);
-  if (it.pbeg >= it.pend) return 0;
-  it.kind = it.L > 0 ? 2 : 1;
-  return it.kind;
-}
-
 // Groups of 8 fit two CTAs per SM (shared memory), so registers are held to 128 per
 // thread; groups of 16 need more shared memory and run one CTA per SM.
 template <typename TQ, int G, int BS, int NST>
 __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
     decode_tc_fp8_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
-                         const __grid_constant__ CUtensorMap tmv, int ppc, int num_items,
-                         int balanced) {
+                         const __grid_constant__ CUtensorMap tmv) {
   using C = TcCfg<TQ, G, BS, NST>;
   constexpr int TM = C::TM, NS = C::NS, NO = C::NO, BPT = C::BPT, D = C::D;
   constexpr unsigned FULL = 0xffffffffu;
@@ -200,7 +178,7 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
   // launched to overlap the end of the kernel before it on the stream: the set-up above
   // touches no global memory; from here on everything may depend on that kernel
   grid_dependency_wait();
-  if (warp == 2 && balanced) {
+  if (warp == 2) {
     // Balanced split: every (sequence row, kv head) contributes its partitions; the
     // flat list of all partitions (row-major) is cut into gridDim.x equal ranges and
     // this CTA takes its range as runs of consecutive partitions.  Per sequence row:
@@ -253,19 +231,6 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
       }
       sh_nitems = n;
     }
-  } else if (warp == 2) {
-    // Round-robin: list positions blockIdx.x + k * gridDim.x (chunks of ppc
-    // partitions), evaluated 32 at a time and compacted
-    int n = 0;
-    for (int k0 = 0; k0 < kTcMaxItems; k0 += 32) {
-      const int idx = blockIdx.x + (k0 + lane) * gridDim.x;
-      TcItem it;
-      const bool keep = k0 + lane < kTcMaxItems && idx < num_items && tc_item(p, idx, ppc, it) != 0;
-      const uint32_t m = __ballot_sync(FULL, keep);
-      if (keep) sh_items[n + __popc(m & ((1u << lane) - 1u))] = it;
-      n += __popc(m);
-    }
-    if (lane == 0) sh_nitems = n;
   }
   tc_fence_before();
   __syncthreads();
@@ -789,10 +754,8 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st) {
   constexpr auto kern = decode_tc_fp8_kernel<TQ, G, BS, NST>;
   cudaError_t e = ensure_smem_limit<kern>(C::SMEM);
   if (e != cudaSuccess) return e;
-  // Persistent CTAs, kTcCtasPerSm per SM.  With few (sequence, kv head) rows the
-  // partitions are split into equal contiguous ranges (balanced); otherwise the CTAs
-  // walk items of up to 2048 tokens of consecutive partitions round-robin (each
-  // partition is still its own partial either way).
+  // Persistent CTAs, kTcCtasPerSm per SM; the partitions are split into equal
+  // contiguous ranges, one per CTA (callers check tc_fp8_eligible: few rows).
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
@@ -817,23 +780,12 @@ cudaError_t launch_tc(const DecodeParams& p, cudaStream_t st) {
   }();
   const int parts = p.max_parts - p.part_base;
   const int64_t rows = static_cast<int64_t>(p.num_seqs) * p.num_kv_heads;
+  if (p.num_seqs > kTcMaxSeqs || rows > kTcMaxItems - 1 || parts < 1) return cudaErrorInvalidValue;
   const int64_t slots = static_cast<int64_t>(per_sm) * sms;
-  const bool balanced = p.num_seqs <= 256 && rows <= kTcMaxItems - 1;
-  const int ppc = p.partition_size >= 2048 ? 1 : 2048 / p.partition_size;
-  const int64_t items = static_cast<int64_t>((parts + ppc - 1) / ppc) * rows;
-  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-  int64_t ctas;
-  if (balanced) {
-    const int64_t work = rows * parts;  // an upper bound of the partitions to split
-    ctas = work < slots ? work : slots;
-  } else {
-    // more CTAs when one would otherwise look at more than kTcMaxItems list positions
-    ctas = items < slots ? items : slots;
-    if (ctas * kTcMaxItems < items) ctas = (items + kTcMaxItems - 1) / kTcMaxItems;
-  }
-  if (ctas < 1) ctas = 1;
+  const int64_t work = rows * parts;  // an upper bound of the partitions to split
+  const int64_t ctas = work < slots ? work : slots;
   return launch_dependent(kern, dim3(static_cast<unsigned>(ctas)), dim3(kTcThreads), C::SMEM,
-                          st, p, tmk, tmv, ppc, static_cast<int>(items), balanced ? 1 : 0);
+                          st, p, tmk, tmv);
 }
 
 constexpr int kTcStages = 3;
@@ -858,8 +810,14 @@ cudaError_t by_group(const DecodeParams& p, cudaStream_t st) {
 
 }  // namespace
 
-bool tc_fp8_eligible(int group, int head_dim, int block_size) {
-  return head_dim == 128 && (group == 8 || group == 16) && (block_size == 16 || block_size == 32);
+// Shapes the kernel serves, and where it is the faster one: few (sequence, kv head)
+// rows, split evenly over every SM.  With many short rows the per-item set-up (q, the
+// pipeline's first tiles, the epilogue) outweighs what the tensor cores save, and the
+// mma.sync kernel, one CTA per (row, partition), was faster (GQA-8 with 512 sequences
+// of 128-2048 tokens: 110 against 118 us; 1024 log-normal sequences: 186 against 218 us).
+bool tc_fp8_eligible(int group, int head_dim, int block_size, int num_seqs, int num_kv_heads) {
+  return head_dim == 128 && (group == 8 || group == 16) && (block_size == 16 || block_size == 32) &&
+         num_seqs <= kTcMaxSeqs && static_cast<int64_t>(num_seqs) * num_kv_heads <= kTcMaxItems - 1;
 }
 
 cudaError_t launch_decode_tc_fp8(const DecodeParams& p, int q_dtype, cudaStream_t st) {

@@ -226,11 +226,11 @@ def _random_codes(shape, seed, stream):
     return (g.integers(0, 0x60, shape) | (g.integers(0, 2, shape) << 7)).astype(np.uint8)
 
 
-def test_fp8_tensor_cores_several_partitions_per_cta(pa):
-    """A grid large enough that each CTA of the tensor-core kernel walks several
-    partitions (152 (sequence, kv head) rows of 8 partitions of 64 tokens: items of
-    consecutive partitions, round-robin), each partition computed on its own and
-    combined with its item's others before the merge."""
+def test_fp8_many_rows_on_the_mma_kernel(pa):
+    """152 (sequence, kv head) rows of up to 8 partitions of 64 tokens: more rows than
+    the tcgen05 kernel takes (it serves few rows, split evenly over the SMs), so the
+    mma.sync tensor-core kernel runs it, one CTA per (row, partition), and the dense
+    merge combines the partitions."""
     S, Hq, Hkv, D, bs, ps = 19, 64, 8, 128, 16, 64
     g = np.random.default_rng(15)
     lens = np.concatenate([[512, 449, 1, 64, 65], g.integers(380, 513, S - 5)]).astype(np.int64)
@@ -254,6 +254,36 @@ def test_fp8_tensor_cores_several_partitions_per_cta(pa):
                                        fp8.dequantize(vc, vs), tables, lens, 1 / math.sqrt(D),
                                        bs, Hkv, "f64")
     assert_close(out_f64(out), want, "bf16", "several partitions per CTA")
+
+
+@pytest.mark.parametrize("S,Hq,Hkv", [(19, 40, 5), (12, 64, 8)], ids=["95-rows-tcgen05", "96-rows-mma"])
+def test_fp8_rows_at_the_kernel_boundary(pa, S, Hq, Hkv):
+    """95 (sequence, kv head) rows, the most the tcgen05 kernel takes, and 96, the
+    fewest the mma.sync kernel takes: both match the oracle."""
+    D, bs, ps = 128, 16, 64
+    g = np.random.default_rng(S)
+    lens = g.integers(1, 700, S).astype(np.int64)
+    lens[0] = 700
+    NB = int(sum(-(-int(L) // bs) for L in lens)) + 3
+    kc, vc = _random_codes((NB, Hkv, bs, D), S, 1), _random_codes((NB, Hkv, bs, D), S, 2)
+    ks, vs = 1.0 / 64, 1.0 / 32
+    q = normal_fill((S, Hq, D), "bf16", 1.0, S, 3)
+    tables = tables_from_order(lens, bs, g.permutation(NB).astype(np.int32),
+                               int(-(-lens.max() // bs)) + 1)
+    max_len = int(lens.max())
+    out = torch.full((S, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps), dtype=torch.uint8,
+                     device="cuda")
+    pa.pa_decode_attention_fp8(out, to_dev(q, "bf16"), torch.from_numpy(kc).cuda(),
+                               torch.from_numpy(vc).cuda(), torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens.astype(np.int32)).cuda(), 1 / math.sqrt(D),
+                               bs, Hkv, max_len, ks, vs, ps, ws)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error_read() == 0
+    want = oatt.paged_decode_attention(to_f64(q, "bf16"), fp8.dequantize(kc, ks),
+                                       fp8.dequantize(vc, vs), tables, lens, 1 / math.sqrt(D),
+                                       bs, Hkv, "f64")
+    assert_close(out_f64(out), want, "bf16", f"{S * Hkv} rows")
 
 
 def test_fp8_tensor_cores_balanced_split_any_workspace(pa):
