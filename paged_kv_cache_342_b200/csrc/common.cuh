@@ -48,8 +48,6 @@ struct DecodeParams {
   // [S] or null: grid row y of the per-sequence kernels serves sequence seq_order[y]
   // (longest first, so that the long rows start early and the short ones fill the end)
   const int32_t* seq_order;
-  // partitions one CTA of the fp8 tensor-core kernel walks (0 or 1: one)
-  int parts_per_cta;
 };
 
 // Index of (query row, partition) in the partition maxima / exp-sums ws_m, ws_l:
