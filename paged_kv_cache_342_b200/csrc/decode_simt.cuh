@@ -51,7 +51,8 @@ struct SimtCfg {
       (kStageArea > kRedBytes ? kStageArea : kRedBytes) + NW * NST * 8;
   static_assert(kVecPerRow % kLanesPerRow == 0, "head_dim too small for 8 lanes per row");
   static_assert(BS % kRowsPerPass == 0, "block_size must be a multiple of 4");
-  static_assert(kChunkBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
+  static_assert(kChunkBytes % 16 == 0 && (D * sizeof(T)) % 16 == 0,
+                "bulk copies move multiples of 16 bytes (whole rows)");
 };
 
 // Sequence length as the kernels use it: an out-of-range value counts as 0 and is
@@ -225,10 +226,14 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
       if (ok) {
         const int64_t off = (static_cast<int64_t>(blk) * p.num_kv_heads + kvh) * (BS * D);
         const uint32_t dst = smem_u32(my_stages + st * C::kStageBytes);
+        // only the rows that hold tokens (the sequence's last block may be part-filled;
+        // the rows past it are never read: their scores are -inf and their V is skipped)
+        const int rows = min(BS, tok_end - (tok_begin + (warp + k * NW) * BS));
+        const uint32_t bytes = static_cast<uint32_t>(rows) * D * sizeof(T);  // 16-byte multiple
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(bar, C::kStageBytes);
-        bulk_g2s(dst, kc + off, C::kChunkBytes, bar);
-        bulk_g2s(dst + C::kChunkBytes, vc + off, C::kChunkBytes, bar);
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        bulk_g2s(dst, kc + off, bytes, bar);
+        bulk_g2s(dst + C::kChunkBytes, vc + off, bytes, bar);
       } else {
         set_error(p.err, PA_DEVERR_TABLE);
         mbar_arrive(bar);
