@@ -45,6 +45,10 @@ struct DecodeParams {
   int num_chunks, group_zparts;
   float v_scale;  // output multiplier (the fp8 cache's V scale; 1 otherwise)
   int part_base;  // partition index of grid z = 0 in the per-sequence kernels
+  // partitions per CTA of the per-sequence tensor-core kernel (0 or 1: one): a CTA
+  // folds its consecutive partitions into one partial, in the slot of the first; the
+  // merge reads every part_step-th slot
+  int part_step;
   // [S] or null: grid row y of the per-sequence kernels serves sequence seq_order[y]
   // (longest first, so that the long rows start early and the short ones fill the end)
   const int32_t* seq_order;

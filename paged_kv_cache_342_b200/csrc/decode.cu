@@ -93,10 +93,14 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
   const int rows_per_cta = 8 / wpr;
   const int wsub = warp % wpr;
   const int row = blockIdx.x * rows_per_cta + warp / wpr;
+  // slots: partitions 0, step, 2 step, ... (a partition kernel that ran `step`
+  // consecutive partitions per CTA left one partial in the first one's slot)
+  const int step = p.part_step > 1 ? p.part_step : 1;
   int nparts = 0;
   if (row < p.num_seqs * p.num_heads) {
     const int L = checked_len(p, row / p.num_heads, false);
     nparts = L > 0 ? (L + p.partition_size - 1) / p.partition_size : 1;
+    nparts = (nparts + step - 1) / step;
   }
   float acc[DPL];
 #pragma unroll
@@ -104,18 +108,19 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeParams p, int wp
   float den = 0.f, M = -INFINITY;
   if (nparts > 1) {
     const int64_t mstride = static_cast<int64_t>(p.num_seqs) * p.num_heads;
-    const float* mrow = p.ws_m + row;  // partition pi at mrow[pi * mstride]
+    const int64_t sstride = mstride * step;  // slot pi (partition pi * step): pi * sstride
+    const float* mrow = p.ws_m + row;
     const float* lrow = p.ws_l + row;
-    const float* orow = p.ws_o + static_cast<int64_t>(row) * D + lane * DPL;  // pi: + pi*mstride*D
+    const float* orow = p.ws_o + static_cast<int64_t>(row) * D + lane * DPL;
     for (int i = wsub; i < nparts; i += U * wpr) {
       float mv[U], lv[U], o[U][DPL];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int pi = i + u * wpr;
         if (pi < nparts) {
-          mv[u] = mrow[pi * mstride];
-          lv[u] = lrow[pi * mstride];
-          load_lane<DPL>(orow + pi * mstride * D, o[u]);
+          mv[u] = mrow[pi * sstride];
+          lv[u] = lrow[pi * sstride];
+          load_lane<DPL>(orow + pi * sstride * D, o[u]);
         } else {
           mv[u] = -INFINITY;
           lv[u] = 0.f;
@@ -276,9 +281,11 @@ cudaError_t launch_merge_d(const DecodeParams& p, int grid, int wpr, bool depend
 // sparse: the partials come from a kernel that combines consecutive partitions itself
 template <typename T>
 cudaError_t launch_merge(const DecodeParams& p, bool dependent, bool sparse, cudaStream_t st) {
-  // warps per row: enough that each walks at most ~32 partitions
+  // warps per row: enough that each walks at most ~32 slots
+  const int step = p.part_step > 1 ? p.part_step : 1;
+  const int slots = (p.max_parts + step - 1) / step;
   int wpr = 1;
-  while (wpr < 8 && p.max_parts > 32 * wpr) wpr *= 2;
+  while (wpr < 8 && slots > 32 * wpr) wpr *= 2;
   const int rows = p.num_seqs * p.num_heads;
   const int rows_per_cta = 8 / wpr;
   const int grid = (rows + rows_per_cta - 1) / rows_per_cta;
@@ -304,6 +311,15 @@ bool mma_eligible(int dtype, int group, int head_dim, int block_size) {
   return (dtype == PA_BF16 || dtype == PA_F16) && group % 8 == 0 && group <= 16 &&
          (head_dim == 64 || head_dim == 128 || head_dim == 256) &&
          (block_size == 16 || block_size == 32);
+}
+
+// Partitions per CTA of the per-sequence tensor-core kernels: about 2048 tokens, the
+// partitions folded in registers (each keeping its own max and exp-sum), where the
+// tile leaves the registers for a second set of accumulators (head_dim / 16 k-steps
+// times group / 8 column tiles at most 8: the kernel's own rule); 1 otherwise.
+int mma_part_step(int head_dim, int group, int partition_size) {
+  if ((head_dim / 16) * (group / 8) > 8 || partition_size >= 2048) return 1;
+  return 2048 / partition_size;
 }
 
 bool mma_fp8_eligible(int group, int block_size) {
@@ -568,10 +584,12 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   } else if (tc) {
     e = launch_decode_tc_fp8(p, dtype, st);
   } else if (fp8 && mma_fp8_eligible(group, block_size)) {
+    p.part_step = mma_part_step(head_dim, group, partition_size);
     e = launch_decode_mma_fp8(p, dtype, st);
   } else if (fp8) {
     e = launch_decode_simt_fp8(p, dtype, simt_heads_per_cta(group, head_dim), st);
   } else if (mma_eligible(dtype, group, head_dim, block_size)) {
+    p.part_step = mma_part_step(head_dim, group, partition_size);
     e = dtype == PA_BF16 ? launch_decode_mma_bf16(p, st) : launch_decode_mma_f16(p, st);
   } else {
     const int gs = simt_heads_per_cta(group, head_dim);

@@ -161,9 +161,10 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 //   part_base on), the columns the group's query heads of that kv head.  So the long
 //   shared partitions start first, the short own ones fill the end, and neither kind
 //   has a last wave of its own.
-// T = MMA operand type, TQ = query / output type, FP8 = e4m3 cache converted to T.
+// T = MMA operand type, TQ = query / output type, FP8 = e4m3 cache converted to T,
+// CHUNK = several partitions per CTA (per-sequence form, p.part_step of them).
 template <typename T, typename TQ, int D, int BS, int NT, int NW, int NST, bool GROUP,
-          bool FP8>
+          bool FP8, bool CHUNK = false>
 __global__ void __launch_bounds__(NW * 32)
     decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -174,6 +175,12 @@ __global__ void __launch_bounds__(NW * 32)
   using Ops = MmaOps<T>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int TT = C::kTT, KS = C::kKS;
+  // Several partitions per CTA (per-sequence form): each keeps its own running max and
+  // exp-sum per warp; a finished partition is folded into the warp's running result by
+  // the log-sum-exp rule, which takes a second set of accumulators - registers the
+  // small tiles have to spare
+  constexpr bool kChunked = CHUNK && !GROUP && KS * NT <= 8;
+  static_assert(!CHUNK || kChunked, "several partitions per CTA need a small tile");
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ int col_row[C::kHeads];  // q / out row (sequence * Hq + head) of each column
@@ -193,7 +200,9 @@ __global__ void __launch_bounds__(NW * 32)
         row_sequence(p, blockIdx.y, threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0);
     if (s < 0) return;
     const int h0 = blockIdx.x * C::kHeads;
-    part = p.part_base + blockIdx.z;
+    // a CTA runs `step` consecutive partitions (one chunk) of the sequence
+    const int step = kChunked && p.part_step > 1 ? p.part_step : 1;
+    part = p.part_base + blockIdx.z * step;
     kvh = h0 / G;
     const int L = checked_len(p, s, threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0);
     nparts = L > 0 ? (L + ps - 1) / ps : 1;
@@ -202,7 +211,9 @@ __global__ void __launch_bounds__(NW * 32)
       set_error(p.err, PA_DEVERR_GROUP);
     if (part >= nparts || part < own) return;
     tok_begin = part * ps;
-    tok_end = min(L, tok_begin + ps);
+    tok_end = min(L, min(nparts, part + step) * ps);
+    // one chunk covering the whole sequence writes the output rows themselves
+    if (part == 0 && nparts <= step) nparts = 1;
     table_seq = s;
     if (threadIdx.x < C::kHeads) {
       col_row[threadIdx.x] = s * p.num_heads + h0 + threadIdx.x;
@@ -234,9 +245,10 @@ __global__ void __launch_bounds__(NW * 32)
       tok_begin = part * ps;
       tok_end = min(L, tok_begin + ps);
       table_seq = s;
-      if (threadIdx.x < C::kHeads) {
-        col_row[threadIdx.x] = threadIdx.x < G ? s * p.num_heads + kvh * G + threadIdx.x : -1;
-        col_ok[threadIdx.x] = threadIdx.x < G ? 1 : 0;
+      const int c = static_cast<int>(threadIdx.x);
+      if (c < C::kHeads) {
+        col_row[c] = c < G ? s * p.num_heads + kvh * G + c : -1;
+        col_ok[c] = c < G ? 1 : 0;
       }
     }
     if (!own_item) {
@@ -295,15 +307,52 @@ __global__ void __launch_bounds__(NW * 32)
   // per thread: heads nt*8 + 2t4 + {0,1}
   float m[NT][2], l[NT][2];
   float oacc[KS][NT][4];
+  auto reset = [&]() {
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    m[nt][0] = m[nt][1] = -INFINITY;
-    l[nt][0] = l[nt][1] = 0.f;
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
 #pragma unroll
-    for (int mt = 0; mt < KS; ++mt)
+      for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.f;
+        for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.f;
+    }
+  };
+  reset();
+  // chunked form: the warp's finished partitions, combined (max, exp-sum, output)
+  constexpr int RN = kChunked ? NT : 1, RK = kChunked ? KS : 1;
+  float mr[RN][2], lr[RN][2], ar[RK][RN][4];
+#pragma unroll
+  for (int nt = 0; nt < RN; ++nt) {
+    mr[nt][0] = mr[nt][1] = -INFINITY;
+    lr[nt][0] = lr[nt][1] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < RK; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ar[mt][nt][i] = 0.f;
   }
+  int cur_part = -1;  // the partition the warp's (m, l, oacc) belong to
+  int cur_end = 0;    // ... and its end, in tokens from tok_begin
+  // M = max(mr, m), result = result * 2^(mr - M) + partition * 2^(m - M), per column
+  auto fold = [&]() {
+    if constexpr (kChunked) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float mn = fmaxf(mr[nt][j], m[nt][j]);
+          const float co = exp2_safe(mr[nt][j], mn), cn = exp2_safe(m[nt][j], mn);
+          lr[nt][j] = fmaf(lr[nt][j], co, l[nt][j] * cn);
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            ar[mt][nt][j] = fmaf(ar[mt][nt][j], co, oacc[mt][nt][j] * cn);
+            ar[mt][nt][2 + j] = fmaf(ar[mt][nt][2 + j], co, oacc[mt][nt][2 + j] * cn);
+          }
+          mr[nt][j] = mn;
+        }
+      reset();
+    }
+  };
 
   const int nb_w = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;
   int tab_base = 0;
@@ -354,6 +403,15 @@ __global__ void __launch_bounds__(NW * 32)
   bool aborted = false;
   for (; k < nb_w; ++k) {
     const int st = k % NST;
+    if constexpr (kChunked) {
+      // a block of the next partition: fold the finished one into the running result
+      const int off = (warp + k * NW) * BS;
+      if (off >= cur_end) {
+        if (cur_part >= 0) fold();
+        cur_part = part + off / ps;
+        cur_end = (cur_part - part + 1) * ps;
+      }
+    }
     const bool ok = mbar_wait_bounded(bar0 + 8 * st, (k / NST) & 1);
     if (!__all_sync(FULL, ok)) {
       aborted = true;
@@ -530,6 +588,21 @@ __global__ void __launch_bounds__(NW * 32)
     }
   }
   allow_dependents();  // the merge may launch now; it waits for this grid's writes
+  if constexpr (kChunked) {
+    if (cur_part >= 0) fold();
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        m[nt][j] = mr[nt][j];
+        l[nt][j] = lr[nt][j];
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          oacc[mt][nt][j] = ar[mt][nt][j];
+          oacc[mt][nt][2 + j] = ar[mt][nt][2 + j];
+        }
+      }
+  }
   if (aborted) {
     if (lane == 0) set_error(p.err, PA_DEVERR_TIMEOUT);
     for (; k < issued; ++k) mbar_wait_bounded(bar0 + 8 * (k % NST), (k / NST) & 1);

@@ -6,7 +6,7 @@
 namespace pa {
 namespace {
 
-template <int D, int BS, int NT, bool GROUP>
+template <int D, int BS, int NT, bool GROUP, bool CHUNK>
 cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   // about 64 KiB of stages per CTA: warps with two stages each (1-4), then 2-4 stages;
   // about 16 KiB (one warp) for a grouped call, whose many short own partitions want
@@ -27,30 +27,40 @@ cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   if (!make_cache_tensor_map(&tmk, p.k_cache, rows, D, BS, dt, 2) ||
       !make_cache_tensor_map(&tmv, p.v_cache, rows, D, BS, dt, 2))
     return cudaErrorInvalidValue;
-  constexpr auto kern = decode_mma_kernel<__half, __half, D, BS, NT, NW, NST, GROUP, false>;
+  constexpr auto kern = decode_mma_kernel<__half, __half, D, BS, NT, NW, NST, GROUP, false, CHUNK>;
   cudaError_t e = ensure_smem_limit<kern>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   return launch_dependent(kern, grid, dim3(NW * 32), C::kSmemBytes, st, p, tmk, tmv);
 }
 
-template <int D, int NT, bool GROUP>
+template <int D, int NT, bool GROUP, bool CHUNK>
 cudaError_t by_bs(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   switch (p.block_size) {
-    case 16: return launch<D, 16, NT, GROUP>(p, grid, st);
-    case 32: return launch<D, 32, NT, GROUP>(p, grid, st);
+    case 16: return launch<D, 16, NT, GROUP, CHUNK>(p, grid, st);
+    case 32: return launch<D, 32, NT, GROUP, CHUNK>(p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
+// several partitions per CTA (p.part_step > 1) only where the kernel folds them
+// (head_dim / 16 k-steps times column tiles at most 8)
 template <bool GROUP>
 cudaError_t by_shape(const DecodeParams& p, int nt, dim3 grid, cudaStream_t st) {
+  const bool chunk = !GROUP && p.part_step > 1;
   switch (p.head_dim * 4 + nt) {
-    case 64 * 4 + 1: return by_bs<64, 1, GROUP>(p, grid, st);
-    case 64 * 4 + 2: return by_bs<64, 2, GROUP>(p, grid, st);
-    case 128 * 4 + 1: return by_bs<128, 1, GROUP>(p, grid, st);
-    case 128 * 4 + 2: return by_bs<128, 2, GROUP>(p, grid, st);
-    case 256 * 4 + 1: return by_bs<256, 1, GROUP>(p, grid, st);
-    case 256 * 4 + 2: return by_bs<256, 2, GROUP>(p, grid, st);
+    case 64 * 4 + 1:
+      return chunk ? by_bs<64, 1, GROUP, !GROUP>(p, grid, st) : by_bs<64, 1, GROUP, false>(p, grid, st);
+    case 64 * 4 + 2:
+      return chunk ? by_bs<64, 2, GROUP, !GROUP>(p, grid, st) : by_bs<64, 2, GROUP, false>(p, grid, st);
+    case 128 * 4 + 1:
+      return chunk ? by_bs<128, 1, GROUP, !GROUP>(p, grid, st)
+                   : by_bs<128, 1, GROUP, false>(p, grid, st);
+    case 128 * 4 + 2:
+      return chunk ? cudaErrorInvalidValue : by_bs<128, 2, GROUP, false>(p, grid, st);
+    case 256 * 4 + 1:
+      return chunk ? cudaErrorInvalidValue : by_bs<256, 1, GROUP, false>(p, grid, st);
+    case 256 * 4 + 2:
+      return chunk ? cudaErrorInvalidValue : by_bs<256, 2, GROUP, false>(p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -60,7 +70,8 @@ cudaError_t by_shape(const DecodeParams& p, int nt, dim3 grid, cudaStream_t st) 
 // Per-sequence partitions: 8*NT query heads of one kv head per CTA (NT = group / 8).
 cudaError_t launch_decode_mma_f16(const DecodeParams& p, cudaStream_t st) {
   const int nt = (p.num_heads / p.num_kv_heads) / 8;
-  dim3 grid(p.num_heads / (8 * nt), p.num_seqs, p.max_parts - p.part_base);
+  const int step = p.part_step > 1 ? p.part_step : 1;
+  dim3 grid(p.num_heads / (8 * nt), p.num_seqs, (p.max_parts - p.part_base + step - 1) / step);
   return by_shape<false>(p, nt, grid, st);
 }
 
