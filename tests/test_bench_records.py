@@ -52,7 +52,9 @@ def test_records_are_consistent(name):
     assert rec["read_bytes"] + rec["write_bytes"] > 0
     ratio = (rec["read_bytes"] + rec["write_bytes"]) / rec["algorithmic_bytes_of_capture"]
     assert ratio == pytest.approx(rec["traffic_over_algorithmic"], abs=1e-4)
-    assert 1.0 <= ratio < 1.1          # no wasted re-reads
+    # no wasted re-reads; a little below 1 where the small inputs (q, tables, lengths)
+    # were still in L2
+    assert 0.99 <= ratio < 1.1
     if rec["captured_on"] == name:     # captured at full size
         assert rec["traffic_bytes_per_launch"] == rec["read_bytes"] + rec["write_bytes"]
     assert rec["kernels"]
