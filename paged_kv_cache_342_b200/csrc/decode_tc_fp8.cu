@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
     uint64_t* empty = is_k ? bar_k_empty : bar_v_empty;
     const CUtensorMap* map = is_k ? &tmk : &tmv;
     const uint32_t half = is_k ? 0u : static_cast<uint32_t>(C::TILE);
+    const uint64_t stream_policy = l2_evict_first_policy();  // K/V are read once
     int g = 0;
     for (int k = 0; k < nitems && !aborted; ++k) {
       const TcItem it = sh_items[k];
@@ -281,8 +282,8 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
           }
           __syncwarp();
           if (ok)
-            tma_load_2d(base + st * C::STAGE + half + lane * BS * 128, map, 0,
-                        (blk * p.num_kv_heads + it.kvh) * BS, b32(full[st]));
+            tma_load_2d_hint(base + st * C::STAGE + half + lane * BS * 128, map, 0,
+                             (blk * p.num_kv_heads + it.kvh) * BS, b32(full[st]), stream_policy);
         }
       }
     }
@@ -520,9 +521,11 @@ __global__ void __launch_bounds__(kTcThreads, G == 8 ? 2 : 1)
         if (single) {
           bulk_s2g(static_cast<TQ*>(p.out) + row0 * D, sa, G * D * sizeof(TQ));
         } else {
-          bulk_s2g(p.ws_o + o_index(p, row0, e.pbeg), sa, G * 512);  // G contiguous rows
-          bulk_s2g(p.ws_m + ml_index(p, row0, e.pbeg), sa + G * 512, G * 4);
-          bulk_s2g(p.ws_l + ml_index(p, row0, e.pbeg), sa + G * 512 + G * 4, G * 4);
+          // partials stay in L2 for the merge
+          const uint64_t keep = l2_evict_last_policy();
+          bulk_s2g_hint(p.ws_o + o_index(p, row0, e.pbeg), sa, G * 512, keep);  // G rows
+          bulk_s2g_hint(p.ws_m + ml_index(p, row0, e.pbeg), sa + G * 512, G * 4, keep);
+          bulk_s2g_hint(p.ws_l + ml_index(p, row0, e.pbeg), sa + G * 512 + G * 4, G * 4, keep);
         }
         bulk_commit();
       }
