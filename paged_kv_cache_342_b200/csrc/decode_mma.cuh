@@ -359,6 +359,7 @@ __global__ void __launch_bounds__(NW * 32)
   int32_t tab = (lane < nb_w) ? __ldg(table + warp + lane * NW) : -1;
   uint32_t bad = 0;
 
+  const uint64_t stream_policy = l2_evict_first_policy();  // K/V are read once
   auto issue = [&](int k) {
     if (k - tab_base >= 32) {
       tab_base += 32;
@@ -379,14 +380,16 @@ __global__ void __launch_bounds__(NW * 32)
         if constexpr (FP8) {
 #pragma unroll
           for (int h = 0; h < C::kF8Slabs; ++h) {
-            tma_load_2d(dst + h * C::kSlabBytes, &tmk, 128 * h, row0, bar);
-            tma_load_2d(dst + C::kF8Tile + h * C::kSlabBytes, &tmv, 128 * h, row0, bar);
+            tma_load_2d_hint(dst + h * C::kSlabBytes, &tmk, 128 * h, row0, bar, stream_policy);
+            tma_load_2d_hint(dst + C::kF8Tile + h * C::kSlabBytes, &tmv, 128 * h, row0, bar,
+                             stream_policy);
           }
         } else {
 #pragma unroll
           for (int h = 0; h < C::kHalves; ++h) {
-            tma_load_2d(dst + h * C::kSlabBytes, &tmk, 64 * h, row0, bar);
-            tma_load_2d(dst + C::kTileBytes + h * C::kSlabBytes, &tmv, 64 * h, row0, bar);
+            tma_load_2d_hint(dst + h * C::kSlabBytes, &tmk, 64 * h, row0, bar, stream_policy);
+            tma_load_2d_hint(dst + C::kTileBytes + h * C::kSlabBytes, &tmv, 64 * h, row0, bar,
+                             stream_policy);
           }
         }
       } else {
@@ -666,6 +669,7 @@ __global__ void __launch_bounds__(NW * 32)
     col_l[hh] = den;
   }
   __syncthreads();
+  const uint64_t keep_policy = l2_evict_last_policy();
   for (int idx = threadIdx.x; idx < C::kHeads * D; idx += NW * 32) {
     const int hh = idx / D, d = idx - hh * D;
     if (!col_ok[hh]) continue;
@@ -679,10 +683,10 @@ __global__ void __launch_bounds__(NW * 32)
     if (nparts == 1) {
       store_elem(static_cast<TQ*>(p.out) + row * D + d, o);
     } else {
-      p.ws_o[o_index(p, row, part) + d] = o;
+      st_hint(p.ws_o + o_index(p, row, part) + d, o, keep_policy);  // L2, for the merge
       if (d == 0) {
-        p.ws_m[ml_index(p, row, part)] = col_m[hh];
-        p.ws_l[ml_index(p, row, part)] = den;
+        st_hint(p.ws_m + ml_index(p, row, part), col_m[hh], keep_policy);
+        st_hint(p.ws_l + ml_index(p, row, part), den, keep_policy);
       }
     }
   }
