@@ -211,6 +211,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
   const T* kc = static_cast<const T*>(p.k_cache);
   const T* vc = static_cast<const T*>(p.v_cache);
 
+  const uint64_t stream_policy = l2_evict_first_policy();  // K/V are read once
   auto issue = [&](int k) {
     if (k - tab_base >= 32) {
       tab_base += 32;
@@ -232,8 +233,8 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
         const uint32_t bytes = static_cast<uint32_t>(rows) * D * sizeof(T);  // 16-byte multiple
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(bar, 2 * bytes);
-        bulk_g2s(dst, kc + off, bytes, bar);
-        bulk_g2s(dst + C::kChunkBytes, vc + off, bytes, bar);
+        bulk_g2s_hint(dst, kc + off, bytes, bar, stream_policy);
+        bulk_g2s_hint(dst + C::kChunkBytes, vc + off, bytes, bar, stream_policy);
       } else {
         set_error(p.err, PA_DEVERR_TABLE);
         mbar_arrive(bar);
