@@ -314,12 +314,13 @@ int pa_decode_attention_fp8(void* out, const void* q, const void* k_cache, const
  * partition_size / block_size logical blocks to the same physical blocks (what
  * pa_build_prefix_groups guarantees); prefix_parts[i] equals its chunk's parts.
  * A sequence never has its last token's partition computed by the group, so every
- * grouped sequence is finished by the merge kernel.  first_part: the lowest partition
- * any sequence computes itself, min over s of min(prefix_parts[s], (seq_lens[s]-1) /
- * partition_size) (0 when any sequence has no group); the per-sequence kernel's grid
- * starts there, so the partitions every group covers launch no CTAs at all.  A
- * sequence whose own partitions start lower is reported (PA_DEVERR_GROUP) and those
- * partitions are left out.  When the shape does not qualify
+ * grouped sequence is finished by the merge kernel.  The call is one grid: the groups'
+ * shared partitions first, then every sequence's own partitions, then the merge.
+ * first_part: the lowest partition any sequence computes itself, min over s of
+ * min(prefix_parts[s], (seq_lens[s]-1) / partition_size) (0 when any sequence has no
+ * group); the sequences' own part of the grid starts there, so the partitions every
+ * group covers launch no CTAs at all.  A sequence whose own partitions start lower is
+ * reported (PA_DEVERR_GROUP) and those partitions are left out.  When the shape does not qualify
  * (f32 cache, block_size not 16/32, max_members * num_heads/num_kv_heads > 16, or a
  * single partition) the groups are ignored and the plain path runs.
  */

@@ -35,7 +35,8 @@ struct DecodeParams {
   float* ws_l;  // [P, S, Hq]     partition exp-sum
   uint32_t* err;
   // prefix groups (all null / 0 for the plain call): whole partitions that a group of
-  // sequences shares are computed once per group by the group kernel
+  // sequences shares are computed once per group, by the tensor-core kernel's grouped
+  // form
   const int32_t* prefix_parts;   // [S] shared partitions of each sequence (0 = none)
   const int32_t* chunk_members;  // [num_chunks, max_members] batch positions, -1 padded
   const int32_t* chunk_parts;    // [num_chunks] shared partitions of each chunk

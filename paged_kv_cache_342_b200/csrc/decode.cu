@@ -342,7 +342,7 @@ int64_t head_ctas(int cache_dtype, int num_heads, int num_kv_heads, int head_dim
 // are resident per SM; the automatic partition size aims at four waves of those.
 constexpr int kAutoCtasPerSm = 3 * 4;
 
-// The group kernel is the tensor-core kernel with (member, head) columns.
+// The grouped form is the tensor-core kernel with (member, head) columns.
 bool group_eligible(int dtype, int group, int head_dim, int block_size, int max_members) {
   return (dtype == PA_BF16 || dtype == PA_F16) && max_members >= 1 &&
          max_members * group <= 16 && (head_dim == 64 || head_dim == 128 || head_dim == 256) &&

@@ -70,8 +70,8 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int s, bool re
 // Leading partitions of sequence s that its prefix group's kernel computes (0 when
 // the call has no groups).  Never the partition holding the last token, so every
 // sequence keeps at least one partition of its own and a grouped sequence always
-// goes through the merge.  The per-sequence and group kernels evaluate this same
-// expression, so every partition is written by exactly one of them.
+// goes through the merge.  The per-sequence kernels and the grouped form evaluate this
+// same expression, so every partition is written exactly once.
 __device__ __forceinline__ int group_parts(const DecodeParams& p, int s, int L) {
   if (!p.prefix_parts || L <= 0) return 0;
   const int g = __ldg(p.prefix_parts + s);
