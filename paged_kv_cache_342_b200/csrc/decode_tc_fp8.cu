@@ -20,13 +20,15 @@
 //   warps 4-7   one thread per token row: read S from tensor memory, online softmax per
 //               head, write P; a partition's output (one thread per dim row) is read
 //               from tensor memory after the next partition's first tile, from the
-//               other of two O accumulators, so it never stalls the pipeline.
+//               other of two O accumulators, so it never stalls the pipeline, and is
+//               combined with the item's earlier partitions (log-sum-exp rule); one
+//               partial per item leaves by bulk copy.
 // The codes are never converted: K and V tiles are the MMA operands as TMA lands
 // them.  q (bf16: 2 terms, f16: 3 terms) is carried as exact e4m3 terms t_j of
 // q * 2^qe (qe per head puts the largest |q| in [128, 256)), the terms as separate
 // columns of S, summed per head; the next item's q is prefetched into registers and
-// written to the other of two Q buffers during the current item.  P is split into
-// hi = e4m3(p) and lo = e4m3((p - hi) * 32), again as separate columns of O:
+// written to the Q operand once the current item's last S has been computed.  P is
+// split into hi = e4m3(p) and lo = e4m3((p - hi) * 32), again as separate columns of O:
 // o = O_hi + O_lo / 32.  Weights stay in (0, 2^8] under the lazy running max, so both
 // fit e4m3 (|p - hi| <= 8).  Tokens past the end (or in blocks whose table entry is
 // out of range) get -inf scores, and their V rows are zeroed in shared memory
