@@ -160,9 +160,11 @@ int pa_swap_blocks(void* dst_k, void* dst_v, int64_t dst_num_blocks, const void*
  * partition's weights were taken against; it may trail the true maximum logit by up
  * to 8 in base 2, and the merge uses each pair as a whole).  A kernel that computes
  * several consecutive partitions of a row may combine them itself and leave one
- * partial in the first one's slot, the others with exp-sum 0.  The contents need no
- * initialisation and are not kept between calls.  Returns 0 when P <= 1 (no merge
- * needed) and 0 for invalid sizes.
+ * partial in the first one's slot, the others with exp-sum 0.  After the partials, one
+ * int32 arrival counter per (sequence, head) row [num_seqs, num_heads], which the
+ * grouped call clears itself before use.  The contents need no initialisation and
+ * are not kept between calls.  Returns 0 when P <= 1 (no merge needed) and 0 for
+ * invalid sizes.
  */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_seq_len,
                                  int partition_size);
@@ -314,8 +316,11 @@ int pa_decode_attention_fp8(void* out, const void* q, const void* k_cache, const
  * partition_size / block_size logical blocks to the same physical blocks (what
  * pa_build_prefix_groups guarantees); prefix_parts[i] equals its chunk's parts.
  * A sequence never has its last token's partition computed by the group, so every
- * grouped sequence is finished by the merge kernel.  The call is one grid: the groups'
- * shared partitions first, then every sequence's own partitions, then the merge.
+ * grouped sequence is finished by a log-sum-exp merge of its partitions.  The call is
+ * one grid: the groups' shared partitions first, then every sequence's own
+ * partitions; the CTA that stores the last partial of a (sequence, kv head) merges
+ * that sequence's heads itself (arrival counters in the workspace, cleared by a small
+ * kernel launched just before the grid), so no merge kernel follows.
  * first_part: the lowest partition any sequence computes itself, min over s of
  * min(prefix_parts[s], (seq_lens[s]-1) / partition_size) (0 when any sequence has no
  * group); the sequences' own part of the grid starts there, so the partitions every

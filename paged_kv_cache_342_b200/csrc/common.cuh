@@ -33,6 +33,10 @@ struct DecodeParams {
   float* ws_o;  // [P, S, Hq, D]  normalised partial outputs, see o_index
   float* ws_m;  // [P, S, Hq]     partition max (base-2 logits), see ml_index
   float* ws_l;  // [P, S, Hq]     partition exp-sum
+  // [S, Hq] arrival counters of the grouped form, zeroed before its grid: the CTA
+  // that writes the last partial of a (sequence, kv head) combines that row
+  // group's partials itself (entry s * Hq + kv head * group)
+  int* ws_cnt;
   uint32_t* err;
   // prefix groups (all null / 0 for the plain call): whole partitions that a group of
   // sequences shares are computed once per group, by the tensor-core kernel's grouped

@@ -7,6 +7,7 @@
 // attention); "PagedAttention" attention-lab explainer (divagr.pages.dev), "Keep
 // pages in order" and "Measure memory use across requests" (the attention equation
 // is unchanged by paging).
+#include <algorithm>
 #include <cmath>
 
 #include "common.cuh"
@@ -34,7 +35,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WsLayout {
   int parts = 1;
-  size_t o_off = 0, m_off = 0, l_off = 0, bytes = 0;
+  size_t o_off = 0, m_off = 0, l_off = 0, cnt_off = 0, bytes = 0;
 };
 
 WsLayout ws_layout(int64_t num_seqs, int64_t num_heads, int64_t head_dim, int64_t max_seq_len,
@@ -46,7 +47,8 @@ WsLayout ws_layout(int64_t num_seqs, int64_t num_heads, int64_t head_dim, int64_
   w.o_off = 0;
   w.m_off = align256(rows * head_dim * sizeof(float));
   w.l_off = w.m_off + align256(rows * sizeof(float));
-  w.bytes = w.l_off + align256(rows * sizeof(float));
+  w.cnt_off = w.l_off + align256(rows * sizeof(float));
+  w.bytes = w.cnt_off + align256(static_cast<size_t>(num_seqs) * num_heads * sizeof(int));
   return w;
 }
 
@@ -295,6 +297,20 @@ cudaError_t launch_merge(const DecodeParams& p, bool dependent, bool sparse, cud
     case 256: return launch_merge_d<T, 256>(p, grid, wpr, dependent, sparse, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// The arrival counters of a grouped call set to zero, launched in the chain before its
+// grid: lets that grid launch at once, then waits for the kernel before it on the
+// stream (the previous call on this workspace may still be counting) and clears them.
+__global__ void __launch_bounds__(256) zero_counters_kernel(int* cnt, int n) {
+  allow_dependents();
+  grid_dependency_wait();
+  for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) cnt[i] = 0;
+}
+
+cudaError_t launch_zero_counters(int* cnt, int n, cudaStream_t st) {
+  const int grid = std::max(1, std::min((n + 255) / 256, 1184));
+  return launch_dependent(zero_counters_kernel, dim3(grid), dim3(256), 0, st, cnt, n);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -557,6 +573,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.ws_o = reinterpret_cast<float*>(base + ws.o_off);
     p.ws_m = reinterpret_cast<float*>(base + ws.m_off);
     p.ws_l = reinterpret_cast<float*>(base + ws.l_off);
+    p.ws_cnt = reinterpret_cast<int*>(base + ws.cnt_off);
   }
   p.err = device_error_word();
   if (!p.err) {
@@ -568,6 +585,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
   const bool tc = fp8 && tc_fp8_eligible(group, head_dim, block_size, num_seqs, num_kv_heads);
+  bool merged = false;  // the partition grid also combines the partitions
   if (!fp8 && groups && groups->num_chunks > 0 && groups->max_chunk_parts > 0 && ws.parts > 1 &&
       group_eligible(dtype, group, head_dim, block_size, groups->max_members)) {
     // Prefix groups (only useful when sequences span several partitions): one grid of
@@ -580,7 +598,12 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.group_zparts = groups->max_chunk_parts < ws.parts ? groups->max_chunk_parts : ws.parts;
     // partitions below first_part belong to the groups for every sequence
     p.part_base = groups->first_part < ws.parts - 1 ? groups->first_part : ws.parts - 1;
-    e = dtype == PA_BF16 ? launch_decode_grouped_bf16(p, st) : launch_decode_grouped_f16(p, st);
+    // the grid combines every row itself (the CTA that writes a row's last partial):
+    // its counters start at zero, and no merge launch follows
+    e = launch_zero_counters(p.ws_cnt, num_seqs * num_heads, st);
+    if (e == cudaSuccess)
+      e = dtype == PA_BF16 ? launch_decode_grouped_bf16(p, st) : launch_decode_grouped_f16(p, st);
+    merged = true;
   } else if (tc) {
     e = launch_decode_tc_fp8(p, dtype, st);
   } else if (fp8 && mma_fp8_eligible(group, block_size)) {
@@ -601,7 +624,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     note_cuda_error(e);
     return PA_ERR_CUDA;
   }
-  if (ws.parts > 1) {
+  if (ws.parts > 1 && !merged) {
     e = dtype == PA_F32    ? launch_merge<float>(p, true, tc, st)
         : dtype == PA_BF16 ? launch_merge<__nv_bfloat16>(p, true, tc, st)
                            : launch_merge<__half>(p, true, tc, st);

@@ -151,6 +151,143 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return static_cast<uint32_t>((c >> 3) * (BS * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+// One warp combines the partials of query row `row` (sequence s, one head) into its
+// output by the merge rule: M = max m_j, w_j = l_j 2^(m_j - M), out = sum w_j o_j /
+// sum w_j, over the slots j in [0, a) and [b, n) (eight in flight, in increasing j,
+// the same arithmetic as the merge kernel).  Slot own_part (-1: none) is this CTA's
+// own partial, taken from shared memory (own_o, own_m, own_l); the others come from
+// other CTAs of the grid: read from L2 (ld.global.cg) unless L1 holds lines fetched
+// after an acquire of the row's counter (L1 = true).
+template <typename TQ, int D, bool L1>
+__device__ __forceinline__ void combine_row(const DecodeParams& p, int row, int a, int b, int n,
+                                            int lane, int own_part, const float* own_o,
+                                            float own_m, float own_l) {
+  constexpr int DPL = D / 32, U = 8;
+  const int ns = a + (n > b ? n - b : 0);
+  float acc[DPL];
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) acc[j] = 0.f;
+  float den = 0.f, M = -INFINITY;
+  for (int i = 0; i < ns; i += U) {
+    float mv[U], lv[U], o[U][DPL];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = i + u;
+      const int part = k < a ? k : b + (k - a);
+      if (k < ns && part == own_part) {
+        mv[u] = own_m;
+        lv[u] = own_l;
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) o[u][j] = own_o[lane * DPL + j];
+      } else if (k < ns) {
+        const float* src = p.ws_o + o_index(p, row, part) + lane * DPL;
+        if constexpr (L1) {
+          mv[u] = __ldca(p.ws_m + ml_index(p, row, part));
+          lv[u] = __ldca(p.ws_l + ml_index(p, row, part));
+        } else {
+          mv[u] = __ldcg(p.ws_m + ml_index(p, row, part));
+          lv[u] = __ldcg(p.ws_l + ml_index(p, row, part));
+        }
+        if constexpr (DPL % 4 == 0) {
+#pragma unroll
+          for (int j = 0; j < DPL; j += 4) {
+            const float4* q4 = reinterpret_cast<const float4*>(src + j);
+            const float4 v = L1 ? __ldca(q4) : __ldcg(q4);
+            o[u][j] = v.x;
+            o[u][j + 1] = v.y;
+            o[u][j + 2] = v.z;
+            o[u][j + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < DPL; j += 2) {
+            const float2* q2 = reinterpret_cast<const float2*>(src + j);
+            const float2 v = L1 ? __ldca(q2) : __ldcg(q2);
+            o[u][j] = v.x;
+            o[u][j + 1] = v.y;
+          }
+        }
+      } else {
+        mv[u] = -INFINITY;
+        lv[u] = 0.f;
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) o[u][j] = 0.f;
+      }
+    }
+    float mx = M;
+#pragma unroll
+    for (int u = 0; u < U; ++u) mx = fmaxf(mx, mv[u]);
+    const float c = exp2_safe(M, mx);
+    den *= c;
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) acc[j] *= c;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float w = lv[u] * exp2_safe(mv[u], mx);
+      den += w;
+#pragma unroll
+      for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w, o[u][j], acc[j]);
+    }
+    M = mx;
+  }
+  TQ* out = static_cast<TQ*>(p.out) + static_cast<int64_t>(row) * D + lane * DPL;
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) store_elem(out + j, acc[j] * inv);
+}
+
+// Grouped form, after a CTA has stored its partials: it counts them on the arrival
+// counter of each (sequence, kv head) it wrote (entry s * Hq + kv head * G), and the
+// CTA whose count completes a counter combines that sequence's G heads itself, so
+// no merge launch follows the grid.  A (sequence, kv head) expects one partial per
+// partition the call writes for it: the group's below a = group_parts(s), then its
+// own from b = max(a, part_base) to its last, n - 1.  col_n / col_a / col_b hold n, a
+// and b for a column that counts (its first head), col_n 0 for the others.  The count
+// is one acquire-release atomic by the counting thread after a block barrier: it
+// publishes every thread's partial stores before it, and the CTA that completes the
+// count sees the other CTAs' partials after it (read from L2 after a second barrier).
+// Called by every thread of the CTA.
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+               : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* addr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void prefetch_l1(const void* addr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(addr));
+}
+
+template <typename TQ, int D, int NW, int H>
+__device__ __forceinline__ void finish_rows(const DecodeParams& p, const int* col_row,
+                                            const int* col_n, const int* col_a,
+                                            const int* col_b, int G) {
+  __shared__ int fin[H];
+  __syncthreads();  // the CTA's partial stores are issued
+  const int c = static_cast<int>(threadIdx.x);
+  if (c < H) {
+    const int n = col_n[c], b = col_b[c];
+    const int expect = col_a[c] + (n > b ? n - b : 0);
+    fin[c] = n > 0 && atomic_add_acq_rel_gpu(p.ws_cnt + col_row[c], 1) == expect - 1;
+  }
+  __syncthreads();
+  const int warp = c >> 5, lane = c & 31;
+  int k = 0;  // finished rows, dealt to the warps in turn
+  for (int c2 = 0; c2 < H; ++c2) {
+    if (!fin[c2]) continue;
+    for (int j = 0; j < G; ++j, ++k)
+      if (k % NW == warp)
+        combine_row<TQ, D, false>(p, col_row[c2] + j, col_a[c2], col_b[c2], col_n[c2], lane,
+                                  -1, nullptr, 0.f, 0.f);
+  }
+}
+
 // GROUP = false: one CTA per (sequence, 8*NT query heads of one kv head, partition).
 // GROUP = true : a grouped call in one flat grid of two kinds of work.  First the
 //   prefix groups' shared partitions, one CTA per (kv head, chunk of a group, shared
@@ -185,6 +322,10 @@ __global__ void __launch_bounds__(NW * 32)
   extern __shared__ uint8_t smem_raw[];
   __shared__ int col_row[C::kHeads];  // q / out row (sequence * Hq + head) of each column
   __shared__ int col_ok[C::kHeads];   // the column's result is written by this CTA
+  // grouped form: partitions of the column's sequence (n), the group's (a) and where
+  // its own start (b), set on the column that counts the sequence's partials
+  __shared__ int col_n[GROUP ? C::kHeads : 1], col_a[GROUP ? C::kHeads : 1],
+      col_b[GROUP ? C::kHeads : 1];
   // 1024-byte alignment for the swizzle atoms
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -195,6 +336,7 @@ __global__ void __launch_bounds__(NW * 32)
   const int G = p.num_heads / p.num_kv_heads;
   const int ps = p.partition_size;
   int kvh, part, nparts, tok_begin, tok_end, table_seq;
+  bool own_row = false;  // grouped form: a sequence's own partition, one of several
   if constexpr (!GROUP) {
     const int s =
         row_sequence(p, blockIdx.y, threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0);
@@ -242,6 +384,7 @@ __global__ void __launch_bounds__(NW * 32)
       const int own = group_parts(p, s, L);
       if (report && own < p.part_base) set_error(p.err, PA_DEVERR_GROUP);
       if (part >= nparts || part < own) return;
+      own_row = nparts > 1;
       tok_begin = part * ps;
       tok_end = min(L, tok_begin + ps);
       table_seq = s;
@@ -249,6 +392,9 @@ __global__ void __launch_bounds__(NW * 32)
       if (c < C::kHeads) {
         col_row[c] = c < G ? s * p.num_heads + kvh * G + c : -1;
         col_ok[c] = c < G ? 1 : 0;
+        col_n[c] = c == 0 ? nparts : 0;
+        col_a[c] = own;
+        col_b[c] = own > p.part_base ? own : p.part_base;
       }
     }
     if (!own_item) {
@@ -261,7 +407,12 @@ __global__ void __launch_bounds__(NW * 32)
         const int m = mi < p.max_members ? __ldg(p.chunk_members + chunk * p.max_members + mi) : -1;
         const bool member = m >= 0 && m < p.num_seqs;
         col_row[c] = member ? m * p.num_heads + kvh * G + (c - mi * G) : -1;
-        col_ok[c] = member && part < group_parts(p, m, checked_len(p, m, false));
+        const int Lm = member ? checked_len(p, m, false) : 0;
+        const int gm = member ? group_parts(p, m, Lm) : 0;
+        col_ok[c] = member && part < gm;
+        col_n[c] = col_ok[c] && c == mi * G ? (Lm + ps - 1) / ps : 0;
+        col_a[c] = gm;
+        col_b[c] = gm > p.part_base ? gm : p.part_base;
       }
       __syncthreads();
       // blocks come from the table of the first member that owns this partition
@@ -401,6 +552,44 @@ __global__ void __launch_bounds__(NW * 32)
 
   const int npre = nb_w < NST ? nb_w : NST;
   for (int k = 0; k < npre; ++k) issue(k);
+  // Grouped form, a sequence's own partition: when every other partial of its
+  // (sequence, kv head) is stored already (the counter, read with acquire, is one
+  // short of complete), this CTA combines the rows at its end without counting; the
+  // other partials' lines are fetched into L1 while the blocks stream.  Otherwise it
+  // counts at its end like every other CTA.
+  bool pre = false;
+  if constexpr (GROUP) {
+    __shared__ int sh_pre;
+    if (own_row) {  // the same for the whole CTA
+      if (threadIdx.x == 0) {
+        const int n = col_n[0], b = col_b[0];
+        const int expect = col_a[0] + (n > b ? n - b : 0);
+        sh_pre = ld_acquire_gpu(p.ws_cnt + col_row[0]) == expect - 1;
+      }
+      __syncthreads();
+      pre = sh_pre;
+      if (pre && warp == 0) {
+        // 128-byte lines: D / 32 of each partial output row, one each for m and l
+        const int a = col_a[0], b = col_b[0], n = col_n[0];
+        const int others = a + (n > b ? n - b : 0) - 1;
+        const int per = D / 32 + 2, total = G * others * per;
+        if (total <= 8 * 32) {
+          for (int i = lane; i < total; i += 32) {
+            // slot list [0, a) then [b, n); this CTA's own partition (list index
+            // a + part - b) is skipped
+            const int line = i % per, t = i / per, r = t % G, k2 = t / G;
+            const int k = k2 < a + (part - b) ? k2 : k2 + 1;
+            const int j = k < a ? k : b + (k - a);
+            const int row = col_row[0] + r;
+            const float* addr = line < D / 32 ? p.ws_o + o_index(p, row, j) + line * 32
+                                : line == D / 32 ? p.ws_m + ml_index(p, row, j)
+                                                 : p.ws_l + ml_index(p, row, j);
+            prefetch_l1(addr);
+          }
+        }
+      }
+    }
+  }
   int issued = npre;
   int k = 0;
   bool aborted = false;
@@ -682,12 +871,24 @@ __global__ void __launch_bounds__(NW * 32)
     const int64_t row = col_row[hh];
     if (nparts == 1) {
       store_elem(static_cast<TQ*>(p.out) + row * D + d, o);
+    } else if (pre) {
+      red[hh * (D + 2) + d] = o;  // this CTA's own partial, combined below (read in place)
     } else {
       st_hint(p.ws_o + o_index(p, row, part) + d, o, keep_policy);  // L2, for the merge
       if (d == 0) {
         st_hint(p.ws_m + ml_index(p, row, part), col_m[hh], keep_policy);
         st_hint(p.ws_l + ml_index(p, row, part), den, keep_policy);
       }
+    }
+  }
+  if constexpr (GROUP) {
+    if (pre) {
+      __syncthreads();  // the own partial is in shared memory
+      for (int r = warp; r < G; r += NW)
+        combine_row<TQ, D, true>(p, col_row[0] + r, col_a[0], col_b[0], col_n[0], lane, part,
+                                 red + r * (D + 2), col_m[r], col_l[r]);
+    } else if (nparts > 1) {
+      finish_rows<TQ, D, NW, C::kHeads>(p, col_row, col_n, col_a, col_b, G);
     }
   }
 }

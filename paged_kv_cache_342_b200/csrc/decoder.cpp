@@ -311,14 +311,15 @@ int prepare(pa_decoder* d, cudaStream_t comp, pa_step_info_t* info) {
     return PA_ERR_CUDA;
   }
 
-  const bool grouped = num_chunks > 0;
   info->num_cow = ncow;
   info->max_seq_len = max_len;
   info->partition_size = d->partition;
   info->num_chunks = num_chunks;
   info->max_chunk_parts = max_chunk_parts;
   info->first_part = first_part;
-  info->kernels = (ncow ? 1 : 0) + 1 + 1 + (grouped ? 1 : 0) + (parts > 1 ? 1 : 0);
+  // copies, the new tokens' write, the partition grid, then the merge (a grouped
+  // call launches its counters' clear before the grid instead)
+  info->kernels = (ncow ? 1 : 0) + 1 + 1 + (parts > 1 ? 1 : 0);
   info->slots = slots;
   info->cow_pairs = pairs;
   info->block_tables = tables;

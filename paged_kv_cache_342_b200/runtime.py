@@ -247,7 +247,8 @@ class PagedDecoder:
         _check(lib.pa_decoder_drain(self._h, self._stream_handle()), "pa_decoder_drain")
 
     def kernel_launches(self, meta: StepInfo) -> int:
-        """Library kernels one step launches (copy, write, group, partitions, merge)."""
+        """Library kernels one step launches (copies, new tokens' write, partition grid, merge
+        or, for a grouped batch, the clear of its arrival counters)."""
         return meta.kernels
 
     def _check_io(self, q, new_k, new_v, out, cuda: bool) -> None:

@@ -50,7 +50,8 @@ def test_workspace_bytes(pa):
     b = pa.pa_decode_workspace_bytes(8, 64, 128, 131072, 512)
     rows = 8 * 64 * 256
     align = lambda x: (x + 255) // 256 * 256
-    assert b == align(rows * 128 * 4) + 2 * align(rows * 4)
+    # partial outputs, maxima, exp-sums, then one int32 arrival counter per query row
+    assert b == align(rows * 128 * 4) + 2 * align(rows * 4) + align(8 * 64 * 4)
     assert pa.pa_decode_workspace_bytes(2, 4, 64, 1000, 0) == \
         pa.pa_decode_workspace_bytes(2, 4, 64, 1000, 512)
     assert pa.pa_decode_workspace_bytes(-1, 4, 64, 1000, 512) == 0

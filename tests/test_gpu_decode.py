@@ -163,10 +163,12 @@ def test_length_beyond_bound_is_skipped_and_reported(pa):
 # ---------------------------------------------------------------------------
 
 def run_grouped_case(pa, dtype, Hq, Hkv, D, bs, ps, prefix_len, tails, group_sizes, mm,
-                     seed=3):
+                     seed=3, ws_fill=None, calls=1):
     """Groups of sequences forked from one prefix through the block manager, with
     private tails written into their own blocks; compare the grouped call with the
-    oracle (and with the plain call)."""
+    oracle (and with the plain call).  ws_fill: a byte value, or "random", written over
+    the workspace first; calls: grouped calls made back to back on that workspace (the
+    result is the last one's, and every call must give the same bits)."""
     from oracle.allocator import BlockManager
     sizes = list(group_sizes)
     S = sum(sizes)
@@ -201,14 +203,24 @@ def run_grouped_case(pa, dtype, Hq, Hkv, D, bs, ps, prefix_len, tails, group_siz
     td, ld = torch.from_numpy(tables).cuda(), torch.from_numpy(sl).cuda()
     wsb = pa.pa_decode_workspace_bytes(S, Hq, D, max_len, ps)
     ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
-    out = torch.full((S, Hq, D), float("nan"), dtype=TORCH_DT[dtype], device="cuda")
+    if ws_fill == "random":
+        ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8,
+                               generator=torch.Generator().manual_seed(seed)))
+    elif ws_fill is not None:
+        ws.fill_(ws_fill)
     own = [min(p_, (int(L) - 1) // ps) if L > 0 else 0 for p_, L in zip(pp, sl)]
     first = min(own) if chunks else 0
-    pa.pa_decode_attention_grouped(out, qd, kd, vd, td, ld, scale, bs, Hkv, max_len,
-                                   torch.from_numpy(np.array(pp, np.int32)).cuda(),
-                                   torch.from_numpy(cm).cuda(), torch.from_numpy(cp).cuda(),
-                                   len(chunks), max([c[1] for c in chunks], default=0), ps,
-                                   ws if wsb else None, first_part=first)
+    results = []
+    for _ in range(calls):
+        out = torch.full((S, Hq, D), float("nan"), dtype=TORCH_DT[dtype], device="cuda")
+        pa.pa_decode_attention_grouped(out, qd, kd, vd, td, ld, scale, bs, Hkv, max_len,
+                                       torch.from_numpy(np.array(pp, np.int32)).cuda(),
+                                       torch.from_numpy(cm).cuda(), torch.from_numpy(cp).cuda(),
+                                       len(chunks), max([c[1] for c in chunks], default=0), ps,
+                                       ws if wsb else None, first_part=first)
+        results.append(out)
+    for r in results[1:]:
+        assert torch.equal(r.view(torch.int16), results[0].view(torch.int16))
     plain = torch.full_like(out, float("nan"))
     pa.pa_decode_attention(plain, qd, kd, vd, td, ld, scale, bs, Hkv, max_len, ps,
                            ws if wsb else None)
@@ -229,6 +241,10 @@ GROUP_CASES = [
     # a group beside two sequences of no group (their own prefixes): in the one grid the
     # group's shared partitions, then every sequence's own partitions from partition 0
     ("bf16", 8, 8, 128, 16, 64, 200, [3, 50, 0, 7, 130, 9], [4, 1, 1], 8),
+    # long shared partitions and one-token tails: the group CTAs finish last, so they
+    # combine their members' rows (8 members of one head; 4 members of 4 heads)
+    ("bf16", 8, 8, 128, 16, 512, 4100, [1] * 16, [16], 8),
+    ("bf16", 8, 2, 128, 16, 256, 2100, [1, 0, 2, 1], [4], 4),
 ]
 
 
@@ -240,6 +256,18 @@ def test_grouped_matches_oracle_and_plain(pa, case):
     assert_close(got, want, dtype, "grouped")
     assert_close(plain, want, dtype, "plain")
     assert np.abs(got - plain).max() <= 2e-2
+
+
+@pytest.mark.parametrize("fill", [0xFF, 0x00, "random"])
+def test_grouped_result_does_not_depend_on_workspace_contents(pa, fill):
+    """The grouped grid combines each row in the CTA that writes its last partial, on
+    arrival counters in the workspace that the call clears first: whatever the
+    workspace held, and on back-to-back calls, the bits are the same."""
+    case = GROUP_CASES[0]
+    got, _, want, _ = run_grouped_case(pa, *case, ws_fill=fill, calls=2)
+    ref, *_ = run_grouped_case(pa, *case)
+    assert np.array_equal(got, ref)
+    assert_close(got, want, case[0], "grouped")
 
 
 def test_grouped_call_uses_groups(pa):
