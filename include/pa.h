@@ -73,6 +73,8 @@ typedef void* pa_stream_t; /* a cudaStream_t */
                                     below first_part (those partitions were skipped)  */
 #define PA_DEVERR_ORDER 64u      /* pa_decode: a seq_order entry outside [0, num_seqs)
                                     (that grid row was skipped)                       */
+#define PA_DEVERR_SMEM 128u      /* grouped decode: a CTA's dynamic shared memory did
+                                    not start 1024-byte aligned (the CTA did nothing) */
 
 /* ------------------------------------------------------------------------- */
 /* GPU entry points                                                           */

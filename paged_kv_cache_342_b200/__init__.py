@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "NO_FREE_BLOCKS", 3: "UNKNOWN_SEQ"
 PA_STATIC_WORKSPACE_BYTES = 16 << 20
 PA_F32, PA_BF16, PA_F16, PA_FP8_E4M3 = 0, 1, 2, 3
 DEVERR_SLOT, DEVERR_COPY_BLOCK, DEVERR_TABLE, DEVERR_SEQ_LEN, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
-DEVERR_GROUP, DEVERR_ORDER = 32, 64
+DEVERR_GROUP, DEVERR_ORDER, DEVERR_SMEM = 32, 64, 128
 DEFAULT_PARTITION = 512
 
 

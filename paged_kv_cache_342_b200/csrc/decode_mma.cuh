@@ -110,7 +110,7 @@ __device__ __forceinline__ void e4m3_pairs_to_f16x2_bits(uint32_t w, uint32_t& e
 // the integer ALU busy: converting K by bit placement as well made the kernel ALU
 // bound (294 us against 254 us on the long-context GQA shape).  Codes 0x7F / 0xFF (NaN) are not special-cased
 // on that path; a cache holds them only for NaN inputs.
-template <typename T, int D, int BS, int NT, int NW, int NST, bool FP8 = false>
+template <typename T, int D, int BS, int NT, int NW, int NST, bool FP8 = false, bool PAD = true>
 struct MmaCfg {
   static constexpr int kHalves = D / 64;         // 128-byte column slabs per 16-bit row
   static constexpr int kSlabBytes = BS * 128;    // one slab of one tile
@@ -123,8 +123,15 @@ struct MmaCfg {
   static constexpr int kHeads = 8 * NT;
   static constexpr int kStageArea = NW * NST * kStageBytes;
   static constexpr int kRedBytes = NW * kHeads * (D + 2) * 4;
-  static constexpr int kSmemBytes =
-      1024 + (kStageArea > kRedBytes ? kStageArea : kRedBytes) + NW * NST * 8;
+  // dynamic shared memory from its 1024-aligned base: the stages (the warps' partial
+  // results reuse them at the end), the copy barriers, then the CTA's small per-column
+  // arrays (8 + NW arrays of kHeads 4-byte words and one flag word); PAD reserves 1024
+  // bytes in front for aligning a base that may not be aligned
+  static constexpr int kAreaBytes = kStageArea > kRedBytes ? kStageArea : kRedBytes;
+  static constexpr int kBarOff = kAreaBytes;
+  static constexpr int kSmallOff = kBarOff + NW * NST * 8;
+  static constexpr int kSmallBytes = ((8 + NW) * kHeads + 1) * 4;
+  static constexpr int kSmemBytes = (PAD ? 1024 : 0) + kSmallOff + kSmallBytes;
   static_assert(sizeof(T) == 2, "tensor-core path computes in 16-bit types");
   static_assert(BS % 16 == 0 && kSlabBytes % 1024 == 0, "slabs must stay 1024-byte aligned");
   static_assert(!FP8 || D % 128 == 0, "fp8 tiles are whole 128-byte slabs");
@@ -267,8 +274,7 @@ __device__ __forceinline__ void prefetch_l1(const void* addr) {
 template <typename TQ, int D, int NW, int H>
 __device__ __forceinline__ void finish_rows(const DecodeParams& p, const int* col_row,
                                             const int* col_n, const int* col_a,
-                                            const int* col_b, int G) {
-  __shared__ int fin[H];
+                                            const int* col_b, int* fin, int G) {
   __syncthreads();  // the CTA's partial stores are issued
   const int c = static_cast<int>(threadIdx.x);
   if (c < H) {
@@ -308,7 +314,8 @@ __global__ void __launch_bounds__(NW * 32)
   // launched to overlap the end of the kernel before it on the stream (typically the
   // write of the new tokens' K/V): nothing is read before that kernel is done
   grid_dependency_wait();
-  using C = MmaCfg<T, D, BS, NT, NW, NST, FP8>;
+  // the grouped form's one-warp CTAs keep no padding (one more CTA fits on an SM)
+  using C = MmaCfg<T, D, BS, NT, NW, NST, FP8, !GROUP>;
   using Ops = MmaOps<T>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int TT = C::kTT, KS = C::kKS;
@@ -319,17 +326,33 @@ __global__ void __launch_bounds__(NW * 32)
   constexpr bool kChunked = CHUNK && !GROUP && KS * NT <= 8;
   static_assert(!CHUNK || kChunked, "several partitions per CTA need a small tile");
 
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ int col_row[C::kHeads];  // q / out row (sequence * Hq + head) of each column
-  __shared__ int col_ok[C::kHeads];   // the column's result is written by this CTA
-  // grouped form: partitions of the column's sequence (n), the group's (a) and where
-  // its own start (b), set on the column that counts the sequence's partials
-  __shared__ int col_n[GROUP ? C::kHeads : 1], col_a[GROUP ? C::kHeads : 1],
-      col_b[GROUP ? C::kHeads : 1];
-  // 1024-byte alignment for the swizzle atoms
+  // All of the CTA's shared memory is dynamic (no static arrays): with nothing in
+  // front of it, the window's dynamic part starts 1024-byte aligned, as the 128-byte
+  // swizzle atoms need, and the grouped form relies on that (checked: a CTA that
+  // finds it otherwise reports PA_DEVERR_SMEM and does nothing)
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
+  if constexpr (!GROUP) {
+  } else if (base != raw) {
+    if (threadIdx.x == 0) set_error(p.err, PA_DEVERR_SMEM);
+    return;
+  }
   uint8_t* smem = smem_raw + (base - raw);
+  constexpr int H = C::kHeads;
+  int* const small = reinterpret_cast<int*>(smem + C::kSmallOff);
+  int* const col_row = small;       // q / out row (sequence * Hq + head) of each column
+  int* const col_ok = small + H;    // the column's result is written by this CTA
+  // grouped form: partitions of the column's sequence (n), the group's (a) and where
+  // its own start (b), set on the column that counts the sequence's partials
+  int* const col_n = small + 2 * H;
+  int* const col_a = small + 3 * H;
+  int* const col_b = small + 4 * H;
+  float* const col_m = reinterpret_cast<float*>(small + 5 * H);  // epilogue: max,
+  float* const col_l = reinterpret_cast<float*>(small + 6 * H);  // exp-sum per column
+  int* const fin = small + 7 * H;   // grouped form: this CTA merges the column's rows
+  float* const col_w = reinterpret_cast<float*>(small + 8 * H);  // [NW][H] warp weights
+  int* const sh_pre = small + (8 + NW) * H;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t4 = lane & 3;  // fragment row group / thread in group
@@ -431,7 +454,7 @@ __global__ void __launch_bounds__(NW * 32)
       p.block_tables + static_cast<int64_t>(table_seq) * p.max_blocks_per_seq + tok_begin / BS;
 
   const uint32_t stage0 = base + warp * NST * C::kStageBytes;
-  const uint32_t bar0 = base + (C::kSmemBytes - 1024 - NW * NST * 8) + warp * NST * 8;
+  const uint32_t bar0 = base + C::kBarOff + warp * NST * 8;
   if (lane == 0) {
 #pragma unroll
     for (int i = 0; i < NST; ++i) mbar_init(bar0 + 8 * i, 1);
@@ -559,15 +582,14 @@ __global__ void __launch_bounds__(NW * 32)
   // counts at its end like every other CTA.
   bool pre = false;
   if constexpr (GROUP) {
-    __shared__ int sh_pre;
     if (own_row) {  // the same for the whole CTA
       if (threadIdx.x == 0) {
         const int n = col_n[0], b = col_b[0];
         const int expect = col_a[0] + (n > b ? n - b : 0);
-        sh_pre = ld_acquire_gpu(p.ws_cnt + col_row[0]) == expect - 1;
+        *sh_pre = ld_acquire_gpu(p.ws_cnt + col_row[0]) == expect - 1;
       }
       __syncthreads();
-      pre = sh_pre;
+      pre = *sh_pre;
       if (pre && warp == 0) {
         // 128-byte lines: D / 32 of each partial output row, one each for m and l
         const int a = col_a[0], b = col_b[0], n = col_n[0];
@@ -836,8 +858,6 @@ __global__ void __launch_bounds__(NW * 32)
   __syncthreads();
   // per head column, once: the max M, the exp-sum and each warp's weight
   // exp2(m_w - M) * v_scale / sum, so that an output element is NW fused multiply-adds
-  __shared__ float col_w[NW][C::kHeads];
-  __shared__ float col_m[C::kHeads], col_l[C::kHeads];
   if (threadIdx.x < C::kHeads) {
     const int hh = threadIdx.x;
     float M = -INFINITY;
@@ -853,7 +873,7 @@ __global__ void __launch_bounds__(NW * 32)
     // FP8: the V operands carry the code values times 2^-8
     const float sc = den > 0.f ? (FP8 ? p.v_scale * 256.f : p.v_scale) / den : 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) col_w[w][hh] = f[w] * sc;
+    for (int w = 0; w < NW; ++w) col_w[w * H + hh] = f[w] * sc;
     col_m[hh] = M;
     col_l[hh] = den;
   }
@@ -865,7 +885,7 @@ __global__ void __launch_bounds__(NW * 32)
     float o = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w)
-      o = fmaf(red[(w * C::kHeads + hh) * (D + 2) + d], col_w[w][hh], o);
+      o = fmaf(red[(w * C::kHeads + hh) * (D + 2) + d], col_w[w * H + hh], o);
     const float den = col_l[hh];
     if (!(den > 0.f)) o = 0.f;
     const int64_t row = col_row[hh];
@@ -888,7 +908,7 @@ __global__ void __launch_bounds__(NW * 32)
         combine_row<TQ, D, true>(p, col_row[0] + r, col_a[0], col_b[0], col_n[0], lane, part,
                                  red + r * (D + 2), col_m[r], col_l[r]);
     } else if (nparts > 1) {
-      finish_rows<TQ, D, NW, C::kHeads>(p, col_row, col_n, col_a, col_b, G);
+      finish_rows<TQ, D, NW, C::kHeads>(p, col_row, col_n, col_a, col_b, fin, G);
     }
   }
 }

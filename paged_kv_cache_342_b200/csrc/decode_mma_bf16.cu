@@ -17,7 +17,7 @@ cudaError_t launch(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   constexpr int NW = kW < 1 ? 1 : (kW > 4 ? 4 : kW);
   constexpr int kRaw = kBudget / (NW * kStage);
   constexpr int NST = kRaw < 2 ? 2 : (kRaw > 4 ? 4 : kRaw);
-  using C = MmaCfg<__nv_bfloat16, D, BS, NT, NW, NST, false>;
+  using C = MmaCfg<__nv_bfloat16, D, BS, NT, NW, NST, false, !GROUP>;
   const uint64_t rows = static_cast<uint64_t>(p.num_blocks) * p.num_kv_heads * BS;
   if (rows > 0x7fffffffull) return cudaErrorInvalidValue;  // int32 row coordinates
   CUtensorMap tmk, tmv;
