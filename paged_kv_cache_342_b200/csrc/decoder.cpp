@@ -373,10 +373,10 @@ int launch(pa_decoder* d, const pa_step_info_t* info, const void* q, const void*
   a.cache_dtype = c.cache_dtype;
   a.k_scale = c.k_scale;
   a.v_scale = c.v_scale;
-  // longest first, except for batches with prefix groups: there the per-sequence
-  // kernel reads only short tails, and the order measured slower (202 us against 191 us
-  // on the 256-sequence shared-prefix batch)
-  a.seq_order = info->num_chunks > 0 ? nullptr : d->d<int32_t>(st, d->off_order);
+  // longest first, prefix groups included: in the grouped grid the sequences' own
+  // partitions follow the groups' shared ones, and taking them longest first shortens
+  // the end of the grid (173.1 against 174.9 us on the 256-sequence shared-prefix batch)
+  a.seq_order = d->d<int32_t>(st, d->off_order);
   if (info->num_chunks > 0) {
     a.prefix_parts = d->d<int32_t>(st, d->off_pparts);
     a.chunk_members = d->d<int32_t>(st, d->off_cmembers);
