@@ -243,17 +243,7 @@ __device__ __forceinline__ void combine_row(const DecodeParams& p, int row, int 
   for (int j = 0; j < DPL; ++j) store_elem(out + j, acc[j] * inv);
 }
 
-// Grouped form, after a CTA has stored its partials: it counts them on the arrival
-// counter of each (sequence, kv head) it wrote (entry s * Hq + kv head * G), and the
-// CTA whose count completes a counter combines that sequence's G heads itself, so
-// no merge launch follows the grid.  A (sequence, kv head) expects one partial per
-// partition the call writes for it: the group's below a = group_parts(s), then its
-// own from b = max(a, part_base) to its last, n - 1.  col_n / col_a / col_b hold n, a
-// and b for a column that counts (its first head), col_n 0 for the others.  The count
-// is one acquire-release atomic by the counting thread after a block barrier: it
-// publishes every thread's partial stores before it, and the CTA that completes the
-// count sees the other CTAs' partials after it (read from L2 after a second barrier).
-// Called by every thread of the CTA.
+// Arrival counters and the partials they guard (device scope).
 __device__ __forceinline__ int atomic_add_acq_rel_gpu(int* addr, int v) {
   int old;
   asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
@@ -271,6 +261,17 @@ __device__ __forceinline__ void prefetch_l1(const void* addr) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(addr));
 }
 
+// Grouped form, after a CTA has stored its partials: it counts them on the arrival
+// counter of each (sequence, kv head) it wrote (entry s * Hq + kv head * G), and the
+// CTA whose count completes a counter combines that sequence's G heads itself, so
+// no merge launch follows the grid.  A (sequence, kv head) expects one partial per
+// partition the call writes for it: the group's below a = group_parts(s), then its
+// own from b = max(a, part_base) to its last, n - 1.  col_n / col_a / col_b hold n, a
+// and b for a column that counts (its first head), col_n 0 for the others.  The count
+// is one acquire-release atomic by the counting thread after a block barrier: it
+// publishes every thread's partial stores before it, and the CTA that completes the
+// count sees the other CTAs' partials after it (read from L2 after a second barrier).
+// Called by every thread of the CTA.
 template <typename TQ, int D, int NW, int H>
 __device__ __forceinline__ void finish_rows(const DecodeParams& p, const int* col_row,
                                             const int* col_n, const int* col_a,
