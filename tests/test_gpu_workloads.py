@@ -91,6 +91,10 @@ def test_workload_step(pa, name, fork_step, seed):
     assert np.array_equal(tables_c, res["tables"]) and np.array_equal(lens_c, res["seq_lens"])
     if fork_step:
         assert len(pairs_c) == 224
+    # kernels of the step: copies (if any), the cache write, the partition grid, then
+    # the merge - or, for a grouped batch, the clear of its arrival counters before it
+    several = -(-meta.max_len // meta.partition_size) > 1
+    assert meta.kernels == (1 if meta.num_cow else 0) + 2 + (1 if several else 0)
 
     # ---- caches ---------------------------------------------------------------
     touched = set((res["slots"] // cfg.block_size).tolist()) | set(res["pairs"][:, 1].tolist())
